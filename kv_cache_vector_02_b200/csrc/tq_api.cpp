@@ -1,0 +1,290 @@
+// C ABI of libtq: validation, parameter upload, dispatch.  The arithmetic of
+// the hot path runs in the CUDA translation units; this file only checks
+// arguments, owns the context and launches.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include <cuda_fp16.h>
+
+#include "tq_internal.h"
+
+using tq::kDim;
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+
+void tq::count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+namespace {
+
+tq::ChunkLayout make_layout(int code_bits, bool prod) {
+    tq::ChunkLayout L{};
+    L.prod = prod;
+    L.code_row = kDim * tq::container_width(code_bits) / 8;
+    int off = tq::kPage * L.code_row;
+    if (prod) {
+        L.signs_off = off;
+        off += tq::kPage * (kDim / 8);
+    } else {
+        L.signs_off = -1;
+    }
+    L.norm_off = off;
+    off += tq::kPage * 4;
+    if (prod) {
+        L.gamma_off = off;
+        off += tq::kPage * 4;
+    } else {
+        L.gamma_off = -1;
+    }
+    L.bytes = off;
+    return L;
+}
+
+tq::Codebook make_codebook(const std::vector<double>& c, const std::vector<double>& t, int bits) {
+    tq::Codebook cb{};
+    cb.bits = bits;
+    cb.levels = 1 << bits;
+    cb.width = tq::container_width(bits);
+    for (int j = 0; j < tq::kMaxLevels; ++j) {
+        cb.c[j] = j < cb.levels ? float(c[j]) : 0.f;
+        cb.t[j] = j < cb.levels - 1 ? float(t[j]) : INFINITY;
+    }
+    return cb;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+uint64_t tq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* tq_status_string(tq_status s) {
+    switch (s) {
+        case TQ_OK: return "TQ_OK";
+        case TQ_ERR_INVALID_ARG: return "TQ_ERR_INVALID_ARG";
+        case TQ_ERR_UNSUPPORTED: return "TQ_ERR_UNSUPPORTED";
+        case TQ_ERR_CUDA: return "TQ_ERR_CUDA";
+        case TQ_ERR_OOM: return "TQ_ERR_OOM";
+        case TQ_ERR_DEVICE: return "TQ_ERR_DEVICE";
+    }
+    return "TQ_ERR_UNKNOWN";
+}
+
+static tq_status validate_init(int head_dim, int bits, int rotation, int key_mode) {
+    if (head_dim != kDim) return TQ_ERR_UNSUPPORTED;
+    if (bits < 2 || bits > 4) return TQ_ERR_UNSUPPORTED;
+    if (rotation != TQ_ROT_HAAR && rotation != TQ_ROT_HADAMARD) return TQ_ERR_UNSUPPORTED;
+    if (key_mode != TQ_KEY_PROD && key_mode != TQ_KEY_MSE) return TQ_ERR_UNSUPPORTED;
+    return TQ_OK;
+}
+
+static void fill_host(tq_ctx* ctx, int head_dim, int bits, uint64_t seed, int rotation, int key_mode) {
+    ctx->host = tq::make_host_params(head_dim, bits, seed, rotation, key_mode);
+    const tq::HostParams& H = ctx->host;
+    ctx->cb_value = make_codebook(H.cv, H.tv, H.vbits);
+    ctx->cb_key = make_codebook(H.ck, H.tk, H.kbits);
+    ctx->lay_value = make_layout(H.vbits, false);
+    ctx->lay_key = make_layout(H.kbits, key_mode == TQ_KEY_PROD);
+}
+
+tq_status tq_init_host(int head_dim, int bits, uint64_t seed, int rotation, int key_mode, tq_ctx** out) {
+    if (!out) return TQ_ERR_INVALID_ARG;
+    *out = nullptr;
+    const tq_status v = validate_init(head_dim, bits, rotation, key_mode);
+    if (v != TQ_OK) return v;
+    tq_ctx* ctx = new (std::nothrow) tq_ctx();
+    if (!ctx) return TQ_ERR_OOM;
+    ctx->host_only = true;
+    fill_host(ctx, head_dim, bits, seed, rotation, key_mode);
+    *out = ctx;
+    return TQ_OK;
+}
+
+tq_status tq_init(int head_dim, int bits, uint64_t seed, int rotation, int key_mode, tq_ctx** out) {
+    if (!out) return TQ_ERR_INVALID_ARG;
+    *out = nullptr;
+    const tq_status v = validate_init(head_dim, bits, rotation, key_mode);
+    if (v != TQ_OK) return v;
+
+    tq_ctx* ctx = new (std::nothrow) tq_ctx();
+    if (!ctx) return TQ_ERR_OOM;
+    if (cudaGetDevice(&ctx->device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&ctx->sm_count, cudaDevAttrMultiProcessorCount, ctx->device) != cudaSuccess) {
+        delete ctx;
+        cudaGetLastError();
+        return TQ_ERR_CUDA;
+    }
+    fill_host(ctx, head_dim, bits, seed, rotation, key_mode);
+    const tq::HostParams& H = ctx->host;
+
+    // fp32 device copies: R, R^T, M^T, S, S^T
+    const size_t n = size_t(kDim) * kDim;
+    std::vector<float> blob(5 * n);
+    float* R = blob.data();
+    float* RT = R + n;
+    float* MT = RT + n;
+    float* S = MT + n;
+    float* ST = S + n;
+    for (int i = 0; i < kDim; ++i)
+        for (int j = 0; j < kDim; ++j) {
+            R[i * kDim + j] = float(H.R[size_t(i) * kDim + j]);
+            RT[j * kDim + i] = float(H.R[size_t(i) * kDim + j]);
+            MT[j * kDim + i] = float(H.M[size_t(i) * kDim + j]);
+            S[i * kDim + j] = float(H.S[size_t(i) * kDim + j]);
+            ST[j * kDim + i] = float(H.S[size_t(i) * kDim + j]);
+        }
+    const size_t bytes = blob.size() * sizeof(float);
+    if (cudaMalloc(&ctx->dev_block, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        delete ctx;
+        return TQ_ERR_OOM;
+    }
+    if (cudaMalloc(reinterpret_cast<void**>(&ctx->dev_error), sizeof(uint32_t)) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(ctx->dev_block);
+        delete ctx;
+        return TQ_ERR_OOM;
+    }
+    if (cudaMemcpy(ctx->dev_block, blob.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemset(ctx->dev_error, 0, sizeof(uint32_t)) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(ctx->dev_block);
+        cudaFree(ctx->dev_error);
+        delete ctx;
+        return TQ_ERR_CUDA;
+    }
+    const float* base = static_cast<const float*>(ctx->dev_block);
+    ctx->dev.R = base;
+    ctx->dev.RT = base + n;
+    ctx->dev.MT = base + 2 * n;
+    ctx->dev.S = base + 3 * n;
+    ctx->dev.ST = base + 4 * n;
+    *out = ctx;
+    return TQ_OK;
+}
+
+tq_status tq_destroy(tq_ctx* ctx) {
+    if (!ctx) return TQ_OK;
+    if (ctx->host_only) {
+        delete ctx;
+        return TQ_OK;
+    }
+    cudaDeviceSynchronize();
+    cudaFree(ctx->dev_block);
+    cudaFree(ctx->dev_error);
+    cudaGetLastError();
+    delete ctx;
+    return TQ_OK;
+}
+
+size_t tq_chunk_bytes(const tq_ctx* ctx, int kind) {
+    if (!ctx) return 0;
+    if (kind == TQ_KIND_KEY) return size_t(ctx->lay_key.bytes);
+    if (kind == TQ_KIND_VALUE) return size_t(ctx->lay_value.bytes);
+    return 0;
+}
+
+int tq_code_bits(const tq_ctx* ctx, int kind) {
+    if (!ctx) return -1;
+    if (kind == TQ_KIND_KEY) return ctx->host.kbits;
+    if (kind == TQ_KIND_VALUE) return ctx->host.vbits;
+    return -1;
+}
+
+tq_status tq_export_params(const tq_ctx* ctx, double* R, int8_t* S, int8_t* hsigns, double* cv, double* tv,
+                           double* ck, double* tk) {
+    if (!ctx) return TQ_ERR_INVALID_ARG;
+    const tq::HostParams& H = ctx->host;
+    if (R) std::memcpy(R, H.R.data(), H.R.size() * sizeof(double));
+    if (S) std::memcpy(S, H.S.data(), H.S.size());
+    if (hsigns && !H.hsigns.empty()) std::memcpy(hsigns, H.hsigns.data(), H.hsigns.size());
+    if (cv) std::memcpy(cv, H.cv.data(), H.cv.size() * sizeof(double));
+    if (tv) std::memcpy(tv, H.tv.data(), H.tv.size() * sizeof(double));
+    if (ck) std::memcpy(ck, H.ck.data(), H.ck.size() * sizeof(double));
+    if (tk) std::memcpy(tk, H.tk.data(), H.tk.size() * sizeof(double));
+    return TQ_OK;
+}
+
+tq_status tq_compress(const tq_ctx* ctx, const uint16_t* k, const uint16_t* v, int T, int Hkv,
+                      const int32_t* slot_mapping, uint8_t* k_cache, uint8_t* v_cache, int num_blocks,
+                      void* stream) {
+    if (!ctx || ctx->host_only || T < 0 || Hkv < 1 || num_blocks < 0) return TQ_ERR_INVALID_ARG;
+    if (T == 0) return TQ_OK;
+    if (!slot_mapping || (!k && !v)) return TQ_ERR_INVALID_ARG;
+    if ((k && !k_cache) || (v && !v_cache)) return TQ_ERR_INVALID_ARG;
+    if ((k && (!aligned16(k) || !aligned16(k_cache))) || (v && (!aligned16(v) || !aligned16(v_cache))))
+        return TQ_ERR_INVALID_ARG;
+    if ((long long)T * Hkv > (1ll << 31) - 1) return TQ_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (k && tq::launch_compress(ctx, TQ_KIND_KEY, k, T, Hkv, slot_mapping, k_cache, num_blocks, s) != cudaSuccess)
+        return TQ_ERR_CUDA;
+    if (v && tq::launch_compress(ctx, TQ_KIND_VALUE, v, T, Hkv, slot_mapping, v_cache, num_blocks, s) != cudaSuccess)
+        return TQ_ERR_CUDA;
+    return TQ_OK;
+}
+
+tq_status tq_decompress(const tq_ctx* ctx, int kind, const uint8_t* cache, int num_blocks,
+                        const int32_t* slot_mapping, int T, int Hkv, void* out, int out_fp32, void* stream) {
+    if (!ctx || ctx->host_only || T < 0 || Hkv < 1 || num_blocks < 0) return TQ_ERR_INVALID_ARG;
+    if (kind != TQ_KIND_KEY && kind != TQ_KIND_VALUE) return TQ_ERR_INVALID_ARG;
+    if (T == 0) return TQ_OK;
+    if (!cache || !slot_mapping || !out) return TQ_ERR_INVALID_ARG;
+    if (!aligned16(cache) || !aligned16(out)) return TQ_ERR_INVALID_ARG;
+    if (tq::launch_decompress(ctx, kind, cache, num_blocks, slot_mapping, T, Hkv, out, out_fp32,
+                              static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return TQ_ERR_CUDA;
+    return TQ_OK;
+}
+
+size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_seq_len) {
+    if (!ctx || ctx->host_only || B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || max_seq_len < 0) return 0;
+    return tq::plan_decode(ctx, B, Hq, Hkv, max_seq_len).bytes;
+}
+
+tq_status tq_decode_attention(const tq_ctx* ctx, const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                              int num_blocks, const int32_t* block_table, int max_blocks, const int32_t* seq_lens,
+                              int B, int Hq, int Hkv, int max_seq_len, float scale, void* out, int out_fp32,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    if (!ctx || ctx->host_only || B < 0 || Hq < 1 || Hkv < 1 || max_blocks < 0 || num_blocks < 0 || max_seq_len < 0)
+        return TQ_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0 || Hq / Hkv > 16) return TQ_ERR_INVALID_ARG;
+    if (B == 0) return TQ_OK;
+    if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !out || !workspace) return TQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(workspace))
+        return TQ_ERR_INVALID_ARG;
+    if (!(scale >= 0.f) || !std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
+    const tq::DecodePlan plan = tq::plan_decode(ctx, B, Hq, Hkv, max_seq_len);
+    if (workspace_bytes < plan.bytes) return TQ_ERR_INVALID_ARG;
+    if (scale == 0.f) scale = 1.0f / std::sqrt(float(kDim));
+    if (tq::launch_decode(ctx, plan, q, k_cache, v_cache, num_blocks, block_table, max_blocks, seq_lens, B, Hq, Hkv,
+                          max_seq_len, scale, out, out_fp32, workspace, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+        return TQ_ERR_CUDA;
+    return TQ_OK;
+}
+
+tq_status tq_get_device_error(const tq_ctx* ctx, void* stream, uint32_t* code) {
+    if (!ctx || ctx->host_only || !code) return TQ_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t h = 0;
+    if (cudaMemcpyAsync(&h, ctx->dev_error, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return TQ_ERR_CUDA;
+    }
+    if (h && (cudaMemsetAsync(ctx->dev_error, 0, sizeof(uint32_t), s) != cudaSuccess ||
+              cudaStreamSynchronize(s) != cudaSuccess)) {
+        cudaGetLastError();
+        return TQ_ERR_CUDA;
+    }
+    *code = h;
+    return h ? TQ_ERR_DEVICE : TQ_OK;
+}
+
+}  // extern "C"

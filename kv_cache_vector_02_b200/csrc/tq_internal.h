@@ -1,0 +1,103 @@
+// Internal declarations shared by the host API and the CUDA launchers of libtq.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "../../include/tq.h"
+
+namespace tq {
+
+constexpr int kDim = 128;       // head_dim supported on the device
+constexpr int kPage = 16;       // tokens per page chunk
+constexpr int kMaxLevels = 16;  // up to 4-bit codebooks
+
+// fp64 parameters built on the host by tq_init.
+struct HostParams {
+    int d = 0, bits = 0, rotation = 0, key_mode = 0;
+    int vbits = 0, kbits = 0;
+    std::vector<double> R;        // [d*d] row-major, y = R^T x
+    std::vector<int8_t> S;        // [d*d] row-major, (S r)_j = sum_i S[j][i] r_i
+    std::vector<int8_t> hsigns;   // [d] Hadamard signs (rotation == 1)
+    std::vector<double> M;        // [d*d] row-major, M = S R
+    std::vector<double> cv, tv;   // value codebook / interior boundaries
+    std::vector<double> ck, tk;   // key codebook / interior boundaries
+};
+
+HostParams make_host_params(int d, int bits, uint64_t seed, int rotation, int key_mode);
+
+// Codebook of one kind as the kernels see it (by value, kernel parameter space).
+struct Codebook {
+    float c[kMaxLevels];      // levels (unit variance)
+    float t[kMaxLevels];      // interior boundaries t[0..L-2]
+    int bits;                 // code bits
+    int width;                // container width (4, 2 or 1)
+    int levels;               // 2^bits
+};
+
+// Byte geometry of one 16-token chunk.
+struct ChunkLayout {
+    int code_row;     // bytes of packed codes per token (d * width / 8)
+    int signs_off;    // offset of signs[16][d/8] (prod keys), else -1
+    int norm_off;     // offset of norm f32[16]
+    int gamma_off;    // offset of gamma f32[16] (prod keys), else -1
+    int bytes;        // chunk size
+    bool prod;        // QJL key chunk
+};
+
+// Device copies of the parameters (one allocation owned by the context).
+struct DeviceParams {
+    const float* R;    // [d*d] R[i][j] row-major
+    const float* RT;   // [d*d] R^T row-major
+    const float* MT;   // [d*d] M^T row-major, MT[i][j] = (S R)[j][i]
+    const float* S;    // [d*d] S row-major as +-1.0f
+    const float* ST;   // [d*d] S^T row-major
+};
+
+inline int container_width(int b) { return b >= 3 ? 4 : (b == 2 ? 2 : 1); }
+
+}  // namespace tq
+
+struct tq_ctx {
+    bool host_only = false;         // built by tq_init_host: no device state
+    int device = 0;
+    int sm_count = 0;
+    tq::HostParams host;
+    tq::Codebook cb_value{}, cb_key{};
+    tq::ChunkLayout lay_value{}, lay_key{};
+    tq::DeviceParams dev{};
+    void* dev_block = nullptr;      // all device parameters
+    uint32_t* dev_error = nullptr;  // device error word
+};
+
+namespace tq {
+
+// Adds n to the process-wide launch counter (tq_launch_count).
+void count_launches(unsigned n);
+
+// Kernel launchers (CUDA translation units).  Each returns cudaSuccess or the
+// launch error.
+cudaError_t launch_compress(const tq_ctx* ctx, int kind, const uint16_t* x, int T, int H, const int32_t* slots,
+                            uint8_t* cache, int num_blocks, cudaStream_t stream);
+cudaError_t launch_decompress(const tq_ctx* ctx, int kind, const uint8_t* cache, int num_blocks,
+                              const int32_t* slots, int T, int H, void* out, int out_fp32, cudaStream_t stream);
+
+struct DecodePlan {
+    int splits;          // split-K factor over the pages of a sequence
+    int pages_per_split; // pages handled by one split
+    int max_pages;       // ceil(max_seq_len / 16)
+    size_t partial_off;  // workspace offsets (bytes)
+    size_t qprep_off;
+    size_t ticket_off;
+    size_t bytes;        // total workspace
+};
+DecodePlan plan_decode(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_seq_len);
+cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint16_t* q, const uint8_t* kc,
+                          const uint8_t* vc, int num_blocks, const int32_t* block_table, int max_blocks,
+                          const int32_t* seq_lens, int B, int Hq, int Hkv, int max_seq_len, float scale, void* out,
+                          int out_fp32, void* workspace, cudaStream_t stream);
+
+}  // namespace tq

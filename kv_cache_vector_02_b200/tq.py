@@ -1,0 +1,211 @@
+"""Thin ctypes binding of libtq (include/tq.h).
+
+Argument marshalling only: every step of the compress / decode path runs in the
+CUDA kernels of libtq.so.  Functions keep the C names; tensors are torch CUDA
+tensors (device pointers are taken with ``data_ptr()``), streams default to
+torch's current stream.  A non-OK status raises :class:`TQError`.
+
+The library must have been built (``python -m kv_cache_vector_02_b200.build``
+or ``__graft_entry__.build()``); importing this module without it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import numpy as np
+
+_LIB_PATH = Path(__file__).resolve().parent / "libtq.so"
+
+TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA, TQ_ERR_OOM, TQ_ERR_DEVICE = range(6)
+ROT_HAAR, ROT_HADAMARD = 0, 1
+KEY_PROD, KEY_MSE = 0, 1
+KIND_KEY, KIND_VALUE = 0, 1
+DEVERR_SLOT, DEVERR_BLOCK, DEVERR_SEQLEN, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+
+EXPORTED = ("tq_init", "tq_init_host", "tq_destroy", "tq_chunk_bytes", "tq_code_bits", "tq_export_params", "tq_compress",
+            "tq_decompress", "tq_decode_workspace_bytes", "tq_decode_attention", "tq_get_device_error",
+            "tq_launch_count", "tq_status_string")
+
+
+class TQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s: %s" % (what, _lib.tq_status_string(status).decode()))
+
+
+def _load():
+    if not _LIB_PATH.exists():
+        raise ImportError("libtq.so not built: run `python -m kv_cache_vector_02_b200.build`")
+    L = ctypes.CDLL(str(_LIB_PATH))
+    P, I, Z, U64, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64, ctypes.c_float
+    sig = {
+        "tq_init": (I, [I, I, U64, I, I, ctypes.POINTER(P)]),
+        "tq_init_host": (I, [I, I, U64, I, I, ctypes.POINTER(P)]),
+        "tq_destroy": (I, [P]),
+        "tq_chunk_bytes": (Z, [P, I]),
+        "tq_code_bits": (I, [P, I]),
+        "tq_export_params": (I, [P, P, P, P, P, P, P, P]),
+        "tq_compress": (I, [P, P, P, I, I, P, P, P, I, P]),
+        "tq_decompress": (I, [P, I, P, I, P, I, I, P, I, P]),
+        "tq_decode_workspace_bytes": (Z, [P, I, I, I, I]),
+        "tq_decode_attention": (I, [P, P, P, P, I, P, I, P, I, I, I, I, F, P, I, P, Z, P]),
+        "tq_get_device_error": (I, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
+        "tq_launch_count": (ctypes.c_uint64, []),
+        "tq_status_string": (ctypes.c_char_p, [I]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
+_lib = _load()
+
+
+def library_path() -> str:
+    return str(_LIB_PATH)
+
+
+def _check(status: int, what: str):
+    if status != TQ_OK:
+        raise TQError(status, what)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class Context:
+    """Owns one libtq context (tq_init / tq_destroy)."""
+
+    def __init__(self, handle: int, head_dim: int, bits: int, seed: int, rotation: int, key_mode: int):
+        self.handle = handle
+        self.head_dim, self.bits, self.seed, self.rotation, self.key_mode = head_dim, bits, seed, rotation, key_mode
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h:
+            _lib.tq_destroy(h)
+            self.handle = None
+
+    @property
+    def _as_parameter_(self):
+        return self.handle
+
+
+def tq_init(head_dim: int = 128, bits: int = 4, seed: int = 0, rotation: int = ROT_HAAR,
+            key_mode: int = KEY_PROD) -> Context:
+    h = ctypes.c_void_p()
+    _check(_lib.tq_init(head_dim, bits, seed, rotation, key_mode, ctypes.byref(h)), "tq_init")
+    return Context(h.value, head_dim, bits, seed, rotation, key_mode)
+
+
+def tq_init_host(head_dim: int = 128, bits: int = 4, seed: int = 0, rotation: int = ROT_HAAR,
+                 key_mode: int = KEY_PROD) -> Context:
+    """Host-only context (parameters on the host, no device touched)."""
+    h = ctypes.c_void_p()
+    _check(_lib.tq_init_host(head_dim, bits, seed, rotation, key_mode, ctypes.byref(h)), "tq_init_host")
+    return Context(h.value, head_dim, bits, seed, rotation, key_mode)
+
+
+def tq_destroy(ctx: Context):
+    if ctx.handle:
+        _check(_lib.tq_destroy(ctx.handle), "tq_destroy")
+        ctx.handle = None
+
+
+def tq_chunk_bytes(ctx: Context, kind: int) -> int:
+    return int(_lib.tq_chunk_bytes(ctx.handle, kind))
+
+
+def tq_code_bits(ctx: Context, kind: int) -> int:
+    return int(_lib.tq_code_bits(ctx.handle, kind))
+
+
+def tq_export_params(ctx: Context) -> dict:
+    d = ctx.head_dim
+    bv = tq_code_bits(ctx, KIND_VALUE)
+    bk = tq_code_bits(ctx, KIND_KEY)
+    out = {
+        "R": np.empty((d, d), np.float64), "S": np.empty((d, d), np.int8), "hsigns": np.zeros(d, np.int8),
+        "cv": np.empty(1 << bv, np.float64), "tv": np.empty((1 << bv) - 1, np.float64),
+        "ck": np.empty(1 << bk, np.float64), "tk": np.empty(max((1 << bk) - 1, 1), np.float64),
+    }
+    p = {k: v.ctypes.data_as(ctypes.c_void_p) for k, v in out.items()}
+    _check(_lib.tq_export_params(ctx.handle, p["R"], p["S"], p["hsigns"], p["cv"], p["tv"], p["ck"], p["tk"]),
+           "tq_export_params")
+    out["tk"] = out["tk"][: (1 << bk) - 1]
+    if ctx.rotation != ROT_HADAMARD:
+        out["hsigns"] = None
+    return out
+
+
+def tq_compress(ctx: Context, k, v, slot_mapping, k_cache, v_cache, stream=None):
+    """k, v: [T, Hkv, 128] fp16 CUDA tensors (either may be None); caches [num_blocks, Hkv, chunk] uint8."""
+    ref = k if k is not None else v
+    T, Hkv = int(ref.shape[0]), int(ref.shape[1])
+    cache = k_cache if k_cache is not None else v_cache
+    num_blocks = int(cache.shape[0])
+    _check(_lib.tq_compress(ctx.handle, _ptr(k), _ptr(v), T, Hkv, _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
+                            num_blocks, _stream(stream)), "tq_compress")
+
+
+def tq_decompress(ctx: Context, kind: int, cache, slot_mapping, out, stream=None):
+    """out: [T, Hkv, 128] fp16 or fp32 CUDA tensor."""
+    import torch
+    T, Hkv = int(out.shape[0]), int(out.shape[1])
+    _check(_lib.tq_decompress(ctx.handle, kind, _ptr(cache), int(cache.shape[0]), _ptr(slot_mapping), T, Hkv,
+                              _ptr(out), 1 if out.dtype == torch.float32 else 0, _stream(stream)), "tq_decompress")
+
+
+def tq_decode_workspace_bytes(ctx: Context, B: int, Hq: int, Hkv: int, max_seq_len: int) -> int:
+    n = int(_lib.tq_decode_workspace_bytes(ctx.handle, B, Hq, Hkv, max_seq_len))
+    if n == 0:
+        raise TQError(TQ_ERR_INVALID_ARG, "tq_decode_workspace_bytes")
+    return n
+
+
+def tq_decode_attention(ctx: Context, q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int, out,
+                        workspace, scale: float = 0.0, Hkv: int | None = None, stream=None):
+    """q: [B, Hq, 128] fp16; caches [num_blocks, Hkv, chunk] uint8; block_table [B, max_blocks] int32;
+    seq_lens [B] int32; out [B, Hq, 128] fp16 or fp32; workspace uint8 tensor (zeroed once)."""
+    import torch
+    B, Hq = int(q.shape[0]), int(q.shape[1])
+    if Hkv is None:
+        Hkv = int(k_cache.shape[1])
+    _check(_lib.tq_decode_attention(ctx.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache), int(k_cache.shape[0]),
+                                    _ptr(block_table), int(block_table.shape[1]), _ptr(seq_lens), B, Hq, Hkv,
+                                    int(max_seq_len), float(scale), _ptr(out), 1 if out.dtype == torch.float32 else 0,
+                                    _ptr(workspace), int(workspace.numel() * workspace.element_size()),
+                                    _stream(stream)), "tq_decode_attention")
+
+
+def tq_get_device_error(ctx: Context, stream=None) -> int:
+    code = ctypes.c_uint32(0)
+    st = _lib.tq_get_device_error(ctx.handle, _stream(stream), ctypes.byref(code))
+    if st not in (TQ_OK, TQ_ERR_DEVICE):
+        raise TQError(st, "tq_get_device_error")
+    return int(code.value)
+
+
+def tq_launch_count() -> int:
+    return int(_lib.tq_launch_count())
+
+
+def tq_status_string(status: int) -> str:
+    return _lib.tq_status_string(status).decode()

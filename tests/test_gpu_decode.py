@@ -1,0 +1,186 @@
+"""GPU decode attention and decompress parity against the oracle."""
+import math
+
+import numpy as np
+import pytest
+
+from parity import DECODE_ATOL, gpu_compress, gpu_ctx
+
+pytestmark = pytest.mark.gpu
+
+
+def _decode_gpu(ctx, q, kc, vc, bt, seq_lens, max_seq_len, Hkv, out_fp32=True, scale=0.0):
+    import torch
+    from kv_cache_vector_02_b200 import tq
+    dev = torch.device("cuda")
+    q = torch.as_tensor(q).to(dev)
+    B, Hq = q.shape[0], q.shape[1]
+    kc = torch.as_tensor(kc).to(dev)
+    vc = torch.as_tensor(vc).to(dev)
+    bt = torch.as_tensor(np.asarray(bt, np.int32)).to(dev)
+    sl = torch.as_tensor(np.asarray(seq_lens, np.int32)).to(dev)
+    out = torch.empty((B, Hq, 128), dtype=torch.float32 if out_fp32 else torch.float16, device=dev)
+    ws = torch.zeros(tq.tq_decode_workspace_bytes(ctx, B, Hq, Hkv, max_seq_len), dtype=torch.uint8, device=dev)
+    tq.tq_decode_attention(ctx, q, kc, vc, bt, sl, max_seq_len, out, ws, scale=scale, Hkv=Hkv)
+    torch.cuda.synchronize()
+    err = tq.tq_get_device_error(ctx)
+    return out.float().cpu().numpy(), err
+
+
+def _pool_cache(orc, o, w, nb_pool, seed):
+    """Oracle-compressed chunks of the workload's law: [nb_pool, Hkv, chunk] per kind."""
+    from kv_cache_vector_02_b200 import workloads as W
+    wp = w.with_(B=1, T=nb_pool * 16, layers=1, decode_steps=0, data_seed=seed)
+    caches = []
+    slots = np.arange(nb_pool * 16, dtype=np.int32)
+    for kind in (0, 1):
+        x = W.gen_kv(wp, kind).numpy()
+        c = o.new_cache(kind, nb_pool, w.Hkv)
+        o.compress_paged(kind, x, slots, c)
+        caches.append(c)
+    return caches
+
+
+@pytest.mark.parametrize("rot,bits,km", [(0, 4, 0), (1, 4, 0), (0, 2, 0), (1, 3, 1)])
+def test_tiny_decode_on_oracle_cache(orc, rot, bits, km):
+    from kv_cache_vector_02_b200 import workloads as W
+    w = W.WORKLOADS["tiny"].with_(rotation=rot, bits=bits, key_mode=km)
+    o = orc.Oracle(128, bits, w.param_seed, rot=rot, key_mode=km)
+    bt = W.block_table(w)
+    slots = W.prefill_slots(w, bt)
+    kc, vc = o.new_cache(0, w.num_blocks, 1), o.new_cache(1, w.num_blocks, 1)
+    o.compress_paged(0, W.gen_kv(w, 0).numpy(), slots, kc)
+    o.compress_paged(1, W.gen_kv(w, 1).numpy(), slots, vc)
+    q = W.gen_q(w).numpy()
+    seq = np.array([w.T], np.int32)
+    want = o.decode(q.astype(np.float64), kc, vc, bt, seq, w.Hkv)
+    ctx = gpu_ctx(bits, w.param_seed, rot, km)
+    got, err = _decode_gpu(ctx, q, kc, vc, bt, seq, w.T, w.Hkv)
+    assert err == 0
+    assert np.abs(got - want).max() <= DECODE_ATOL
+
+
+@pytest.mark.parametrize("B,T,Hkv,G,maxlen", [(3, 45, 2, 3, 64), (2, 1, 1, 16, 16), (4, 300, 2, 4, 300),
+                                               (1, 700, 1, 8, 4096)])
+def test_ragged_decode_on_oracle_cache(orc, B, T, Hkv, G, maxlen):
+    o = orc.Oracle(128, 4, 9)
+    rng = np.random.default_rng(B * 1000 + T)
+    nbps = (maxlen + 15) // 16
+    nb = B * nbps + 3
+    bt = rng.permutation(nb)[: B * nbps].reshape(B, nbps).astype(np.int32)
+    seq = rng.integers(max(T // 2, 0), T + 1, size=B).astype(np.int32)
+    seq[0] = T
+    kc, vc = o.new_cache(0, nb, Hkv), o.new_cache(1, nb, Hkv)
+    for b in range(B):
+        t = np.arange(T)
+        sl = (bt[b][t // 16] * 16 + t % 16).astype(np.int32)
+        o.compress_paged(0, (rng.standard_normal((T, Hkv, 128)) * 2).astype(np.float16), sl, kc)
+        o.compress_paged(1, rng.standard_normal((T, Hkv, 128)).astype(np.float16), sl, vc)
+    q = (rng.standard_normal((B, G * Hkv, 128)) / math.sqrt(128)).astype(np.float16)
+    want = o.decode(q.astype(np.float64), kc, vc, bt, seq, Hkv)
+    ctx = gpu_ctx(4, 9, 0, 0)
+    got, err = _decode_gpu(ctx, q, kc, vc, bt, seq, maxlen, Hkv)
+    assert err == 0
+    assert np.abs(got - want).max() <= DECODE_ATOL
+
+
+def test_llama8b_compress_append_decode_end_to_end(orc):
+    """Compress the 4096-token context, then 64 steps: append one token (compress)
+    and decode over seq_len + 1 tokens; GPU path end to end vs oracle end to end."""
+    import torch
+    from kv_cache_vector_02_b200 import tq, workloads as W
+    w = W.WORKLOADS["llama8b"]
+    o = orc.Oracle(128, w.bits, w.param_seed)
+    ctx = gpu_ctx(w.bits, w.param_seed, 0, 0)
+    bt = W.block_table(w)
+    slots = W.prefill_slots(w, bt)
+    k, v = W.gen_kv(w, 0), W.gen_kv(w, 1)
+    kc_g, vc_g = gpu_compress(ctx, k, v, slots, w.num_blocks, w.Hkv)
+    kc_o, vc_o = o.new_cache(0, w.num_blocks, w.Hkv), o.new_cache(1, w.num_blocks, w.Hkv)
+    o.compress_paged(0, k.numpy(), slots, kc_o)
+    o.compress_paged(1, v.numpy(), slots, vc_o)
+    dev = torch.device("cuda")
+    bt_d = torch.as_tensor(bt, device=dev)
+    ws = torch.zeros(tq.tq_decode_workspace_bytes(ctx, w.B, w.Hq, w.Hkv, w.max_seq_len), dtype=torch.uint8,
+                     device=dev)
+    worst = 0.0
+    for step in range(w.decode_steps):
+        ks, vs = W.gen_step_kv(w, 0, step), W.gen_step_kv(w, 1, step)
+        ss = W.step_slots(w, bt, step)
+        tq.tq_compress(ctx, ks.to(dev), vs.to(dev), torch.as_tensor(ss, device=dev), kc_g, vc_g)
+        o.compress_paged(0, ks.numpy(), ss, kc_o)
+        o.compress_paged(1, vs.numpy(), ss, vc_o)
+        q = W.gen_q(w, step)
+        seq = np.full(w.B, w.T + step + 1, np.int32)
+        out = torch.empty((w.B, w.Hq, 128), dtype=torch.float32, device=dev)
+        tq.tq_decode_attention(ctx, q.to(dev), kc_g, vc_g, bt_d, torch.as_tensor(seq, device=dev), w.max_seq_len,
+                               out, ws)
+        if step % 16 == 15 or step == 0:
+            want = o.decode(q.numpy().astype(np.float64), kc_o, vc_o, bt, seq, w.Hkv)
+            worst = max(worst, float(np.abs(out.cpu().numpy() - want).max()))
+    assert tq.tq_get_device_error(ctx) == 0
+    assert worst <= DECODE_ATOL, worst
+
+
+@pytest.mark.parametrize("name,bits,rot,nseq", [("batched", 4, 0, 3), ("long70b", 4, 0, 1), ("long70b", 2, 1, 1)])
+def test_full_size_decode(orc, name, bits, rot, nseq):
+    """Full-size decode on a cache tiled from oracle-compressed pages; the oracle
+    recomputes `nseq` sequences (all their query heads)."""
+    import torch
+    from kv_cache_vector_02_b200 import workloads as W
+    w = W.WORKLOADS[name].with_(bits=bits, rotation=rot)
+    o = orc.Oracle(128, bits, w.param_seed, rot=rot)
+    pool = _pool_cache(orc, o, w, 512, seed=41)
+    rng = np.random.default_rng(43)
+    pick = rng.integers(0, 512, size=w.num_blocks)
+    kc, vc = pool[0][pick], pool[1][pick]
+    bt = W.block_table(w)
+    seq = np.full(w.B, w.T, np.int32)
+    q = W.gen_q(w).numpy()
+    ctx = gpu_ctx(bits, w.param_seed, rot, 0)
+    got, err = _decode_gpu(ctx, q, kc, vc, bt, seq, w.T, w.Hkv)
+    assert err == 0
+    sel = rng.choice(w.B, size=nseq, replace=False)
+    want = o.decode(q[sel].astype(np.float64), kc, vc, bt[sel], seq[sel], w.Hkv)
+    assert np.abs(got[sel] - want).max() <= DECODE_ATOL
+    torch.cuda.empty_cache()
+
+
+def test_fp16_output_matches_fp32_output(orc):
+    from kv_cache_vector_02_b200 import workloads as W
+    w = W.WORKLOADS["tiny"]
+    o = orc.Oracle(128, 4, 0)
+    bt = W.block_table(w)
+    slots = W.prefill_slots(w, bt)
+    kc, vc = o.new_cache(0, w.num_blocks, 1), o.new_cache(1, w.num_blocks, 1)
+    o.compress_paged(0, W.gen_kv(w, 0).numpy(), slots, kc)
+    o.compress_paged(1, W.gen_kv(w, 1).numpy(), slots, vc)
+    q = W.gen_q(w).numpy()
+    ctx = gpu_ctx(4, 0, 0, 0)
+    a, _ = _decode_gpu(ctx, q, kc, vc, bt, [w.T], w.T, 1, out_fp32=True)
+    b, _ = _decode_gpu(ctx, q, kc, vc, bt, [w.T], w.T, 1, out_fp32=False)
+    assert np.abs(a - b).max() <= np.abs(a).max() * 2 ** -10
+
+
+@pytest.mark.parametrize("rot,bits,km", [(0, 4, 0), (1, 2, 0), (0, 3, 1)])
+def test_decompress_matches_oracle(orc, rot, bits, km):
+    import torch
+    from kv_cache_vector_02_b200 import tq
+    o = orc.Oracle(128, bits, 4, rot=rot, key_mode=km)
+    rng = np.random.default_rng(8)
+    T, H = 77, 3
+    nb = 8
+    perm = rng.permutation(nb)
+    slots = (perm[np.arange(T) // 16] * 16 + np.arange(T) % 16).astype(np.int32)
+    ctx = gpu_ctx(bits, 4, rot, km)
+    dev = torch.device("cuda")
+    for kind in (0, 1):
+        x = (rng.standard_normal((T, H, 128)) * 2).astype(np.float16)
+        c = o.new_cache(kind, nb, H)
+        o.compress_paged(kind, x, slots, c)
+        want = o.decompress_paged(kind, c, slots, H)
+        out = torch.empty((T, H, 128), dtype=torch.float32, device=dev)
+        tq.tq_decompress(ctx, kind, torch.as_tensor(c, device=dev), torch.as_tensor(slots, device=dev), out)
+        got = out.cpu().numpy()
+        scale = np.linalg.norm(x.astype(np.float64), axis=-1, keepdims=True)
+        assert np.abs(got - want).max() <= 1e-5 * scale.max()
