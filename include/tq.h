@@ -81,6 +81,7 @@ typedef enum { TQ_KIND_KEY = 0, TQ_KIND_VALUE = 1 } tq_kind;
 #define TQ_DEVERR_BLOCK     0x2u  /* decode: block id outside [0, num_blocks) (page skipped)   */
 #define TQ_DEVERR_SEQLEN    0x4u  /* decode: seq_len < 0 or > min(max_blocks*16, max_seq_len)  */
 #define TQ_DEVERR_TIMEOUT   0x8u  /* a bounded wait inside a kernel gave up (work abandoned)   */
+#define TQ_DEVERR_INTERNAL  0x10u /* a kernel found its launch set-up unusable (nothing done)   */
 
 /*
  * tq_init -- build the compressor parameters from one seed

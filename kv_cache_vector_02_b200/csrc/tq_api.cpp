@@ -102,6 +102,11 @@ tq_status tq_init_host(int head_dim, int bits, uint64_t seed, int rotation, int 
     if (!ctx) return TQ_ERR_OOM;
     ctx->host_only = true;
     fill_host(ctx, head_dim, bits, seed, rotation, key_mode);
+    tq::TcBlob tcb;  // same tables as a device context, built to surface any failure here too
+    if (!tq::build_tc_blob(ctx->host, tcb)) {
+        delete ctx;
+        return TQ_ERR_UNSUPPORTED;
+    }
     *out = ctx;
     return TQ_OK;
 }
@@ -123,7 +128,7 @@ tq_status tq_init(int head_dim, int bits, uint64_t seed, int rotation, int key_m
     fill_host(ctx, head_dim, bits, seed, rotation, key_mode);
     const tq::HostParams& H = ctx->host;
 
-    // fp32 device copies: R, R^T, M^T, S, S^T
+    // fp32 device copies: R, R^T, M^T, S, S^T; then the tensor-core blob
     const size_t n = size_t(kDim) * kDim;
     std::vector<float> blob(5 * n);
     float* R = blob.data();
@@ -139,7 +144,14 @@ tq_status tq_init(int head_dim, int bits, uint64_t seed, int rotation, int key_m
             S[i * kDim + j] = float(H.S[size_t(i) * kDim + j]);
             ST[j * kDim + i] = float(H.S[size_t(i) * kDim + j]);
         }
-    const size_t bytes = blob.size() * sizeof(float);
+    tq::TcBlob tcb;
+    if (!tq::build_tc_blob(H, tcb)) {
+        delete ctx;
+        return TQ_ERR_UNSUPPORTED;
+    }
+    const size_t f32_bytes = blob.size() * sizeof(float);
+    const size_t tc_off = (f32_bytes + 1023) & ~size_t(1023);
+    const size_t bytes = tc_off + tcb.bytes.size();
     if (cudaMalloc(&ctx->dev_block, bytes) != cudaSuccess) {
         cudaGetLastError();
         delete ctx;
@@ -151,7 +163,9 @@ tq_status tq_init(int head_dim, int bits, uint64_t seed, int rotation, int key_m
         delete ctx;
         return TQ_ERR_OOM;
     }
-    if (cudaMemcpy(ctx->dev_block, blob.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+    uint8_t* base8 = static_cast<uint8_t*>(ctx->dev_block);
+    if (cudaMemcpy(base8, blob.data(), f32_bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(base8 + tc_off, tcb.bytes.data(), tcb.bytes.size(), cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemset(ctx->dev_error, 0, sizeof(uint32_t)) != cudaSuccess) {
         cudaGetLastError();
         cudaFree(ctx->dev_block);
@@ -165,6 +179,11 @@ tq_status tq_init(int head_dim, int bits, uint64_t seed, int rotation, int key_m
     ctx->dev.MT = base + 2 * n;
     ctx->dev.S = base + 3 * n;
     ctx->dev.ST = base + 4 * n;
+    ctx->tc.images = base8 + tc_off + tcb.off_images;
+    ctx->tc.lut_value = base8 + tc_off + tcb.off_lut_value;
+    ctx->tc.lut_key = base8 + tc_off + tcb.off_lut_key;
+    ctx->tc.lp_value = tcb.lp_value;
+    ctx->tc.lp_key = tcb.lp_key;
     *out = ctx;
     return TQ_OK;
 }

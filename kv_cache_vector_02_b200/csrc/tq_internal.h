@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/tq.h"
+#include "tc_params.h"
 
 namespace tq {
 
@@ -69,6 +70,7 @@ struct tq_ctx {
     tq::Codebook cb_value{}, cb_key{};
     tq::ChunkLayout lay_value{}, lay_key{};
     tq::DeviceParams dev{};
+    tq::TcTables tc{};              // tensor-core compress operands and tables (in dev_block)
     void* dev_block = nullptr;      // all device parameters
     uint32_t* dev_error = nullptr;  // device error word
 };
@@ -80,6 +82,8 @@ void count_launches(unsigned n);
 
 // Kernel launchers (CUDA translation units).  Each returns cudaSuccess or the
 // launch error.
+cudaError_t launch_compress_tc(const tq_ctx* ctx, int kind, const uint16_t* x, int T, int H, const int32_t* slots,
+                               uint8_t* cache, int num_blocks, cudaStream_t stream);
 cudaError_t launch_compress(const tq_ctx* ctx, int kind, const uint16_t* x, int T, int H, const int32_t* slots,
                             uint8_t* cache, int num_blocks, cudaStream_t stream);
 cudaError_t launch_decompress(const tq_ctx* ctx, int kind, const uint8_t* cache, int num_blocks,
