@@ -1,18 +1,30 @@
-// Split-K decode attention over the paged compressed cache.
+// Split-K decode attention over the paged compressed cache, on tensor cores.
 //
 // [FQ-TQ] "FlashQuant：生产级KV缓存压缩方案…":
 //   - section "注意力计算的特殊挑战与QJL校正": score estimator
 //       <q,k> ~ <q,k_hat> + gamma sqrt(pi/2)/d <S q, sign(S r)>
 //   - section "架构设计" / "关键工程改进": Paged Decode as split-K FlashDecoding.
-// Scores are taken in the rotated domain: <q, k_hat> = n/sqrt(d) <R^T q, c[idx]>,
-// values are accumulated as sum_t p_t n_t c[idx_t]/sqrt(d) and un-rotated once
-// per query head (o = R acc).
+// Everything happens in the rotated domain: <q, k_hat> = n/sqrt(d) <R^T q, c[idx]>,
+// the value sum is accumulated as sum_t p_t n_t c[idx_t]/sqrt(d) and un-rotated
+// once per query head (o = R acc / l).
 //
-// Three stages: (1) prep: q' = R^T q and s = S q per (sequence, query head);
-// (2) split: each CTA scans a contiguous range of pages of one (sequence, kv
-// head) for all of its G query heads with an online softmax; (3) merge: the
-// log-sum-exp combination of the splits, the division by the softmax
-// denominator and the un-rotation.
+// Kernels:
+//   prep   one CTA per (sequence, kv head): q' = R^T q and s = S q for its G query
+//          heads, stored fp16.
+//   split  persistent CTAs over items (sequence, kv head, page range); each warp
+//          takes one 16-token page at a time:
+//            scores  D[16 tok x 8 heads] = sum_k Khat[tok][k] q'[k][h]   (mma m16n8k16)
+//                    plus the sign term with +-1 fragments against s
+//            softmax online, base 2, per head column
+//            values  D[16 coords x 8 heads] += Vhat^T[coord][tok] P'[tok][h]
+//          Packed codes become fp16 fragments in registers: key codes (<= 8 levels)
+//          through byte permutes of an 8-entry table, sign nibbles and value bytes
+//          through small shared-memory tables (the value table is replicated per
+//          lane so a warp's 32 lookups never share a bank).  Coordinates are
+//          permuted inside each contraction so that a thread's fragment elements
+//          are contiguous packed bytes.  The warps of a CTA merge their states;
+//          each item's partial (m, l, acc) goes to the workspace.
+//   merge  log-sum-exp combination of the splits, division by l, un-rotation.
 #include <cmath>
 
 #include "device_util.cuh"
@@ -20,12 +32,17 @@
 namespace tq {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
 constexpr int kMaxG = 16;
 constexpr int kPartStride = kDim + 2;  // m, l, acc[128]
 
+enum KMode { kKPrmt = 0, kKByte4 = 1, kKByte2 = 2, kKBit1 = 3 };
+enum VMode { kVByte4 = 0, kVByte2 = 1 };
+
 struct DecodeArgs {
     const uint16_t* q;
+    __half* qf;  // [B][Hq][2][128] fp16: q' then s
     const uint8_t* kc;
     const uint8_t* vc;
     int num_blocks;
@@ -33,185 +50,546 @@ struct DecodeArgs {
     int max_blocks;
     const int32_t* seq_lens;
     int B, Hq, Hkv, G, max_seq_len;
-    float scale;
-    void* out;
-    int out_fp32;
-    float* qprep;     // [B*Hq][2][128]: R^T q, S q
-    float* partial;   // [B*Hq][splits][130]
-    int splits, pages_per_split;
+    float scale_log2;  // softmax scale * log2(e)
+    float* partial;    // [B*Hkv][splits][G][130]
+    int splits, pages_per_item;
+    int merge_heads, merge_parts;
     const float* R;   // row-major
     const float* RT;  // row-major R^T
     const float* ST;  // row-major S^T
     Codebook cbk, cbv;
     ChunkLayout lk, lv;
+    void* out;
+    int out_fp32;
     uint32_t* err;
 };
-
-__global__ void __launch_bounds__(kThreads) decode_prep_kernel(DecodeArgs a) {
-    __shared__ float qs[kDim];
-    const int bh = blockIdx.x, j = threadIdx.x;
-    qs[j] = half_bits_to_float(a.q[(size_t)bh * kDim + j]);
-    __syncthreads();
-    float qr = 0.f, sq = 0.f;
-    for (int i = 0; i < kDim; ++i) {
-        qr = fmaf(a.R[i * kDim + j], qs[i], qr);    // (R^T q)_j = sum_i R[i][j] q_i
-        sq = fmaf(a.ST[i * kDim + j], qs[i], sq);   // (S q)_j = sum_i S[j][i] q_i
-    }
-    a.qprep[(size_t)bh * 2 * kDim + j] = qr;
-    a.qprep[(size_t)bh * 2 * kDim + kDim + j] = sq;
-}
 
 __device__ __forceinline__ bool seq_len_ok(const DecodeArgs& a, int L) {
     return L >= 0 && L <= a.max_blocks * kPage && L <= a.max_seq_len;
 }
 
-__global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
-    __shared__ float qp[kMaxG][kDim];
-    __shared__ float sq[kMaxG][kDim];
-    __shared__ __align__(16) uint8_t kchunk[1536];
-    __shared__ __align__(16) uint8_t vchunk[1152];
-    __shared__ float sc[kMaxG][kPage];
-    __shared__ float corr[kMaxG];
-    __shared__ float msh[kMaxG], lsh[kMaxG];
-    const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int G = a.G;
-    int L = a.seq_lens[b];
-    if (!seq_len_ok(a, L)) {
-        if (tid == 0 && split == 0 && hk == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
-        L = 0;
-    }
-    const int npages = (L + kPage - 1) / kPage;
-    const int p0 = split * a.pages_per_split;
-    const int p1 = min(p0 + a.pages_per_split, npages);
-    for (int g = 0; g < G; ++g) {
-        const size_t bh = (size_t)b * a.Hq + hk * G + g;
-        qp[g][tid] = a.qprep[bh * 2 * kDim + tid];
-        sq[g][tid] = a.qprep[bh * 2 * kDim + kDim + tid];
-    }
-    if (tid < kMaxG) {
-        msh[tid] = -INFINITY;
-        lsh[tid] = 0.f;
-    }
-    float acc[kMaxG];
-#pragma unroll
-    for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
-    const float sqrt_d = sqrtf((float)kDim);
-    const float qjl = sqrtf(3.14159265358979f / 2.f) / kDim;
+// ------------------------------------------------------------------ prep
+// q' = R^T q, s = S q for the G query heads of one (sequence, kv head).
+__global__ void __launch_bounds__(kDim) decode_prep_kernel(DecodeArgs a) {
+    __shared__ float qs[kMaxG][kDim];
+    const int unit = blockIdx.x;  // b * Hkv + hk
+    const int j = threadIdx.x;
+    const size_t q0 = (size_t)unit * a.G;  // first query head row of this unit in [B][Hq]
+    for (int g = 0; g < a.G; ++g) qs[g][j] = half_bits_to_float(a.q[(q0 + g) * kDim + j]);
     __syncthreads();
-
-    for (int p = p0; p < p1; ++p) {
-        const int blk = a.block_table[(size_t)b * a.max_blocks + p];
-        if (blk < 0 || blk >= a.num_blocks) {
-            if (tid == 0) atomicOr(a.err, TQ_DEVERR_BLOCK);
-            continue;  // uniform across the CTA
-        }
-        const int ntok = min(kPage, L - p * kPage);
-        const uint4* ksrc = reinterpret_cast<const uint4*>(a.kc + ((size_t)blk * a.Hkv + hk) * a.lk.bytes);
-        const uint4* vsrc = reinterpret_cast<const uint4*>(a.vc + ((size_t)blk * a.Hkv + hk) * a.lv.bytes);
-        for (int i = tid; i < a.lk.bytes / 16; i += kThreads) reinterpret_cast<uint4*>(kchunk)[i] = ksrc[i];
-        for (int i = tid; i < a.lv.bytes / 16; i += kThreads) reinterpret_cast<uint4*>(vchunk)[i] = vsrc[i];
-        __syncthreads();
-        // scores: warp w takes tokens w, w+4, w+8, w+12; lane covers coordinates 4*lane .. 4*lane+3
-        for (int t = warp; t < ntok; t += kThreads / 32) {
-            const uint8_t* crow = kchunk + t * a.lk.code_row;
-            float cval[4], sg[4];
+    float qr[kMaxG], sq[kMaxG];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int j = 4 * lane + e;
-                const int c = extract_code(crow, j, a.cbk.width);
-                float cv = 0.f;
+    for (int g = 0; g < kMaxG; ++g) qr[g] = sq[g] = 0.f;
+    for (int i = 0; i < kDim; ++i) {
+        const float r = a.R[i * kDim + j];   // (R^T q)_j = sum_i R[i][j] q_i
+        const float s = a.ST[i * kDim + j];  // (S q)_j   = sum_i S[j][i] q_i
 #pragma unroll
-                for (int k = 0; k < kMaxLevels; ++k) cv = (k == c) ? a.cbk.c[k] : cv;
-                cval[e] = cv;
-                sg[e] = a.lk.prod ? (extract_code(kchunk + a.lk.signs_off + t * (kDim / 8), j, 1) ? 1.f : -1.f) : 0.f;
+        for (int g = 0; g < kMaxG; ++g)
+            if (g < a.G) {
+                qr[g] = fmaf(r, qs[g][i], qr[g]);
+                sq[g] = fmaf(s, qs[g][i], sq[g]);
             }
-            const float n = reinterpret_cast<const float*>(kchunk + a.lk.norm_off)[t];
-            const float gm = a.lk.prod ? reinterpret_cast<const float*>(kchunk + a.lk.gamma_off)[t] : 0.f;
-            for (int g = 0; g < G; ++g) {
-                float d1 = 0.f, d2 = 0.f;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    d1 = fmaf(qp[g][4 * lane + e], cval[e], d1);
-                    d2 = fmaf(sq[g][4 * lane + e], sg[e], d2);
-                }
-                d1 = warp_sum(d1);
-                d2 = warp_sum(d2);
-                if (lane == 0) sc[g][t] = a.scale * (n / sqrt_d * d1 + gm * qjl * d2);
-            }
-        }
-        __syncthreads();
-        // online softmax, one thread per query head
-        if (tid < G) {
-            const int g = tid;
-            float mnew = msh[g];
-            for (int t = 0; t < ntok; ++t) mnew = fmaxf(mnew, sc[g][t]);
-            const float c = __expf(msh[g] - mnew);
-            float l = lsh[g] * c;
-            for (int t = 0; t < ntok; ++t) {
-                const float e = __expf(sc[g][t] - mnew);
-                sc[g][t] = e;
-                l += e;
-            }
-            corr[g] = c;
-            msh[g] = mnew;
-            lsh[g] = l;
-        }
-        __syncthreads();
-        // values: thread owns rotated coordinate tid
-        {
-            const int j = tid;
-#pragma unroll
-            for (int g = 0; g < kMaxG; ++g)
-                if (g < G) acc[g] *= corr[g];
-            for (int t = 0; t < ntok; ++t) {
-                const int c = extract_code(vchunk + t * a.lv.code_row, j, a.cbv.width);
-                float cv = 0.f;
-#pragma unroll
-                for (int k = 0; k < kMaxLevels; ++k) cv = (k == c) ? a.cbv.c[k] : cv;
-                const float vh = reinterpret_cast<const float*>(vchunk + a.lv.norm_off)[t] / sqrt_d * cv;
-#pragma unroll
-                for (int g = 0; g < kMaxG; ++g)
-                    if (g < G) acc[g] = fmaf(sc[g][t], vh, acc[g]);
-            }
-        }
-        __syncthreads();
     }
-    for (int g = 0; g < G; ++g) {
-        float* part = a.partial + (((size_t)b * a.Hq + hk * G + g) * a.splits + split) * kPartStride;
-        if (tid == 0) {
-            part[0] = msh[g];
-            part[1] = lsh[g];
-        }
-        float av = 0.f;
 #pragma unroll
-        for (int k = 0; k < kMaxG; ++k) av = (k == g) ? acc[k] : av;
-        part[2 + tid] = av;
+    for (int g = 0; g < kMaxG; ++g)
+        if (g < a.G) {
+            a.qf[((q0 + g) * 2 + 0) * kDim + j] = __float2half_rn(qr[g]);
+            a.qf[((q0 + g) * 2 + 1) * kDim + j] = __float2half_rn(sq[g]);
+        }
+}
+
+// ------------------------------------------------------------------ helpers
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t h2bits(__half lo, __half hi) {
+    return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+}
+
+__device__ __forceinline__ __half cb_half(const Codebook& cb, int code) {
+    float v = 0.f;
+#pragma unroll
+    for (int k = 0; k < kMaxLevels; ++k) v = (k == code) ? cb.c[k] : v;
+    return __float2half_rn(v);
+}
+
+// Raw bytes of one page that one thread needs (lane = 4 g + c).
+template <int KM, int VM, bool PROD>
+struct PageRegs {
+    uint32_t k[2][4];    // key code bytes of token rows g, g+8 (coords 32c .. 32c+31)
+    uint32_t s[2];       // sign word c of rows g, g+8
+    float kn[2], kg[2];  // key norm / gamma of tokens g, g+8
+    uint32_t v[4][2];    // value code bytes of token rows 2c, 2c+1, 2c+8, 2c+9 (coords 16g .. 16g+15)
+    float vn[2];         // value norms of tokens g, g+8
+};
+
+template <int KM, int VM, bool PROD>
+__device__ __forceinline__ void load_page(PageRegs<KM, VM, PROD>& r, const uint8_t* kchunk, const uint8_t* vchunk,
+                                          const DecodeArgs& a, int g, int c) {
+    constexpr int kBytes = KM == kKBit1 ? 4 : (KM == kKByte2 ? 8 : 16);  // per key row per thread
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const uint8_t* row = kchunk + (g + 8 * i) * a.lk.code_row + kBytes * c;
+        if (kBytes == 16) {
+            const uint4 w = __ldg(reinterpret_cast<const uint4*>(row));
+            r.k[i][0] = w.x, r.k[i][1] = w.y, r.k[i][2] = w.z, r.k[i][3] = w.w;
+        } else if (kBytes == 8) {
+            const uint2 w = __ldg(reinterpret_cast<const uint2*>(row));
+            r.k[i][0] = w.x, r.k[i][1] = w.y;
+        } else {
+            r.k[i][0] = __ldg(reinterpret_cast<const uint32_t*>(row));
+        }
+        if (PROD) {
+            r.s[i] = __ldg(reinterpret_cast<const uint32_t*>(kchunk + a.lk.signs_off + (g + 8 * i) * 16) + c);
+            r.kg[i] = __ldg(reinterpret_cast<const float*>(kchunk + a.lk.gamma_off) + g + 8 * i);
+        }
+        r.kn[i] = __ldg(reinterpret_cast<const float*>(kchunk + a.lk.norm_off) + g + 8 * i);
+        r.vn[i] = __ldg(reinterpret_cast<const float*>(vchunk + a.lv.norm_off) + g + 8 * i);
+    }
+    constexpr int vBytes = VM == kVByte4 ? 8 : 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int tok = 2 * c + (i & 1) + 8 * (i >> 1);
+        const uint8_t* row = vchunk + tok * a.lv.code_row + vBytes * g;
+        if (vBytes == 8) {
+            const uint2 w = __ldg(reinterpret_cast<const uint2*>(row));
+            r.v[i][0] = w.x, r.v[i][1] = w.y;
+        } else {
+            r.v[i][0] = __ldg(reinterpret_cast<const uint32_t*>(row));
+        }
     }
 }
 
-__global__ void __launch_bounds__(kThreads) decode_merge_kernel(DecodeArgs a) {
-    __shared__ float orot[kDim];
-    const int bh = blockIdx.x, i = threadIdx.x;
-    const float* part = a.partial + (size_t)bh * a.splits * kPartStride;
-    float M = -INFINITY;
-    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, part[s * kPartStride]);
-    float l = 0.f, acc = 0.f;
-    if (M != -INFINITY) {
-        for (int s = 0; s < a.splits; ++s) {
-            const float w = __expf(part[s * kPartStride] - M);  // exp(-inf) = 0 for empty splits
-            l = fmaf(w, part[s * kPartStride + 1], l);
-            acc = fmaf(w, part[s * kPartStride + 2 + i], acc);
+// Shared memory of the split kernel.
+//   V   value byte table, lane-replicated: [256][32] half2 (nibbles) or [256][16] 2 x half2 (crumbs)
+//   K   key byte table (same layouts) when keys are not byte-permuted
+//   S   sign nibble table [16] 2 x half2 of +-1 (bit set -> +1)
+//   K1  1-bit key nibble table [16] 2 x half2 of c[bit]
+//   P   per warp P' transpose [2 n-tiles][8 heads][16 tokens] fp16
+//   M   per warp m[16], l[16];  Acc  per warp acc[16 heads][128]
+constexpr int kTabBytes = 32768;
+
+template <int KM, int VM, bool PROD>
+struct SmemLayout {
+    static constexpr bool kKTab = (KM == kKByte4 || KM == kKByte2);
+    static constexpr uint32_t kOffV = 0;
+    static constexpr uint32_t kOffK = kOffV + kTabBytes;
+    static constexpr uint32_t kOffS = kOffK + (kKTab ? kTabBytes : 0);
+    static constexpr uint32_t kOffK1 = kOffS + 128;
+    static constexpr uint32_t kOffP = kOffK1 + 128;
+    static constexpr uint32_t kOffM = kOffP + kWarps * 2 * 8 * 16 * 2;
+    static constexpr uint32_t kOffAcc = kOffM + kWarps * 2 * kMaxG * 4;
+    static constexpr uint32_t kBytes = kOffAcc + kWarps * kMaxG * kDim * 4;
+};
+
+template <int KM, int VM, bool PROD>
+__device__ void build_tables(uint8_t* smem, const DecodeArgs& a) {
+    using L = SmemLayout<KM, VM, PROD>;
+    const int tid = threadIdx.x;
+    for (int e = tid; e < 256; e += kThreads) {
+        if (VM == kVByte4) {
+            const uint32_t w = h2bits(cb_half(a.cbv, e & 15), cb_half(a.cbv, e >> 4));
+            uint32_t* t = reinterpret_cast<uint32_t*>(smem + L::kOffV) + e * 32;
+#pragma unroll
+            for (int l = 0; l < 32; ++l) t[l] = w;
+        } else {
+            const uint2 w = make_uint2(h2bits(cb_half(a.cbv, e & 3), cb_half(a.cbv, (e >> 2) & 3)),
+                                       h2bits(cb_half(a.cbv, (e >> 4) & 3), cb_half(a.cbv, e >> 6)));
+            uint2* t = reinterpret_cast<uint2*>(smem + L::kOffV) + e * 16;
+#pragma unroll
+            for (int l = 0; l < 16; ++l) t[l] = w;
+        }
+        if (KM == kKByte4) {
+            const uint32_t w = h2bits(cb_half(a.cbk, e & 15), cb_half(a.cbk, e >> 4));
+            uint32_t* t = reinterpret_cast<uint32_t*>(smem + L::kOffK) + e * 32;
+#pragma unroll
+            for (int l = 0; l < 32; ++l) t[l] = w;
+        } else if (KM == kKByte2) {
+            const uint2 w = make_uint2(h2bits(cb_half(a.cbk, e & 3), cb_half(a.cbk, (e >> 2) & 3)),
+                                       h2bits(cb_half(a.cbk, (e >> 4) & 3), cb_half(a.cbk, e >> 6)));
+            uint2* t = reinterpret_cast<uint2*>(smem + L::kOffK) + e * 16;
+#pragma unroll
+            for (int l = 0; l < 16; ++l) t[l] = w;
         }
     }
-    orot[i] = (l > 0.f) ? acc / l : 0.f;
+    if (tid < 16) {
+        const __half one = __float2half_rn(1.f), mone = __float2half_rn(-1.f);
+        auto pm = [&](int bit) { return ((tid >> bit) & 1) ? one : mone; };
+        reinterpret_cast<uint2*>(smem + L::kOffS)[tid] = make_uint2(h2bits(pm(0), pm(1)), h2bits(pm(2), pm(3)));
+        const __half lo = cb_half(a.cbk, 0), hi = cb_half(a.cbk, 1);
+        auto pk = [&](int bit) { return ((tid >> bit) & 1) ? hi : lo; };
+        reinterpret_cast<uint2*>(smem + L::kOffK1)[tid] = make_uint2(h2bits(pk(0), pk(1)), h2bits(pk(2), pk(3)));
+    }
+}
+
+// ------------------------------------------------------------------ split
+template <int KM, int VM, bool PROD, int NT>
+__global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
+    using L = SmemLayout<KM, VM, PROD>;
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, c = lane & 3;
+    build_tables<KM, VM, PROD>(smem, a);
+    // 8-entry key tables (low / high bytes of the fp16 levels) for the byte-permute path
+    uint32_t klo0 = 0, klo1 = 0, khi0 = 0, khi1 = 0;
+    if (KM == kKPrmt) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const uint32_t hb = __half_as_ushort(cb_half(a.cbk, k));
+            if (k < 4) {
+                klo0 |= (hb & 0xffu) << (8 * k);
+                khi0 |= (hb >> 8) << (8 * k);
+            } else {
+                klo1 |= (hb & 0xffu) << (8 * (k - 4));
+                khi1 |= (hb >> 8) << (8 * (k - 4));
+            }
+        }
+    }
     __syncthreads();
-    float o = 0.f;
-    for (int j = 0; j < kDim; ++j) o = fmaf(a.RT[j * kDim + i], orot[j], o);  // o_i = sum_j R[i][j] orot_j
+    const float inv_sqrt_d = 0.08838834764831845f;
+    const float qjl = 1.2533141373155003f / kDim;  // sqrt(pi/2) / d
+    const uint32_t* vtab4 = reinterpret_cast<const uint32_t*>(smem + L::kOffV);
+    const uint2* vtab2 = reinterpret_cast<const uint2*>(smem + L::kOffV);
+    const uint32_t* ktab4 = reinterpret_cast<const uint32_t*>(smem + L::kOffK);
+    const uint2* ktab2 = reinterpret_cast<const uint2*>(smem + L::kOffK);
+    const uint2* stab = reinterpret_cast<const uint2*>(smem + L::kOffS);
+    const uint2* ktab1 = reinterpret_cast<const uint2*>(smem + L::kOffK1);
+    __half* pt = reinterpret_cast<__half*>(smem + L::kOffP) + warp * 2 * 8 * 16;
+    float* wm = reinterpret_cast<float*>(smem + L::kOffM);      // [warp][2][16]: m then l
+    float* wacc = reinterpret_cast<float*>(smem + L::kOffAcc);  // [warp][16 heads][128]
+
+    const int items = a.B * a.Hkv * a.splits;
+    for (int item = blockIdx.x; item < items; item += gridDim.x) {
+        const int unit = item / a.splits, split = item - unit * a.splits;
+        const int b = unit / a.Hkv, hk = unit - b * a.Hkv;
+        int Ls = a.seq_lens[b];
+        if (!seq_len_ok(a, Ls)) {
+            if (tid == 0 && split == 0 && hk == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
+            Ls = 0;
+        }
+        const int npages = (Ls + kPage - 1) / kPage;
+        const int p0 = split * a.pages_per_item;
+        const int p1 = min(p0 + a.pages_per_item, npages);
+
+        // query fragments (B operand): head nt*8 + g, coords 32c .. 32c+31; K-step ks
+        // uses coords 32c + 4ks + {0,1} (b0) and {2,3} (b1)
+        uint32_t bq[NT][8][2], bs[NT][8][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int h = nt * 8 + g;
+            if (h < a.G) {
+                const uint4* src =
+                    reinterpret_cast<const uint4*>(a.qf + (((size_t)unit * a.G + h) * 2) * kDim + 32 * c);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 w = src[i];
+                    bq[nt][2 * i][0] = w.x, bq[nt][2 * i][1] = w.y;
+                    bq[nt][2 * i + 1][0] = w.z, bq[nt][2 * i + 1][1] = w.w;
+                    if (PROD) {
+                        const uint4 u = src[i + kDim / 8];
+                        bs[nt][2 * i][0] = u.x, bs[nt][2 * i][1] = u.y;
+                        bs[nt][2 * i + 1][0] = u.z, bs[nt][2 * i + 1][1] = u.w;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) bq[nt][i][0] = bq[nt][i][1] = bs[nt][i][0] = bs[nt][i][1] = 0u;
+            }
+        }
+        float m[NT][2], l[NT][2], acc[NT][8][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            m[nt][0] = m[nt][1] = -INFINITY;
+            l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) acc[nt][mt][0] = acc[nt][mt][1] = acc[nt][mt][2] = acc[nt][mt][3] = 0.f;
+        }
+
+        // ---- page loop: one page per warp at a time, the next one prefetched
+        auto chunk_of = [&](int page, const uint8_t*& kch, const uint8_t*& vch) -> bool {
+            const int blk = a.block_table[(size_t)b * a.max_blocks + page];
+            if (blk < 0 || blk >= a.num_blocks) return false;
+            kch = a.kc + ((size_t)blk * a.Hkv + hk) * a.lk.bytes;
+            vch = a.vc + ((size_t)blk * a.Hkv + hk) * a.lv.bytes;
+            return true;
+        };
+        PageRegs<KM, VM, PROD> cur, nxt;
+        int p = p0 + warp;
+        bool have = p < p1;
+        bool cur_ok = false;
+        if (have) {
+            const uint8_t *kch, *vch;
+            cur_ok = chunk_of(p, kch, vch);
+            if (cur_ok) load_page<KM, VM, PROD>(cur, kch, vch, a, g, c);
+        }
+        while (have) {
+            const int pn = p + kWarps;
+            const bool have_n = pn < p1;
+            bool nxt_ok = false;
+            if (have_n) {
+                const uint8_t *kch, *vch;
+                nxt_ok = chunk_of(pn, kch, vch);
+                if (nxt_ok) load_page<KM, VM, PROD>(nxt, kch, vch, a, g, c);
+            }
+            if (!cur_ok) {
+                if (lane == 0) atomicOr(a.err, TQ_DEVERR_BLOCK);
+            } else {
+                const int ntok = min(kPage, Ls - p * kPage);
+                const bool valid0 = g < ntok, valid1 = g + 8 < ntok;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    // ---- scores: 8 K-steps of 16 coordinates
+                    float d1[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        uint32_t ak[2][2];  // [row g / g+8][coords (4ks,4ks+1) / (4ks+2,4ks+3)]
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            if (KM == kKPrmt) {
+                                const uint32_t w = cur.k[i][ks >> 1];
+                                const uint32_t sel = (ks & 1) ? (w >> 16) : w;
+                                const uint32_t lo = __byte_perm(klo0, klo1, sel);
+                                const uint32_t hi = __byte_perm(khi0, khi1, sel);
+                                ak[i][0] = __byte_perm(lo, hi, 0x5140);
+                                ak[i][1] = __byte_perm(lo, hi, 0x7362);
+                            } else if (KM == kKByte4) {
+                                const uint32_t w = cur.k[i][ks >> 1];
+                                const int sh = 16 * (ks & 1);
+                                ak[i][0] = ktab4[((w >> sh) & 0xffu) * 32 + lane];
+                                ak[i][1] = ktab4[((w >> (sh + 8)) & 0xffu) * 32 + lane];
+                            } else if (KM == kKByte2) {
+                                const uint32_t w = cur.k[i][ks >> 2];
+                                const uint2 e = ktab2[((w >> (8 * (ks & 3))) & 0xffu) * 16 + (lane & 15)];
+                                ak[i][0] = e.x;
+                                ak[i][1] = e.y;
+                            } else {
+                                const uint2 e = ktab1[(cur.k[i][0] >> (4 * ks)) & 0xfu];
+                                ak[i][0] = e.x;
+                                ak[i][1] = e.y;
+                            }
+                        }
+                        mma16816(d1, ak[0][0], ak[1][0], ak[0][1], ak[1][1], bq[nt][ks][0], bq[nt][ks][1]);
+                        if (PROD) {
+                            const uint2 s0 = stab[(cur.s[0] >> (4 * ks)) & 0xfu];
+                            const uint2 s1 = stab[(cur.s[1] >> (4 * ks)) & 0xfu];
+                            mma16816(d2, s0.x, s1.x, s0.y, s1.y, bs[nt][ks][0], bs[nt][ks][1]);
+                        }
+                    }
+                    // ---- base-2 logits of tokens g, g+8 for heads nt*8 + 2c + e
+                    float sc[2][2];
+#pragma unroll
+                    for (int i = 0; i < 2; ++i)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            float s = cur.kn[i] * inv_sqrt_d * d1[2 * i + e];
+                            if (PROD) s = fmaf(cur.kg[i] * qjl, d2[2 * i + e], s);
+                            sc[i][e] = (i == 0 ? valid0 : valid1) ? s * a.scale_log2 : -INFINITY;
+                        }
+                    float pw[2][2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        float mx = fmaxf(sc[0][e], sc[1][e]);
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                        const float mnew = fmaxf(m[nt][e], mx);
+                        const float corr = exp2f(m[nt][e] - mnew);
+                        const float p0v = exp2f(sc[0][e] - mnew), p1v = exp2f(sc[1][e] - mnew);
+                        float ps = p0v + p1v;
+                        ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+                        ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+                        ps += __shfl_xor_sync(0xffffffffu, ps, 16);
+                        l[nt][e] = fmaf(l[nt][e], corr, ps);
+                        m[nt][e] = mnew;
+#pragma unroll
+                        for (int mt = 0; mt < 8; ++mt) {
+                            acc[nt][mt][e] *= corr;
+                            acc[nt][mt][2 + e] *= corr;
+                        }
+                        pw[0][e] = valid0 ? p0v * cur.vn[0] * inv_sqrt_d : 0.f;
+                        pw[1][e] = valid1 ? p1v * cur.vn[1] * inv_sqrt_d : 0.f;
+                    }
+                    // ---- P' to the B-operand layout through shared memory: ptn[head][token]
+                    __half* ptn = pt + nt * 8 * 16;
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        ptn[(2 * c + e) * 16 + g] = __float2half_rn(pw[0][e]);
+                        ptn[(2 * c + e) * 16 + g + 8] = __float2half_rn(pw[1][e]);
+                    }
+                    __syncwarp();
+                    const uint32_t pb0 = *reinterpret_cast<const uint32_t*>(ptn + g * 16 + 2 * c);
+                    const uint32_t pb1 = *reinterpret_cast<const uint32_t*>(ptn + g * 16 + 2 * c + 8);
+                    __syncwarp();
+                    // ---- values: m-tile mt, row g -> coord vc0(g, mt), row g+8 -> vc0 + 1
+#pragma unroll
+                    for (int mt = 0; mt < 8; ++mt) {
+                        uint32_t av[4];
+                        if (VM == kVByte4) {
+                            uint32_t t[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const uint32_t w = cur.v[i][mt >> 2];
+                                t[i] = vtab4[((w >> (8 * (mt & 3))) & 0xffu) * 32 + lane];
+                            }
+                            av[0] = __byte_perm(t[0], t[1], 0x5410);  // lower coord, tokens 2c, 2c+1
+                            av[1] = __byte_perm(t[0], t[1], 0x7632);  // upper coord
+                            av[2] = __byte_perm(t[2], t[3], 0x5410);  // tokens 2c+8, 2c+9
+                            av[3] = __byte_perm(t[2], t[3], 0x7632);
+                        } else {
+                            uint2 t[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const uint32_t w = cur.v[i][0];
+                                t[i] = vtab2[((w >> (8 * (mt >> 1))) & 0xffu) * 16 + (lane & 15)];
+                            }
+                            const uint32_t x0 = (mt & 1) ? t[0].y : t[0].x, x1 = (mt & 1) ? t[1].y : t[1].x;
+                            const uint32_t x2 = (mt & 1) ? t[2].y : t[2].x, x3 = (mt & 1) ? t[3].y : t[3].x;
+                            av[0] = __byte_perm(x0, x1, 0x5410);
+                            av[1] = __byte_perm(x0, x1, 0x7632);
+                            av[2] = __byte_perm(x2, x3, 0x5410);
+                            av[3] = __byte_perm(x2, x3, 0x7632);
+                        }
+                        mma16816(acc[nt][mt], av[0], av[1], av[2], av[3], pb0, pb1);
+                    }
+                }
+            }
+            p = pn;
+            have = have_n;
+            cur = nxt;
+            cur_ok = nxt_ok;
+        }
+
+        // ---- merge the warps of the CTA (coordinates back in natural order)
+        __syncthreads();
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int h = nt * 8 + 2 * c + e;
+                if (g == 0) {
+                    wm[(warp * 2 + 0) * kMaxG + h] = m[nt][e];
+                    wm[(warp * 2 + 1) * kMaxG + h] = l[nt][e];
+                }
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    const int c0 = (VM == kVByte4) ? 16 * g + 2 * mt : 16 * g + 4 * (mt >> 1) + 2 * (mt & 1);
+                    wacc[(warp * kMaxG + h) * kDim + c0] = acc[nt][mt][e];
+                    wacc[(warp * kMaxG + h) * kDim + c0 + 1] = acc[nt][mt][2 + e];
+                }
+            }
+        __syncthreads();
+        for (int h = 0; h < a.G; ++h) {  // thread = coordinate
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wm[(w * 2) * kMaxG + h]);
+            float Lsum = 0.f, A = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+                const float mw = wm[(w * 2) * kMaxG + h];
+                const float wt = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+                Lsum = fmaf(wt, wm[(w * 2 + 1) * kMaxG + h], Lsum);
+                A = fmaf(wt, wacc[(w * kMaxG + h) * kDim + tid], A);
+            }
+            float* part = a.partial + (((size_t)unit * a.splits + split) * a.G + h) * kPartStride;
+            if (tid == 0) {
+                part[0] = M;
+                part[1] = Lsum;
+            }
+            part[2 + tid] = A;
+        }
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------------ merge
+// grid (B*Hkv, ceil(G / merge_heads)); threads = 128 * merge_heads * merge_parts.
+// Thread (part, head, coord): the splits s = part, part + parts, ... of one head.
+__global__ void decode_merge_kernel(DecodeArgs a) {
+    extern __shared__ float sm[];  // [parts][heads][3][128]: M, L, A; then orot [heads][128]
+    const int unit = blockIdx.x;
+    const int H = a.merge_heads, P = a.merge_parts;
+    const int i = threadIdx.x % kDim, hl = (threadIdx.x / kDim) % H, part = threadIdx.x / (kDim * H);
+    const int h = blockIdx.y * H + hl;
+    const bool active = h < a.G;
+    float M = -INFINITY, Lsum = 0.f, A = 0.f;
+    if (active) {
+        const float* base = a.partial + ((size_t)unit * a.splits * a.G + h) * kPartStride;
+        const size_t stride = (size_t)a.G * kPartStride;
+        for (int s = part; s < a.splits; s += P) M = fmaxf(M, base[s * stride]);
+        if (M != -INFINITY) {
+#pragma unroll 4
+            for (int s = part; s < a.splits; s += P) {
+                const float ms = base[s * stride];
+                const float wt = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+                Lsum = fmaf(wt, base[s * stride + 1], Lsum);
+                A = fmaf(wt, base[s * stride + 2 + i], A);
+            }
+        }
+    }
+    float* slot = sm + ((part * H + hl) * 3) * kDim;
+    slot[i] = M;
+    slot[kDim + i] = Lsum;
+    slot[2 * kDim + i] = A;
+    __syncthreads();
+    float* orot = sm + (size_t)P * H * 3 * kDim;
+    if (part == 0) {
+        float MM = -INFINITY;
+        for (int q = 0; q < P; ++q) MM = fmaxf(MM, sm[((q * H + hl) * 3) * kDim + i]);
+        float LL = 0.f, AA = 0.f;
+        if (MM != -INFINITY)
+            for (int q = 0; q < P; ++q) {
+                const float* sq = sm + ((q * H + hl) * 3) * kDim;
+                const float wt = (sq[i] == -INFINITY) ? 0.f : exp2f(sq[i] - MM);
+                LL = fmaf(wt, sq[kDim + i], LL);
+                AA = fmaf(wt, sq[2 * kDim + i], AA);
+            }
+        orot[hl * kDim + i] = LL > 0.f ? AA / LL : 0.f;
+    }
+    __syncthreads();
+    if (part != 0 || !active) return;
+    float y = 0.f;
+    const float* orh = orot + hl * kDim;
+#pragma unroll 8
+    for (int j = 0; j < kDim; ++j) y = fmaf(a.RT[j * kDim + i], orh[j], y);  // o_i = sum_j R[i][j] orot_j
+    const size_t oi = ((size_t)unit * a.G + h) * kDim + i;
     if (a.out_fp32)
-        static_cast<float*>(a.out)[(size_t)bh * kDim + i] = o;
+        static_cast<float*>(a.out)[oi] = y;
     else
-        static_cast<__half*>(a.out)[(size_t)bh * kDim + i] = __float2half_rn(o);
+        static_cast<__half*>(a.out)[oi] = __float2half_rn(y);
+}
+
+int kmode_of(const tq_ctx* ctx) {
+    const int w = ctx->cb_key.width;
+    if (w == 4) return ctx->cb_key.levels <= 8 ? kKPrmt : kKByte4;
+    if (w == 2) return kKByte2;
+    return kKBit1;
+}
+
+size_t split_smem(int km) {
+    return (km == kKByte4 || km == kKByte2) ? SmemLayout<kKByte4, kVByte4, true>::kBytes
+                                            : SmemLayout<kKPrmt, kVByte4, true>::kBytes;
+}
+
+int ctas_per_sm_for(size_t smem) {
+    int n = (int)((227 * 1024) / (smem + 1024));
+    if (n > 4) n = 4;
+    return n < 1 ? 1 : n;
+}
+
+template <int KM, int VM, bool PROD, int NT>
+cudaError_t launch_split(const DecodeArgs& a, int grid, cudaStream_t stream) {
+    using L = SmemLayout<KM, VM, PROD>;
+    auto k = decode_split_kernel<KM, VM, PROD, NT>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kThreads, L::kBytes, stream>>>(a);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -219,23 +597,24 @@ __global__ void __launch_bounds__(kThreads) decode_merge_kernel(DecodeArgs a) {
 DecodePlan plan_decode(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_seq_len) {
     DecodePlan p{};
     p.max_pages = (max_seq_len + kPage - 1) / kPage;
-    // enough splits that (B * Hkv) * splits CTAs cover two waves of the SMs
-    long work = (long)B * Hkv;
-    if (work < 1) work = 1;
-    long splits = (2L * ctx->sm_count + work - 1) / work;
-    if (splits > p.max_pages) splits = p.max_pages;
+    const long resident = (long)ctx->sm_count * ctas_per_sm_for(split_smem(kmode_of(ctx)));
+    const long units = (long)B * Hkv;
+    // about two items per resident CTA, and at least 16 pages (4 per warp) per item
+    long splits = (2 * resident + units - 1) / units;
+    const long max_splits = (p.max_pages + 4 * kWarps - 1) / (4 * kWarps);
+    if (splits > max_splits) splits = max_splits;
     if (splits < 1) splits = 1;
     p.splits = (int)splits;
     p.pages_per_split = p.max_pages > 0 ? (p.max_pages + p.splits - 1) / p.splits : 0;
     size_t off = 0;
     p.qprep_off = off;
-    off += (size_t)B * Hq * 2 * kDim * sizeof(float);
+    off += (size_t)B * Hq * 2 * kDim * sizeof(__half);
+    off = (off + 255) & ~size_t(255);
     p.partial_off = off;
     off += (size_t)B * Hq * p.splits * kPartStride * sizeof(float);
     off = (off + 255) & ~size_t(255);
     p.ticket_off = off;
-    off += (size_t)B * Hq * sizeof(uint32_t);
-    p.bytes = (off + 255) & ~size_t(255);
+    p.bytes = off;
     return p;
 }
 
@@ -244,13 +623,69 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
                           const int32_t* seq_lens, int B, int Hq, int Hkv, int max_seq_len, float scale, void* out,
                           int out_fp32, void* workspace, cudaStream_t stream) {
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    DecodeArgs a{q, kc, vc, num_blocks, block_table, max_blocks, seq_lens, B, Hq, Hkv, Hq / Hkv, max_seq_len, scale,
-                 out, out_fp32, reinterpret_cast<float*>(ws + plan.qprep_off),
-                 reinterpret_cast<float*>(ws + plan.partial_off), plan.splits, plan.pages_per_split, ctx->dev.R,
-                 ctx->dev.RT, ctx->dev.ST, ctx->cb_key, ctx->cb_value, ctx->lay_key, ctx->lay_value, ctx->dev_error};
-    decode_prep_kernel<<<B * Hq, kThreads, 0, stream>>>(a);
-    decode_split_kernel<<<dim3(plan.splits, Hkv, B), kThreads, 0, stream>>>(a);
-    decode_merge_kernel<<<B * Hq, kThreads, 0, stream>>>(a);
+    DecodeArgs a{};
+    a.q = q;
+    a.qf = reinterpret_cast<__half*>(ws + plan.qprep_off);
+    a.kc = kc;
+    a.vc = vc;
+    a.num_blocks = num_blocks;
+    a.block_table = block_table;
+    a.max_blocks = max_blocks;
+    a.seq_lens = seq_lens;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.G = Hq / Hkv;
+    a.max_seq_len = max_seq_len;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.partial = reinterpret_cast<float*>(ws + plan.partial_off);
+    a.splits = plan.splits;
+    a.pages_per_item = plan.pages_per_split;
+    a.R = ctx->dev.R;
+    a.RT = ctx->dev.RT;
+    a.ST = ctx->dev.ST;
+    a.cbk = ctx->cb_key;
+    a.cbv = ctx->cb_value;
+    a.lk = ctx->lay_key;
+    a.lv = ctx->lay_value;
+    a.out = out;
+    a.out_fp32 = out_fp32;
+    a.err = ctx->dev_error;
+    // merge: all heads of a unit in one CTA (they share the un-rotation matrix) when
+    // the splits are few; one head per CTA with the splits spread over 8 parts otherwise
+    if (plan.splits <= 16) {
+        a.merge_heads = a.G < 8 ? a.G : 8;
+        a.merge_parts = 1;
+    } else {
+        a.merge_heads = 1;
+        a.merge_parts = 8;
+    }
+
+    decode_prep_kernel<<<B * Hkv, kDim, 0, stream>>>(a);
+    const int KM = kmode_of(ctx);
+    const int VM = ctx->cb_value.width == 4 ? kVByte4 : kVByte2;
+    const bool prod = ctx->lay_key.prod;
+    const int NT = a.G <= 8 ? 1 : 2;
+    const long resident = (long)ctx->sm_count * ctas_per_sm_for(split_smem(KM));
+    const long items = (long)B * Hkv * plan.splits;
+    const int grid = (int)(items < resident ? items : resident);
+    cudaError_t e = cudaErrorInvalidValue;
+#define TQ_DEC_CASE(K_, V_, P_, N_) \
+    if (KM == K_ && VM == V_ && prod == P_ && NT == N_) e = launch_split<K_, V_, P_, N_>(a, grid, stream);
+#define TQ_DEC_NT(K_, V_, P_) TQ_DEC_CASE(K_, V_, P_, 1) TQ_DEC_CASE(K_, V_, P_, 2)
+    TQ_DEC_NT(kKPrmt, kVByte4, true)    // bits 4, prod keys (3-bit codes)
+    TQ_DEC_NT(kKByte2, kVByte4, true)   // bits 3, prod keys (2-bit codes)
+    TQ_DEC_NT(kKBit1, kVByte2, true)    // bits 2, prod keys (1-bit codes)
+    TQ_DEC_NT(kKByte4, kVByte4, false)  // bits 4, MSE keys
+    TQ_DEC_NT(kKPrmt, kVByte4, false)   // bits 3, MSE keys
+    TQ_DEC_NT(kKByte2, kVByte2, false)  // bits 2, MSE keys
+#undef TQ_DEC_NT
+#undef TQ_DEC_CASE
+    if (e != cudaSuccess) return e;
+    dim3 mgrid(B * Hkv, (a.G + a.merge_heads - 1) / a.merge_heads);
+    const int mthreads = kDim * a.merge_heads * a.merge_parts;
+    const size_t msmem = sizeof(float) * kDim * a.merge_heads * (3 * a.merge_parts + 1);
+    decode_merge_kernel<<<mgrid, mthreads, msmem, stream>>>(a);
     count_launches(3);
     return cudaGetLastError();
 }
