@@ -54,9 +54,11 @@ struct DecodeArgs {
     float* partial;    // [B*Hkv][splits][G][130]
     int splits, pages_per_item;
     int merge_heads, merge_parts;
-    const float* R;   // row-major
-    const float* RT;  // row-major R^T
-    const float* ST;  // row-major S^T
+    const float* RT;       // row-major R^T (fp32)
+    const uint16_t* RTh;   // fp16 R^T hi / lo, S (row-major)
+    const uint16_t* RTl;
+    const uint16_t* Sh;
+    float qscale, sscale;  // scale*log2(e)/sqrt(d), scale*log2(e)*sqrt(pi/2)/d
     Codebook cbk, cbv;
     ChunkLayout lk, lv;
     void* out;
@@ -68,36 +70,6 @@ __device__ __forceinline__ bool seq_len_ok(const DecodeArgs& a, int L) {
     return L >= 0 && L <= a.max_blocks * kPage && L <= a.max_seq_len;
 }
 
-// ------------------------------------------------------------------ prep
-// q' = R^T q, s = S q for the G query heads of one (sequence, kv head).
-__global__ void __launch_bounds__(kDim) decode_prep_kernel(DecodeArgs a) {
-    __shared__ float qs[kMaxG][kDim];
-    const int unit = blockIdx.x;  // b * Hkv + hk
-    const int j = threadIdx.x;
-    const size_t q0 = (size_t)unit * a.G;  // first query head row of this unit in [B][Hq]
-    for (int g = 0; g < a.G; ++g) qs[g][j] = half_bits_to_float(a.q[(q0 + g) * kDim + j]);
-    __syncthreads();
-    float qr[kMaxG], sq[kMaxG];
-#pragma unroll
-    for (int g = 0; g < kMaxG; ++g) qr[g] = sq[g] = 0.f;
-    for (int i = 0; i < kDim; ++i) {
-        const float r = a.R[i * kDim + j];   // (R^T q)_j = sum_i R[i][j] q_i
-        const float s = a.ST[i * kDim + j];  // (S q)_j   = sum_i S[j][i] q_i
-#pragma unroll
-        for (int g = 0; g < kMaxG; ++g)
-            if (g < a.G) {
-                qr[g] = fmaf(r, qs[g][i], qr[g]);
-                sq[g] = fmaf(s, qs[g][i], sq[g]);
-            }
-    }
-#pragma unroll
-    for (int g = 0; g < kMaxG; ++g)
-        if (g < a.G) {
-            a.qf[((q0 + g) * 2 + 0) * kDim + j] = __float2half_rn(qr[g]);
-            a.qf[((q0 + g) * 2 + 1) * kDim + j] = __float2half_rn(sq[g]);
-        }
-}
-
 // ------------------------------------------------------------------ helpers
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -106,6 +78,48 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ------------------------------------------------------------------ prep
+// [q' | s] = q [R | S^T] for 16 query heads per CTA, on mma.sync (fp16 inputs, fp32
+// accumulation; R^T enters as fp16 hi + lo, S is exact).  Warp w computes output
+// columns 32w .. 32w+31 of the 256 (q' then s).
+constexpr int kPrepThreads = 256;
+__global__ void __launch_bounds__(kPrepThreads) decode_prep_kernel(DecodeArgs a) {
+    const int NQ = a.B * a.Hq;
+    const int h0 = blockIdx.x * 16;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+    const bool r0 = h0 + g < NQ, r1 = h0 + g + 8 < NQ;
+    const uint32_t* q0 = reinterpret_cast<const uint32_t*>(a.q + (size_t)(r0 ? h0 + g : 0) * kDim);
+    const uint32_t* q1 = reinterpret_cast<const uint32_t*>(a.q + (size_t)(r1 ? h0 + g + 8 : 0) * kDim);
+    uint32_t A[8][4];
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        A[ks][0] = r0 ? q0[8 * ks + c] : 0u;
+        A[ks][1] = r1 ? q1[8 * ks + c] : 0u;
+        A[ks][2] = r0 ? q0[8 * ks + c + 4] : 0u;
+        A[ks][3] = r1 ? q1[8 * ks + c + 4] : 0u;
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const int nt = warp * 4 + t;  // 0..15 -> q', 16..31 -> s
+        const bool isq = nt < 16;
+        const int n = (nt & 15) * 8 + g;
+        const uint32_t* bh = reinterpret_cast<const uint32_t*>((isq ? a.RTh : a.Sh) + (size_t)n * kDim);
+        const uint32_t* bl = reinterpret_cast<const uint32_t*>(a.RTl + (size_t)n * kDim);
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            mma16816(d, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bh[8 * ks + c], bh[8 * ks + c + 4]);
+            if (isq) mma16816(d, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bl[8 * ks + c], bl[8 * ks + c + 4]);
+        }
+        const int col = (nt & 15) * 8 + 2 * c, which = isq ? 0 : 1;
+        if (r0)
+            *reinterpret_cast<__half2*>(a.qf + ((size_t)(h0 + g) * 2 + which) * kDim + col) = __floats2half2_rn(d[0], d[1]);
+        if (r1)
+            *reinterpret_cast<__half2*>(a.qf + ((size_t)(h0 + g + 8) * 2 + which) * kDim + col) =
+                __floats2half2_rn(d[2], d[3]);
+    }
 }
 
 __device__ __forceinline__ uint32_t h2bits(__half lo, __half hi) {
@@ -119,14 +133,15 @@ __device__ __forceinline__ __half cb_half(const Codebook& cb, int code) {
     return __float2half_rn(v);
 }
 
-// Raw bytes of one page that one thread needs (lane = 4 g + c).
+// Raw bytes of one page that one thread needs (lane = 4 g + c), with the per-token
+// scalars already multiplied by the constants of the score and of P'.
 template <int KM, int VM, bool PROD>
 struct PageRegs {
     uint32_t k[2][4];    // key code bytes of token rows g, g+8 (coords 32c .. 32c+31)
     uint32_t s[2];       // sign word c of rows g, g+8
-    float kn[2], kg[2];  // key norm / gamma of tokens g, g+8
+    float kn[2], kg[2];  // key norm * qscale, gamma * sscale of tokens g, g+8
     uint32_t v[4][2];    // value code bytes of token rows 2c, 2c+1, 2c+8, 2c+9 (coords 16g .. 16g+15)
-    float vn[2];         // value norms of tokens g, g+8
+    float vn[2];         // value norm / sqrt(d) of tokens g, g+8
 };
 
 template <int KM, int VM, bool PROD>
@@ -147,10 +162,10 @@ __device__ __forceinline__ void load_page(PageRegs<KM, VM, PROD>& r, const uint8
         }
         if (PROD) {
             r.s[i] = __ldg(reinterpret_cast<const uint32_t*>(kchunk + a.lk.signs_off + (g + 8 * i) * 16) + c);
-            r.kg[i] = __ldg(reinterpret_cast<const float*>(kchunk + a.lk.gamma_off) + g + 8 * i);
+            r.kg[i] = __ldg(reinterpret_cast<const float*>(kchunk + a.lk.gamma_off) + g + 8 * i) * a.sscale;
         }
-        r.kn[i] = __ldg(reinterpret_cast<const float*>(kchunk + a.lk.norm_off) + g + 8 * i);
-        r.vn[i] = __ldg(reinterpret_cast<const float*>(vchunk + a.lv.norm_off) + g + 8 * i);
+        r.kn[i] = __ldg(reinterpret_cast<const float*>(kchunk + a.lk.norm_off) + g + 8 * i) * a.qscale;
+        r.vn[i] = __ldg(reinterpret_cast<const float*>(vchunk + a.lv.norm_off) + g + 8 * i) * 0.08838834764831845f;
     }
     constexpr int vBytes = VM == kVByte4 ? 8 : 4;
 #pragma unroll
@@ -166,7 +181,7 @@ __device__ __forceinline__ void load_page(PageRegs<KM, VM, PROD>& r, const uint8
     }
 }
 
-// Shared memory of the split kernel.
+// Shared memory of the split kernel (byte offsets; V at offset 0).
 //   V   value byte table, lane-replicated: [256][32] half2 (nibbles) or [256][16] 2 x half2 (crumbs)
 //   K   key byte table (same layouts) when keys are not byte-permuted
 //   S   sign nibble table [16] 2 x half2 of +-1 (bit set -> +1)
@@ -228,7 +243,197 @@ __device__ void build_tables(uint8_t* smem, const DecodeArgs& a) {
     }
 }
 
+// byte k (0..3) of w, times `scale` (a power of two), as a shared-memory byte offset
+template <int K, int LOG2SCALE>
+__device__ __forceinline__ uint32_t byte_off(uint32_t w) {
+    constexpr int sh = 8 * K - LOG2SCALE;
+    const uint32_t x = sh >= 0 ? (w >> sh) : (w << (-sh));
+    return x & (0xffu << LOG2SCALE);
+}
+// nibble k (0..7) of w, times 8 (a uint2 table index as a byte offset)
+template <int K>
+__device__ __forceinline__ uint32_t nib_off8(uint32_t w) {
+    constexpr int sh = 4 * K - 3;
+    const uint32_t x = sh >= 0 ? (w >> sh) : (w << (-sh));
+    return x & 0x78u;
+}
+
+// Lazy softmax rescaling: the running maximum only moves when a page exceeds it by
+// more than 2^kSlack (log2 units), so exponentials stay <= 2^kSlack in fp32 / fp16.
+constexpr float kSlack = 8.f;
+
 // ------------------------------------------------------------------ split
+template <int KM, int VM, bool PROD, int NT>
+struct SplitCtx {
+    uint32_t klo0, klo1, khi0, khi1;
+    const uint8_t* smem;
+    __half* pt;
+    int lane, lane4, g, c;
+};
+
+template <int KM, int VM, bool PROD, int NT>
+__device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, int ntok,
+                                             const SplitCtx<KM, VM, PROD, NT>& x, const uint32_t (&bq)[NT][8][2],
+                                             const uint32_t (&bs)[NT][8][2], float (&m)[NT][2], float (&l)[NT][2],
+                                             float (&acc)[NT][8][4]) {
+    using L = SmemLayout<KM, VM, PROD>;
+    const int g = x.g, c = x.c;
+    const bool valid0 = g < ntok, valid1 = g + 8 < ntok;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        // ---- scores: 8 K-steps of 16 coordinates
+        float d1[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            uint32_t ak[2][2];  // [row g / g+8][coords (4ks,4ks+1) / (4ks+2,4ks+3)]
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                if (KM == kKPrmt) {
+                    const uint32_t w = cur.k[i][ks >> 1];
+                    const uint32_t sel = (ks & 1) ? (w >> 16) : w;
+                    const uint32_t lo = __byte_perm(x.klo0, x.klo1, sel);
+                    const uint32_t hi = __byte_perm(x.khi0, x.khi1, sel);
+                    ak[i][0] = __byte_perm(lo, hi, 0x5140);
+                    ak[i][1] = __byte_perm(lo, hi, 0x7362);
+                } else if (KM == kKByte4) {
+                    const uint32_t w = cur.k[i][ks >> 1];
+                    const uint32_t o0 = (ks & 1) ? byte_off<2, 7>(w) : byte_off<0, 7>(w);
+                    const uint32_t o1 = (ks & 1) ? byte_off<3, 7>(w) : byte_off<1, 7>(w);
+                    ak[i][0] = *reinterpret_cast<const uint32_t*>(x.smem + L::kOffK + (o0 | x.lane4));
+                    ak[i][1] = *reinterpret_cast<const uint32_t*>(x.smem + L::kOffK + (o1 | x.lane4));
+                } else if (KM == kKByte2) {
+                    const uint32_t w = cur.k[i][ks >> 2];
+                    uint32_t o;
+                    switch (ks & 3) {
+                        case 0: o = byte_off<0, 7>(w); break;
+                        case 1: o = byte_off<1, 7>(w); break;
+                        case 2: o = byte_off<2, 7>(w); break;
+                        default: o = byte_off<3, 7>(w); break;
+                    }
+                    const uint2 e = *reinterpret_cast<const uint2*>(x.smem + L::kOffK + (o | ((x.lane & 15) << 3)));
+                    ak[i][0] = e.x;
+                    ak[i][1] = e.y;
+                } else {
+                    const uint2 e = reinterpret_cast<const uint2*>(x.smem + L::kOffK1)[(cur.k[i][0] >> (4 * ks)) & 0xfu];
+                    ak[i][0] = e.x;
+                    ak[i][1] = e.y;
+                }
+            }
+            mma16816(d1, ak[0][0], ak[1][0], ak[0][1], ak[1][1], bq[nt][ks][0], bq[nt][ks][1]);
+            if (PROD) {
+                const uint32_t oa = nib_off8<0>(cur.s[0] >> (4 * ks));
+                const uint32_t ob = nib_off8<0>(cur.s[1] >> (4 * ks));
+                const uint2 s0 = *reinterpret_cast<const uint2*>(x.smem + L::kOffS + oa);
+                const uint2 s1 = *reinterpret_cast<const uint2*>(x.smem + L::kOffS + ob);
+                mma16816(d2, s0.x, s1.x, s0.y, s1.y, bs[nt][ks][0], bs[nt][ks][1]);
+            }
+        }
+        // ---- base-2 logits of tokens g, g+8 for heads nt*8 + 2c + e
+        float sc[2][2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float s = cur.kn[i] * d1[2 * i + e];
+                if (PROD) s = fmaf(cur.kg[i], d2[2 * i + e], s);
+                sc[i][e] = (i == 0 ? valid0 : valid1) ? s : -INFINITY;
+            }
+        float pw[2][2];
+        bool need = false;
+        float mnew[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            float mx = fmaxf(sc[0][e], sc[1][e]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const bool up = mx > m[nt][e] + kSlack;
+            mnew[e] = up ? mx : m[nt][e];
+            need |= up;
+        }
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float corr = exp2f(m[nt][e] - mnew[e]);  // 1 when unchanged, 0 from -inf
+                l[nt][e] *= corr;
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    acc[nt][mt][e] *= corr;
+                    acc[nt][mt][2 + e] *= corr;
+                }
+                m[nt][e] = mnew[e];
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float p0v = exp2f(sc[0][e] - m[nt][e]), p1v = exp2f(sc[1][e] - m[nt][e]);
+            float ps = p0v + p1v;
+            ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 16);
+            l[nt][e] += ps;
+            pw[0][e] = valid0 ? p0v * cur.vn[0] : 0.f;
+            pw[1][e] = valid1 ? p1v * cur.vn[1] : 0.f;
+        }
+        // ---- P' to the B-operand layout through shared memory: ptn[head][token]
+        __half* ptn = x.pt + nt * 8 * 16;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            ptn[(2 * c + e) * 16 + g] = __float2half_rn(pw[0][e]);
+            ptn[(2 * c + e) * 16 + g + 8] = __float2half_rn(pw[1][e]);
+        }
+        __syncwarp();
+        const uint32_t pb0 = *reinterpret_cast<const uint32_t*>(ptn + g * 16 + 2 * c);
+        const uint32_t pb1 = *reinterpret_cast<const uint32_t*>(ptn + g * 16 + 2 * c + 8);
+        __syncwarp();
+        // ---- values: m-tile mt, row g -> coord 16g + 2mt (nibbles), row g+8 -> +1
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            uint32_t av[4];
+            if (VM == kVByte4) {
+                uint32_t t[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t w = cur.v[i][mt >> 2];
+                    uint32_t o;
+                    switch (mt & 3) {
+                        case 0: o = byte_off<0, 7>(w); break;
+                        case 1: o = byte_off<1, 7>(w); break;
+                        case 2: o = byte_off<2, 7>(w); break;
+                        default: o = byte_off<3, 7>(w); break;
+                    }
+                    t[i] = *reinterpret_cast<const uint32_t*>(x.smem + L::kOffV + (o | x.lane4));
+                }
+                av[0] = __byte_perm(t[0], t[1], 0x5410);  // lower coord, tokens 2c, 2c+1
+                av[1] = __byte_perm(t[0], t[1], 0x7632);  // upper coord
+                av[2] = __byte_perm(t[2], t[3], 0x5410);  // tokens 2c+8, 2c+9
+                av[3] = __byte_perm(t[2], t[3], 0x7632);
+            } else {
+                uint2 t[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t w = cur.v[i][0];
+                    uint32_t o;
+                    switch (mt >> 1) {
+                        case 0: o = byte_off<0, 7>(w); break;
+                        case 1: o = byte_off<1, 7>(w); break;
+                        case 2: o = byte_off<2, 7>(w); break;
+                        default: o = byte_off<3, 7>(w); break;
+                    }
+                    t[i] = *reinterpret_cast<const uint2*>(x.smem + L::kOffV + (o | ((x.lane & 15) << 3)));
+                }
+                const uint32_t x0 = (mt & 1) ? t[0].y : t[0].x, x1 = (mt & 1) ? t[1].y : t[1].x;
+                const uint32_t x2 = (mt & 1) ? t[2].y : t[2].x, x3 = (mt & 1) ? t[3].y : t[3].x;
+                av[0] = __byte_perm(x0, x1, 0x5410);
+                av[1] = __byte_perm(x0, x1, 0x7632);
+                av[2] = __byte_perm(x2, x3, 0x5410);
+                av[3] = __byte_perm(x2, x3, 0x7632);
+            }
+            mma16816(acc[nt][mt], av[0], av[1], av[2], av[3], pb0, pb1);
+        }
+    }
+}
+
 template <int KM, int VM, bool PROD, int NT>
 __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
     using L = SmemLayout<KM, VM, PROD>;
@@ -236,31 +441,27 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, c = lane & 3;
     build_tables<KM, VM, PROD>(smem, a);
-    // 8-entry key tables (low / high bytes of the fp16 levels) for the byte-permute path
-    uint32_t klo0 = 0, klo1 = 0, khi0 = 0, khi1 = 0;
-    if (KM == kKPrmt) {
+    SplitCtx<KM, VM, PROD, NT> x{};
+    x.smem = smem;
+    x.pt = reinterpret_cast<__half*>(smem + L::kOffP) + warp * 2 * 8 * 16;
+    x.lane = lane;
+    x.lane4 = lane << 2;
+    x.g = g;
+    x.c = c;
+    if (KM == kKPrmt) {  // 8-entry key tables: low / high bytes of the fp16 levels
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const uint32_t hb = __half_as_ushort(cb_half(a.cbk, k));
             if (k < 4) {
-                klo0 |= (hb & 0xffu) << (8 * k);
-                khi0 |= (hb >> 8) << (8 * k);
+                x.klo0 |= (hb & 0xffu) << (8 * k);
+                x.khi0 |= (hb >> 8) << (8 * k);
             } else {
-                klo1 |= (hb & 0xffu) << (8 * (k - 4));
-                khi1 |= (hb >> 8) << (8 * (k - 4));
+                x.klo1 |= (hb & 0xffu) << (8 * (k - 4));
+                x.khi1 |= (hb >> 8) << (8 * (k - 4));
             }
         }
     }
     __syncthreads();
-    const float inv_sqrt_d = 0.08838834764831845f;
-    const float qjl = 1.2533141373155003f / kDim;  // sqrt(pi/2) / d
-    const uint32_t* vtab4 = reinterpret_cast<const uint32_t*>(smem + L::kOffV);
-    const uint2* vtab2 = reinterpret_cast<const uint2*>(smem + L::kOffV);
-    const uint32_t* ktab4 = reinterpret_cast<const uint32_t*>(smem + L::kOffK);
-    const uint2* ktab2 = reinterpret_cast<const uint2*>(smem + L::kOffK);
-    const uint2* stab = reinterpret_cast<const uint2*>(smem + L::kOffS);
-    const uint2* ktab1 = reinterpret_cast<const uint2*>(smem + L::kOffK1);
-    __half* pt = reinterpret_cast<__half*>(smem + L::kOffP) + warp * 2 * 8 * 16;
     float* wm = reinterpret_cast<float*>(smem + L::kOffM);      // [warp][2][16]: m then l
     float* wacc = reinterpret_cast<float*>(smem + L::kOffAcc);  // [warp][16 heads][128]
 
@@ -311,158 +512,34 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
             for (int mt = 0; mt < 8; ++mt) acc[nt][mt][0] = acc[nt][mt][1] = acc[nt][mt][2] = acc[nt][mt][3] = 0.f;
         }
 
-        // ---- page loop: one page per warp at a time, the next one prefetched
-        auto chunk_of = [&](int page, const uint8_t*& kch, const uint8_t*& vch) -> bool {
+        // ---- page loop: one page per warp at a time; two register sets alternate
+        // so that the next page is in flight while the current one is processed
+        auto fetch = [&](int page, PageRegs<KM, VM, PROD>& r) -> bool {
             const int blk = a.block_table[(size_t)b * a.max_blocks + page];
             if (blk < 0 || blk >= a.num_blocks) return false;
-            kch = a.kc + ((size_t)blk * a.Hkv + hk) * a.lk.bytes;
-            vch = a.vc + ((size_t)blk * a.Hkv + hk) * a.lv.bytes;
+            load_page<KM, VM, PROD>(r, a.kc + ((size_t)blk * a.Hkv + hk) * a.lk.bytes,
+                                    a.vc + ((size_t)blk * a.Hkv + hk) * a.lv.bytes, a, g, c);
             return true;
         };
-        PageRegs<KM, VM, PROD> cur, nxt;
-        int p = p0 + warp;
-        bool have = p < p1;
-        bool cur_ok = false;
-        if (have) {
-            const uint8_t *kch, *vch;
-            cur_ok = chunk_of(p, kch, vch);
-            if (cur_ok) load_page<KM, VM, PROD>(cur, kch, vch, a, g, c);
-        }
-        while (have) {
-            const int pn = p + kWarps;
-            const bool have_n = pn < p1;
-            bool nxt_ok = false;
-            if (have_n) {
-                const uint8_t *kch, *vch;
-                nxt_ok = chunk_of(pn, kch, vch);
-                if (nxt_ok) load_page<KM, VM, PROD>(nxt, kch, vch, a, g, c);
-            }
-            if (!cur_ok) {
+        auto handle = [&](int page, bool ok, const PageRegs<KM, VM, PROD>& r) {
+            if (!ok) {
                 if (lane == 0) atomicOr(a.err, TQ_DEVERR_BLOCK);
-            } else {
-                const int ntok = min(kPage, Ls - p * kPage);
-                const bool valid0 = g < ntok, valid1 = g + 8 < ntok;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    // ---- scores: 8 K-steps of 16 coordinates
-                    float d1[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        uint32_t ak[2][2];  // [row g / g+8][coords (4ks,4ks+1) / (4ks+2,4ks+3)]
-#pragma unroll
-                        for (int i = 0; i < 2; ++i) {
-                            if (KM == kKPrmt) {
-                                const uint32_t w = cur.k[i][ks >> 1];
-                                const uint32_t sel = (ks & 1) ? (w >> 16) : w;
-                                const uint32_t lo = __byte_perm(klo0, klo1, sel);
-                                const uint32_t hi = __byte_perm(khi0, khi1, sel);
-                                ak[i][0] = __byte_perm(lo, hi, 0x5140);
-                                ak[i][1] = __byte_perm(lo, hi, 0x7362);
-                            } else if (KM == kKByte4) {
-                                const uint32_t w = cur.k[i][ks >> 1];
-                                const int sh = 16 * (ks & 1);
-                                ak[i][0] = ktab4[((w >> sh) & 0xffu) * 32 + lane];
-                                ak[i][1] = ktab4[((w >> (sh + 8)) & 0xffu) * 32 + lane];
-                            } else if (KM == kKByte2) {
-                                const uint32_t w = cur.k[i][ks >> 2];
-                                const uint2 e = ktab2[((w >> (8 * (ks & 3))) & 0xffu) * 16 + (lane & 15)];
-                                ak[i][0] = e.x;
-                                ak[i][1] = e.y;
-                            } else {
-                                const uint2 e = ktab1[(cur.k[i][0] >> (4 * ks)) & 0xfu];
-                                ak[i][0] = e.x;
-                                ak[i][1] = e.y;
-                            }
-                        }
-                        mma16816(d1, ak[0][0], ak[1][0], ak[0][1], ak[1][1], bq[nt][ks][0], bq[nt][ks][1]);
-                        if (PROD) {
-                            const uint2 s0 = stab[(cur.s[0] >> (4 * ks)) & 0xfu];
-                            const uint2 s1 = stab[(cur.s[1] >> (4 * ks)) & 0xfu];
-                            mma16816(d2, s0.x, s1.x, s0.y, s1.y, bs[nt][ks][0], bs[nt][ks][1]);
-                        }
-                    }
-                    // ---- base-2 logits of tokens g, g+8 for heads nt*8 + 2c + e
-                    float sc[2][2];
-#pragma unroll
-                    for (int i = 0; i < 2; ++i)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            float s = cur.kn[i] * inv_sqrt_d * d1[2 * i + e];
-                            if (PROD) s = fmaf(cur.kg[i] * qjl, d2[2 * i + e], s);
-                            sc[i][e] = (i == 0 ? valid0 : valid1) ? s * a.scale_log2 : -INFINITY;
-                        }
-                    float pw[2][2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        float mx = fmaxf(sc[0][e], sc[1][e]);
-                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                        const float mnew = fmaxf(m[nt][e], mx);
-                        const float corr = exp2f(m[nt][e] - mnew);
-                        const float p0v = exp2f(sc[0][e] - mnew), p1v = exp2f(sc[1][e] - mnew);
-                        float ps = p0v + p1v;
-                        ps += __shfl_xor_sync(0xffffffffu, ps, 4);
-                        ps += __shfl_xor_sync(0xffffffffu, ps, 8);
-                        ps += __shfl_xor_sync(0xffffffffu, ps, 16);
-                        l[nt][e] = fmaf(l[nt][e], corr, ps);
-                        m[nt][e] = mnew;
-#pragma unroll
-                        for (int mt = 0; mt < 8; ++mt) {
-                            acc[nt][mt][e] *= corr;
-                            acc[nt][mt][2 + e] *= corr;
-                        }
-                        pw[0][e] = valid0 ? p0v * cur.vn[0] * inv_sqrt_d : 0.f;
-                        pw[1][e] = valid1 ? p1v * cur.vn[1] * inv_sqrt_d : 0.f;
-                    }
-                    // ---- P' to the B-operand layout through shared memory: ptn[head][token]
-                    __half* ptn = pt + nt * 8 * 16;
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        ptn[(2 * c + e) * 16 + g] = __float2half_rn(pw[0][e]);
-                        ptn[(2 * c + e) * 16 + g + 8] = __float2half_rn(pw[1][e]);
-                    }
-                    __syncwarp();
-                    const uint32_t pb0 = *reinterpret_cast<const uint32_t*>(ptn + g * 16 + 2 * c);
-                    const uint32_t pb1 = *reinterpret_cast<const uint32_t*>(ptn + g * 16 + 2 * c + 8);
-                    __syncwarp();
-                    // ---- values: m-tile mt, row g -> coord vc0(g, mt), row g+8 -> vc0 + 1
-#pragma unroll
-                    for (int mt = 0; mt < 8; ++mt) {
-                        uint32_t av[4];
-                        if (VM == kVByte4) {
-                            uint32_t t[4];
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const uint32_t w = cur.v[i][mt >> 2];
-                                t[i] = vtab4[((w >> (8 * (mt & 3))) & 0xffu) * 32 + lane];
-                            }
-                            av[0] = __byte_perm(t[0], t[1], 0x5410);  // lower coord, tokens 2c, 2c+1
-                            av[1] = __byte_perm(t[0], t[1], 0x7632);  // upper coord
-                            av[2] = __byte_perm(t[2], t[3], 0x5410);  // tokens 2c+8, 2c+9
-                            av[3] = __byte_perm(t[2], t[3], 0x7632);
-                        } else {
-                            uint2 t[4];
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const uint32_t w = cur.v[i][0];
-                                t[i] = vtab2[((w >> (8 * (mt >> 1))) & 0xffu) * 16 + (lane & 15)];
-                            }
-                            const uint32_t x0 = (mt & 1) ? t[0].y : t[0].x, x1 = (mt & 1) ? t[1].y : t[1].x;
-                            const uint32_t x2 = (mt & 1) ? t[2].y : t[2].x, x3 = (mt & 1) ? t[3].y : t[3].x;
-                            av[0] = __byte_perm(x0, x1, 0x5410);
-                            av[1] = __byte_perm(x0, x1, 0x7632);
-                            av[2] = __byte_perm(x2, x3, 0x5410);
-                            av[3] = __byte_perm(x2, x3, 0x7632);
-                        }
-                        mma16816(acc[nt][mt], av[0], av[1], av[2], av[3], pb0, pb1);
-                    }
-                }
+                return;
             }
-            p = pn;
-            have = have_n;
-            cur = nxt;
-            cur_ok = nxt_ok;
+            process_page<KM, VM, PROD, NT>(r, min(kPage, Ls - page * kPage), x, bq, bs, m, l, acc);
+        };
+        PageRegs<KM, VM, PROD> ra, rb;
+        int p = p0 + warp;
+        bool oka = (p < p1) && fetch(p, ra);
+        while (p < p1) {
+            const int pb = p + kWarps;
+            const bool okb = (pb < p1) && fetch(pb, rb);
+            handle(p, oka, ra);
+            if (pb >= p1) break;
+            const int pa = pb + kWarps;
+            oka = (pa < p1) && fetch(pa, ra);
+            handle(pb, okb, rb);
+            p = pa;
         }
 
         // ---- merge the warps of the CTA (coordinates back in natural order)
@@ -509,14 +586,21 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
 
 // ------------------------------------------------------------------ merge
 // grid (B*Hkv, ceil(G / merge_heads)); threads = 128 * merge_heads * merge_parts.
-// Thread (part, head, coord): the splits s = part, part + parts, ... of one head.
+// Thread (part, head, coord) combines the splits s = part, part + parts, ... of one
+// head; R^T is staged in shared memory for the un-rotation.
 __global__ void decode_merge_kernel(DecodeArgs a) {
-    extern __shared__ float sm[];  // [parts][heads][3][128]: M, L, A; then orot [heads][128]
+    extern __shared__ __align__(16) float sm[];  // RT [128*128] | [parts][heads][3][128] | orot [heads][128]
     const int unit = blockIdx.x;
     const int H = a.merge_heads, P = a.merge_parts;
     const int i = threadIdx.x % kDim, hl = (threadIdx.x / kDim) % H, part = threadIdx.x / (kDim * H);
     const int h = blockIdx.y * H + hl;
     const bool active = h < a.G;
+    float* rts = sm;
+    {
+        const float4* src = reinterpret_cast<const float4*>(a.RT);
+        float4* dst = reinterpret_cast<float4*>(rts);
+        for (int k = threadIdx.x; k < kDim * kDim / 4; k += blockDim.x) dst[k] = src[k];
+    }
     float M = -INFINITY, Lsum = 0.f, A = 0.f;
     if (active) {
         const float* base = a.partial + ((size_t)unit * a.splits * a.G + h) * kPartStride;
@@ -532,19 +616,20 @@ __global__ void decode_merge_kernel(DecodeArgs a) {
             }
         }
     }
-    float* slot = sm + ((part * H + hl) * 3) * kDim;
+    float* red = sm + kDim * kDim;
+    float* slot = red + ((part * H + hl) * 3) * kDim;
     slot[i] = M;
     slot[kDim + i] = Lsum;
     slot[2 * kDim + i] = A;
     __syncthreads();
-    float* orot = sm + (size_t)P * H * 3 * kDim;
+    float* orot = red + (size_t)P * H * 3 * kDim;
     if (part == 0) {
         float MM = -INFINITY;
-        for (int q = 0; q < P; ++q) MM = fmaxf(MM, sm[((q * H + hl) * 3) * kDim + i]);
+        for (int q = 0; q < P; ++q) MM = fmaxf(MM, red[((q * H + hl) * 3) * kDim + i]);
         float LL = 0.f, AA = 0.f;
         if (MM != -INFINITY)
             for (int q = 0; q < P; ++q) {
-                const float* sq = sm + ((q * H + hl) * 3) * kDim;
+                const float* sq = red + ((q * H + hl) * 3) * kDim;
                 const float wt = (sq[i] == -INFINITY) ? 0.f : exp2f(sq[i] - MM);
                 LL = fmaf(wt, sq[kDim + i], LL);
                 AA = fmaf(wt, sq[2 * kDim + i], AA);
@@ -556,7 +641,7 @@ __global__ void decode_merge_kernel(DecodeArgs a) {
     float y = 0.f;
     const float* orh = orot + hl * kDim;
 #pragma unroll 8
-    for (int j = 0; j < kDim; ++j) y = fmaf(a.RT[j * kDim + i], orh[j], y);  // o_i = sum_j R[i][j] orot_j
+    for (int j = 0; j < kDim; ++j) y = fmaf(rts[j * kDim + i], orh[j], y);  // o_i = sum_j R[i][j] orot_j
     const size_t oi = ((size_t)unit * a.G + h) * kDim + i;
     if (a.out_fp32)
         static_cast<float*>(a.out)[oi] = y;
@@ -638,12 +723,15 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
     a.G = Hq / Hkv;
     a.max_seq_len = max_seq_len;
     a.scale_log2 = scale * 1.4426950408889634f;
+    a.qscale = a.scale_log2 / sqrtf((float)kDim);
+    a.sscale = a.scale_log2 * 1.2533141373155003f / (float)kDim;
     a.partial = reinterpret_cast<float*>(ws + plan.partial_off);
     a.splits = plan.splits;
     a.pages_per_item = plan.pages_per_split;
-    a.R = ctx->dev.R;
     a.RT = ctx->dev.RT;
-    a.ST = ctx->dev.ST;
+    a.RTh = ctx->dev.RTh;
+    a.RTl = ctx->dev.RTl;
+    a.Sh = ctx->dev.Sh;
     a.cbk = ctx->cb_key;
     a.cbv = ctx->cb_value;
     a.lk = ctx->lay_key;
@@ -651,8 +739,8 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
     a.out = out;
     a.out_fp32 = out_fp32;
     a.err = ctx->dev_error;
-    // merge: all heads of a unit in one CTA (they share the un-rotation matrix) when
-    // the splits are few; one head per CTA with the splits spread over 8 parts otherwise
+    // merge: all heads of a unit in one CTA when the splits are few; one head per
+    // CTA with the splits spread over 8 parts otherwise
     if (plan.splits <= 16) {
         a.merge_heads = a.G < 8 ? a.G : 8;
         a.merge_parts = 1;
@@ -661,7 +749,7 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
         a.merge_parts = 8;
     }
 
-    decode_prep_kernel<<<B * Hkv, kDim, 0, stream>>>(a);
+    decode_prep_kernel<<<(B * Hq + 15) / 16, kPrepThreads, 0, stream>>>(a);
     const int KM = kmode_of(ctx);
     const int VM = ctx->cb_value.width == 4 ? kVByte4 : kVByte2;
     const bool prod = ctx->lay_key.prod;
@@ -684,7 +772,9 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
     if (e != cudaSuccess) return e;
     dim3 mgrid(B * Hkv, (a.G + a.merge_heads - 1) / a.merge_heads);
     const int mthreads = kDim * a.merge_heads * a.merge_parts;
-    const size_t msmem = sizeof(float) * kDim * a.merge_heads * (3 * a.merge_parts + 1);
+    const size_t msmem = sizeof(float) * (kDim * kDim + kDim * a.merge_heads * (3 * a.merge_parts + 1));
+    e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+    if (e != cudaSuccess) return e;
     decode_merge_kernel<<<mgrid, mthreads, msmem, stream>>>(a);
     count_launches(3);
     return cudaGetLastError();

@@ -128,21 +128,25 @@ tq_status tq_init(int head_dim, int bits, uint64_t seed, int rotation, int key_m
     fill_host(ctx, head_dim, bits, seed, rotation, key_mode);
     const tq::HostParams& H = ctx->host;
 
-    // fp32 device copies: R, R^T, M^T, S, S^T; then the tensor-core blob
+    // device copies: R, R^T, S, S^T (fp32), R^T hi / lo and S (fp16); then the tensor-core blob
     const size_t n = size_t(kDim) * kDim;
-    std::vector<float> blob(5 * n);
+    std::vector<float> blob(4 * n);
+    std::vector<__half> blob16(3 * n);
     float* R = blob.data();
     float* RT = R + n;
-    float* MT = RT + n;
-    float* S = MT + n;
+    float* S = RT + n;
     float* ST = S + n;
     for (int i = 0; i < kDim; ++i)
         for (int j = 0; j < kDim; ++j) {
-            R[i * kDim + j] = float(H.R[size_t(i) * kDim + j]);
-            RT[j * kDim + i] = float(H.R[size_t(i) * kDim + j]);
-            MT[j * kDim + i] = float(H.M[size_t(i) * kDim + j]);
+            const double r = H.R[size_t(i) * kDim + j];
+            R[i * kDim + j] = float(r);
+            RT[j * kDim + i] = float(r);
             S[i * kDim + j] = float(H.S[size_t(i) * kDim + j]);
             ST[j * kDim + i] = float(H.S[size_t(i) * kDim + j]);
+            const __half hi = __double2half(r);
+            blob16[size_t(j) * kDim + i] = hi;
+            blob16[n + size_t(j) * kDim + i] = __double2half(r - double(__half2float(hi)));
+            blob16[2 * n + size_t(i) * kDim + j] = __double2half(double(H.S[size_t(i) * kDim + j]));
         }
     tq::TcBlob tcb;
     if (!tq::build_tc_blob(H, tcb)) {
@@ -150,7 +154,9 @@ tq_status tq_init(int head_dim, int bits, uint64_t seed, int rotation, int key_m
         return TQ_ERR_UNSUPPORTED;
     }
     const size_t f32_bytes = blob.size() * sizeof(float);
-    const size_t tc_off = (f32_bytes + 1023) & ~size_t(1023);
+    const size_t f16_off = f32_bytes;
+    const size_t f16_bytes = blob16.size() * sizeof(__half);
+    const size_t tc_off = (f16_off + f16_bytes + 1023) & ~size_t(1023);
     const size_t bytes = tc_off + tcb.bytes.size();
     if (cudaMalloc(&ctx->dev_block, bytes) != cudaSuccess) {
         cudaGetLastError();
@@ -165,6 +171,7 @@ tq_status tq_init(int head_dim, int bits, uint64_t seed, int rotation, int key_m
     }
     uint8_t* base8 = static_cast<uint8_t*>(ctx->dev_block);
     if (cudaMemcpy(base8, blob.data(), f32_bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(base8 + f16_off, blob16.data(), f16_bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(base8 + tc_off, tcb.bytes.data(), tcb.bytes.size(), cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemset(ctx->dev_error, 0, sizeof(uint32_t)) != cudaSuccess) {
         cudaGetLastError();
@@ -176,9 +183,12 @@ tq_status tq_init(int head_dim, int bits, uint64_t seed, int rotation, int key_m
     const float* base = static_cast<const float*>(ctx->dev_block);
     ctx->dev.R = base;
     ctx->dev.RT = base + n;
-    ctx->dev.MT = base + 2 * n;
-    ctx->dev.S = base + 3 * n;
-    ctx->dev.ST = base + 4 * n;
+    ctx->dev.S = base + 2 * n;
+    ctx->dev.ST = base + 3 * n;
+    const uint16_t* base16 = reinterpret_cast<const uint16_t*>(base8 + f16_off);
+    ctx->dev.RTh = base16;
+    ctx->dev.RTl = base16 + n;
+    ctx->dev.Sh = base16 + 2 * n;
     ctx->tc.images = base8 + tc_off + tcb.off_images;
     ctx->tc.lut_value = base8 + tc_off + tcb.off_lut_value;
     ctx->tc.lut_key = base8 + tc_off + tcb.off_lut_key;

@@ -51,11 +51,13 @@ struct ChunkLayout {
 
 // Device copies of the parameters (one allocation owned by the context).
 struct DeviceParams {
-    const float* R;    // [d*d] R[i][j] row-major
-    const float* RT;   // [d*d] R^T row-major
-    const float* MT;   // [d*d] M^T row-major, MT[i][j] = (S R)[j][i]
-    const float* S;    // [d*d] S row-major as +-1.0f
-    const float* ST;   // [d*d] S^T row-major
+    const float* R;       // [d*d] R[i][j] row-major
+    const float* RT;      // [d*d] R^T row-major
+    const float* S;       // [d*d] S row-major as +-1.0f
+    const float* ST;      // [d*d] S^T row-major
+    const uint16_t* RTh;  // [d*d] fp16 R^T, high part
+    const uint16_t* RTl;  // [d*d] fp16 R^T - RTh
+    const uint16_t* Sh;   // [d*d] fp16 S (+-1, exact)
 };
 
 inline int container_width(int b) { return b >= 3 ? 4 : (b == 2 ? 2 : 1); }
