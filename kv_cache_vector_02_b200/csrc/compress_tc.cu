@@ -49,13 +49,17 @@ constexpr uint32_t kHalf = kTile / 2;      // one 128-byte-swizzled K-half
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kSmemMax = 232448;
 
-// TMEM: two tile buffers of 256 columns: [A 128 | B 128].  For keys, once A and
-// B have been read, rho_hi / rho_lo take A's columns [0,64) / [64,128) and the
-// sketch accumulates over B.
+// TMEM (512 columns).  Values: two tile buffers [A 128 | B 128] at 0 and 256.
+// Keys: one rotation buffer [A | B] at 0 (released as soon as it has been read, so
+// the next tile's rotation overlaps this tile's epilogue) and a sketch region at
+// 256: rho_hi [256,320), rho_lo [320,384) (the A operand, fp16 pairs) and the
+// sketch accumulator [384,512).  The epilogue reads tile k-1's sketch before it
+// writes tile k's rho, so the sketch contraction overlaps the epilogue too.
 constexpr uint32_t kBufCols = 256;
 constexpr uint32_t kColB = 128;
-constexpr uint32_t kColRhoHi = 0;
-constexpr uint32_t kColRhoLo = 64;
+constexpr uint32_t kColRhoHi = 256;
+constexpr uint32_t kColRhoLo = 320;
+constexpr uint32_t kColQjl = 384;
 
 template <int ROT, bool PROD>
 struct Cfg {
@@ -202,9 +206,11 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
                 return smem_desc_sw128(base + (uint32_t)(step >> 2) * kHalf + (uint32_t)(step & 3) * 32u);
             };
             auto issue_rot = [&](int k) -> bool {
-                const int s = k % C::kStages, b = k & 1;
+                const int s = k % C::kStages;
+                const int b = PROD ? 0 : (k & 1);
+                const uint32_t use = PROD ? (uint32_t)k : (uint32_t)(k >> 1);  // use count of buffer b
                 if (!mbar_wait(bar(kBarXFull + s), (uint32_t)(k / C::kStages) & 1u, abort, kWaitNs)) return false;
-                if (!mbar_wait(bar(kBarRotEmpty + b), ((uint32_t)(k >> 1) & 1u) ^ 1u, abort, kWaitNs)) return false;
+                if (!mbar_wait(bar(kBarRotEmpty + b), (use & 1u) ^ 1u, abort, kWaitNs)) return false;
                 tc_fence_after();
                 const uint32_t dA = tmem + kBufCols * b, dB = dA + kColB;
                 const uint32_t xs = sbase + C::kOffX + s * kTile;
@@ -230,22 +236,21 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
             auto issue_qjl = [&](int k) -> bool {
                 if (!mbar_wait(bar(kBarRhoFull), (uint32_t)k & 1u, abort, kWaitNs)) return false;
                 tc_fence_after();
-                const uint32_t base = tmem + kBufCols * (uint32_t)(k & 1);
-                const uint32_t d = base + kColB;
+                const uint32_t d = tmem + kColQjl;
                 const uint32_t m0 = img + C::kRotImages * kTile;
                 uint32_t acc2 = 0u;
                 // the small terms first: rho_lo M_hi (+ rho_hi M_lo for Haar), then rho_hi M_hi
 #pragma unroll
                 for (int st = 0; st < 8; ++st) {
-                    umma_ts(d, base + kColRhoLo + 8u * st, kdesc(m0, st), idesc, acc2);
+                    umma_ts(d, tmem + kColRhoLo + 8u * st, kdesc(m0, st), idesc, acc2);
                     acc2 = 1u;
                 }
                 if (ROT == 0) {
 #pragma unroll
-                    for (int st = 0; st < 8; ++st) umma_ts(d, base + kColRhoHi + 8u * st, kdesc(m0 + kTile, st), idesc, 1u);
+                    for (int st = 0; st < 8; ++st) umma_ts(d, tmem + kColRhoHi + 8u * st, kdesc(m0 + kTile, st), idesc, 1u);
                 }
 #pragma unroll
-                for (int st = 0; st < 8; ++st) umma_ts(d, base + kColRhoHi + 8u * st, kdesc(m0, st), idesc, 1u);
+                for (int st = 0; st < 8; ++st) umma_ts(d, tmem + kColRhoHi + 8u * st, kdesc(m0, st), idesc, 1u);
                 umma_commit(bar(kBarQjlFull));
                 return true;
             };
@@ -271,18 +276,84 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
         float* part = reinterpret_cast<float*>(smem + C::kOffPart);
         const uint8_t* lut = smem + C::kOffLut;
         const float sqrt_d = 11.313708498984761f;
+        constexpr int kPer = 32 / W;      // codes per 32-bit word
+        constexpr int kWords = 64 / kPer;  // words of this thread's half row
         bool ok = mbar_wait(bar(kBarConst), 0, abort, kWaitNs);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) set_abort(abort, a.err);
+
+        // destination of this thread's row of a tile (null when nothing is stored)
+        auto dest = [&](int tile) -> uint8_t* {
+            const int vi = tile * 128 + row;
+            if (vi >= a.N) return nullptr;
+            const int t = vi / a.H, head = vi - t * a.H;
+            const long s = a.slots[t];
+            if (s >= (long)a.num_blocks * kPage) {
+                if (h == 0) atomicOr(a.err, TQ_DEVERR_SLOT);
+                return nullptr;
+            }
+            if (s < 0) return nullptr;
+            return a.cache + ((size_t)(s / kPage) * a.H + head) * (size_t)a.lay.bytes + (size_t)(s % kPage);
+        };
+        // (a chunk pointer plus the row inside the page in the low 4 bits; chunks are 16-byte aligned)
+        auto store = [&](uint8_t* d, const uint32_t (&words)[kWords], float norm, float gamma, uint32_t sg0,
+                         uint32_t sg1) {
+            if (!d) return;
+            const int pr = (int)((uintptr_t)d & 15u);
+            uint8_t* chunk = d - pr;
+            uint8_t* cp = chunk + pr * a.lay.code_row + h * (a.lay.code_row / 2);
+            if (W == 4) {
+                reinterpret_cast<uint4*>(cp)[0] = make_uint4(words[0], words[1], words[2], words[3]);
+                reinterpret_cast<uint4*>(cp)[1] = make_uint4(words[4], words[5], words[6], words[7]);
+            } else if (W == 2) {
+                reinterpret_cast<uint4*>(cp)[0] = make_uint4(words[0], words[1], words[2], words[3]);
+            } else {
+                reinterpret_cast<uint2*>(cp)[0] = make_uint2(words[0], words[1]);
+            }
+            if (PROD)
+                *reinterpret_cast<uint2*>(chunk + a.lay.signs_off + pr * (kDim / 8) + h * 8) = make_uint2(sg0, sg1);
+            if (h == 0) {
+                reinterpret_cast<float*>(chunk + a.lay.norm_off)[pr] = norm;
+                if (PROD) reinterpret_cast<float*>(chunk + a.lay.gamma_off)[pr] = gamma;
+            }
+        };
+        // read tile k's sketch accumulator and turn it into sign bits (bit set when >= 0)
+        auto read_signs = [&](int k, bool nonzero, uint32_t& sg0, uint32_t& sg1) -> bool {
+            bool ok3 = mbar_wait(bar(kBarQjlFull), (uint32_t)k & 1u, abort, kWaitNs);
+            ok3 = __all_sync(0xffffffffu, ok3);
+            if (!ok3) return false;
+            tc_fence_after();
+            uint32_t q0[32], q1[32];
+            tmem_ld32(tmem + lane_addr + kColQjl + 64u * h, q0);
+            tmem_ld32(tmem + lane_addr + kColQjl + 64u * h + 32u, q1);
+            tmem_ld_wait();
+            uint32_t n0 = 0u, n1 = 0u;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                n0 |= (q0[j] >> 31) << j;
+                n1 |= (q1[j] >> 31) << j;
+            }
+            sg0 = nonzero ? ~n0 : 0xffffffffu;
+            sg1 = nonzero ? ~n1 : 0xffffffffu;
+            return true;
+        };
+
+        // the previous tile's outputs wait here until its sketch is ready (keys)
+        uint32_t pw[kWords];
+        float pnorm = 0.f, pgamma = 0.f;
+        bool pnz = false;
+        uint8_t* pdst = nullptr;
         for (int k = 0; k < my_tiles; ++k) {
             const int tile = (int)blockIdx.x + k * (int)gridDim.x;
-            const int b = k & 1;
+            const int b = PROD ? 0 : (k & 1);
+            const uint32_t use = PROD ? (uint32_t)k : (uint32_t)(k >> 1);
             float* pn = part + ((k & 1) * 2 + 0) * 256;
             float* pg = part + ((k & 1) * 2 + 1) * 256;
+            uint8_t* dst = dest(tile);  // issued early: the slot load overlaps the wait below
             // ---- rotation accumulators A + B -> registers
             float acc[64];
             const uint32_t buf = tmem + lane_addr + kBufCols * (uint32_t)b;
-            ok = !*abort && mbar_wait(bar(kBarRotFull + b), (uint32_t)(k >> 1) & 1u, abort, kWaitNs);
+            ok = !*abort && mbar_wait(bar(kBarRotFull + b), use & 1u, abort, kWaitNs);
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
                 tc_fence_after();
@@ -303,10 +374,8 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
                     acc[j] += __uint_as_float(r0[j]);
                     acc[32 + j] += __uint_as_float(r1[j]);
                 }
-                if (!PROD) {
-                    tc_fence_before();
-                    mbar_arrive(bar(kBarRotEmpty + b));
-                }
+                tc_fence_before();
+                mbar_arrive(bar(kBarRotEmpty + b));
             } else {
                 set_abort(abort, a.err);
 #pragma unroll
@@ -327,113 +396,79 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
             const float norm = sqrtf(nsq * a.n2_scale);
 
             // ---- bucketize + pack (+ residual for keys)
-            constexpr int kPer = 32 / W;  // codes per 32-bit word
-            uint32_t words[64 / kPer];
+            uint32_t words[kWords];
 #pragma unroll
-            for (int i = 0; i < 64 / kPer; ++i) words[i] = 0u;
+            for (int i = 0; i < kWords; ++i) words[i] = 0u;
             uint32_t rho_hi[32], rho_lo[32];
             float gs[4] = {0.f, 0.f, 0.f, 0.f};
             const float chat_scale = nacc / sqrt_d;
             const float kappa = nacc > 0.f ? 32.f * sqrt_d / nacc : 0.f;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                const float v = acc[j] * inv;
-                const float g = fmaf(v, a.lut_scale, a.lut_magic);
-                const int cell = __float_as_int(g) & (C::kCells - 1);
-                int code;
-                if (PROD) {
-                    const LutProd e = reinterpret_cast<const LutProd*>(lut)[cell];
-                    const bool up = e.bnd < v;
-                    code = e.base + (up ? 1 : 0);
-                    const float ch = up ? e.c_hi : e.c_lo;
-                    const float r = fmaf(-ch, chat_scale, acc[j]);
-                    gs[j & 3] = fmaf(r, r, gs[j & 3]);
-                    const float rho = r * kappa;
-                    const __half hh = __float2half_rn(rho);
-                    const __half hl = __float2half_rn(rho - __half2float(hh));
-                    if (j & 1) {
-                        rho_hi[j >> 1] |= (uint32_t)__half_as_ushort(hh) << 16;
-                        rho_lo[j >> 1] |= (uint32_t)__half_as_ushort(hl) << 16;
-                    } else {
-                        rho_hi[j >> 1] = (uint32_t)__half_as_ushort(hh);
-                        rho_lo[j >> 1] = (uint32_t)__half_as_ushort(hl);
-                    }
-                } else {
-                    const LutMse e = reinterpret_cast<const LutMse*>(lut)[cell];
-                    code = e.base + (e.bnd < v ? 1 : 0);
-                }
-                words[j / kPer] |= (uint32_t)code << (W * (j % kPer));
-            }
-            float gamma = 0.f;
-            uint32_t sgn0 = 0xffffffffu, sgn1 = 0xffffffffu;
-            if (PROD) {
-                pg[h * 128 + row] = (gs[0] + gs[1]) + (gs[2] + gs[3]);
-                // rho -> tensor memory over the tile's accumulator A (both warps of the
-                // row finished reading A and B before the norm barrier above)
-                if (!*abort) {
-                    tmem_st32(buf + kColRhoHi + 32u * h, rho_hi);
-                    tmem_st32(buf + kColRhoLo + 32u * h, rho_lo);
-                    tmem_st_wait();
-                    tc_fence_before();
-                    mbar_arrive(bar(kBarRhoFull));
-                }
-                named_barrier(1, kEpiThreads);
-                if (*abort) break;
-                gamma = sqrtf((pg[row] + pg[128 + row]) * a.n2_scale);
-                // sketch accumulator -> sign bits
-                bool ok3 = mbar_wait(bar(kBarQjlFull), (uint32_t)k & 1u, abort, kWaitNs);
-                ok3 = __all_sync(0xffffffffu, ok3);
-                if (!ok3) {
-                    set_abort(abort, a.err);
-                    continue;  // the next tile's first barrier sees the abort
-                }
-                tc_fence_after();
-                uint32_t q0[32], q1[32];
-                tmem_ld32(buf + kColB + 64u * h, q0);
-                tmem_ld32(buf + kColB + 64u * h + 32u, q1);
-                tmem_ld_wait();
-                tc_fence_before();
-                mbar_arrive(bar(kBarRotEmpty + b));  // the whole tile buffer is free again
-                // bit j set when the sketch is >= 0 (sign bit clear)
-                uint32_t n0 = 0u, n1 = 0u;
+            for (int j = 0; j < 64; j += 2) {
+                float rho2[2];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    n0 |= (q0[j] >> 31) << j;
-                    n1 |= (q1[j] >> 31) << j;
-                }
-                if (nsq > 0.f) {
-                    sgn0 = ~n0;
-                    sgn1 = ~n1;
-                }
-            }
-            // ---- store row `row` of this tile
-            const int vi = tile * 128 + row;
-            if (vi < a.N) {
-                const int t = vi / a.H, head = vi - t * a.H;
-                const long s = a.slots[t];
-                if (s >= (long)a.num_blocks * kPage) {
-                    if (h == 0) atomicOr(a.err, TQ_DEVERR_SLOT);
-                } else if (s >= 0) {
-                    uint8_t* chunk = a.cache + ((size_t)(s / kPage) * a.H + head) * (size_t)a.lay.bytes;
-                    const int pr = (int)(s % kPage);
-                    uint8_t* cp = chunk + pr * a.lay.code_row + h * (a.lay.code_row / 2);
-                    if (W == 4) {
-                        reinterpret_cast<uint4*>(cp)[0] = make_uint4(words[0], words[1], words[2], words[3]);
-                        reinterpret_cast<uint4*>(cp)[1] = make_uint4(words[4], words[5], words[6], words[7]);
-                    } else if (W == 2) {
-                        reinterpret_cast<uint4*>(cp)[0] = make_uint4(words[0], words[1], words[2], words[3]);
+                for (int u = 0; u < 2; ++u) {
+                    const float v = acc[j + u] * inv;
+                    const float gg = fmaf(v, a.lut_scale, a.lut_magic);
+                    const int cell = __float_as_int(gg) & (C::kCells - 1);
+                    int code;
+                    if (PROD) {
+                        const LutProd e = reinterpret_cast<const LutProd*>(lut)[cell];
+                        const bool upc = e.bnd < v;
+                        code = e.base + (upc ? 1 : 0);
+                        const float r = fmaf(upc ? -e.c_hi : -e.c_lo, chat_scale, acc[j + u]);
+                        gs[(j + u) & 3] = fmaf(r, r, gs[(j + u) & 3]);
+                        rho2[u] = r * kappa;
                     } else {
-                        reinterpret_cast<uint2*>(cp)[0] = make_uint2(words[0], words[1]);
+                        const LutMse e = reinterpret_cast<const LutMse*>(lut)[cell];
+                        code = e.base + (e.bnd < v ? 1 : 0);
                     }
-                    if (PROD)
-                        *reinterpret_cast<uint2*>(chunk + a.lay.signs_off + pr * (kDim / 8) + h * 8) =
-                            make_uint2(sgn0, sgn1);
-                    if (h == 0) {
-                        reinterpret_cast<float*>(chunk + a.lay.norm_off)[pr] = norm;
-                        if (PROD) reinterpret_cast<float*>(chunk + a.lay.gamma_off)[pr] = gamma;
-                    }
+                    words[(j + u) / kPer] |= (uint32_t)code << (W * ((j + u) % kPer));
+                }
+                if (PROD) {  // rho = hi + lo in fp16
+                    const __half2 hi = __floats2half2_rn(rho2[0], rho2[1]);
+                    const float2 hf = __half22float2(hi);
+                    const __half2 lo = __floats2half2_rn(rho2[0] - hf.x, rho2[1] - hf.y);
+                    rho_hi[j >> 1] = *reinterpret_cast<const uint32_t*>(&hi);
+                    rho_lo[j >> 1] = *reinterpret_cast<const uint32_t*>(&lo);
                 }
             }
+            if (!PROD) {
+                store(dst, words, norm, 0.f, 0u, 0u);
+                continue;
+            }
+            pg[h * 128 + row] = (gs[0] + gs[1]) + (gs[2] + gs[3]);
+            // tile k-1's sketch leaves the sketch region before tile k's rho enters it
+            uint32_t sg0 = 0xffffffffu, sg1 = 0xffffffffu;
+            bool have_prev = (k > 0) && !*abort;
+            if (have_prev && !read_signs(k - 1, pnz, sg0, sg1)) {
+                set_abort(abort, a.err);
+                have_prev = false;
+            }
+            if (!*abort) {
+                tmem_st32(tmem + lane_addr + kColRhoHi + 32u * h, rho_hi);
+                tmem_st32(tmem + lane_addr + kColRhoLo + 32u * h, rho_lo);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(bar(kBarRhoFull));
+            }
+            named_barrier(1, kEpiThreads);
+            if (*abort) break;
+            if (have_prev) store(pdst, pw, pnorm, pgamma, sg0, sg1);
+            // this tile's outputs wait for its sketch
+#pragma unroll
+            for (int i = 0; i < kWords; ++i) pw[i] = words[i];
+            pnorm = norm;
+            pgamma = sqrtf((pg[row] + pg[128 + row]) * a.n2_scale);
+            pnz = nsq > 0.f;
+            pdst = dst;
+        }
+        if (PROD && my_tiles > 0 && !*abort) {
+            uint32_t sg0, sg1;
+            if (read_signs(my_tiles - 1, pnz, sg0, sg1))
+                store(pdst, pw, pnorm, pgamma, sg0, sg1);
+            else
+                set_abort(abort, a.err);
         }
     }
     __syncthreads();
