@@ -7,9 +7,9 @@
 // Walsh-Hadamard rotation).
 //
 // One CTA per SM walks 128-vector tiles of the flattened [T*Hkv, 128] input:
-//   warp 0      TMA producer: 128x128 fp16 tiles (two 128-byte-swizzled boxes)
-//   warp 1      TMEM owner and single-thread MMA issuer
-//   warps 2..9  epilogue, two warps per TMEM lane quarter (64 columns each)
+//   warp 0       TMA producer: 128x128 fp16 tiles (two 128-byte-swizzled boxes)
+//   warp 1       TMEM owner and single-thread MMA issuer
+//   warps 2..17  epilogue, four warps per TMEM lane quarter (32 columns each)
 // Rotation: D[v][n] = sum_k x[v][k] B[n][k] with B the rotation split into
 // fp16 parts held in shared memory for the whole kernel:
 //   Haar      B = 16 R^T = hi + lo (two passes, x is exact in fp16, products are
@@ -41,8 +41,10 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;
 constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kSpan = 4 * 128 / kEpiWarps;  // columns per epilogue thread
+constexpr int kQ = 128 / kSpan;             // epilogue threads per row
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kTile = 128 * 128 * 2;  // one 128 x 128 fp16 operand
 constexpr uint32_t kHalf = kTile / 2;      // one 128-byte-swizzled K-half
@@ -68,7 +70,7 @@ struct Cfg {
     static constexpr int kImages = kRotImages + kQjlImages;
     static constexpr int kCells = PROD ? kLutCellsProd : kLutCellsMse;
     static constexpr int kLutBytes = PROD ? kLutBytesProd : kLutBytesMse;
-    static constexpr uint32_t kPartBytes = 2 * 2 * 2 * 128 * 4;  // [tile parity][norm, gamma][half][row]
+    static constexpr uint32_t kPartBytes = 2 * 2 * kQ * 128 * 4;  // [tile parity][norm, gamma][span][row]
     static constexpr uint32_t kBarBytes = 512;
     static constexpr uint32_t kFixed = kImages * kTile + kLutBytes + kPartBytes + kBarBytes;
     static constexpr int kStagesFit = (int)((kSmemMax - kFixed) / kTile);
@@ -270,19 +272,21 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
         // ------------------------------------------------------------ epilogue
         const int ew = warp - 2;
         const int quarter = warp & 3;  // TMEM lanes this warp may access
-        const int h = ew >> 2;         // column half
+        const int h = ew >> 2;         // column span [kSpan h, kSpan (h+1))
         const int row = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         float* part = reinterpret_cast<float*>(smem + C::kOffPart);
-        const uint8_t* lut = smem + C::kOffLut;
+        // this lane's replica of the bucketize table (see tc_params.h)
+        const uint8_t* lut = smem + C::kOffLut + (PROD ? 16 * (lane & (kLutReplProd - 1)) : 8 * (lane & (kLutReplMse - 1)));
         const float sqrt_d = 11.313708498984761f;
-        constexpr int kPer = 32 / W;      // codes per 32-bit word
-        constexpr int kWords = 64 / kPer;  // words of this thread's half row
+        constexpr int kPer = 32 / W;          // codes per 32-bit word
+        constexpr int kWords = kSpan / kPer;  // words of this thread's span
         bool ok = mbar_wait(bar(kBarConst), 0, abort, kWaitNs);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) set_abort(abort, a.err);
 
-        // destination of this thread's row of a tile (null when nothing is stored)
+        // destination of this thread's row of a tile: the chunk pointer with the row
+        // inside the page in its low 4 bits (chunks are 16-byte aligned), or null
         auto dest = [&](int tile) -> uint8_t* {
             const int vi = tile * 128 + row;
             if (vi >= a.N) return nullptr;
@@ -295,47 +299,41 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
             if (s < 0) return nullptr;
             return a.cache + ((size_t)(s / kPage) * a.H + head) * (size_t)a.lay.bytes + (size_t)(s % kPage);
         };
-        // (a chunk pointer plus the row inside the page in the low 4 bits; chunks are 16-byte aligned)
-        auto store = [&](uint8_t* d, const uint32_t (&words)[kWords], float norm, float gamma, uint32_t sg0,
-                         uint32_t sg1) {
+        auto store = [&](uint8_t* d, const uint32_t (&words)[kWords], float norm, float gamma, uint32_t sg) {
             if (!d) return;
             const int pr = (int)((uintptr_t)d & 15u);
             uint8_t* chunk = d - pr;
-            uint8_t* cp = chunk + pr * a.lay.code_row + h * (a.lay.code_row / 2);
-            if (W == 4) {
-                reinterpret_cast<uint4*>(cp)[0] = make_uint4(words[0], words[1], words[2], words[3]);
-                reinterpret_cast<uint4*>(cp)[1] = make_uint4(words[4], words[5], words[6], words[7]);
-            } else if (W == 2) {
-                reinterpret_cast<uint4*>(cp)[0] = make_uint4(words[0], words[1], words[2], words[3]);
+            uint8_t* cp = chunk + pr * a.lay.code_row + h * (a.lay.code_row / kQ);
+            if (kWords == 4) {
+                *reinterpret_cast<uint4*>(cp) = make_uint4(words[0], words[1], words[2], words[kWords - 1]);
+            } else if (kWords == 2) {
+                *reinterpret_cast<uint2*>(cp) = make_uint2(words[0], words[kWords - 1]);
             } else {
-                reinterpret_cast<uint2*>(cp)[0] = make_uint2(words[0], words[1]);
+                *reinterpret_cast<uint32_t*>(cp) = words[0];
             }
-            if (PROD)
-                *reinterpret_cast<uint2*>(chunk + a.lay.signs_off + pr * (kDim / 8) + h * 8) = make_uint2(sg0, sg1);
+            if (PROD) *reinterpret_cast<uint32_t*>(chunk + a.lay.signs_off + pr * (kDim / 8) + h * 4) = sg;
             if (h == 0) {
                 reinterpret_cast<float*>(chunk + a.lay.norm_off)[pr] = norm;
                 if (PROD) reinterpret_cast<float*>(chunk + a.lay.gamma_off)[pr] = gamma;
             }
         };
         // read tile k's sketch accumulator and turn it into sign bits (bit set when >= 0)
-        auto read_signs = [&](int k, bool nonzero, uint32_t& sg0, uint32_t& sg1) -> bool {
+        auto read_signs = [&](int k, bool nonzero, uint32_t& sg) -> bool {
             bool ok3 = mbar_wait(bar(kBarQjlFull), (uint32_t)k & 1u, abort, kWaitNs);
             ok3 = __all_sync(0xffffffffu, ok3);
             if (!ok3) return false;
             tc_fence_after();
-            uint32_t q0[32], q1[32];
-            tmem_ld32(tmem + lane_addr + kColQjl + 64u * h, q0);
-            tmem_ld32(tmem + lane_addr + kColQjl + 64u * h + 32u, q1);
+            uint32_t q[32];
+            tmem_ld32(tmem + lane_addr + kColQjl + kSpan * h, q);
             tmem_ld_wait();
-            uint32_t n0 = 0u, n1 = 0u;
+            uint32_t n0 = 0u;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                n0 |= (q0[j] >> 31) << j;
-                n1 |= (q1[j] >> 31) << j;
-            }
-            sg0 = nonzero ? ~n0 : 0xffffffffu;
-            sg1 = nonzero ? ~n1 : 0xffffffffu;
+            for (int j = 0; j < 32; ++j) n0 |= (q[j] >> 31) << j;
+            sg = nonzero ? ~n0 : 0xffffffffu;
             return true;
+        };
+        auto sum4 = [&](const float* pp) {
+            return (pp[row] + pp[128 + row]) + (pp[256 + row] + pp[384 + row]);
         };
 
         // the previous tile's outputs wait here until its sketch is ready (keys)
@@ -347,50 +345,39 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
             const int tile = (int)blockIdx.x + k * (int)gridDim.x;
             const int b = PROD ? 0 : (k & 1);
             const uint32_t use = PROD ? (uint32_t)k : (uint32_t)(k >> 1);
-            float* pn = part + ((k & 1) * 2 + 0) * 256;
-            float* pg = part + ((k & 1) * 2 + 1) * 256;
+            float* pn = part + ((k & 1) * 2 + 0) * (kQ * 128);
+            float* pg = part + ((k & 1) * 2 + 1) * (kQ * 128);
             uint8_t* dst = dest(tile);  // issued early: the slot load overlaps the wait below
             // ---- rotation accumulators A + B -> registers
-            float acc[64];
-            const uint32_t buf = tmem + lane_addr + kBufCols * (uint32_t)b;
+            float acc[kSpan];
+            const uint32_t buf = tmem + lane_addr + kBufCols * (uint32_t)b + kSpan * h;
             ok = !*abort && mbar_wait(bar(kBarRotFull + b), use & 1u, abort, kWaitNs);
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
                 tc_fence_after();
                 uint32_t r0[32], r1[32];
-                tmem_ld32(buf + 64u * h, r0);
-                tmem_ld32(buf + 64u * h + 32u, r1);
+                tmem_ld32(buf, r0);
+                tmem_ld32(buf + kColB, r1);
                 tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    acc[j] = __uint_as_float(r0[j]);
-                    acc[32 + j] = __uint_as_float(r1[j]);
-                }
-                tmem_ld32(buf + kColB + 64u * h, r0);
-                tmem_ld32(buf + kColB + 64u * h + 32u, r1);
-                tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    acc[j] += __uint_as_float(r0[j]);
-                    acc[32 + j] += __uint_as_float(r1[j]);
-                }
                 tc_fence_before();
                 mbar_arrive(bar(kBarRotEmpty + b));
+#pragma unroll
+                for (int j = 0; j < kSpan; ++j) acc[j] = __uint_as_float(r0[j]) + __uint_as_float(r1[j]);
             } else {
                 set_abort(abort, a.err);
 #pragma unroll
-                for (int j = 0; j < 64; ++j) acc[j] = 0.f;
+                for (int j = 0; j < kSpan; ++j) acc[j] = 0.f;
             }
-            // ---- ||acc||^2: 8 interleaved partial sums, then the two halves
+            // ---- ||acc||^2: 8 interleaved partial sums, then the spans of the row
             float ps[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) ps[i] = 0.f;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) ps[j & 7] = fmaf(acc[j], acc[j], ps[j & 7]);
+            for (int j = 0; j < kSpan; ++j) ps[j & 7] = fmaf(acc[j], acc[j], ps[j & 7]);
             pn[h * 128 + row] = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
             named_barrier(1, kEpiThreads);
             if (*abort) break;
-            const float nsq = pn[row] + pn[128 + row];
+            const float nsq = sum4(pn);
             const float nacc = sqrtf(nsq);
             const float inv = nacc > 0.f ? sqrt_d / nacc : 0.f;
             const float norm = sqrtf(nsq * a.n2_scale);
@@ -399,12 +386,12 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
             uint32_t words[kWords];
 #pragma unroll
             for (int i = 0; i < kWords; ++i) words[i] = 0u;
-            uint32_t rho_hi[32], rho_lo[32];
+            uint32_t rho_hi[kSpan / 2], rho_lo[kSpan / 2];
             float gs[4] = {0.f, 0.f, 0.f, 0.f};
             const float chat_scale = nacc / sqrt_d;
             const float kappa = nacc > 0.f ? 32.f * sqrt_d / nacc : 0.f;
 #pragma unroll
-            for (int j = 0; j < 64; j += 2) {
+            for (int j = 0; j < kSpan; j += 2) {
                 float rho2[2];
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
@@ -413,14 +400,14 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
                     const int cell = __float_as_int(gg) & (C::kCells - 1);
                     int code;
                     if (PROD) {
-                        const LutProd e = reinterpret_cast<const LutProd*>(lut)[cell];
+                        const LutProd e = *reinterpret_cast<const LutProd*>(lut + cell * 128);
                         const bool upc = e.bnd < v;
                         code = e.base + (upc ? 1 : 0);
                         const float r = fmaf(upc ? -e.c_hi : -e.c_lo, chat_scale, acc[j + u]);
                         gs[(j + u) & 3] = fmaf(r, r, gs[(j + u) & 3]);
                         rho2[u] = r * kappa;
                     } else {
-                        const LutMse e = reinterpret_cast<const LutMse*>(lut)[cell];
+                        const LutMse e = *reinterpret_cast<const LutMse*>(lut + cell * 128);
                         code = e.base + (e.bnd < v ? 1 : 0);
                     }
                     words[(j + u) / kPer] |= (uint32_t)code << (W * ((j + u) % kPer));
@@ -434,39 +421,39 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
                 }
             }
             if (!PROD) {
-                store(dst, words, norm, 0.f, 0u, 0u);
+                store(dst, words, norm, 0.f, 0u);
                 continue;
             }
             pg[h * 128 + row] = (gs[0] + gs[1]) + (gs[2] + gs[3]);
             // tile k-1's sketch leaves the sketch region before tile k's rho enters it
-            uint32_t sg0 = 0xffffffffu, sg1 = 0xffffffffu;
+            uint32_t sg = 0xffffffffu;
             bool have_prev = (k > 0) && !*abort;
-            if (have_prev && !read_signs(k - 1, pnz, sg0, sg1)) {
+            if (have_prev && !read_signs(k - 1, pnz, sg)) {
                 set_abort(abort, a.err);
                 have_prev = false;
             }
             if (!*abort) {
-                tmem_st32(tmem + lane_addr + kColRhoHi + 32u * h, rho_hi);
-                tmem_st32(tmem + lane_addr + kColRhoLo + 32u * h, rho_lo);
+                tmem_st16(tmem + lane_addr + kColRhoHi + (kSpan / 2) * h, rho_hi);
+                tmem_st16(tmem + lane_addr + kColRhoLo + (kSpan / 2) * h, rho_lo);
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(bar(kBarRhoFull));
             }
             named_barrier(1, kEpiThreads);
             if (*abort) break;
-            if (have_prev) store(pdst, pw, pnorm, pgamma, sg0, sg1);
+            if (have_prev) store(pdst, pw, pnorm, pgamma, sg);
             // this tile's outputs wait for its sketch
 #pragma unroll
             for (int i = 0; i < kWords; ++i) pw[i] = words[i];
             pnorm = norm;
-            pgamma = sqrtf((pg[row] + pg[128 + row]) * a.n2_scale);
+            pgamma = sqrtf(sum4(pg) * a.n2_scale);
             pnz = nsq > 0.f;
             pdst = dst;
         }
         if (PROD && my_tiles > 0 && !*abort) {
-            uint32_t sg0, sg1;
-            if (read_signs(my_tiles - 1, pnz, sg0, sg1))
-                store(pdst, pw, pnorm, pgamma, sg0, sg1);
+            uint32_t sg;
+            if (read_signs(my_tiles - 1, pnz, sg))
+                store(pdst, pw, pnorm, pgamma, sg);
             else
                 set_abort(abort, a.err);
         }

@@ -12,10 +12,15 @@ struct HostParams;
 
 // Bucketize tables: uniform cells over v = sqrt(d) y / ||x|| in [-V, V]; a cell
 // holds at most one interior boundary, far from its edges.
+// Each entry is stored once per lane group, interleaved, so that the lanes of
+// one shared-memory phase (16 for 8-byte loads, 8 for 16-byte loads) always hit
+// distinct banks: byte offset = cell * 128 + replica * entry_size.
 constexpr int kLutCellsMse = 256;   // entry {float bnd; int base}
 constexpr int kLutCellsProd = 128;  // entry {float bnd; int base; float c_lo; float c_hi}
-constexpr int kLutBytesMse = kLutCellsMse * 8;
-constexpr int kLutBytesProd = kLutCellsProd * 16;
+constexpr int kLutReplMse = 16;
+constexpr int kLutReplProd = 8;
+constexpr int kLutBytesMse = kLutCellsMse * 8 * kLutReplMse;
+constexpr int kLutBytesProd = kLutCellsProd * 16 * kLutReplProd;
 
 // cell = bits(fma(v, scale, magic)) & (cells - 1), magic = 1.5 * 2^23 + cells / 2
 struct LutParams {

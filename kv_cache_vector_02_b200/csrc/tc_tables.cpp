@@ -85,13 +85,19 @@ bool build_lut(const std::vector<double>& t, const std::vector<double>& c, int c
             if (prod) {
                 const float clo = float(c[base]);
                 const float chi = float(c[base + 1 < L ? base + 1 : base]);
-                std::memcpy(dst + 16 * cell + 0, &bnd, 4);
-                std::memcpy(dst + 16 * cell + 4, &base, 4);
-                std::memcpy(dst + 16 * cell + 8, &clo, 4);
-                std::memcpy(dst + 16 * cell + 12, &chi, 4);
+                for (int r = 0; r < kLutReplProd; ++r) {
+                    uint8_t* e = dst + 128 * cell + 16 * r;
+                    std::memcpy(e + 0, &bnd, 4);
+                    std::memcpy(e + 4, &base, 4);
+                    std::memcpy(e + 8, &clo, 4);
+                    std::memcpy(e + 12, &chi, 4);
+                }
             } else {
-                std::memcpy(dst + 8 * cell + 0, &bnd, 4);
-                std::memcpy(dst + 8 * cell + 4, &base, 4);
+                for (int r = 0; r < kLutReplMse; ++r) {
+                    uint8_t* e = dst + 128 * cell + 8 * r;
+                    std::memcpy(e + 0, &bnd, 4);
+                    std::memcpy(e + 4, &base, 4);
+                }
             }
         }
         return true;

@@ -99,7 +99,7 @@ class Context:
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h:
+        if h and _lib is not None:
             _lib.tq_destroy(h)
             self.handle = None
 
