@@ -200,6 +200,38 @@ TQ_API tq_status tq_decode_attention(const tq_ctx* ctx, const uint16_t* q_dev, c
                               void* stream);
 
 /*
+ * Size of the device array behind tq_decode_attention_noalloc.  Every GPU that
+ * loads libtq reserves this much device memory for it until the process exits.
+ */
+#define TQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * tq_decode_attention_noalloc -- tq_decode_attention without a workspace
+ * argument, for callers that cannot allocate device memory at the call site:
+ * code whose device memory is all owned by another allocator (for example a
+ * serving runtime that reserves nearly all HBM for its KV cache at start-up,
+ * so a fresh cudaMalloc would fail), and code that must not risk the device-wide
+ * synchronisation a cudaMalloc / cudaFree may cause.  The pages describe no such
+ * variant; it is an addition of this library.
+ * The scratch is one file-scope device array of TQ_NOALLOC_SCRATCH_BYTES per
+ * device, shared by every call: the decode needs
+ * tq_decode_workspace_bytes(ctx, B, Hq, Hkv, max_seq_len) of it, and a larger
+ * request is refused with TQ_ERR_INVALID_ARG before anything is launched.
+ * Nothing in the scratch has to start at zero (every byte read is written
+ * earlier in the same call).  Calls that overlap on the GPU (other streams, other
+ * threads, the same device) race on the array and must be serialised by the
+ * caller.  The first call on a device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.  The
+ * current device must be the context's.  Arguments and results are otherwise
+ * those of tq_decode_attention.  Allocates nothing.
+ */
+TQ_API tq_status tq_decode_attention_noalloc(const tq_ctx* ctx, const uint16_t* q_dev, const uint8_t* k_cache_dev,
+                                             const uint8_t* v_cache_dev, int num_blocks,
+                                             const int32_t* block_table_dev, int max_blocks,
+                                             const int32_t* seq_lens_dev, int B, int Hq, int Hkv, int max_seq_len,
+                                             float scale, void* out_dev, int out_fp32, void* stream);
+
+/*
  * tq_get_device_error -- synchronize stream, return the device error word in
  * *code (TQ_DEVERR_* bits, 0 if clean) and clear it.  Returns TQ_ERR_DEVICE when
  * the word was non-zero, TQ_OK otherwise.

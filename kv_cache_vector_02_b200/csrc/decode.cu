@@ -26,6 +26,7 @@
 //          each item's partial (m, l, acc) goes to the workspace.
 //   merge  log-sum-exp combination of the splits, division by l, un-rotation.
 #include <cmath>
+#include <mutex>
 
 #include "device_util.cuh"
 
@@ -780,4 +781,54 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ allocation-free variant
+// The scratch of tq_decode_attention_noalloc: one array per device, reserved when
+// the module loads and kept until the process exits.  Host code cannot use the
+// symbol itself (that is a host-side stand-in); its device address is looked up
+// once per device with cudaGetSymbolAddress and cached.
+namespace {
+__device__ __align__(256) uint8_t g_noalloc_scratch[TQ_NOALLOC_SCRATCH_BYTES];
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+}  // namespace
+
+cudaError_t noalloc_scratch(int device, void** out) {
+    if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[device]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // with `device` current
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[device] = p;
+    }
+    *out = g_noalloc_ptr[device];
+    return cudaSuccess;
+}
+
 }  // namespace tq
+
+extern "C" tq_status tq_decode_attention_noalloc(const tq_ctx* ctx, const uint16_t* q, const uint8_t* k_cache,
+                                                 const uint8_t* v_cache, int num_blocks, const int32_t* block_table,
+                                                 int max_blocks, const int32_t* seq_lens, int B, int Hq, int Hkv,
+                                                 int max_seq_len, float scale, void* out, int out_fp32,
+                                                 void* stream) {
+    if (!ctx || ctx->host_only) return TQ_ERR_INVALID_ARG;
+    if (B > 0) {
+        const size_t need = tq_decode_workspace_bytes(ctx, B, Hq, Hkv, max_seq_len);
+        if (need > TQ_NOALLOC_SCRATCH_BYTES) return TQ_ERR_INVALID_ARG;
+    }
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) {
+        cudaGetLastError();
+        return TQ_ERR_CUDA;
+    }
+    if (cur != ctx->device) return TQ_ERR_INVALID_ARG;
+    void* scratch = nullptr;
+    if (tq::noalloc_scratch(cur, &scratch) != cudaSuccess) {
+        cudaGetLastError();
+        return TQ_ERR_CUDA;
+    }
+    return tq_decode_attention(ctx, q, k_cache, v_cache, num_blocks, block_table, max_blocks, seq_lens, B, Hq, Hkv,
+                               max_seq_len, scale, out, out_fp32, scratch, TQ_NOALLOC_SCRATCH_BYTES, stream);
+}

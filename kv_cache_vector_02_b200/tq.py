@@ -24,8 +24,8 @@ KIND_KEY, KIND_VALUE = 0, 1
 DEVERR_SLOT, DEVERR_BLOCK, DEVERR_SEQLEN, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 
 EXPORTED = ("tq_init", "tq_init_host", "tq_destroy", "tq_chunk_bytes", "tq_code_bits", "tq_export_params", "tq_compress",
-            "tq_decompress", "tq_decode_workspace_bytes", "tq_decode_attention", "tq_get_device_error",
-            "tq_launch_count", "tq_status_string")
+            "tq_decompress", "tq_decode_workspace_bytes", "tq_decode_attention", "tq_decode_attention_noalloc",
+            "tq_get_device_error", "tq_launch_count", "tq_status_string")
 
 
 class TQError(RuntimeError):
@@ -50,6 +50,7 @@ def _load():
         "tq_decompress": (I, [P, I, P, I, P, I, I, P, I, P]),
         "tq_decode_workspace_bytes": (Z, [P, I, I, I, I]),
         "tq_decode_attention": (I, [P, P, P, P, I, P, I, P, I, I, I, I, F, P, I, P, Z, P]),
+        "tq_decode_attention_noalloc": (I, [P, P, P, P, I, P, I, P, I, I, I, I, F, P, I, P]),
         "tq_get_device_error": (I, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
         "tq_launch_count": (ctypes.c_uint64, []),
         "tq_status_string": (ctypes.c_char_p, [I]),
@@ -193,6 +194,25 @@ def tq_decode_attention(ctx: Context, q, k_cache, v_cache, block_table, seq_lens
                                     int(max_seq_len), float(scale), _ptr(out), 1 if out.dtype == torch.float32 else 0,
                                     _ptr(workspace), int(workspace.numel() * workspace.element_size()),
                                     _stream(stream)), "tq_decode_attention")
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def tq_decode_attention_noalloc(ctx: Context, q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int, out,
+                                scale: float = 0.0, Hkv: int | None = None, stream=None):
+    """tq_decode_attention with the library's own per-device scratch instead of a
+    workspace argument, for callers that cannot allocate device memory (see tq.h).
+    Calls that overlap on the GPU race on that scratch."""
+    import torch
+    B, Hq = int(q.shape[0]), int(q.shape[1])
+    if Hkv is None:
+        Hkv = int(k_cache.shape[1])
+    _check(_lib.tq_decode_attention_noalloc(ctx.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache), int(k_cache.shape[0]),
+                                            _ptr(block_table), int(block_table.shape[1]), _ptr(seq_lens), B, Hq, Hkv,
+                                            int(max_seq_len), float(scale), _ptr(out),
+                                            1 if out.dtype == torch.float32 else 0, _stream(stream)),
+           "tq_decode_attention_noalloc")
 
 
 def tq_get_device_error(ctx: Context, stream=None) -> int:
