@@ -29,6 +29,7 @@
 #include <mutex>
 
 #include "device_util.cuh"
+#include "sm100.cuh"
 
 namespace tq {
 namespace {
@@ -145,51 +146,59 @@ struct PageRegs {
     float vn[2];         // value norm / sqrt(d) of tokens g, g+8
 };
 
+// Fragment bytes of one page from its shared-memory stage (key chunk at kst, value
+// chunk at vst).
 template <int KM, int VM, bool PROD>
-__device__ __forceinline__ void load_page(PageRegs<KM, VM, PROD>& r, const uint8_t* kchunk, const uint8_t* vchunk,
+__device__ __forceinline__ void load_page(PageRegs<KM, VM, PROD>& r, const uint8_t* kst, const uint8_t* vst,
                                           const DecodeArgs& a, int g, int c) {
     constexpr int kBytes = KM == kKBit1 ? 4 : (KM == kKByte2 ? 8 : 16);  // per key row per thread
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-        const uint8_t* row = kchunk + (g + 8 * i) * a.lk.code_row + kBytes * c;
+        const uint8_t* row = kst + (g + 8 * i) * a.lk.code_row + kBytes * c;
         if (kBytes == 16) {
-            const uint4 w = __ldg(reinterpret_cast<const uint4*>(row));
+            const uint4 w = *reinterpret_cast<const uint4*>(row);
             r.k[i][0] = w.x, r.k[i][1] = w.y, r.k[i][2] = w.z, r.k[i][3] = w.w;
         } else if (kBytes == 8) {
-            const uint2 w = __ldg(reinterpret_cast<const uint2*>(row));
+            const uint2 w = *reinterpret_cast<const uint2*>(row);
             r.k[i][0] = w.x, r.k[i][1] = w.y;
         } else {
-            r.k[i][0] = __ldg(reinterpret_cast<const uint32_t*>(row));
+            r.k[i][0] = *reinterpret_cast<const uint32_t*>(row);
         }
         if (PROD) {
-            r.s[i] = __ldg(reinterpret_cast<const uint32_t*>(kchunk + a.lk.signs_off + (g + 8 * i) * 16) + c);
-            r.kg[i] = __ldg(reinterpret_cast<const float*>(kchunk + a.lk.gamma_off) + g + 8 * i) * a.sscale;
+            r.s[i] = reinterpret_cast<const uint32_t*>(kst + a.lk.signs_off + (g + 8 * i) * 16)[c];
+            r.kg[i] = reinterpret_cast<const float*>(kst + a.lk.gamma_off)[g + 8 * i] * a.sscale;
         }
-        r.kn[i] = __ldg(reinterpret_cast<const float*>(kchunk + a.lk.norm_off) + g + 8 * i) * a.qscale;
-        r.vn[i] = __ldg(reinterpret_cast<const float*>(vchunk + a.lv.norm_off) + g + 8 * i) * 0.08838834764831845f;
+        r.kn[i] = reinterpret_cast<const float*>(kst + a.lk.norm_off)[g + 8 * i] * a.qscale;
+        r.vn[i] = reinterpret_cast<const float*>(vst + a.lv.norm_off)[g + 8 * i] * 0.08838834764831845f;
     }
     constexpr int vBytes = VM == kVByte4 ? 8 : 4;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int tok = 2 * c + (i & 1) + 8 * (i >> 1);
-        const uint8_t* row = vchunk + tok * a.lv.code_row + vBytes * g;
+        const uint8_t* row = vst + tok * a.lv.code_row + vBytes * g;
         if (vBytes == 8) {
-            const uint2 w = __ldg(reinterpret_cast<const uint2*>(row));
+            const uint2 w = *reinterpret_cast<const uint2*>(row);
             r.v[i][0] = w.x, r.v[i][1] = w.y;
         } else {
-            r.v[i][0] = __ldg(reinterpret_cast<const uint32_t*>(row));
+            r.v[i][0] = *reinterpret_cast<const uint32_t*>(row);
         }
     }
 }
 
 // Shared memory of the split kernel (byte offsets; V at offset 0).
-//   V   value byte table, lane-replicated: [256][32] half2 (nibbles) or [256][16] 2 x half2 (crumbs)
-//   K   key byte table (same layouts) when keys are not byte-permuted
-//   S   sign nibble table [16] 2 x half2 of +-1 (bit set -> +1)
-//   K1  1-bit key nibble table [16] 2 x half2 of c[bit]
-//   P   per warp P' transpose [2 n-tiles][8 heads][16 tokens] fp16
-//   M   per warp m[16], l[16];  Acc  per warp acc[16 heads][128]
+//   V    value byte table, lane-replicated: [256][32] half2 (nibbles) or [256][16] 2 x half2 (crumbs)
+//   K    key byte table (same layouts) when keys are not byte-permuted
+//   S    sign nibble table [16] 2 x half2 of +-1 (bit set -> +1)
+//   K1   1-bit key nibble table [16] 2 x half2 of c[bit]
+//   P    per warp P' transpose [2 n-tiles][8 heads][16 tokens] fp16
+//   M    per warp m[16], l[16]
+//   Bar  per warp kStagesD mbarriers of the page ring
+//   Ring per warp kStagesD stages of one page (key chunk, then value chunk), filled
+//        by bulk copies; after the page loop the same bytes hold the warps'
+//        accumulators for the CTA merge (Acc: per warp acc[16 heads][128])
 constexpr int kTabBytes = 32768;
+constexpr int kStagesD = 4;
+constexpr int kStageBytes = 2496;  // >= key chunk + value chunk for every bit width (16-byte multiple)
 
 template <int KM, int VM, bool PROD>
 struct SmemLayout {
@@ -200,8 +209,12 @@ struct SmemLayout {
     static constexpr uint32_t kOffK1 = kOffS + 128;
     static constexpr uint32_t kOffP = kOffK1 + 128;
     static constexpr uint32_t kOffM = kOffP + kWarps * 2 * 8 * 16 * 2;
-    static constexpr uint32_t kOffAcc = kOffM + kWarps * 2 * kMaxG * 4;
-    static constexpr uint32_t kBytes = kOffAcc + kWarps * kMaxG * kDim * 4;
+    static constexpr uint32_t kOffBar = kOffM + kWarps * 2 * kMaxG * 4;
+    static constexpr uint32_t kOffRing = (kOffBar + kWarps * kStagesD * 8 + 127) & ~127u;
+    static constexpr uint32_t kRingBytes = kWarps * kStagesD * kStageBytes;
+    static constexpr uint32_t kAccBytes = kWarps * kMaxG * kDim * 4;
+    static constexpr uint32_t kOffAcc = kOffRing;
+    static constexpr uint32_t kBytes = kOffRing + (kRingBytes > kAccBytes ? kRingBytes : kAccBytes);
 };
 
 template <int KM, int VM, bool PROD>
@@ -462,9 +475,18 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
             }
         }
     }
+    const uint32_t ring = sm100::smem_u32(smem + L::kOffRing) + warp * kStagesD * kStageBytes;
+    const uint32_t bars = sm100::smem_u32(smem + L::kOffBar) + warp * kStagesD * 8;
+    if (lane == 0) {
+        for (int st = 0; st < kStagesD; ++st) sm100::mbar_init(bars + 8 * st, 1);
+        sm100::fence_mbar_init();
+    }
     __syncthreads();
     float* wm = reinterpret_cast<float*>(smem + L::kOffM);      // [warp][2][16]: m then l
     float* wacc = reinterpret_cast<float*>(smem + L::kOffAcc);  // [warp][16 heads][128]
+    const volatile int never = 0;
+    uint32_t issued = 0, consumed = 0;  // pages this warp has requested / processed (all items)
+    bool dead = false;                  // a page copy never arrived: this warp stops working
 
     const int items = a.B * a.Hkv * a.splits;
     for (int item = blockIdx.x; item < items; item += gridDim.x) {
@@ -513,34 +535,67 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
             for (int mt = 0; mt < 8; ++mt) acc[nt][mt][0] = acc[nt][mt][1] = acc[nt][mt][2] = acc[nt][mt][3] = 0.f;
         }
 
-        // ---- page loop: one page per warp at a time; two register sets alternate
-        // so that the next page is in flight while the current one is processed
-        auto fetch = [&](int page, PageRegs<KM, VM, PROD>& r) -> bool {
-            const int blk = a.block_table[(size_t)b * a.max_blocks + page];
-            if (blk < 0 || blk >= a.num_blocks) return false;
-            load_page<KM, VM, PROD>(r, a.kc + ((size_t)blk * a.Hkv + hk) * a.lk.bytes,
-                                    a.vc + ((size_t)blk * a.Hkv + hk) * a.lv.bytes, a, g, c);
-            return true;
-        };
-        auto handle = [&](int page, bool ok, const PageRegs<KM, VM, PROD>& r) {
-            if (!ok) {
-                if (lane == 0) atomicOr(a.err, TQ_DEVERR_BLOCK);
-                return;
+        // ---- page loop: the warp takes pages first, first + 4, ...; a ring of
+        // kStagesD shared-memory stages keeps the next pages' bulk copies in flight
+        const int first = p0 + warp;
+        const int nj = first < p1 ? (p1 - first + kWarps - 1) / kWarps : 0;
+        const int* btab = a.block_table + (size_t)b * a.max_blocks + first;
+        const int win = (lane < nj) ? btab[lane * kWarps] : -1;  // block ids of the first 32 pages
+        auto blk_of = [&](int j) -> int {
+            int v = __shfl_sync(0xffffffffu, win, j & 31);
+            if (j >= 32) {
+                v = lane == 0 ? btab[j * kWarps] : 0;
+                v = __shfl_sync(0xffffffffu, v, 0);
             }
-            process_page<KM, VM, PROD, NT>(r, min(kPage, Ls - page * kPage), x, bq, bs, m, l, acc);
+            return v;
         };
-        PageRegs<KM, VM, PROD> ra, rb;
-        int p = p0 + warp;
-        bool oka = (p < p1) && fetch(p, ra);
-        while (p < p1) {
-            const int pb = p + kWarps;
-            const bool okb = (pb < p1) && fetch(pb, rb);
-            handle(p, oka, ra);
-            if (pb >= p1) break;
-            const int pa = pb + kWarps;
-            oka = (pa < p1) && fetch(pa, ra);
-            handle(pb, okb, rb);
-            p = pa;
+        const uint32_t kb = (uint32_t)a.lk.bytes, vb = (uint32_t)a.lv.bytes;
+        auto issue = [&](int j) {
+            const int blk = blk_of(j);
+            const uint32_t st = ring + (issued % kStagesD) * kStageBytes;
+            const uint32_t bar = bars + 8 * (issued % kStagesD);
+            if (lane == 0) {
+                if (blk >= 0 && blk < a.num_blocks) {
+                    const size_t chunk = (size_t)blk * a.Hkv + hk;
+                    sm100::mbar_arrive_expect_tx(bar, kb + vb);
+                    sm100::bulk_g2s(st, a.kc + chunk * kb, kb, bar);
+                    sm100::bulk_g2s(st + kb, a.vc + chunk * vb, vb, bar);
+                } else {
+                    sm100::mbar_arrive(bar);  // nothing to copy: the stage completes at once
+                }
+            }
+            ++issued;
+        };
+        if (!dead)
+            for (int j = 0; j < nj && j < kStagesD; ++j) issue(j);
+        for (int j = 0; j < nj && !dead; ++j) {
+            const uint32_t sidx = consumed % kStagesD;
+            bool ok = sm100::mbar_wait(bars + 8 * sidx, (consumed / kStagesD) & 1u, &never, 2000000000ull);
+            ok = __all_sync(0xffffffffu, ok);
+            const int blk = blk_of(j);
+            if (!ok) {
+                if (lane == 0) atomicOr(a.err, TQ_DEVERR_TIMEOUT);
+                dead = true;
+                break;
+            }
+            ++consumed;
+            const int page = first + j * kWarps;
+            if (blk < 0 || blk >= a.num_blocks) {
+                if (lane == 0) atomicOr(a.err, TQ_DEVERR_BLOCK);
+            } else {
+                const uint8_t* st = smem + L::kOffRing + (size_t)(warp * kStagesD + sidx) * kStageBytes;
+                PageRegs<KM, VM, PROD> r;
+                load_page<KM, VM, PROD>(r, st, st + kb, a, g, c);
+                process_page<KM, VM, PROD, NT>(r, min(kPage, Ls - page * kPage), x, bq, bs, m, l, acc);
+            }
+            __syncwarp();  // every lane is done with the stage before it is refilled
+            if (j + kStagesD < nj) issue(j + kStagesD);
+        }
+        if (dead) {  // let copies already in flight land before the stages are reused
+            while (consumed < issued) {
+                sm100::mbar_wait(bars + 8 * (consumed % kStagesD), (consumed / kStagesD) & 1u, &never, 2000000000ull);
+                ++consumed;
+            }
         }
 
         // ---- merge the warps of the CTA (coordinates back in natural order)
@@ -663,7 +718,7 @@ size_t split_smem(int km) {
 }
 
 int ctas_per_sm_for(size_t smem) {
-    int n = (int)((227 * 1024) / (smem + 1024));
+    int n = (int)(233472 / (smem + 1024));  // 228 KB of shared memory per SM, 1 KB reserved per CTA
     if (n > 4) n = 4;
     return n < 1 ? 1 : n;
 }
