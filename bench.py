@@ -41,8 +41,8 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--workload", default="batched")
     ap.add_argument("--bits", type=int, default=4)
@@ -149,7 +149,8 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- distributed
-def dist_setup(args):
+def dist_setup(backend: str = "nccl"):
+    """One process per GPU (torchrun env).  Returns (world_size, rank, local_rank)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -158,9 +159,11 @@ def dist_setup(args):
 
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return ws, rank, local
 
 
@@ -170,14 +173,26 @@ def barrier(ws):
         dist.barrier()
 
 
-def max_over_ranks(ws, x: float) -> float:
+def max_over_ranks(ws, x: float, device: str = "cuda") -> float:
+    """Largest x over all ranks (every rank gets it)."""
     if ws == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_data_seed(rank: int) -> int:
+    """Each replica compresses and attends over its own seeded batch."""
+    return 1 + 1000003 * rank
+
+
+def whole_job_gbs(ws: int, bytes_per_rank_step: float, ms_step_max: float) -> float:
+    """Weak scaling: every rank moves the same bytes per step; the step time is
+    the slowest rank's."""
+    return ws * bytes_per_rank_step / (ms_step_max * 1e-3) / 1e9
 
 
 # ---------------------------------------------------------------- oracle (CPU) leg
@@ -266,7 +281,7 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
-    ws, rank, local = dist_setup(args)
+    ws, rank, local = dist_setup("nccl")
     import numpy as np
     import torch
 
@@ -275,7 +290,7 @@ def main():
     dev = torch.device("cuda", local)
     rot = 1 if args.rotation == "hadamard" else 0
     w = W.WORKLOADS[args.workload].with_(bits=args.bits, rotation=rot, decode_steps=0,
-                                         data_seed=1 + 1000003 * rank)
+                                         data_seed=rank_data_seed(rank))
     ctx = tq.tq_init(D, w.bits, w.param_seed, w.rotation, w.key_mode)
     bt_np = W.block_table(w)
     slots_np = W.prefill_slots(w, bt_np)
@@ -339,7 +354,7 @@ def main():
 
     cbytes, dbytes = step_bytes(w)
     ms_step = ms_total / args.steps
-    value = ws * (cbytes + dbytes) / (ms_step * 1e-3) / 1e9
+    value = whole_job_gbs(ws, cbytes + dbytes, ms_step)
     peak, peak_kind = measured_peak()
     comp_avg = max_over_ranks(ws, sum(comp_ms) / len(comp_ms))
     dec_avg = max_over_ranks(ws, sum(dec_ms) / len(dec_ms))
@@ -388,7 +403,7 @@ def main():
     torch.cuda.synchronize()
     barrier(ws)
     e2e_ms = max_over_ranks(ws, a.elapsed_time(b)) / args.e2e_steps
-    e2e_val = ws * (cbytes + dbytes) / (e2e_ms * 1e-3) / 1e9
+    e2e_val = whole_job_gbs(ws, cbytes + dbytes, e2e_ms)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
