@@ -1,5 +1,6 @@
 """One rank of the world_size-2 CPU test of the benchmark's multi-rank host logic
-(run under torchrun with the gloo backend; prints one JSON line per rank)."""
+(run under torchrun with the gloo backend; each rank writes rank<r>.json into
+the directory given as the first argument)."""
 import json
 import os
 import sys
@@ -24,8 +25,10 @@ def main():
     sums = [torch.zeros(1, dtype=torch.float64) for _ in range(ws)]
     import torch.distributed as dist
     dist.all_gather(sums, torch.tensor([csum], dtype=torch.float64))
-    print(json.dumps({"rank": rank, "ws": ws, "tmax": t, "sums": [float(s) for s in sums],
-                      "value": bench.whole_job_gbs(ws, 1e9, t)}), flush=True)
+    rec = {"rank": rank, "ws": ws, "tmax": t, "sums": [float(s) for s in sums],
+           "value": bench.whole_job_gbs(ws, 1e9, t)}
+    with open(os.path.join(sys.argv[1], "rank%d.json" % rank), "w") as f:
+        json.dump(rec, f)
     bench.barrier(ws)
     dist.destroy_process_group()
 
