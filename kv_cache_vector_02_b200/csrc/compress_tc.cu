@@ -9,7 +9,10 @@
 // One CTA per SM walks 128-vector tiles of the flattened [T*Hkv, 128] input:
 //   warp 0       TMA producer: 128x128 fp16 tiles (two 128-byte-swizzled boxes)
 //   warp 1       TMEM owner and single-thread MMA issuer
-//   warps 2..17  epilogue, four warps per TMEM lane quarter (32 columns each)
+//   warps 2..17  epilogue, two teams of eight warps; team t takes the CTA's
+//                tiles k with k % 2 == t in TMEM buffer t, so one team's waits
+//                overlap the other team's arithmetic.  In a team, the two warps
+//                of each TMEM lane quarter split a row's 128 columns in halves.
 // Rotation: D[v][n] = sum_k x[v][k] B[n][k] with B the rotation split into
 // fp16 parts held in shared memory for the whole kernel:
 //   Haar      B = 16 R^T = hi + lo (two passes, x is exact in fp16, products are
@@ -19,17 +22,20 @@
 // 1e-6 the rotation goes to two accumulators, A = (lo pass) + K-steps 0-3 of the
 // hi pass and B = K-steps 4-7, summed in registers (acc = A + B).
 // In both cases v = sqrt(d) y / ||x|| = sqrt(d) acc / ||acc||, so the epilogue
-// only needs ||acc||.  Codes come from a 2 KB shared-memory table of uniform
-// cells over v (each cell holds at most one boundary), one exact fp32 compare.
-// Keys (prod mode): r = acc - c[code] ||acc|| / sqrt(d) (the residual in the
-// rotated domain, scaled), gamma = ||r|| / scale, and the sign sketch
+// only needs ||acc||; it works in cell units u = v * scale of a shared-memory
+// table of uniform cells (each holds at most one boundary): round(u) addresses
+// the cell, one fp32 compare with its boundary gives the code.
+// Keys (prod mode): the residual d = u - c[code] (cell units) gives
+// gamma = ||x - x_hat|| and rho = 32 (v - c[code]), and the sign sketch
 //   S (x - x_hat) = (S R) (y - y_hat)
-// is a second contraction whose A operand rho ~ r (split into fp16 hi + lo) is
-// written by the epilogue straight into tensor memory (over the tile's own,
-// already read, accumulator A; the sketch accumulates over B):
-//   Haar      acc2 = rho_hi M_hi + rho_lo M_hi + rho_hi M_lo   (M = S R)
-//   Hadamard  acc2 = (rho_hi + rho_lo) M',   M' = S D H integer, exact in fp16
+// is a second contraction whose A operand rho (split into fp16 hi + lo) the
+// epilogue writes back into tensor memory over the accumulator columns it has
+// just read; the sketch accumulates over the tile's B accumulator:
+//   Haar      acc2 = rho_lo M_hi + rho_hi M_lo + rho_hi M_hi   (M = S R)
+//   Hadamard  acc2 = (rho_lo + rho_hi) M',   M' = S D H integer, exact in fp16
 // sign bit j = [acc2_j >= 0].  Every wait is bounded (TQ_DEVERR_TIMEOUT).
+#include <cmath>
+
 #include <cuda.h>
 
 #include "device_util.cuh"
@@ -41,36 +47,31 @@ namespace {
 
 using namespace sm100;
 
+constexpr int kTeams = 2;
 constexpr int kEpiWarps = 16;
-constexpr int kEpiThreads = kEpiWarps * 32;
-constexpr int kSpan = 4 * 128 / kEpiWarps;  // columns per epilogue thread
-constexpr int kQ = 128 / kSpan;             // epilogue threads per row
-constexpr int kThreads = 64 + kEpiThreads;
+constexpr int kTeamThreads = kEpiWarps * 32 / kTeams;  // 256
+constexpr int kHalfCols = 64;                            // columns of a row per thread
+constexpr int kThreads = 64 + kEpiWarps * 32;
 constexpr uint32_t kTile = 128 * 128 * 2;  // one 128 x 128 fp16 operand
 constexpr uint32_t kHalf = kTile / 2;      // one 128-byte-swizzled K-half
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kSmemMax = 232448;
 
-// TMEM (512 columns).  Values: two tile buffers [A 128 | B 128] at 0 and 256.
-// Keys: one rotation buffer [A | B] at 0 (released as soon as it has been read, so
-// the next tile's rotation overlaps this tile's epilogue) and a sketch region at
-// 256: rho_hi [256,320), rho_lo [320,384) (the A operand, fp16 pairs) and the
-// sketch accumulator [384,512).  The epilogue reads tile k-1's sketch before it
-// writes tile k's rho, so the sketch contraction overlaps the epilogue too.
+// TMEM (512 columns): buffer t at 256 t holds team t's tile: the rotation
+// accumulators A [0,128) and B [128,256).  Keys then reuse A for rho: the 16
+// coordinates of K-step st (A columns [16 st, 16 st + 16)) become 8 columns of
+// rho_hi pairs followed by 8 of rho_lo pairs, written by the thread that has
+// just read those A columns, and the sketch accumulates over B.
 constexpr uint32_t kBufCols = 256;
 constexpr uint32_t kColB = 128;
-constexpr uint32_t kColRhoHi = 256;
-constexpr uint32_t kColRhoLo = 320;
-constexpr uint32_t kColQjl = 384;
 
 template <int ROT, bool PROD>
 struct Cfg {
     static constexpr int kRotImages = ROT == 0 ? 2 : 1;
     static constexpr int kQjlImages = PROD ? (ROT == 0 ? 2 : 1) : 0;
     static constexpr int kImages = kRotImages + kQjlImages;
-    static constexpr int kCells = PROD ? kLutCellsProd : kLutCellsMse;
     static constexpr int kLutBytes = PROD ? kLutBytesProd : kLutBytesMse;
-    static constexpr uint32_t kPartBytes = 2 * 2 * kQ * 128 * 4;  // [tile parity][norm, gamma][span][row]
+    static constexpr uint32_t kPartBytes = kTeams * 2 * 2 * 128 * 4;  // [team][norm, gamma][half][row]
     static constexpr uint32_t kBarBytes = 512;
     static constexpr uint32_t kFixed = kImages * kTile + kLutBytes + kPartBytes + kBarBytes;
     static constexpr int kStagesFit = (int)((kSmemMax - kFixed) / kTile);
@@ -89,14 +90,14 @@ struct Cfg {
 // barrier indices
 enum : int {
     kBarConst = 0,
-    kBarXFull = 1,    // +stage (4)
-    kBarXEmpty = 5,   // +stage (4)
-    kBarRotFull = 9,  // +buffer (2)
-    kBarRotEmpty = 11,
-    kBarRhoFull = 13,
-    kBarQjlFull = 14,
-    kBarDrain = 15,
-    kNumBars = 16
+    kBarXFull = 1,     // +stage (4)
+    kBarXEmpty = 5,    // +stage (4)
+    kBarRotFull = 9,   // +team: rotation accumulators ready
+    kBarRotEmpty = 11, // +team: the team is done with its buffer
+    kBarRhoFull = 13,  // +team: rho written (keys)
+    kBarQjlFull = 15,  // +team: sketch ready (keys)
+    kBarDrain = 17,
+    kNumBars = 18
 };
 
 struct TcArgs {
@@ -108,24 +109,51 @@ struct TcArgs {
     const uint8_t* images;  // kImages pre-swizzled 32 KB operands
     const uint8_t* lut;     // bucketize table
     ChunkLayout lay;
-    float lut_scale, lut_magic;
-    float n2_scale;  // ||x||^2 = n2_scale * ||acc||^2
+    float lut_kscale;  // sqrt(d) * table scale: u = acc * lut_kscale / ||acc|| is v in cell units
+    float lut_magic;   // 1.5 * 2^23 + cells / 2
+    float rho_scale;   // 32 / table scale: rho = 32 (v - c) from the cell-unit residual
+    float n_scale;     // ||x|| = n_scale * ||acc||
+    float gamma_scale; // n_scale / (sqrt(d) * table scale): gamma = ||d|| ||acc|| gamma_scale
     uint32_t* err;
-};
-
-struct LutMse {
-    float bnd;
-    int base;
-};
-struct LutProd {
-    float bnd;
-    int base;
-    float c_lo, c_hi;
 };
 
 __device__ __forceinline__ void set_abort(volatile int* abort, uint32_t* err) {
     *abort = 1;
     atomicOr(err, TQ_DEVERR_TIMEOUT);
+}
+
+// 1/sqrt(x) for finite x > 0: the hardware estimate and one Newton step
+// r' = r + r (1 - x r^2) / 2, within about an ulp.
+__device__ __forceinline__ float rsqrt_refined(float x) {
+    const float r = rsqrtf(x);
+    const float e = fmaf(-x * r, r, 1.0f);
+    return fmaf(0.5f * r, e, r);
+}
+
+// Table reads at a 32-bit shared-memory address.
+__device__ __forceinline__ void lds_v2(uint32_t addr, uint32_t& x, uint32_t& y) {
+    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(x), "=r"(y) : "r"(addr));
+}
+__device__ __forceinline__ void lds_v4(uint32_t addr, uint32_t& x, uint32_t& y, uint32_t& z, uint32_t& w) {
+    asm("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(x), "=r"(y), "=r"(z), "=r"(w) : "r"(addr));
+}
+
+// Named barrier `id` over `count` threads that also ORs a predicate across them:
+// every participant gets the same answer.
+__device__ __forceinline__ bool bar_any(int id, int count, bool p) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)p), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ float2 ld_sum(const uint32_t (&r0)[32], const uint32_t (&r1)[32], int i) {
+    return __fadd2_rn(make_float2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1])),
+                      make_float2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1])));
 }
 
 template <int ROT, bool PROD, int W>
@@ -151,12 +179,12 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
             mbar_init(bar(kBarXFull + s), 1);
             mbar_init(bar(kBarXEmpty + s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(bar(kBarRotFull + b), 1);
-            mbar_init(bar(kBarRotEmpty + b), kEpiThreads);
+        for (int t = 0; t < kTeams; ++t) {
+            mbar_init(bar(kBarRotFull + t), 1);
+            mbar_init(bar(kBarRotEmpty + t), kTeamThreads);
+            mbar_init(bar(kBarRhoFull + t), kTeamThreads);
+            mbar_init(bar(kBarQjlFull + t), 1);
         }
-        mbar_init(bar(kBarRhoFull), kEpiThreads);
-        mbar_init(bar(kBarQjlFull), 1);
         mbar_init(bar(kBarDrain), 1);
         *abort = 0;
         fence_mbar_init();
@@ -207,14 +235,15 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
             auto kdesc = [](uint32_t base, int step) {  // K-step of 16 elements inside a 128x128 operand
                 return smem_desc_sw128(base + (uint32_t)(step >> 2) * kHalf + (uint32_t)(step & 3) * 32u);
             };
-            auto issue_rot = [&](int k) -> bool {
+            // rotation of local tile k into its team's buffer; false when not ready yet
+            auto try_rot = [&](int k) -> bool {
                 const int s = k % C::kStages;
-                const int b = PROD ? 0 : (k & 1);
-                const uint32_t use = PROD ? (uint32_t)k : (uint32_t)(k >> 1);  // use count of buffer b
-                if (!mbar_wait(bar(kBarXFull + s), (uint32_t)(k / C::kStages) & 1u, abort, kWaitNs)) return false;
-                if (!mbar_wait(bar(kBarRotEmpty + b), (use & 1u) ^ 1u, abort, kWaitNs)) return false;
+                const int t = k & 1;
+                const uint32_t use = (uint32_t)(k >> 1);
+                if (!mbar_try_wait(bar(kBarXFull + s), (uint32_t)(k / C::kStages) & 1u)) return false;
+                if (!mbar_try_wait(bar(kBarRotEmpty + t), (use & 1u) ^ 1u)) return false;
                 tc_fence_after();
-                const uint32_t dA = tmem + kBufCols * b, dB = dA + kColB;
+                const uint32_t dA = tmem + kBufCols * (uint32_t)t, dB = dA + kColB;
                 const uint32_t xs = sbase + C::kOffX + s * kTile;
                 uint32_t accA = 0u;
                 if (ROT == 0) {  // the small lo pass first, then K-steps 0-3 of the hi pass
@@ -232,34 +261,65 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
 #pragma unroll
                 for (int st = 4; st < 8; ++st) umma_ss(dB, kdesc(xs, st), kdesc(img, st), idesc, st > 4 ? 1u : 0u);
                 umma_commit(bar(kBarXEmpty + s));
-                umma_commit(bar(kBarRotFull + b));
+                umma_commit(bar(kBarRotFull + t));
                 return true;
             };
-            auto issue_qjl = [&](int k) -> bool {
-                if (!mbar_wait(bar(kBarRhoFull), (uint32_t)k & 1u, abort, kWaitNs)) return false;
+            // sketch of local tile k (keys); false when its rho is not written yet
+            auto try_qjl = [&](int k) -> bool {
+                const int t = k & 1;
+                if (!mbar_try_wait(bar(kBarRhoFull + t), (uint32_t)(k >> 1) & 1u)) return false;
                 tc_fence_after();
-                const uint32_t d = tmem + kColQjl;
+                const uint32_t buf = tmem + kBufCols * (uint32_t)t;
+                const uint32_t d = buf + kColB;
                 const uint32_t m0 = img + C::kRotImages * kTile;
+                // rho of K-step st: columns 16 st (hi pairs) and 16 st + 8 (lo pairs)
+                auto rho_col = [&](int st) { return buf + 16u * (uint32_t)st; };
                 uint32_t acc2 = 0u;
                 // the small terms first: rho_lo M_hi (+ rho_hi M_lo for Haar), then rho_hi M_hi
 #pragma unroll
                 for (int st = 0; st < 8; ++st) {
-                    umma_ts(d, tmem + kColRhoLo + 8u * st, kdesc(m0, st), idesc, acc2);
+                    umma_ts(d, rho_col(st) + 8u, kdesc(m0, st), idesc, acc2);
                     acc2 = 1u;
                 }
                 if (ROT == 0) {
 #pragma unroll
-                    for (int st = 0; st < 8; ++st) umma_ts(d, tmem + kColRhoHi + 8u * st, kdesc(m0 + kTile, st), idesc, 1u);
+                    for (int st = 0; st < 8; ++st) umma_ts(d, rho_col(st), kdesc(m0 + kTile, st), idesc, 1u);
                 }
 #pragma unroll
-                for (int st = 0; st < 8; ++st) umma_ts(d, tmem + kColRhoHi + 8u * st, kdesc(m0, st), idesc, 1u);
-                umma_commit(bar(kBarQjlFull));
+                for (int st = 0; st < 8; ++st) umma_ts(d, rho_col(st), kdesc(m0, st), idesc, 1u);
+                umma_commit(bar(kBarQjlFull + t));
                 return true;
             };
-            if (ok && my_tiles > 0) ok = issue_rot(0);
-            for (int k = 0; ok && k < my_tiles; ++k) {
-                if (k + 1 < my_tiles) ok = issue_rot(k + 1);
-                if (ok && PROD) ok = issue_qjl(k);
+            // Rotations go in tile order (the stage ring); each team's sketch goes
+            // as soon as its rho is in.  Polls with a bound on time without progress.
+            int next_rot = 0;
+            int qjl_next[kTeams] = {0, 1};
+            uint64_t t_last = globaltimer_ns();
+            uint32_t spins = 0;
+            while (ok) {
+                bool progress = false;
+                if (PROD) {
+#pragma unroll
+                    for (int t = 0; t < kTeams; ++t) {
+                        const int k = qjl_next[t];
+                        if (k < next_rot && try_qjl(k)) {
+                            qjl_next[t] = k + kTeams;
+                            progress = true;
+                        }
+                    }
+                }
+                if (next_rot < my_tiles && (!PROD || qjl_next[next_rot & 1] >= next_rot - 1) && try_rot(next_rot)) {
+                    ++next_rot;
+                    progress = true;
+                }
+                const bool done = next_rot >= my_tiles && (!PROD || (qjl_next[0] >= my_tiles && qjl_next[1] >= my_tiles));
+                if (done) break;
+                if (progress) {
+                    spins = 0;
+                    t_last = globaltimer_ns();
+                } else if ((++spins & 31u) == 0) {
+                    if (*abort || globaltimer_ns() - t_last > kWaitNs) ok = false;
+                }
             }
             if (!ok) set_abort(abort, a.err);
             // all MMAs of this CTA complete before its tensor memory is released
@@ -271,191 +331,220 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
     } else {
         // ------------------------------------------------------------ epilogue
         const int ew = warp - 2;
-        const int quarter = warp & 3;  // TMEM lanes this warp may access
-        const int h = ew >> 2;         // column span [kSpan h, kSpan (h+1))
+        const int quarter = warp & 3;     // TMEM lanes this warp may access
+        const int team = ew >> 3;         // tiles k with k % 2 == team, buffer team
+        const int hh = (ew >> 2) & 1;     // column half [64 hh, 64 hh + 64)
         const int row = quarter * 32 + lane;
+        const int pbar = 1 + team * 4 + quarter;  // the two warps that share these rows
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        float* part = reinterpret_cast<float*>(smem + C::kOffPart);
-        // this lane's replica of the bucketize table (see tc_params.h)
-        const uint8_t* lut = smem + C::kOffLut + (PROD ? 16 * (lane & (kLutReplProd - 1)) : 8 * (lane & (kLutReplMse - 1)));
-        const float sqrt_d = 11.313708498984761f;
-        constexpr int kPer = 32 / W;          // codes per 32-bit word
-        constexpr int kWords = kSpan / kPer;  // words of this thread's span
+        const uint32_t buf = tmem + lane_addr + kBufCols * (uint32_t)team;
+        float* pn = reinterpret_cast<float*>(smem + C::kOffPart) + team * (2 * 2 * 128);
+        float* pg = pn + 2 * 128;
+        // table entry of u: bits(u + magic) * 128 + lut_off, in this lane's replica
+        // (bits(u + magic) = bits(1.5 * 2^23) + cells / 2 + round(u), see tc_params.h)
+        const uint32_t lut_off = sbase + C::kOffLut +
+                                 (PROD ? 16u * (uint32_t)(lane & (kLutReplProd - 1))
+                                       : 8u * (uint32_t)(lane & (kLutReplMse - 1))) -
+                                 __float_as_uint(12582912.0f) * 128u;
+        const float2 magic2 = make_float2(a.lut_magic, a.lut_magic);
+        const float2 rho_k = make_float2(a.rho_scale, a.rho_scale);
+        constexpr int kPer = 32 / W;               // codes per 32-bit word
+        constexpr int kWords = kHalfCols / kPer;   // words of this thread's 64 columns
+        constexpr int kHW = kWords / 2;            // words of one 32-column half
         bool ok = mbar_wait(bar(kBarConst), 0, abort, kWaitNs);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) set_abort(abort, a.err);
 
-        // destination of this thread's row of a tile: the chunk pointer with the row
-        // inside the page in its low 4 bits (chunks are 16-byte aligned), or null
-        auto dest = [&](int tile) -> uint8_t* {
+        // slot of this thread's row of a tile, and the row's destination: the chunk
+        // pointer with the row inside the page in its low 4 bits (chunks are
+        // 16-byte aligned), or null
+        auto slot_of = [&](int tile) -> int {
             const int vi = tile * 128 + row;
-            if (vi >= a.N) return nullptr;
-            const int t = vi / a.H, head = vi - t * a.H;
-            const long s = a.slots[t];
-            if (s >= (long)a.num_blocks * kPage) {
-                if (h == 0) atomicOr(a.err, TQ_DEVERR_SLOT);
+            return vi < a.N ? __ldg(a.slots + vi / a.H) : -1;
+        };
+        auto dest = [&](int tile, int slot) -> uint8_t* {
+            const int vi = tile * 128 + row;
+            if (vi >= a.N || slot < 0) return nullptr;
+            if (slot >= a.num_blocks * kPage) {
+                if (hh == 0) atomicOr(a.err, TQ_DEVERR_SLOT);
                 return nullptr;
             }
-            if (s < 0) return nullptr;
-            return a.cache + ((size_t)(s / kPage) * a.H + head) * (size_t)a.lay.bytes + (size_t)(s % kPage);
+            const int head = vi % a.H;
+            return a.cache + ((size_t)(slot / kPage) * a.H + head) * (size_t)a.lay.bytes + (size_t)(slot % kPage);
         };
-        auto store = [&](uint8_t* d, const uint32_t (&words)[kWords], float norm, float gamma, uint32_t sg) {
+        auto store = [&](uint8_t* d, const uint32_t (&words)[kWords], float norm, float gamma, uint2 sg) {
             if (!d) return;
             const int pr = (int)((uintptr_t)d & 15u);
             uint8_t* chunk = d - pr;
-            uint8_t* cp = chunk + pr * a.lay.code_row + h * (a.lay.code_row / kQ);
-            if (kWords == 4) {
-                *reinterpret_cast<uint4*>(cp) = make_uint4(words[0], words[1], words[2], words[kWords - 1]);
-            } else if (kWords == 2) {
-                *reinterpret_cast<uint2*>(cp) = make_uint2(words[0], words[kWords - 1]);
+            uint8_t* cp = chunk + pr * a.lay.code_row + hh * (a.lay.code_row / 2);
+            if (kWords == 8) {
+                reinterpret_cast<uint4*>(cp)[0] = make_uint4(words[0], words[1], words[2], words[3]);
+                reinterpret_cast<uint4*>(cp)[1] = make_uint4(words[4 % kWords], words[5 % kWords], words[6 % kWords], words[7 % kWords]);
+            } else if (kWords == 4) {
+                *reinterpret_cast<uint4*>(cp) = make_uint4(words[0], words[1 % kWords], words[2 % kWords], words[3 % kWords]);
             } else {
-                *reinterpret_cast<uint32_t*>(cp) = words[0];
+                *reinterpret_cast<uint2*>(cp) = make_uint2(words[0], words[1 % kWords]);
             }
-            if (PROD) *reinterpret_cast<uint32_t*>(chunk + a.lay.signs_off + pr * (kDim / 8) + h * 4) = sg;
-            if (h == 0) {
+            if (PROD) *reinterpret_cast<uint2*>(chunk + a.lay.signs_off + pr * (kDim / 8) + hh * 8) = sg;
+            if (hh == 0) {
                 reinterpret_cast<float*>(chunk + a.lay.norm_off)[pr] = norm;
                 if (PROD) reinterpret_cast<float*>(chunk + a.lay.gamma_off)[pr] = gamma;
             }
         };
-        // read tile k's sketch accumulator and turn it into sign bits (bit set when >= 0)
-        auto read_signs = [&](int k, bool nonzero, uint32_t& sg) -> bool {
-            bool ok3 = mbar_wait(bar(kBarQjlFull), (uint32_t)k & 1u, abort, kWaitNs);
-            ok3 = __all_sync(0xffffffffu, ok3);
-            if (!ok3) return false;
-            tc_fence_after();
+        // 32 sketch columns as sign bits (bit j set when column j >= 0)
+        auto signs32 = [&](uint32_t col) -> uint32_t {
             uint32_t q[32];
-            tmem_ld32(tmem + lane_addr + kColQjl + kSpan * h, q);
+            tmem_ld32(col, q);
             tmem_ld_wait();
-            uint32_t n0 = 0u;
+            uint32_t neg = 0u;  // bit j = sign bit of column j
 #pragma unroll
-            for (int j = 0; j < 32; ++j) n0 |= (q[j] >> 31) << j;
-            sg = nonzero ? ~n0 : 0xffffffffu;
-            return true;
-        };
-        auto sum4 = [&](const float* pp) {
-            return (pp[row] + pp[128 + row]) + (pp[256 + row] + pp[384 + row]);
+            for (int j = 31; j >= 0; --j) neg = __funnelshift_l(q[j], neg, 1);
+            return ~neg;
         };
 
-        // the previous tile's outputs wait here until its sketch is ready (keys)
-        uint32_t pw[kWords];
-        float pnorm = 0.f, pgamma = 0.f;
-        bool pnz = false;
-        uint8_t* pdst = nullptr;
-        for (int k = 0; k < my_tiles; ++k) {
+        int slot_next = team < my_tiles ? slot_of((int)blockIdx.x + team * (int)gridDim.x) : -1;
+        for (int k = team; k < my_tiles; k += kTeams) {
             const int tile = (int)blockIdx.x + k * (int)gridDim.x;
-            const int b = PROD ? 0 : (k & 1);
-            const uint32_t use = PROD ? (uint32_t)k : (uint32_t)(k >> 1);
-            float* pn = part + ((k & 1) * 2 + 0) * (kQ * 128);
-            float* pg = part + ((k & 1) * 2 + 1) * (kQ * 128);
-            uint8_t* dst = dest(tile);  // issued early: the slot load overlaps the wait below
-            // ---- rotation accumulators A + B -> registers
-            float acc[kSpan];
-            const uint32_t buf = tmem + lane_addr + kBufCols * (uint32_t)b + kSpan * h;
-            ok = !*abort && mbar_wait(bar(kBarRotFull + b), use & 1u, abort, kWaitNs);
-            ok = __all_sync(0xffffffffu, ok);
-            if (ok) {
-                tc_fence_after();
-                uint32_t r0[32], r1[32];
-                tmem_ld32(buf, r0);
-                tmem_ld32(buf + kColB, r1);
-                tmem_ld_wait();
-                tc_fence_before();
-                mbar_arrive(bar(kBarRotEmpty + b));
+            const uint32_t use = (uint32_t)(k >> 1);
+            const int slot = slot_next;
+            if (k + kTeams < my_tiles) slot_next = slot_of(tile + kTeams * (int)gridDim.x);
+            uint8_t* dst = dest(tile, slot);
+            bool good = !*abort && mbar_wait(bar(kBarRotFull + team), use & 1u, abort, kWaitNs);
+            good = __all_sync(0xffffffffu, good);
+            // ---- ||acc||^2 over this thread's 64 columns; the upper 32 stay in registers
+            float2 acc[16];
+            float2 q2[4];
 #pragma unroll
-                for (int j = 0; j < kSpan; ++j) acc[j] = __uint_as_float(r0[j]) + __uint_as_float(r1[j]);
+            for (int i = 0; i < 4; ++i) q2[i] = make_float2(0.f, 0.f);
+            if (good) {
+                tc_fence_after();
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(buf + kHalfCols * hh + 32 * hf, r0);
+                    tmem_ld32(buf + kColB + kHalfCols * hh + 32 * hf, r1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        acc[i] = ld_sum(r0, r1, i);
+                        q2[i & 3] = __ffma2_rn(acc[i], acc[i], q2[i & 3]);
+                    }
+                }
             } else {
                 set_abort(abort, a.err);
 #pragma unroll
-                for (int j = 0; j < kSpan; ++j) acc[j] = 0.f;
+                for (int i = 0; i < 16; ++i) acc[i] = make_float2(0.f, 0.f);
             }
-            // ---- ||acc||^2: 8 interleaved partial sums, then the spans of the row
-            float ps[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) ps[i] = 0.f;
-#pragma unroll
-            for (int j = 0; j < kSpan; ++j) ps[j & 7] = fmaf(acc[j], acc[j], ps[j & 7]);
-            pn[h * 128 + row] = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-            named_barrier(1, kEpiThreads);
-            if (*abort) break;
-            const float nsq = sum4(pn);
-            const float nacc = sqrtf(nsq);
-            const float inv = nacc > 0.f ? sqrt_d / nacc : 0.f;
-            const float norm = sqrtf(nsq * a.n2_scale);
+            pn[hh * 128 + row] = ((q2[0].x + q2[0].y) + (q2[1].x + q2[1].y)) + ((q2[2].x + q2[2].y) + (q2[3].x + q2[3].y));
+            if (bar_any(pbar, 64, !good || *abort)) break;
+            const float nsq = pn[row] + pn[128 + row];
+            // rows with inf / nan inputs are quantized as zero vectors (their norm stays non-finite)
+            const bool finite = nsq <= 3.4e38f;
+            const bool live = finite && nsq > 0.f;
+            const float rn = live ? rsqrt_refined(nsq) : 0.f;  // 1 / ||acc||
+            const float nacc = nsq * rn;
+            const float2 s2 = make_float2(a.lut_kscale * rn, a.lut_kscale * rn);
+            const bool any_bad = __any_sync(0xffffffffu, !finite);
+            const float norm = live ? nacc * a.n_scale : (finite ? 0.f : sqrtf(nsq));
 
-            // ---- bucketize + pack (+ residual for keys)
+            // ---- bucketize + pack (+ residual, rho for keys) in groups of 16 columns,
+            // the upper half (still in registers for values) first
             uint32_t words[kWords];
 #pragma unroll
             for (int i = 0; i < kWords; ++i) words[i] = 0u;
-            uint32_t rho_hi[kSpan / 2], rho_lo[kSpan / 2];
-            float gs[4] = {0.f, 0.f, 0.f, 0.f};
-            const float chat_scale = nacc / sqrt_d;
-            const float kappa = nacc > 0.f ? 32.f * sqrt_d / nacc : 0.f;
+            float2 gs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int j = 0; j < kSpan; j += 2) {
-                float rho2[2];
+            for (int grp = 0; grp < 4; ++grp) {
+                const int hf = grp < 2 ? 1 : 0;
+                const int g = grp & 1;
+                const uint32_t col = buf + kHalfCols * hh + 32 * hf + 16 * g;  // A columns of the group
+                float2 av[8];
+                if (hf == 1 && !PROD) {  // keys reload it too: registers are short there
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const float v = acc[j + u] * inv;
-                    const float gg = fmaf(v, a.lut_scale, a.lut_magic);
-                    const int cell = __float_as_int(gg) & (C::kCells - 1);
-                    int code;
-                    if (PROD) {
-                        const LutProd e = *reinterpret_cast<const LutProd*>(lut + cell * 128);
-                        const bool upc = e.bnd < v;
-                        code = e.base + (upc ? 1 : 0);
-                        const float r = fmaf(upc ? -e.c_hi : -e.c_lo, chat_scale, acc[j + u]);
-                        gs[(j + u) & 3] = fmaf(r, r, gs[(j + u) & 3]);
-                        rho2[u] = r * kappa;
-                    } else {
-                        const LutMse e = *reinterpret_cast<const LutMse*>(lut + cell * 128);
-                        code = e.base + (e.bnd < v ? 1 : 0);
-                    }
-                    words[(j + u) / kPer] |= (uint32_t)code << (W * ((j + u) % kPer));
+                    for (int i = 0; i < 8; ++i) av[i] = acc[8 * g + i];
+                } else {  // reload from tensor memory
+                    uint32_t r0[16], r1[16];
+                    tmem_ld16(col, r0);
+                    tmem_ld16(col + kColB, r1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        av[i] = __fadd2_rn(make_float2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1])),
+                                           make_float2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1])));
                 }
-                if (PROD) {  // rho = hi + lo in fp16
-                    const __half2 hi = __floats2half2_rn(rho2[0], rho2[1]);
-                    const float2 hf = __half22float2(hi);
-                    const __half2 lo = __floats2half2_rn(rho2[0] - hf.x, rho2[1] - hf.y);
-                    rho_hi[j >> 1] = *reinterpret_cast<const uint32_t*>(&hi);
-                    rho_lo[j >> 1] = *reinterpret_cast<const uint32_t*>(&lo);
+                if (any_bad && !finite) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) av[i] = make_float2(0.f, 0.f);
+                }
+                uint32_t rho_hi[8], rho_lo[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float2 u = __fmul2_rn(av[i], s2);
+                    const float2 gg = __fadd2_rn(u, magic2);
+                    const uint32_t ad0 = __float_as_uint(gg.x) * 128u + lut_off;
+                    const uint32_t ad1 = __float_as_uint(gg.y) * 128u + lut_off;
+                    uint32_t code0, code1;
+                    if (PROD) {
+                        uint32_t b0, base0, lo0, hi0, b1, base1, lo1, hi1;
+                        lds_v4(ad0, b0, base0, lo0, hi0);
+                        lds_v4(ad1, b1, base1, lo1, hi1);
+                        const bool p0 = __uint_as_float(b0) < u.x;
+                        const bool p1 = __uint_as_float(b1) < u.y;
+                        code0 = base0 + (p0 ? 1u : 0u);
+                        code1 = base1 + (p1 ? 1u : 0u);
+                        const float c0 = __uint_as_float(p0 ? hi0 : lo0);
+                        const float c1 = __uint_as_float(p1 ? hi1 : lo1);
+                        const float2 d = __ffma2_rn(av[i], s2, make_float2(-c0, -c1));  // residual, cell units
+                        gs[i & 1] = __ffma2_rn(d, d, gs[i & 1]);
+                        const float2 rho = __fmul2_rn(d, rho_k);  // 32 (v - c): rho = hi + lo in fp16
+                        const __half2 hi = __floats2half2_rn(rho.x, rho.y);
+                        const float2 back = __half22float2(hi);
+                        const float2 rem = __fadd2_rn(rho, make_float2(-back.x, -back.y));
+                        const __half2 lo = __floats2half2_rn(rem.x, rem.y);
+                        rho_hi[i] = *reinterpret_cast<const uint32_t*>(&hi);
+                        rho_lo[i] = *reinterpret_cast<const uint32_t*>(&lo);
+                    } else {
+                        uint32_t b0, base0, b1, base1;
+                        lds_v2(ad0, b0, base0);
+                        lds_v2(ad1, b1, base1);
+                        code0 = base0 + (__uint_as_float(b0) < u.x ? 1u : 0u);
+                        code1 = base1 + (__uint_as_float(b1) < u.y ? 1u : 0u);
+                    }
+                    const int j = 32 * hf + 16 * g + 2 * i;  // column within this thread's 64
+                    words[j / kPer] += code0 << (W * (j % kPer));
+                    words[(j + 1) / kPer] += code1 << (W * ((j + 1) % kPer));
+                }
+                if (PROD && good) {  // over the group's A columns, already read
+                    tmem_st8(col, rho_hi);
+                    tmem_st8(col + 8, rho_lo);
                 }
             }
             if (!PROD) {
-                store(dst, words, norm, 0.f, 0u);
+                tc_fence_before();
+                mbar_arrive(bar(kBarRotEmpty + team));
+                store(dst, words, norm, 0.f, make_uint2(0u, 0u));
                 continue;
             }
-            pg[h * 128 + row] = (gs[0] + gs[1]) + (gs[2] + gs[3]);
-            // tile k-1's sketch leaves the sketch region before tile k's rho enters it
-            uint32_t sg = 0xffffffffu;
-            bool have_prev = (k > 0) && !*abort;
-            if (have_prev && !read_signs(k - 1, pnz, sg)) {
+            // ---- keys: release rho, exchange the gamma partials, then read the sketch
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(bar(kBarRhoFull + team));
+            pg[hh * 128 + row] = (gs[0].x + gs[0].y) + (gs[1].x + gs[1].y);
+            if (bar_any(pbar, 64, *abort)) break;
+            const float gsq = pg[row] + pg[128 + row];
+            const float gamma = (live && gsq > 0.f) ? gsq * rsqrt_refined(gsq) * nacc * a.gamma_scale : 0.f;
+            bool sk = mbar_wait(bar(kBarQjlFull + team), use & 1u, abort, kWaitNs);
+            sk = __all_sync(0xffffffffu, sk);
+            if (!sk) {
                 set_abort(abort, a.err);
-                have_prev = false;
+                continue;  // the next barrier sees the abort
             }
-            if (!*abort) {
-                tmem_st16(tmem + lane_addr + kColRhoHi + (kSpan / 2) * h, rho_hi);
-                tmem_st16(tmem + lane_addr + kColRhoLo + (kSpan / 2) * h, rho_lo);
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(bar(kBarRhoFull));
-            }
-            named_barrier(1, kEpiThreads);
-            if (*abort) break;
-            if (have_prev) store(pdst, pw, pnorm, pgamma, sg);
-            // this tile's outputs wait for its sketch
-#pragma unroll
-            for (int i = 0; i < kWords; ++i) pw[i] = words[i];
-            pnorm = norm;
-            pgamma = sqrtf(sum4(pg) * a.n2_scale);
-            pnz = nsq > 0.f;
-            pdst = dst;
-        }
-        if (PROD && my_tiles > 0 && !*abort) {
-            uint32_t sg;
-            if (read_signs(my_tiles - 1, pnz, sg))
-                store(pdst, pw, pnorm, pgamma, sg);
-            else
-                set_abort(abort, a.err);
+            tc_fence_after();
+            uint2 sg = make_uint2(signs32(buf + kColB + kHalfCols * hh), signs32(buf + kColB + kHalfCols * hh + 32));
+            if (!live) sg = make_uint2(0xffffffffu, 0xffffffffu);
+            tc_fence_before();
+            mbar_arrive(bar(kBarRotEmpty + team));
+            store(dst, words, norm, gamma, sg);
         }
     }
     __syncthreads();
@@ -496,9 +585,12 @@ cudaError_t launch_compress_tc(const tq_ctx* ctx, int kind, const uint16_t* x, i
     a.images = tabs.images;
     a.lut = value ? tabs.lut_value : tabs.lut_key;
     const LutParams& lp = value ? tabs.lp_value : tabs.lp_key;
-    a.lut_scale = lp.scale;
+    a.lut_kscale = (float)(std::sqrt((double)kDim) * (double)lp.scale);
     a.lut_magic = lp.magic;
-    a.n2_scale = rot == TQ_ROT_HAAR ? 1.0f / 256.0f : 1.0f / 128.0f;
+    a.rho_scale = (float)(32.0 / (double)lp.scale);
+    const double n_scale = rot == TQ_ROT_HAAR ? 1.0 / 16.0 : 1.0 / std::sqrt(128.0);
+    a.n_scale = (float)n_scale;
+    a.gamma_scale = (float)(n_scale / (std::sqrt((double)kDim) * (double)lp.scale));
     a.lay = lay;
     a.err = ctx->dev_error;
     const int ntiles = (N + 127) / 128;

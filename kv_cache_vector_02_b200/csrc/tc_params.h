@@ -11,7 +11,8 @@ namespace tq {
 struct HostParams;
 
 // Bucketize tables: uniform cells over v = sqrt(d) y / ||x|| in [-V, V]; a cell
-// holds at most one interior boundary, far from its edges.
+// holds at most one interior boundary, far from its edges.  Entries hold the
+// boundary (+inf if none) and the levels in cell units u = v * scale.
 // Each entry is stored once per lane group, interleaved, so that the lanes of
 // one shared-memory phase (16 for 8-byte loads, 8 for 16-byte loads) always hit
 // distinct banks: byte offset = cell * 128 + replica * entry_size.
@@ -22,7 +23,7 @@ constexpr int kLutReplProd = 8;
 constexpr int kLutBytesMse = kLutCellsMse * 8 * kLutReplMse;
 constexpr int kLutBytesProd = kLutCellsProd * 16 * kLutReplProd;
 
-// cell = bits(fma(v, scale, magic)) & (cells - 1), magic = 1.5 * 2^23 + cells / 2
+// u = v * scale; cell = bits(u + magic) - bits(1.5 * 2^23), magic = 1.5 * 2^23 + cells / 2
 struct LutParams {
     float scale = 0.f, magic = 0.f;
 };

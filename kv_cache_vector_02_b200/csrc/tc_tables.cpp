@@ -47,7 +47,8 @@ inline int hadamard_sign(int i, int j) { return (__builtin_popcount(unsigned(i &
 
 // Bucketize table for boundaries t (L-1) and levels c (L).  The cell width w is
 // chosen so that [-sqrt(d), sqrt(d)] maps inside [0, cells) and every boundary
-// sits at least 5% of a cell away from a cell edge.
+// sits at least 5% of a cell away from a cell edge.  Boundaries and levels are
+// stored in cell units (value * scale), the unit the kernel compares in.
 bool build_lut(const std::vector<double>& t, const std::vector<double>& c, int cells, bool prod, uint8_t* dst,
                LutParams& lp) {
     const double vmax = std::sqrt(double(kD));
@@ -79,12 +80,12 @@ bool build_lut(const std::vector<double>& t, const std::vector<double>& c, int c
             for (double tk : t) {
                 const double u = double(float(tk)) * double(scale);
                 if (u < ulo) ++base;
-                else if (u < uhi) bnd = float(tk);
+                else if (u < uhi) bnd = float(tk * double(scale));
             }
             if (base > L - 1) base = L - 1;
             if (prod) {
-                const float clo = float(c[base]);
-                const float chi = float(c[base + 1 < L ? base + 1 : base]);
+                const float clo = float(c[base] * double(scale));
+                const float chi = float(c[base + 1 < L ? base + 1 : base] * double(scale));
                 for (int r = 0; r < kLutReplProd; ++r) {
                     uint8_t* e = dst + 128 * cell + 16 * r;
                     std::memcpy(e + 0, &bnd, 4);
