@@ -7,22 +7,24 @@
 // Walsh-Hadamard rotation).
 //
 // One CTA per SM walks 128-vector tiles of the flattened [T*Hkv, 128] input:
-//   warp 0       TMA producer: 128x128 fp16 tiles (two 128-byte-swizzled boxes)
-//   warp 1       TMEM owner and single-thread MMA issuer
-//   warps 2..17  epilogue, two teams of eight warps; team t takes the CTA's
-//                tiles k with k % 2 == t in TMEM buffer t, so one team's waits
-//                overlap the other team's arithmetic.  In a team, the two warps
-//                of each TMEM lane quarter split a row's 128 columns in halves.
+//   warps 0..4n-1  epilogue, n teams of four warps (one per TMEM lane quarter,
+//                  one thread per row); team t takes the CTA's tiles k with
+//                  k % n == t in TMEM buffer t, so one team's waits overlap the
+//                  other teams' arithmetic (values n = 4, keys n = 2)
+//   warp 4n        TMA producer: 128x128 fp16 tiles (two 128-byte-swizzled boxes)
+//   warp 4n+1      TMEM owner and single-thread MMA issuer
 // Rotation: D[v][n] = sum_k x[v][k] B[n][k] with B the rotation split into
 // fp16 parts held in shared memory for the whole kernel:
 //   Haar      B = 16 R^T = hi + lo (two passes, x is exact in fp16, products are
 //             exact, fp32 accumulation)  -> acc = 16 y
 //   Hadamard  B = H D (entries +-1, exact, one pass)  -> acc = sqrt(d) y
-// The tensor core rounds each accumulation step; to keep ||x|| and gamma within
-// 1e-6 the rotation goes to two accumulators, A = (lo pass) + K-steps 0-3 of the
-// hi pass and B = K-steps 4-7, summed in registers (acc = A + B).
-// In both cases v = sqrt(d) y / ||x|| = sqrt(d) acc / ||acc||, so the epilogue
-// only needs ||acc||; it works in cell units u = v * scale of a shared-memory
+// Values: one accumulator; ||x|| comes from the fp16 tile in shared memory
+// (exact squares, fp32 sums), and the codes only need acc within the 1e-6 window.
+// Keys: gamma needs the residual to ~1e-7 of ||x||, and the tensor core rounds
+// each accumulation step, so the rotation goes to two accumulators,
+// A = (lo pass) + K-steps 0-3 of the hi pass and B = K-steps 4-7, summed in
+// registers (acc = A + B), and ||x|| = ||acc|| / (acc / y).
+// In both cases v = sqrt(d) y / ||x||; the epilogue works in cell units u = v * scale of a shared-memory
 // table of uniform cells (each holds at most one boundary): round(u) addresses
 // the cell, one fp32 compare with its boundary gives the code.
 // Keys (prod mode): the residual d = u - c[code] (cell units) gives
@@ -47,22 +49,18 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTeams = 2;
-constexpr int kEpiWarps = 16;
-constexpr int kTeamThreads = kEpiWarps * 32 / kTeams;  // 256
-constexpr int kHalfCols = 64;                            // columns of a row per thread
-constexpr int kThreads = 64 + kEpiWarps * 32;
+constexpr int kTeamThreads = 128;  // one thread per row
 constexpr uint32_t kTile = 128 * 128 * 2;  // one 128 x 128 fp16 operand
 constexpr uint32_t kHalf = kTile / 2;      // one 128-byte-swizzled K-half
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kSmemMax = 232448;
 
-// TMEM (512 columns): buffer t at 256 t holds team t's tile: the rotation
-// accumulators A [0,128) and B [128,256).  Keys then reuse A for rho: the 16
-// coordinates of K-step st (A columns [16 st, 16 st + 16)) become 8 columns of
-// rho_hi pairs followed by 8 of rho_lo pairs, written by the thread that has
-// just read those A columns, and the sketch accumulates over B.
-constexpr uint32_t kBufCols = 256;
+// TMEM (512 columns): buffer t holds team t's tile.  Values: 128-column
+// accumulators at 128 t.  Keys: at 256 t the rotation accumulators A [0,128) and
+// B [128,256); A is then reused for rho: the 16 coordinates of K-step st
+// (A columns [16 st, 16 st + 16)) become 8 columns of rho_hi pairs followed by 8
+// of rho_lo pairs, written by the thread that has just read those A columns, and
+// the sketch accumulates over B.
 constexpr uint32_t kColB = 128;
 
 template <int ROT, bool PROD>
@@ -71,7 +69,7 @@ struct Cfg {
     static constexpr int kQjlImages = PROD ? (ROT == 0 ? 2 : 1) : 0;
     static constexpr int kImages = kRotImages + kQjlImages;
     static constexpr int kLutBytes = PROD ? kLutBytesProd : kLutBytesMse;
-    static constexpr uint32_t kPartBytes = kTeams * 2 * 2 * 128 * 4;  // [team][norm, gamma][half][row]
+    static constexpr uint32_t kPartBytes = 0;
     static constexpr uint32_t kBarBytes = 512;
     static constexpr uint32_t kFixed = kImages * kTile + kLutBytes + kPartBytes + kBarBytes;
     static constexpr int kStagesFit = (int)((kSmemMax - kFixed) / kTile);
@@ -83,6 +81,15 @@ struct Cfg {
     static constexpr uint32_t kOffBar = kOffPart + kPartBytes;
     static constexpr uint32_t kSmem = kOffBar + kBarBytes;
     static constexpr uint32_t kTmemCols = 512;
+    static constexpr int kTeams = PROD ? 2 : 4;
+    static constexpr int kEpiWarps = 4 * kTeams;
+    static constexpr int kWarpProducer = kEpiWarps;
+    static constexpr int kWarpMma = kEpiWarps + 1;
+    static constexpr int kThreads = kEpiWarps * 32 + 64;
+    // registers: keys 10 warps, three on the busiest SM sub-partition, 3 x 32 x 168
+    // <= 16384 (the bound of 384 threads gives 168); values 18 warps at 96
+    static constexpr int kBound = PROD ? 384 : kThreads;
+    static constexpr uint32_t kBufCols = PROD ? 256 : 128;
     static_assert(kStages >= 1, "shared memory budget");
     static_assert(kSmem <= kSmemMax, "shared memory budget");
 };
@@ -92,12 +99,12 @@ enum : int {
     kBarConst = 0,
     kBarXFull = 1,     // +stage (4)
     kBarXEmpty = 5,    // +stage (4)
-    kBarRotFull = 9,   // +team: rotation accumulators ready
-    kBarRotEmpty = 11, // +team: the team is done with its buffer
-    kBarRhoFull = 13,  // +team: rho written (keys)
-    kBarQjlFull = 15,  // +team: sketch ready (keys)
-    kBarDrain = 17,
-    kNumBars = 18
+    kBarRotFull = 9,    // +team (4): rotation accumulators ready
+    kBarRotEmpty = 13,  // +team (4): the team is done with its buffer
+    kBarRhoFull = 17,   // +team (2): rho written (keys)
+    kBarQjlFull = 19,   // +team (2): sketch ready (keys)
+    kBarDrain = 21,
+    kNumBars = 22
 };
 
 struct TcArgs {
@@ -109,7 +116,8 @@ struct TcArgs {
     const uint8_t* images;  // kImages pre-swizzled 32 KB operands
     const uint8_t* lut;     // bucketize table
     ChunkLayout lay;
-    float lut_kscale;  // sqrt(d) * table scale: u = acc * lut_kscale / ||acc|| is v in cell units
+    float lut_kscale;  // keys: sqrt(d) * table scale, u = acc * lut_kscale / ||acc|| is v in cell units
+    float lut_xscale;  // values: sqrt(d) * table scale / (acc / y), u = acc * lut_xscale / ||x||
     float lut_magic;   // 1.5 * 2^23 + cells / 2
     float rho_scale;   // 32 / table scale: rho = 32 (v - c) from the cell-unit residual
     float n_scale;     // ||x|| = n_scale * ||acc||
@@ -132,23 +140,22 @@ __device__ __forceinline__ float rsqrt_refined(float x) {
 
 // Table reads at a 32-bit shared-memory address.
 __device__ __forceinline__ void lds_v2(uint32_t addr, uint32_t& x, uint32_t& y) {
-    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(x), "=r"(y) : "r"(addr));
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(x), "=r"(y) : "r"(addr));
+}
+// in program order with the other volatile accesses (bounds how far loads are hoisted)
+__device__ __forceinline__ void lds_v4_ordered(uint32_t addr, uint32_t& x, uint32_t& y, uint32_t& z, uint32_t& w) {
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(x), "=r"(y), "=r"(z), "=r"(w) : "r"(addr));
 }
 __device__ __forceinline__ void lds_v4(uint32_t addr, uint32_t& x, uint32_t& y, uint32_t& z, uint32_t& w) {
     asm("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(x), "=r"(y), "=r"(z), "=r"(w) : "r"(addr));
 }
 
-// Named barrier `id` over `count` threads that also ORs a predicate across them:
-// every participant gets the same answer.
-__device__ __forceinline__ bool bar_any(int id, int count, bool p) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)p), "r"(id), "r"(count)
-        : "memory");
-    return r != 0;
+// s0 += lo^2, s1 += hi^2 for the two fp16 halves of w (exact squares, fp32 sums).
+__device__ __forceinline__ void sq_acc2(uint32_t w, float& s0, float& s1) {
+    asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "fma.rn.f32.f16 %0, a, a, %0;\n\tfma.rn.f32.f16 %1, b, b, %1;\n\t}"
+        : "+f"(s0), "+f"(s1)
+        : "r"(w));
 }
 
 __device__ __forceinline__ float2 ld_sum(const uint32_t (&r0)[32], const uint32_t (&r1)[32], int i) {
@@ -157,7 +164,7 @@ __device__ __forceinline__ float2 ld_sum(const uint32_t (&r0)[32], const uint32_
 }
 
 template <int ROT, bool PROD, int W>
-__global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs a) {
+__global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs a) {
     using C = Cfg<ROT, PROD>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
@@ -177,19 +184,22 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
         mbar_init(bar(kBarConst), 1);
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(bar(kBarXFull + s), 1);
-            mbar_init(bar(kBarXEmpty + s), 1);
+            // released by the rotation MMAs and, for values, by the team that reads ||x||
+            mbar_init(bar(kBarXEmpty + s), PROD ? 1 : 1 + kTeamThreads);
         }
-        for (int t = 0; t < kTeams; ++t) {
+        for (int t = 0; t < C::kTeams; ++t) {
             mbar_init(bar(kBarRotFull + t), 1);
             mbar_init(bar(kBarRotEmpty + t), kTeamThreads);
-            mbar_init(bar(kBarRhoFull + t), kTeamThreads);
-            mbar_init(bar(kBarQjlFull + t), 1);
+            if (PROD) {
+                mbar_init(bar(kBarRhoFull + t), kTeamThreads);
+                mbar_init(bar(kBarQjlFull + t), 1);
+            }
         }
         mbar_init(bar(kBarDrain), 1);
         *abort = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == C::kWarpMma) {
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
@@ -198,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
+    if (warp == C::kWarpProducer) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             mbar_arrive_expect_tx(bar(kBarConst), C::kImages * kTile + C::kLutBytes);
@@ -226,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
                 mbar_wait(bar(kBarXFull + k % C::kStages), (uint32_t)(k / C::kStages) & 1u, &never, kWaitNs);
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == C::kWarpMma) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_f16(128, 128);
@@ -238,12 +248,12 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
             // rotation of local tile k into its team's buffer; false when not ready yet
             auto try_rot = [&](int k) -> bool {
                 const int s = k % C::kStages;
-                const int t = k & 1;
-                const uint32_t use = (uint32_t)(k >> 1);
+                const int t = k % C::kTeams;
+                const uint32_t use = (uint32_t)(k / C::kTeams);
                 if (!mbar_try_wait(bar(kBarXFull + s), (uint32_t)(k / C::kStages) & 1u)) return false;
                 if (!mbar_try_wait(bar(kBarRotEmpty + t), (use & 1u) ^ 1u)) return false;
                 tc_fence_after();
-                const uint32_t dA = tmem + kBufCols * (uint32_t)t, dB = dA + kColB;
+                const uint32_t dA = tmem + C::kBufCols * (uint32_t)t, dB = PROD ? dA + kColB : dA;
                 const uint32_t xs = sbase + C::kOffX + s * kTile;
                 uint32_t accA = 0u;
                 if (ROT == 0) {  // the small lo pass first, then K-steps 0-3 of the hi pass
@@ -259,7 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
                     accA = 1u;
                 }
 #pragma unroll
-                for (int st = 4; st < 8; ++st) umma_ss(dB, kdesc(xs, st), kdesc(img, st), idesc, st > 4 ? 1u : 0u);
+                for (int st = 4; st < 8; ++st)
+                    umma_ss(dB, kdesc(xs, st), kdesc(img, st), idesc, (PROD && st == 4) ? 0u : 1u);
                 umma_commit(bar(kBarXEmpty + s));
                 umma_commit(bar(kBarRotFull + t));
                 return true;
@@ -269,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
                 const int t = k & 1;
                 if (!mbar_try_wait(bar(kBarRhoFull + t), (uint32_t)(k >> 1) & 1u)) return false;
                 tc_fence_after();
-                const uint32_t buf = tmem + kBufCols * (uint32_t)t;
+                const uint32_t buf = tmem + C::kBufCols * (uint32_t)t;
                 const uint32_t d = buf + kColB;
                 const uint32_t m0 = img + C::kRotImages * kTile;
                 // rho of K-step st: columns 16 st (hi pairs) and 16 st + 8 (lo pairs)
@@ -293,17 +304,17 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
             // Rotations go in tile order (the stage ring); each team's sketch goes
             // as soon as its rho is in.  Polls with a bound on time without progress.
             int next_rot = 0;
-            int qjl_next[kTeams] = {0, 1};
+            int qjl_next[2] = {0, 1};
             uint64_t t_last = globaltimer_ns();
             uint32_t spins = 0;
             while (ok) {
                 bool progress = false;
                 if (PROD) {
 #pragma unroll
-                    for (int t = 0; t < kTeams; ++t) {
+                    for (int t = 0; t < 2; ++t) {
                         const int k = qjl_next[t];
                         if (k < next_rot && try_qjl(k)) {
-                            qjl_next[t] = k + kTeams;
+                            qjl_next[t] = k + 2;
                             progress = true;
                         }
                     }
@@ -330,16 +341,11 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        const int ew = warp - 2;
-        const int quarter = warp & 3;     // TMEM lanes this warp may access
-        const int team = ew >> 3;         // tiles k with k % 2 == team, buffer team
-        const int hh = (ew >> 2) & 1;     // column half [64 hh, 64 hh + 64)
+        const int quarter = warp & 3;  // TMEM lanes this warp may access
+        const int team = warp >> 2;    // tiles k with k % kTeams == team, buffer team
         const int row = quarter * 32 + lane;
-        const int pbar = 1 + team * 4 + quarter;  // the two warps that share these rows
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        const uint32_t buf = tmem + lane_addr + kBufCols * (uint32_t)team;
-        float* pn = reinterpret_cast<float*>(smem + C::kOffPart) + team * (2 * 2 * 128);
-        float* pg = pn + 2 * 128;
+        const uint32_t buf = tmem + lane_addr + C::kBufCols * (uint32_t)team;
         // table entry of u: bits(u + magic) * 128 + lut_off, in this lane's replica
         // (bits(u + magic) = bits(1.5 * 2^23) + cells / 2 + round(u), see tc_params.h)
         const uint32_t lut_off = sbase + C::kOffLut +
@@ -348,9 +354,8 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
                                  __float_as_uint(12582912.0f) * 128u;
         const float2 magic2 = make_float2(a.lut_magic, a.lut_magic);
         const float2 rho_k = make_float2(a.rho_scale, a.rho_scale);
-        constexpr int kPer = 32 / W;               // codes per 32-bit word
-        constexpr int kWords = kHalfCols / kPer;   // words of this thread's 64 columns
-        constexpr int kHW = kWords / 2;            // words of one 32-column half
+        constexpr int kPer = 32 / W;       // codes per 32-bit word
+        constexpr int kQW = 32 / kPer;     // words of 32 columns' codes
         bool ok = mbar_wait(bar(kBarConst), 0, abort, kWaitNs);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) set_abort(abort, a.err);
@@ -366,103 +371,126 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
             const int vi = tile * 128 + row;
             if (vi >= a.N || slot < 0) return nullptr;
             if (slot >= a.num_blocks * kPage) {
-                if (hh == 0) atomicOr(a.err, TQ_DEVERR_SLOT);
+                atomicOr(a.err, TQ_DEVERR_SLOT);
                 return nullptr;
             }
             const int head = vi % a.H;
             return a.cache + ((size_t)(slot / kPage) * a.H + head) * (size_t)a.lay.bytes + (size_t)(slot % kPage);
         };
-        auto store = [&](uint8_t* d, const uint32_t (&words)[kWords], float norm, float gamma, uint2 sg) {
+        // codes of columns [32 q, 32 q + 32) of the row
+        auto store_codes = [&](uint8_t* d, int q, const uint32_t (&w)[kQW]) {
+            if (!d) return;
+            const int pr = (int)((uintptr_t)d & 15u);
+            uint8_t* cp = d - pr + pr * a.lay.code_row + q * (4 * kQW);
+            if (kQW == 4) *reinterpret_cast<uint4*>(cp) = make_uint4(w[0], w[1 % kQW], w[2 % kQW], w[3 % kQW]);
+            else if (kQW == 2) *reinterpret_cast<uint2*>(cp) = make_uint2(w[0], w[1 % kQW]);
+            else *reinterpret_cast<uint32_t*>(cp) = w[0];
+        };
+        auto store_tail = [&](uint8_t* d, float norm, float gamma, const uint32_t (&sg)[4]) {
             if (!d) return;
             const int pr = (int)((uintptr_t)d & 15u);
             uint8_t* chunk = d - pr;
-            uint8_t* cp = chunk + pr * a.lay.code_row + hh * (a.lay.code_row / 2);
-            if (kWords == 8) {
-                reinterpret_cast<uint4*>(cp)[0] = make_uint4(words[0], words[1], words[2], words[3]);
-                reinterpret_cast<uint4*>(cp)[1] = make_uint4(words[4 % kWords], words[5 % kWords], words[6 % kWords], words[7 % kWords]);
-            } else if (kWords == 4) {
-                *reinterpret_cast<uint4*>(cp) = make_uint4(words[0], words[1 % kWords], words[2 % kWords], words[3 % kWords]);
-            } else {
-                *reinterpret_cast<uint2*>(cp) = make_uint2(words[0], words[1 % kWords]);
-            }
-            if (PROD) *reinterpret_cast<uint2*>(chunk + a.lay.signs_off + pr * (kDim / 8) + hh * 8) = sg;
-            if (hh == 0) {
-                reinterpret_cast<float*>(chunk + a.lay.norm_off)[pr] = norm;
-                if (PROD) reinterpret_cast<float*>(chunk + a.lay.gamma_off)[pr] = gamma;
-            }
-        };
-        // 32 sketch columns as sign bits (bit j set when column j >= 0)
-        auto signs32 = [&](uint32_t col) -> uint32_t {
-            uint32_t q[32];
-            tmem_ld32(col, q);
-            tmem_ld_wait();
-            uint32_t neg = 0u;  // bit j = sign bit of column j
-#pragma unroll
-            for (int j = 31; j >= 0; --j) neg = __funnelshift_l(q[j], neg, 1);
-            return ~neg;
+            if (PROD) *reinterpret_cast<uint4*>(chunk + a.lay.signs_off + pr * (kDim / 8)) = make_uint4(sg[0], sg[1], sg[2], sg[3]);
+            reinterpret_cast<float*>(chunk + a.lay.norm_off)[pr] = norm;
+            if (PROD) reinterpret_cast<float*>(chunk + a.lay.gamma_off)[pr] = gamma;
         };
 
         int slot_next = team < my_tiles ? slot_of((int)blockIdx.x + team * (int)gridDim.x) : -1;
-        for (int k = team; k < my_tiles; k += kTeams) {
+        for (int k = team; k < my_tiles; k += C::kTeams) {
             const int tile = (int)blockIdx.x + k * (int)gridDim.x;
-            const uint32_t use = (uint32_t)(k >> 1);
+            const uint32_t use = (uint32_t)(k / C::kTeams);
             const int slot = slot_next;
-            if (k + kTeams < my_tiles) slot_next = slot_of(tile + kTeams * (int)gridDim.x);
+            if (k + C::kTeams < my_tiles) slot_next = slot_of(tile + C::kTeams * (int)gridDim.x);
             uint8_t* dst = dest(tile, slot);
-            bool good = !*abort && mbar_wait(bar(kBarRotFull + team), use & 1u, abort, kWaitNs);
-            good = __all_sync(0xffffffffu, good);
-            // ---- ||acc||^2 over this thread's 64 columns; the upper 32 stay in registers
-            float2 acc[16];
-            float2 q2[4];
+            float nsq;
+            if (!PROD) {
+                // ---- ||x||^2 of the row from the swizzled fp16 tile (logical 16-byte
+                // chunk c of a 128-byte row sits at chunk c ^ (row % 8))
+                const int stg = k % C::kStages;
+                bool good = !*abort && mbar_wait(bar(kBarXFull + stg), (uint32_t)(k / C::kStages) & 1u, abort, kWaitNs);
+                good = __all_sync(0xffffffffu, good);
+                if (!good) {
+                    set_abort(abort, a.err);
+                    break;
+                }
+                float sq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) q2[i] = make_float2(0.f, 0.f);
-            if (good) {
+                for (int kb = 0; kb < 2; ++kb) {
+                    const uint32_t xr = sbase + C::kOffX + stg * kTile + kb * kHalf + row * 128;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t w0, w1, w2, w3;
+                        lds_v4_ordered(xr + (uint32_t)((c ^ (row & 7)) << 4), w0, w1, w2, w3);
+                        sq_acc2(w0, sq[0], sq[1]);
+                        sq_acc2(w1, sq[2], sq[3]);
+                        sq_acc2(w2, sq[0], sq[1]);
+                        sq_acc2(w3, sq[2], sq[3]);
+                    }
+                }
+                mbar_arrive(bar(kBarXEmpty + stg));
+                nsq = (sq[0] + sq[1]) + (sq[2] + sq[3]);
+                good = mbar_wait(bar(kBarRotFull + team), use & 1u, abort, kWaitNs);
+                good = __all_sync(0xffffffffu, good);
+                if (!good) {
+                    set_abort(abort, a.err);
+                    break;
+                }
                 tc_fence_after();
+            } else {
+                bool good = !*abort && mbar_wait(bar(kBarRotFull + team), use & 1u, abort, kWaitNs);
+                good = __all_sync(0xffffffffu, good);
+                if (!good) {
+                    set_abort(abort, a.err);
+                    break;
+                }
+                tc_fence_after();
+                // ---- ||acc||^2 of the row, acc = A + B
+                float2 q2[4];
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
+                for (int i = 0; i < 4; ++i) q2[i] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
                     uint32_t r0[32], r1[32];
-                    tmem_ld32(buf + kHalfCols * hh + 32 * hf, r0);
-                    tmem_ld32(buf + kColB + kHalfCols * hh + 32 * hf, r1);
+                    tmem_ld32(buf + 32 * c, r0);
+                    tmem_ld32(buf + kColB + 32 * c, r1);
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        acc[i] = ld_sum(r0, r1, i);
-                        q2[i & 3] = __ffma2_rn(acc[i], acc[i], q2[i & 3]);
+                        const float2 v = ld_sum(r0, r1, i);
+                        q2[i & 3] = __ffma2_rn(v, v, q2[i & 3]);
                     }
                 }
-            } else {
-                set_abort(abort, a.err);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) acc[i] = make_float2(0.f, 0.f);
+                nsq = ((q2[0].x + q2[0].y) + (q2[1].x + q2[1].y)) + ((q2[2].x + q2[2].y) + (q2[3].x + q2[3].y));
             }
-            pn[hh * 128 + row] = ((q2[0].x + q2[0].y) + (q2[1].x + q2[1].y)) + ((q2[2].x + q2[2].y) + (q2[3].x + q2[3].y));
-            if (bar_any(pbar, 64, !good || *abort)) break;
-            const float nsq = pn[row] + pn[128 + row];
             // rows with inf / nan inputs are quantized as zero vectors (their norm stays non-finite)
             const bool finite = nsq <= 3.4e38f;
             const bool live = finite && nsq > 0.f;
-            const float rn = live ? rsqrt_refined(nsq) : 0.f;  // 1 / ||acc||
+            const float rn = live ? rsqrt_refined(nsq) : 0.f;  // 1 / ||acc|| (keys), 1 / ||x|| (values)
             const float nacc = nsq * rn;
-            const float2 s2 = make_float2(a.lut_kscale * rn, a.lut_kscale * rn);
+            const float sc = (PROD ? a.lut_kscale : a.lut_xscale) * rn;
+            const float2 s2 = make_float2(sc, sc);
             const bool any_bad = __any_sync(0xffffffffu, !finite);
-            const float norm = live ? nacc * a.n_scale : (finite ? 0.f : sqrtf(nsq));
+            const float norm = live ? (PROD ? nacc * a.n_scale : nacc) : (finite ? 0.f : sqrtf(nsq));
 
-            // ---- bucketize + pack (+ residual, rho for keys) in groups of 16 columns,
-            // the upper half (still in registers for values) first
-            uint32_t words[kWords];
-#pragma unroll
-            for (int i = 0; i < kWords; ++i) words[i] = 0u;
+            // ---- bucketize + pack (+ residual, rho for keys): 32 columns (two K-steps)
+            // per iteration, their codes stored at once
             float2 gs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+              uint32_t words[kQW];
 #pragma unroll
-            for (int grp = 0; grp < 4; ++grp) {
-                const int hf = grp < 2 ? 1 : 0;
-                const int g = grp & 1;
-                const uint32_t col = buf + kHalfCols * hh + 32 * hf + 16 * g;  // A columns of the group
+              for (int i = 0; i < kQW; ++i) words[i] = 0u;
+#pragma unroll
+              for (int sub = 0; sub < 2; ++sub) {
+                const uint32_t col = buf + 32 * q + 16 * sub;
                 float2 av[8];
-                if (hf == 1 && !PROD) {  // keys reload it too: registers are short there
+                if (!PROD) {  // one accumulator
+                    uint32_t r0[16];
+                    tmem_ld16(col, r0);
+                    tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) av[i] = acc[8 * g + i];
-                } else {  // reload from tensor memory
+                    for (int i = 0; i < 8; ++i) av[i] = make_float2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
+                } else {
                     uint32_t r0[16], r1[16];
                     tmem_ld16(col, r0);
                     tmem_ld16(col + kColB, r1);
@@ -510,45 +538,55 @@ __global__ void __launch_bounds__(kThreads, 1) compress_tc_kernel(const __grid_c
                         code0 = base0 + (__uint_as_float(b0) < u.x ? 1u : 0u);
                         code1 = base1 + (__uint_as_float(b1) < u.y ? 1u : 0u);
                     }
-                    const int j = 32 * hf + 16 * g + 2 * i;  // column within this thread's 64
+                    const int j = 16 * sub + 2 * i;  // column within the 32
                     words[j / kPer] += code0 << (W * (j % kPer));
                     words[(j + 1) / kPer] += code1 << (W * ((j + 1) % kPer));
                 }
-                if (PROD && good) {  // over the group's A columns, already read
+                if (PROD) {  // over the K-step's A columns, already read
                     tmem_st8(col, rho_hi);
                     tmem_st8(col + 8, rho_lo);
                 }
+              }
+              store_codes(dst, q, words);
             }
             if (!PROD) {
                 tc_fence_before();
                 mbar_arrive(bar(kBarRotEmpty + team));
-                store(dst, words, norm, 0.f, make_uint2(0u, 0u));
+                const uint32_t none[4] = {0u, 0u, 0u, 0u};
+                store_tail(dst, norm, 0.f, none);
                 continue;
             }
-            // ---- keys: release rho, exchange the gamma partials, then read the sketch
+            // ---- keys: release rho; gamma; then the sketch as sign bits
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(bar(kBarRhoFull + team));
-            pg[hh * 128 + row] = (gs[0].x + gs[0].y) + (gs[1].x + gs[1].y);
-            if (bar_any(pbar, 64, *abort)) break;
-            const float gsq = pg[row] + pg[128 + row];
+            const float gsq = (gs[0].x + gs[0].y) + (gs[1].x + gs[1].y);
             const float gamma = (live && gsq > 0.f) ? gsq * rsqrt_refined(gsq) * nacc * a.gamma_scale : 0.f;
             bool sk = mbar_wait(bar(kBarQjlFull + team), use & 1u, abort, kWaitNs);
             sk = __all_sync(0xffffffffu, sk);
             if (!sk) {
                 set_abort(abort, a.err);
-                continue;  // the next barrier sees the abort
+                break;
             }
             tc_fence_after();
-            uint2 sg = make_uint2(signs32(buf + kColB + kHalfCols * hh), signs32(buf + kColB + kHalfCols * hh + 32));
-            if (!live) sg = make_uint2(0xffffffffu, 0xffffffffu);
+            uint32_t sg[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t q[32];
+                tmem_ld32(buf + kColB + 32 * c, q);
+                tmem_ld_wait();
+                uint32_t neg = 0u;  // bit j = sign bit of column 32 c + j
+#pragma unroll
+                for (int j = 31; j >= 0; --j) neg = __funnelshift_l(q[j], neg, 1);
+                sg[c] = live ? ~neg : 0xffffffffu;
+            }
             tc_fence_before();
             mbar_arrive(bar(kBarRotEmpty + team));
-            store(dst, words, norm, gamma, sg);
+            store_tail(dst, norm, gamma, sg);
         }
     }
     __syncthreads();
-    if (warp == 1) {
+    if (warp == C::kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
@@ -560,7 +598,7 @@ cudaError_t launch_tc(const CUtensorMap& tmap, const TcArgs& a, int grid, cudaSt
     auto k = compress_tc_kernel<ROT, PROD, W>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
     if (e != cudaSuccess) return e;
-    k<<<grid, kThreads, C::kSmem, stream>>>(tmap, a);
+    k<<<grid, C::kThreads, C::kSmem, stream>>>(tmap, a);
     return cudaGetLastError();
 }
 
@@ -586,6 +624,8 @@ cudaError_t launch_compress_tc(const tq_ctx* ctx, int kind, const uint16_t* x, i
     a.lut = value ? tabs.lut_value : tabs.lut_key;
     const LutParams& lp = value ? tabs.lp_value : tabs.lp_key;
     a.lut_kscale = (float)(std::sqrt((double)kDim) * (double)lp.scale);
+    // values: acc = 16 y (Haar) or sqrt(d) y (Hadamard)
+    a.lut_xscale = (float)(std::sqrt((double)kDim) * (double)lp.scale / (rot == TQ_ROT_HAAR ? 16.0 : std::sqrt((double)kDim)));
     a.lut_magic = lp.magic;
     a.rho_scale = (float)(32.0 / (double)lp.scale);
     const double n_scale = rot == TQ_ROT_HAAR ? 1.0 / 16.0 : 1.0 / std::sqrt(128.0);
