@@ -427,6 +427,7 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                         sq_acc2(w3, sq[2], sq[3]);
                     }
                 }
+                fence_proxy_async_shared();  // these reads before the next TMA write of the stage
                 mbar_arrive(bar(kBarXEmpty + stg));
                 nsq = (sq[0] + sq[1]) + (sq[2] + sq[3]);
                 good = mbar_wait(bar(kBarRotFull + team), use & 1u, abort, kWaitNs);

@@ -53,9 +53,9 @@ struct DecodeArgs {
     const int32_t* seq_lens;
     int B, Hq, Hkv, G, max_seq_len;
     float scale_log2;  // softmax scale * log2(e)
-    float* partial;    // [B*Hkv][splits][G][130]
-    int splits, pages_per_item;
-    int merge_heads, merge_parts;
+    float* partial;    // [slots][G][130]: m, l, acc (rotated domain)
+    int* prefix;       // [B + 1] pages of the sequences before b (prep writes it)
+    int split_grid;    // CTAs of the split kernel
     const float* RT;       // row-major R^T (fp32)
     const uint16_t* RTh;   // fp16 R^T hi / lo, S (row-major)
     const uint16_t* RTl;
@@ -73,6 +73,12 @@ __device__ __forceinline__ bool seq_len_ok(const DecodeArgs& a, int L) {
 }
 
 // ------------------------------------------------------------------ helpers
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before its predecessor ends; it reads nothing that the
+// predecessor (or anything before it) writes until griddep_wait() returns.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -84,8 +90,8 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 
 // ------------------------------------------------------------------ prep
 // [q' | s] = q [R | S^T] for 16 query heads per CTA, on mma.sync (fp16 inputs, fp32
-// accumulation; R^T enters as fp16 hi + lo, S is exact).  Warp w computes output
-// columns 32w .. 32w+31 of the 256 (q' then s).
+// accumulation; R^T enters as fp16 hi + lo, S is exact).  CTA (x, y), warp w
+// computes output columns 8 (8 y + w) .. +7 of the 256 (q' then s).
 constexpr int kPrepThreads = 256;
 __global__ void __launch_bounds__(kPrepThreads) decode_prep_kernel(DecodeArgs a) {
     const int NQ = a.B * a.Hq;
@@ -94,6 +100,34 @@ __global__ void __launch_bounds__(kPrepThreads) decode_prep_kernel(DecodeArgs a)
     const bool r0 = h0 + g < NQ, r1 = h0 + g + 8 < NQ;
     const uint32_t* q0 = reinterpret_cast<const uint32_t*>(a.q + (size_t)(r0 ? h0 + g : 0) * kDim);
     const uint32_t* q1 = reinterpret_cast<const uint32_t*>(a.q + (size_t)(r1 ? h0 + g + 8 : 0) * kDim);
+    if (blockIdx.x == 0 && blockIdx.y == 0) {
+        // pages per sequence (invalid lengths count as empty and raise the error
+        // word) and their exclusive prefix sum, in chunks of 256 sequences
+        __shared__ int sc[kPrepThreads];
+        int carry = 0;
+        for (int b0 = 0; b0 < a.B; b0 += kPrepThreads) {
+            const int b = b0 + (int)threadIdx.x;
+            int n = 0;
+            if (b < a.B) {
+                const int L = a.seq_lens[b];
+                if (seq_len_ok(a, L)) n = (L + kPage - 1) / kPage;
+                else atomicOr(a.err, TQ_DEVERR_SEQLEN);
+            }
+            sc[threadIdx.x] = n;
+            __syncthreads();
+            for (int off = 1; off < kPrepThreads; off <<= 1) {  // inclusive scan
+                const int v = threadIdx.x >= off ? sc[threadIdx.x - off] : 0;
+                __syncthreads();
+                sc[threadIdx.x] += v;
+                __syncthreads();
+            }
+            if (b < a.B) a.prefix[b] = carry + sc[threadIdx.x] - n;
+            carry += sc[kPrepThreads - 1];
+            __syncthreads();
+        }
+        if (threadIdx.x == 0) a.prefix[a.B] = carry;
+    }
+    griddep_launch_dependents();  // the split kernel may start its prologue
     uint32_t A[8][4];
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
@@ -102,9 +136,8 @@ __global__ void __launch_bounds__(kPrepThreads) decode_prep_kernel(DecodeArgs a)
         A[ks][2] = r0 ? q0[8 * ks + c + 4] : 0u;
         A[ks][3] = r1 ? q1[8 * ks + c + 4] : 0u;
     }
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        const int nt = warp * 4 + t;  // 0..15 -> q', 16..31 -> s
+    {
+        const int nt = blockIdx.y * 8 + warp;  // 0..15 -> q', 16..31 -> s
         const bool isq = nt < 16;
         const int n = (nt & 15) * 8 + g;
         const uint32_t* bh = reinterpret_cast<const uint32_t*>((isq ? a.RTh : a.Sh) + (size_t)n * kDim);
@@ -482,24 +515,42 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
         sm100::fence_mbar_init();
     }
     __syncthreads();
+    griddep_wait();  // q', s and the page prefix sums from the prep kernel; the caller's inputs
+    griddep_launch_dependents();  // the merge kernel may stage its rotation meanwhile
     float* wm = reinterpret_cast<float*>(smem + L::kOffM);      // [warp][2][16]: m then l
     float* wacc = reinterpret_cast<float*>(smem + L::kOffAcc);  // [warp][16 heads][128]
     const volatile int never = 0;
     uint32_t issued = 0, consumed = 0;  // pages this warp has requested / processed (all items)
     bool dead = false;                  // a page copy never arrived: this warp stops working
 
-    const int items = a.B * a.Hkv * a.splits;
-    for (int item = blockIdx.x; item < items; item += gridDim.x) {
-        const int unit = item / a.splits, split = item - unit * a.splits;
-        const int b = unit / a.Hkv, hk = unit - b * a.Hkv;
-        int Ls = a.seq_lens[b];
-        if (!seq_len_ok(a, Ls)) {
-            if (tid == 0 && split == 0 && hk == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
-            Ls = 0;
+    // this CTA's range [pos, end) of the pages of all units in order (unit
+    // u = b Hkv + h holds the pages of sequence b), cut into pieces by unit
+    const long total = (long)a.Hkv * a.prefix[a.B];
+    long pos = total * (long)blockIdx.x / gridDim.x;
+    const long end = total * (long)(blockIdx.x + 1) / gridDim.x;
+    int b = 0;
+    if (pos < end) {  // the last sequence b with Hkv * prefix[b] <= pos
+        int lo = 0, hi = a.B - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if ((long)a.Hkv * a.prefix[mid] <= pos) lo = mid;
+            else hi = mid - 1;
         }
-        const int npages = (Ls + kPage - 1) / kPage;
-        const int p0 = split * a.pages_per_item;
-        const int p1 = min(p0 + a.pages_per_item, npages);
+        b = lo;
+    }
+    while (pos < end && b < a.B) {
+        const int np = a.prefix[b + 1] - a.prefix[b];  // pages of sequence b (the same for each kv head)
+        const long off = pos - (long)a.Hkv * a.prefix[b];
+        if (np == 0 || off >= (long)a.Hkv * np) {  // past sequence b
+            ++b;
+            continue;
+        }
+        const int hk = (int)(off / np);
+        const int p0 = (int)(off - (long)hk * np);
+        const int p1 = (int)min((long)np, p0 + (end - pos));
+        pos += p1 - p0;
+        const int unit = b * a.Hkv + hk;
+        const int Ls = a.seq_lens[b];  // valid: np > 0
 
         // query fragments (B operand): head nt*8 + g, coords 32c .. 32c+31; K-step ks
         // uses coords 32c + 4ks + {0,1} (b0) and {2,3} (b1)
@@ -588,6 +639,7 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
                 load_page<KM, VM, PROD>(r, st, st + kb, a, g, c);
                 process_page<KM, VM, PROD, NT>(r, min(kPage, Ls - page * kPage), x, bq, bs, m, l, acc);
             }
+            sm100::fence_proxy_async_shared();  // this lane's reads before the refill's bulk copy
             __syncwarp();  // every lane is done with the stage before it is refilled
             if (j + kStagesD < nj) issue(j + kStagesD);
         }
@@ -629,7 +681,7 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
                 Lsum = fmaf(wt, wm[(w * 2 + 1) * kMaxG + h], Lsum);
                 A = fmaf(wt, wacc[(w * kMaxG + h) * kDim + tid], A);
             }
-            float* part = a.partial + (((size_t)unit * a.splits + split) * a.G + h) * kPartStride;
+            float* part = a.partial + (((size_t)unit + blockIdx.x) * a.G + h) * kPartStride;
             if (tid == 0) {
                 part[0] = M;
                 part[1] = Lsum;
@@ -641,68 +693,67 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
 }
 
 // ------------------------------------------------------------------ merge
-// grid (B*Hkv, ceil(G / merge_heads)); threads = 128 * merge_heads * merge_parts.
-// Thread (part, head, coord) combines the splits s = part, part + parts, ... of one
-// head; R^T is staged in shared memory for the un-rotation.
-__global__ void decode_merge_kernel(DecodeArgs a) {
-    extern __shared__ __align__(16) float sm[];  // RT [128*128] | [parts][heads][3][128] | orot [heads][128]
-    const int unit = blockIdx.x;
-    const int H = a.merge_heads, P = a.merge_parts;
-    const int i = threadIdx.x % kDim, hl = (threadIdx.x / kDim) % H, part = threadIdx.x / (kDim * H);
-    const int h = blockIdx.y * H + hl;
-    const bool active = h < a.G;
+// Persistent: CTA i takes units i, i + grid, ...; 128 threads per head, kMergeHeads
+// heads at a time.  R^T is staged once per CTA (while the split kernel runs).
+// Unit u's pieces sit in slots u + c for the split CTAs c whose page range meets
+// it: c(p) = ((p + 1) grid - 1) / total is the CTA of page p.
+constexpr int kMergeHeads = 4;
+constexpr int kMergeThreads = kDim * kMergeHeads;
+__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs a) {
+    extern __shared__ __align__(16) float sm[];  // RT [128*128] | orot [heads][128]
+    const int i = threadIdx.x % kDim, hl = threadIdx.x / kDim;
     float* rts = sm;
+    float* orot = sm + kDim * kDim;
     {
         const float4* src = reinterpret_cast<const float4*>(a.RT);
         float4* dst = reinterpret_cast<float4*>(rts);
         for (int k = threadIdx.x; k < kDim * kDim / 4; k += blockDim.x) dst[k] = src[k];
     }
-    float M = -INFINITY, Lsum = 0.f, A = 0.f;
-    if (active) {
-        const float* base = a.partial + ((size_t)unit * a.splits * a.G + h) * kPartStride;
-        const size_t stride = (size_t)a.G * kPartStride;
-        for (int s = part; s < a.splits; s += P) M = fmaxf(M, base[s * stride]);
-        if (M != -INFINITY) {
-#pragma unroll 4
-            for (int s = part; s < a.splits; s += P) {
-                const float ms = base[s * stride];
-                const float wt = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
-                Lsum = fmaf(wt, base[s * stride + 1], Lsum);
-                A = fmaf(wt, base[s * stride + 2 + i], A);
+    griddep_wait();  // the split partials
+    const long total = (long)a.Hkv * a.prefix[a.B];
+    const long grid = a.split_grid;
+    const int units = a.B * a.Hkv;
+    for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
+        const int b = unit / a.Hkv, hk = unit - b * a.Hkv;
+        const int np = a.prefix[b + 1] - a.prefix[b];
+        int c_lo = 0, c_hi = -1;
+        if (np > 0) {
+            const long first = (long)a.Hkv * a.prefix[b] + (long)hk * np, last = first + np - 1;
+            c_lo = (int)(((first + 1) * grid - 1) / total);
+            c_hi = (int)(((last + 1) * grid - 1) / total);
+        }
+        for (int h0 = 0; h0 < a.G; h0 += kMergeHeads) {
+            const int h = h0 + hl;
+            const bool active = h < a.G;
+            float M = -INFINITY, Lsum = 0.f, A = 0.f;
+            if (active) {
+                for (int c = c_lo; c <= c_hi; ++c)
+                    M = fmaxf(M, a.partial[(((size_t)unit + c) * a.G + h) * kPartStride]);
+                if (M != -INFINITY)
+                    for (int c = c_lo; c <= c_hi; ++c) {
+                        const float* pp = a.partial + (((size_t)unit + c) * a.G + h) * kPartStride;
+                        const float ms = pp[0];
+                        const float wt = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+                        Lsum = fmaf(wt, pp[1], Lsum);
+                        A = fmaf(wt, pp[2 + i], A);
+                    }
+            }
+            __syncthreads();  // the previous heads' un-rotation is done with orot
+            orot[hl * kDim + i] = Lsum > 0.f ? A / Lsum : 0.f;
+            __syncthreads();
+            if (active) {
+                float y = 0.f;
+                const float* orh = orot + hl * kDim;
+#pragma unroll 8
+                for (int j = 0; j < kDim; ++j) y = fmaf(rts[j * kDim + i], orh[j], y);  // o_i = sum_j R[i][j] orot_j
+                const size_t oi = ((size_t)unit * a.G + h) * kDim + i;
+                if (a.out_fp32)
+                    static_cast<float*>(a.out)[oi] = y;
+                else
+                    static_cast<__half*>(a.out)[oi] = __float2half_rn(y);
             }
         }
     }
-    float* red = sm + kDim * kDim;
-    float* slot = red + ((part * H + hl) * 3) * kDim;
-    slot[i] = M;
-    slot[kDim + i] = Lsum;
-    slot[2 * kDim + i] = A;
-    __syncthreads();
-    float* orot = red + (size_t)P * H * 3 * kDim;
-    if (part == 0) {
-        float MM = -INFINITY;
-        for (int q = 0; q < P; ++q) MM = fmaxf(MM, red[((q * H + hl) * 3) * kDim + i]);
-        float LL = 0.f, AA = 0.f;
-        if (MM != -INFINITY)
-            for (int q = 0; q < P; ++q) {
-                const float* sq = red + ((q * H + hl) * 3) * kDim;
-                const float wt = (sq[i] == -INFINITY) ? 0.f : exp2f(sq[i] - MM);
-                LL = fmaf(wt, sq[kDim + i], LL);
-                AA = fmaf(wt, sq[2 * kDim + i], AA);
-            }
-        orot[hl * kDim + i] = LL > 0.f ? AA / LL : 0.f;
-    }
-    __syncthreads();
-    if (part != 0 || !active) return;
-    float y = 0.f;
-    const float* orh = orot + hl * kDim;
-#pragma unroll 8
-    for (int j = 0; j < kDim; ++j) y = fmaf(rts[j * kDim + i], orh[j], y);  // o_i = sum_j R[i][j] orot_j
-    const size_t oi = ((size_t)unit * a.G + h) * kDim + i;
-    if (a.out_fp32)
-        static_cast<float*>(a.out)[oi] = y;
-    else
-        static_cast<__half*>(a.out)[oi] = __float2half_rn(y);
 }
 
 int kmode_of(const tq_ctx* ctx) {
@@ -723,14 +774,30 @@ int ctas_per_sm_for(size_t smem) {
     return n < 1 ? 1 : n;
 }
 
+
+// Launch with programmatic stream serialization (see griddep_wait).
+template <typename K>
+cudaError_t launch_dependent(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, const DecodeArgs& a) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
 template <int KM, int VM, bool PROD, int NT>
 cudaError_t launch_split(const DecodeArgs& a, int grid, cudaStream_t stream) {
     using L = SmemLayout<KM, VM, PROD>;
     auto k = decode_split_kernel<KM, VM, PROD, NT>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes);
     if (e != cudaSuccess) return e;
-    k<<<grid, kThreads, L::kBytes, stream>>>(a);
-    return cudaGetLastError();
+    return launch_dependent(k, dim3(grid), dim3(kThreads), L::kBytes, stream, a);
 }
 
 }  // namespace
@@ -740,21 +807,23 @@ DecodePlan plan_decode(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_seq_le
     p.max_pages = (max_seq_len + kPage - 1) / kPage;
     const long resident = (long)ctx->sm_count * ctas_per_sm_for(split_smem(kmode_of(ctx)));
     const long units = (long)B * Hkv;
-    // about two items per resident CTA, and at least 16 pages (4 per warp) per item
-    long splits = (2 * resident + units - 1) / units;
-    const long max_splits = (p.max_pages + 4 * kWarps - 1) / (4 * kWarps);
-    if (splits > max_splits) splits = max_splits;
-    if (splits < 1) splits = 1;
-    p.splits = (int)splits;
-    p.pages_per_split = p.max_pages > 0 ? (p.max_pages + p.splits - 1) / p.splits : 0;
+    // every resident CTA, but at least 16 pages (4 per warp) per CTA for small batches
+    long grid = (units * p.max_pages + 4 * kWarps - 1) / (4 * kWarps);
+    if (grid > resident) grid = resident;
+    if (grid < 1) grid = 1;
+    p.grid = (int)grid;
+    p.slots = (int)(units + grid);
+    const int G = Hkv > 0 ? Hq / Hkv : 0;
     size_t off = 0;
     p.qprep_off = off;
     off += (size_t)B * Hq * 2 * kDim * sizeof(__half);
     off = (off + 255) & ~size_t(255);
     p.partial_off = off;
-    off += (size_t)B * Hq * p.splits * kPartStride * sizeof(float);
+    off += (size_t)p.slots * G * kPartStride * sizeof(float);
     off = (off + 255) & ~size_t(255);
-    p.ticket_off = off;
+    p.prefix_off = off;
+    off += (size_t)(B + 1) * sizeof(int);
+    off = (off + 255) & ~size_t(255);
     p.bytes = off;
     return p;
 }
@@ -782,8 +851,8 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
     a.qscale = a.scale_log2 / sqrtf((float)kDim);
     a.sscale = a.scale_log2 * 1.2533141373155003f / (float)kDim;
     a.partial = reinterpret_cast<float*>(ws + plan.partial_off);
-    a.splits = plan.splits;
-    a.pages_per_item = plan.pages_per_split;
+    a.prefix = reinterpret_cast<int*>(ws + plan.prefix_off);
+    a.split_grid = plan.grid;
     a.RT = ctx->dev.RT;
     a.RTh = ctx->dev.RTh;
     a.RTl = ctx->dev.RTl;
@@ -795,24 +864,13 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
     a.out = out;
     a.out_fp32 = out_fp32;
     a.err = ctx->dev_error;
-    // merge: all heads of a unit in one CTA when the splits are few; one head per
-    // CTA with the splits spread over 8 parts otherwise
-    if (plan.splits <= 16) {
-        a.merge_heads = a.G < 8 ? a.G : 8;
-        a.merge_parts = 1;
-    } else {
-        a.merge_heads = 1;
-        a.merge_parts = 8;
-    }
 
-    decode_prep_kernel<<<(B * Hq + 15) / 16, kPrepThreads, 0, stream>>>(a);
+    decode_prep_kernel<<<dim3((B * Hq + 15) / 16, 4), kPrepThreads, 0, stream>>>(a);
     const int KM = kmode_of(ctx);
     const int VM = ctx->cb_value.width == 4 ? kVByte4 : kVByte2;
     const bool prod = ctx->lay_key.prod;
     const int NT = a.G <= 8 ? 1 : 2;
-    const long resident = (long)ctx->sm_count * ctas_per_sm_for(split_smem(KM));
-    const long items = (long)B * Hkv * plan.splits;
-    const int grid = (int)(items < resident ? items : resident);
+    const int grid = plan.grid;
     cudaError_t e = cudaErrorInvalidValue;
 #define TQ_DEC_CASE(K_, V_, P_, N_) \
     if (KM == K_ && VM == V_ && prod == P_ && NT == N_) e = launch_split<K_, V_, P_, N_>(a, grid, stream);
@@ -826,12 +884,13 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
 #undef TQ_DEC_NT
 #undef TQ_DEC_CASE
     if (e != cudaSuccess) return e;
-    dim3 mgrid(B * Hkv, (a.G + a.merge_heads - 1) / a.merge_heads);
-    const int mthreads = kDim * a.merge_heads * a.merge_parts;
-    const size_t msmem = sizeof(float) * (kDim * kDim + kDim * a.merge_heads * (3 * a.merge_parts + 1));
+    const int units = B * Hkv;
+    const dim3 mgrid(units < ctx->sm_count ? units : ctx->sm_count);
+    const size_t msmem = sizeof(float) * (kDim * kDim + kDim * kMergeHeads);
     e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<<<mgrid, mthreads, msmem, stream>>>(a);
+    e = launch_dependent(decode_merge_kernel, mgrid, dim3(kMergeThreads), msmem, stream, a);
+    if (e != cudaSuccess) return e;
     count_launches(3);
     return cudaGetLastError();
 }

@@ -91,13 +91,17 @@ cudaError_t launch_compress(const tq_ctx* ctx, int kind, const uint16_t* x, int 
 cudaError_t launch_decompress(const tq_ctx* ctx, int kind, const uint8_t* cache, int num_blocks,
                               const int32_t* slots, int T, int H, void* out, int out_fp32, cudaStream_t stream);
 
+// Split-K decode: the pages of all (sequence, kv head) units, in order, are cut
+// into `grid` equal ranges, one per CTA of the split kernel; the piece of unit u
+// in CTA c leaves its partial softmax state in slot u + c (unique: each slot index
+// counts the unit and CTA boundaries before the piece).
 struct DecodePlan {
-    int splits;          // split-K factor over the pages of a sequence
-    int pages_per_split; // pages handled by one split
+    int grid;            // CTAs of the split kernel
+    int slots;           // units + grid
     int max_pages;       // ceil(max_seq_len / 16)
-    size_t partial_off;  // workspace offsets (bytes)
-    size_t qprep_off;
-    size_t ticket_off;
+    size_t qprep_off;    // workspace offsets (bytes)
+    size_t partial_off;
+    size_t prefix_off;   // int32 [B + 1]: pages of sequences 0 .. b-1
     size_t bytes;        // total workspace
 };
 DecodePlan plan_decode(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_seq_len);
