@@ -276,6 +276,22 @@ def workload_config(w):
                   "cache written one step earlier, evicted by the 700 MB of compress traffic in between"}
 
 
+def bench_slots(w):
+    """Prefill slot mapping and decode block table.  Several layers flatten into the
+    token axis (page-aligned, shuffled blocks); the decode then attends the first
+    layer's pages."""
+    import numpy as np
+
+    from kv_cache_vector_02_b200 import workloads as W
+    if w.layers == 1:
+        bt = W.block_table(w)
+        return W.prefill_slots(w, bt), bt
+    assert w.B == 1, "layered workloads hold one sequence per layer"
+    slots = W.flat_slots(w.tokens, perm_seed=w.data_seed)
+    bt = (slots[: w.T : PAGE] // PAGE).astype(np.int32)[None]
+    return slots, bt
+
+
 # ---------------------------------------------------------------- GPU arm
 def main():
     args = parse()
@@ -292,8 +308,7 @@ def main():
     w = W.WORKLOADS[args.workload].with_(bits=args.bits, rotation=rot, decode_steps=0,
                                          data_seed=rank_data_seed(rank))
     ctx = tq.tq_init(D, w.bits, w.param_seed, w.rotation, w.key_mode)
-    bt_np = W.block_table(w)
-    slots_np = W.prefill_slots(w, bt_np)
+    slots_np, bt_np = bench_slots(w)
     k = W.gen_kv(w, 0, device=dev)
     v = W.gen_kv(w, 1, device=dev)
     q = W.gen_q(w, 0, device=dev)

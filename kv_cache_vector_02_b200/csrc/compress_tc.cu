@@ -49,7 +49,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTeamThreads = 128;  // one thread per row
+constexpr int kTeamWarps = 4;  // one per TMEM lane quarter, one thread per row
 constexpr uint32_t kTile = 128 * 128 * 2;  // one 128 x 128 fp16 operand
 constexpr uint32_t kHalf = kTile / 2;      // one 128-byte-swizzled K-half
 constexpr uint64_t kWaitNs = 2000000000ull;
@@ -185,13 +185,13 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(bar(kBarXFull + s), 1);
             // released by the rotation MMAs and, for values, by the team that reads ||x||
-            mbar_init(bar(kBarXEmpty + s), PROD ? 1 : 1 + kTeamThreads);
+            mbar_init(bar(kBarXEmpty + s), PROD ? 1 : 1 + kTeamWarps);
         }
         for (int t = 0; t < C::kTeams; ++t) {
             mbar_init(bar(kBarRotFull + t), 1);
-            mbar_init(bar(kBarRotEmpty + t), kTeamThreads);
+            mbar_init(bar(kBarRotEmpty + t), kTeamWarps);
             if (PROD) {
-                mbar_init(bar(kBarRhoFull + t), kTeamThreads);
+                mbar_init(bar(kBarRhoFull + t), kTeamWarps);
                 mbar_init(bar(kBarQjlFull + t), 1);
             }
         }
@@ -356,8 +356,7 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
         const float2 rho_k = make_float2(a.rho_scale, a.rho_scale);
         constexpr int kPer = 32 / W;       // codes per 32-bit word
         constexpr int kQW = 32 / kPer;     // words of 32 columns' codes
-        bool ok = mbar_wait(bar(kBarConst), 0, abort, kWaitNs);
-        ok = __all_sync(0xffffffffu, ok);
+        const bool ok = mbar_wait_warp(bar(kBarConst), 0, abort, kWaitNs);
         if (!ok) set_abort(abort, a.err);
 
         // slot of this thread's row of a tile, and the row's destination: the chunk
@@ -407,8 +406,8 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 // ---- ||x||^2 of the row from the swizzled fp16 tile (logical 16-byte
                 // chunk c of a 128-byte row sits at chunk c ^ (row % 8))
                 const int stg = k % C::kStages;
-                bool good = !*abort && mbar_wait(bar(kBarXFull + stg), (uint32_t)(k / C::kStages) & 1u, abort, kWaitNs);
-                good = __all_sync(0xffffffffu, good);
+                bool good = mbar_wait_warp(bar(kBarXFull + stg), (uint32_t)(k / C::kStages) & 1u, abort, kWaitNs);
+                good = __all_sync(0xffffffffu, good && !*abort);
                 if (!good) {
                     set_abort(abort, a.err);
                     break;
@@ -428,18 +427,17 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                     }
                 }
                 fence_proxy_async_shared();  // these reads before the next TMA write of the stage
-                mbar_arrive(bar(kBarXEmpty + stg));
+                mbar_arrive_warp(bar(kBarXEmpty + stg));
                 nsq = (sq[0] + sq[1]) + (sq[2] + sq[3]);
-                good = mbar_wait(bar(kBarRotFull + team), use & 1u, abort, kWaitNs);
-                good = __all_sync(0xffffffffu, good);
+                good = mbar_wait_warp(bar(kBarRotFull + team), use & 1u, abort, kWaitNs);
                 if (!good) {
                     set_abort(abort, a.err);
                     break;
                 }
                 tc_fence_after();
             } else {
-                bool good = !*abort && mbar_wait(bar(kBarRotFull + team), use & 1u, abort, kWaitNs);
-                good = __all_sync(0xffffffffu, good);
+                bool good = mbar_wait_warp(bar(kBarRotFull + team), use & 1u, abort, kWaitNs);
+                good = __all_sync(0xffffffffu, good && !*abort);
                 if (!good) {
                     set_abort(abort, a.err);
                     break;
@@ -552,7 +550,7 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
             }
             if (!PROD) {
                 tc_fence_before();
-                mbar_arrive(bar(kBarRotEmpty + team));
+                mbar_arrive_warp(bar(kBarRotEmpty + team));
                 const uint32_t none[4] = {0u, 0u, 0u, 0u};
                 store_tail(dst, norm, 0.f, none);
                 continue;
@@ -560,11 +558,10 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
             // ---- keys: release rho; gamma; then the sketch as sign bits
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(bar(kBarRhoFull + team));
+            mbar_arrive_warp(bar(kBarRhoFull + team));
             const float gsq = (gs[0].x + gs[0].y) + (gs[1].x + gs[1].y);
             const float gamma = (live && gsq > 0.f) ? gsq * rsqrt_refined(gsq) * nacc * a.gamma_scale : 0.f;
-            bool sk = mbar_wait(bar(kBarQjlFull + team), use & 1u, abort, kWaitNs);
-            sk = __all_sync(0xffffffffu, sk);
+            const bool sk = mbar_wait_warp(bar(kBarQjlFull + team), use & 1u, abort, kWaitNs);
             if (!sk) {
                 set_abort(abort, a.err);
                 break;
@@ -582,7 +579,7 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 sg[c] = live ? ~neg : 0xffffffffu;
             }
             tc_fence_before();
-            mbar_arrive(bar(kBarRotEmpty + team));
+            mbar_arrive_warp(bar(kBarRotEmpty + team));
             store_tail(dst, norm, gamma, sg);
         }
     }

@@ -621,8 +621,7 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
             for (int j = 0; j < nj && j < kStagesD; ++j) issue(j);
         for (int j = 0; j < nj && !dead; ++j) {
             const uint32_t sidx = consumed % kStagesD;
-            bool ok = sm100::mbar_wait(bars + 8 * sidx, (consumed / kStagesD) & 1u, &never, 2000000000ull);
-            ok = __all_sync(0xffffffffu, ok);
+            const bool ok = sm100::mbar_wait_warp(bars + 8 * sidx, (consumed / kStagesD) & 1u, &never, 2000000000ull);
             const int blk = blk_of(j);
             if (!ok) {
                 if (lane == 0) atomicOr(a.err, TQ_DEVERR_TIMEOUT);
@@ -693,8 +692,8 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
 }
 
 // ------------------------------------------------------------------ merge
-// Persistent: CTA i takes units i, i + grid, ...; 128 threads per head, kMergeHeads
-// heads at a time.  R^T is staged once per CTA (while the split kernel runs).
+// Persistent: CTA i takes the (unit, group of kMergeHeads heads) items i, i + grid,
+// ...; 128 threads per head.  R^T is staged once per CTA (while the split kernel runs).
 // Unit u's pieces sit in slots u + c for the split CTAs c whose page range meets
 // it: c(p) = ((p + 1) grid - 1) / total is the CTA of page p.
 constexpr int kMergeHeads = 4;
@@ -712,8 +711,10 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs 
     griddep_wait();  // the split partials
     const long total = (long)a.Hkv * a.prefix[a.B];
     const long grid = a.split_grid;
-    const int units = a.B * a.Hkv;
-    for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
+    const int groups = (a.G + kMergeHeads - 1) / kMergeHeads;
+    const int items = a.B * a.Hkv * groups;
+    for (int item = blockIdx.x; item < items; item += gridDim.x) {
+        const int unit = item / groups, h0 = (item - unit * groups) * kMergeHeads;
         const int b = unit / a.Hkv, hk = unit - b * a.Hkv;
         const int np = a.prefix[b + 1] - a.prefix[b];
         int c_lo = 0, c_hi = -1;
@@ -722,14 +723,16 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs 
             c_lo = (int)(((first + 1) * grid - 1) / total);
             c_hi = (int)(((last + 1) * grid - 1) / total);
         }
-        for (int h0 = 0; h0 < a.G; h0 += kMergeHeads) {
+        {
             const int h = h0 + hl;
             const bool active = h < a.G;
             float M = -INFINITY, Lsum = 0.f, A = 0.f;
-            if (active) {
+            if (active) {  // unrolled: a long sequence spreads over tens of slots
+#pragma unroll 8
                 for (int c = c_lo; c <= c_hi; ++c)
                     M = fmaxf(M, a.partial[(((size_t)unit + c) * a.G + h) * kPartStride]);
                 if (M != -INFINITY)
+#pragma unroll 8
                     for (int c = c_lo; c <= c_hi; ++c) {
                         const float* pp = a.partial + (((size_t)unit + c) * a.G + h) * kPartStride;
                         const float ms = pp[0];
@@ -884,8 +887,8 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
 #undef TQ_DEC_NT
 #undef TQ_DEC_CASE
     if (e != cudaSuccess) return e;
-    const int units = B * Hkv;
-    const dim3 mgrid(units < ctx->sm_count ? units : ctx->sm_count);
+    const int mitems = B * Hkv * ((a.G + kMergeHeads - 1) / kMergeHeads);
+    const dim3 mgrid(mitems < ctx->sm_count ? mitems : ctx->sm_count);
     const size_t msmem = sizeof(float) * (kDim * kDim + kDim * kMergeHeads);
     e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
     if (e != cudaSuccess) return e;

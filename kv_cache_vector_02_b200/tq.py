@@ -156,20 +156,44 @@ def tq_export_params(ctx: Context) -> dict:
     return out
 
 
+def _expect(t, shape, dtypes, what: str, name: str):
+    """The C ABI takes raw pointers plus sizes: every tensor must hold exactly what
+    those sizes promise (shape, dtype, dense row-major), or the call is refused here."""
+    import torch
+    ok = t is not None and t.dim() == len(shape) and t.is_contiguous() and t.dtype in dtypes
+    ok = ok and all(want is None or int(got) == want for got, want in zip(t.shape, shape))
+    if not ok:
+        desc = "None" if t is None else "%s %s" % (tuple(t.shape), t.dtype)
+        raise TQError(TQ_ERR_INVALID_ARG, "%s: %s must be %s of %s, got %s" % (what, name, list(shape), dtypes, desc))
+
+
 def tq_compress(ctx: Context, k, v, slot_mapping, k_cache, v_cache, stream=None):
-    """k, v: [T, Hkv, 128] fp16 CUDA tensors (either may be None); caches [num_blocks, Hkv, chunk] uint8."""
+    """k, v: [T, Hkv, 128] fp16 CUDA tensors (either may be None); slot_mapping [T] int32;
+    caches [num_blocks, Hkv, chunk] uint8."""
+    import torch
     ref = k if k is not None else v
-    T, Hkv = int(ref.shape[0]), int(ref.shape[1])
+    if ref is None:
+        raise TQError(TQ_ERR_INVALID_ARG, "tq_compress: no input")
+    T, Hkv = int(ref.shape[0]), int(ref.shape[1]) if ref.dim() > 1 else 0
     cache = k_cache if k_cache is not None else v_cache
-    num_blocks = int(cache.shape[0])
+    num_blocks = int(cache.shape[0]) if cache is not None else 0
+    for x, c, kind, n in ((k, k_cache, KIND_KEY, "k"), (v, v_cache, KIND_VALUE, "v")):
+        if x is None:
+            continue
+        _expect(x, (T, Hkv, ctx.head_dim), (torch.float16,), "tq_compress", n)
+        _expect(c, (num_blocks, Hkv, tq_chunk_bytes(ctx, kind)), (torch.uint8,), "tq_compress", n + "_cache")
+    _expect(slot_mapping, (T,), (torch.int32,), "tq_compress", "slot_mapping")
     _check(_lib.tq_compress(ctx.handle, _ptr(k), _ptr(v), T, Hkv, _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
                             num_blocks, _stream(stream)), "tq_compress")
 
 
 def tq_decompress(ctx: Context, kind: int, cache, slot_mapping, out, stream=None):
-    """out: [T, Hkv, 128] fp16 or fp32 CUDA tensor."""
+    """out: [T, Hkv, 128] fp16 or fp32 CUDA tensor; slot_mapping [T] int32; cache [num_blocks, Hkv, chunk]."""
     import torch
     T, Hkv = int(out.shape[0]), int(out.shape[1])
+    _expect(out, (T, Hkv, ctx.head_dim), (torch.float16, torch.float32), "tq_decompress", "out")
+    _expect(slot_mapping, (T,), (torch.int32,), "tq_decompress", "slot_mapping")
+    _expect(cache, (None, Hkv, tq_chunk_bytes(ctx, kind)), (torch.uint8,), "tq_decompress", "cache")
     _check(_lib.tq_decompress(ctx.handle, kind, _ptr(cache), int(cache.shape[0]), _ptr(slot_mapping), T, Hkv,
                               _ptr(out), 1 if out.dtype == torch.float32 else 0, _stream(stream)), "tq_decompress")
 
@@ -189,6 +213,8 @@ def tq_decode_attention(ctx: Context, q, k_cache, v_cache, block_table, seq_lens
     B, Hq = int(q.shape[0]), int(q.shape[1])
     if Hkv is None:
         Hkv = int(k_cache.shape[1])
+    _check_decode_args(ctx, q, k_cache, v_cache, block_table, seq_lens, out, Hkv, "tq_decode_attention")
+    _expect(workspace, (None,), (torch.uint8,), "tq_decode_attention", "workspace")
     _check(_lib.tq_decode_attention(ctx.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache), int(k_cache.shape[0]),
                                     _ptr(block_table), int(block_table.shape[1]), _ptr(seq_lens), B, Hq, Hkv,
                                     int(max_seq_len), float(scale), _ptr(out), 1 if out.dtype == torch.float32 else 0,
@@ -197,6 +223,17 @@ def tq_decode_attention(ctx: Context, q, k_cache, v_cache, block_table, seq_lens
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def _check_decode_args(ctx, q, k_cache, v_cache, block_table, seq_lens, out, Hkv, what):
+    import torch
+    B, Hq = int(q.shape[0]), int(q.shape[1])
+    _expect(q, (B, Hq, ctx.head_dim), (torch.float16,), what, "q")
+    _expect(k_cache, (None, Hkv, tq_chunk_bytes(ctx, KIND_KEY)), (torch.uint8,), what, "k_cache")
+    _expect(v_cache, (int(k_cache.shape[0]), Hkv, tq_chunk_bytes(ctx, KIND_VALUE)), (torch.uint8,), what, "v_cache")
+    _expect(block_table, (B, None), (torch.int32,), what, "block_table")
+    _expect(seq_lens, (B,), (torch.int32,), what, "seq_lens")
+    _expect(out, (B, Hq, ctx.head_dim), (torch.float16, torch.float32), what, "out")
 
 
 def tq_decode_attention_noalloc(ctx: Context, q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int, out,
@@ -208,6 +245,7 @@ def tq_decode_attention_noalloc(ctx: Context, q, k_cache, v_cache, block_table, 
     B, Hq = int(q.shape[0]), int(q.shape[1])
     if Hkv is None:
         Hkv = int(k_cache.shape[1])
+    _check_decode_args(ctx, q, k_cache, v_cache, block_table, seq_lens, out, Hkv, "tq_decode_attention_noalloc")
     _check(_lib.tq_decode_attention_noalloc(ctx.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache), int(k_cache.shape[0]),
                                             _ptr(block_table), int(block_table.shape[1]), _ptr(seq_lens), B, Hq, Hkv,
                                             int(max_seq_len), float(scale), _ptr(out),
