@@ -479,72 +479,92 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
               uint32_t words[kQW];
 #pragma unroll
               for (int i = 0; i < kQW; ++i) words[i] = 0u;
+              if (PROD) {
+                // both K-steps of the 32 columns at once: 16 independent column pairs
+                const uint32_t col = buf + 32 * q;
+                float2 av[16];
+                {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(col, r0);
+                    tmem_ld32(col + kColB, r1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) av[i] = ld_sum(r0, r1, i);
+                }
+                if (any_bad && !finite) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) av[i] = make_float2(0.f, 0.f);
+                }
+                uint32_t rho_hi[16], rho_lo[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 u = __fmul2_rn(av[i], s2);
+                    const float2 gg = __fadd2_rn(u, magic2);
+                    uint32_t b0, base0, lo0, hi0, b1, base1, lo1, hi1;
+                    lds_v4(__float_as_uint(gg.x) * 128u + lut_off, b0, base0, lo0, hi0);
+                    lds_v4(__float_as_uint(gg.y) * 128u + lut_off, b1, base1, lo1, hi1);
+                    const bool p0 = __uint_as_float(b0) < u.x;
+                    const bool p1 = __uint_as_float(b1) < u.y;
+                    const uint32_t code0 = base0 + (p0 ? 1u : 0u);
+                    const uint32_t code1 = base1 + (p1 ? 1u : 0u);
+                    const float c0 = __uint_as_float(p0 ? hi0 : lo0);
+                    const float c1 = __uint_as_float(p1 ? hi1 : lo1);
+                    const float2 d = __ffma2_rn(av[i], s2, make_float2(-c0, -c1));  // residual, cell units
+                    gs[i & 1] = __ffma2_rn(d, d, gs[i & 1]);
+                    // rho = 32 (v - c) = hi + lo in fp16: hi keeps the top 11 significant bits
+                    // (exact in fp16 for |rho| < 65504), lo = rho - hi exactly
+                    const float2 rho = __fmul2_rn(d, rho_k);
+                    const float2 hf = make_float2(__uint_as_float(__float_as_uint(rho.x) & 0xffffe000u),
+                                                  __uint_as_float(__float_as_uint(rho.y) & 0xffffe000u));
+                    const float2 rem = __fadd2_rn(rho, make_float2(-hf.x, -hf.y));
+                    const __half2 hi = __floats2half2_rn(hf.x, hf.y);
+                    const __half2 lo = __floats2half2_rn(rem.x, rem.y);
+                    rho_hi[i] = *reinterpret_cast<const uint32_t*>(&hi);
+                    rho_lo[i] = *reinterpret_cast<const uint32_t*>(&lo);
+                    const int j = 2 * i;  // column within the 32
+                    words[j / kPer] += code0 << (W * (j % kPer));
+                    words[(j + 1) / kPer] += code1 << (W * ((j + 1) % kPer));
+                }
+                // over the K-steps' A columns, already read: K-step st -> hi at 16 st, lo at 16 st + 8
+                uint32_t h8[8], l8[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) h8[i] = rho_hi[i], l8[i] = rho_lo[i];
+                tmem_st8(col, h8);
+                tmem_st8(col + 8, l8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) h8[i] = rho_hi[8 + i], l8[i] = rho_lo[8 + i];
+                tmem_st8(col + 16, h8);
+                tmem_st8(col + 24, l8);
+              } else {
 #pragma unroll
               for (int sub = 0; sub < 2; ++sub) {
                 const uint32_t col = buf + 32 * q + 16 * sub;
                 float2 av[8];
-                if (!PROD) {  // one accumulator
+                {  // one accumulator
                     uint32_t r0[16];
                     tmem_ld16(col, r0);
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 8; ++i) av[i] = make_float2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
-                } else {
-                    uint32_t r0[16], r1[16];
-                    tmem_ld16(col, r0);
-                    tmem_ld16(col + kColB, r1);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        av[i] = __fadd2_rn(make_float2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1])),
-                                           make_float2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1])));
                 }
                 if (any_bad && !finite) {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) av[i] = make_float2(0.f, 0.f);
                 }
-                uint32_t rho_hi[8], rho_lo[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float2 u = __fmul2_rn(av[i], s2);
                     const float2 gg = __fadd2_rn(u, magic2);
-                    const uint32_t ad0 = __float_as_uint(gg.x) * 128u + lut_off;
-                    const uint32_t ad1 = __float_as_uint(gg.y) * 128u + lut_off;
-                    uint32_t code0, code1;
-                    if (PROD) {
-                        uint32_t b0, base0, lo0, hi0, b1, base1, lo1, hi1;
-                        lds_v4(ad0, b0, base0, lo0, hi0);
-                        lds_v4(ad1, b1, base1, lo1, hi1);
-                        const bool p0 = __uint_as_float(b0) < u.x;
-                        const bool p1 = __uint_as_float(b1) < u.y;
-                        code0 = base0 + (p0 ? 1u : 0u);
-                        code1 = base1 + (p1 ? 1u : 0u);
-                        const float c0 = __uint_as_float(p0 ? hi0 : lo0);
-                        const float c1 = __uint_as_float(p1 ? hi1 : lo1);
-                        const float2 d = __ffma2_rn(av[i], s2, make_float2(-c0, -c1));  // residual, cell units
-                        gs[i & 1] = __ffma2_rn(d, d, gs[i & 1]);
-                        const float2 rho = __fmul2_rn(d, rho_k);  // 32 (v - c): rho = hi + lo in fp16
-                        const __half2 hi = __floats2half2_rn(rho.x, rho.y);
-                        const float2 back = __half22float2(hi);
-                        const float2 rem = __fadd2_rn(rho, make_float2(-back.x, -back.y));
-                        const __half2 lo = __floats2half2_rn(rem.x, rem.y);
-                        rho_hi[i] = *reinterpret_cast<const uint32_t*>(&hi);
-                        rho_lo[i] = *reinterpret_cast<const uint32_t*>(&lo);
-                    } else {
-                        uint32_t b0, base0, b1, base1;
-                        lds_v2(ad0, b0, base0);
-                        lds_v2(ad1, b1, base1);
-                        code0 = base0 + (__uint_as_float(b0) < u.x ? 1u : 0u);
-                        code1 = base1 + (__uint_as_float(b1) < u.y ? 1u : 0u);
-                    }
+                    uint32_t b0, base0, b1, base1;
+                    lds_v2(__float_as_uint(gg.x) * 128u + lut_off, b0, base0);
+                    lds_v2(__float_as_uint(gg.y) * 128u + lut_off, b1, base1);
+                    const uint32_t code0 = base0 + (__uint_as_float(b0) < u.x ? 1u : 0u);
+                    const uint32_t code1 = base1 + (__uint_as_float(b1) < u.y ? 1u : 0u);
                     const int j = 16 * sub + 2 * i;  // column within the 32
                     words[j / kPer] += code0 << (W * (j % kPer));
                     words[(j + 1) / kPer] += code1 << (W * ((j + 1) % kPer));
                 }
-                if (PROD) {  // over the K-step's A columns, already read
-                    tmem_st8(col, rho_hi);
-                    tmem_st8(col + 8, rho_lo);
-                }
+              }
               }
               store_codes(dst, q, words);
             }
