@@ -692,17 +692,20 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
 }
 
 // ------------------------------------------------------------------ merge
-// Persistent: CTA i takes the (unit, group of kMergeHeads heads) items i, i + grid,
-// ...; 128 threads per head.  R^T is staged once per CTA (while the split kernel runs).
-// Unit u's pieces sit in slots u + c for the split CTAs c whose page range meets
-// it: c(p) = ((p + 1) grid - 1) / total is the CTA of page p.
+// Persistent: CTA i takes the (unit, group of kMergeHeads heads) items
+// i * kMergeItems .. + kMergeItems - 1, then + grid * kMergeItems, ...; 128 threads
+// per item, thread = coordinate, computing all the group's heads so that each
+// element of R is read once per item.  R^T is staged once per CTA (while the split
+// kernel runs).  Unit u's pieces sit in slots u + c for the split CTAs c whose
+// page range meets it: c(p) = ((p + 1) grid - 1) / total is the CTA of page p.
 constexpr int kMergeHeads = 4;
-constexpr int kMergeThreads = kDim * kMergeHeads;
+constexpr int kMergeItems = 4;
+constexpr int kMergeThreads = kDim * kMergeItems;
 __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs a) {
-    extern __shared__ __align__(16) float sm[];  // RT [128*128] | orot [heads][128]
-    const int i = threadIdx.x % kDim, hl = threadIdx.x / kDim;
+    extern __shared__ __align__(16) float sm[];  // RT [128*128] | orot [items][128][kMergeHeads]
+    const int i = threadIdx.x % kDim, il = threadIdx.x / kDim;
     float* rts = sm;
-    float* orot = sm + kDim * kDim;
+    float4* orot = reinterpret_cast<float4*>(sm + kDim * kDim) + il * kDim;  // this item's [j] of 4 heads
     {
         const float4* src = reinterpret_cast<const float4*>(a.RT);
         float4* dst = reinterpret_cast<float4*>(rts);
@@ -713,48 +716,74 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs 
     const long grid = a.split_grid;
     const int groups = (a.G + kMergeHeads - 1) / kMergeHeads;
     const int items = a.B * a.Hkv * groups;
-    for (int item = blockIdx.x; item < items; item += gridDim.x) {
-        const int unit = item / groups, h0 = (item - unit * groups) * kMergeHeads;
-        const int b = unit / a.Hkv, hk = unit - b * a.Hkv;
-        const int np = a.prefix[b + 1] - a.prefix[b];
-        int c_lo = 0, c_hi = -1;
-        if (np > 0) {
-            const long first = (long)a.Hkv * a.prefix[b] + (long)hk * np, last = first + np - 1;
-            c_lo = (int)(((first + 1) * grid - 1) / total);
-            c_hi = (int)(((last + 1) * grid - 1) / total);
+    for (int base = blockIdx.x * kMergeItems; base < items; base += gridDim.x * kMergeItems) {
+        const int item = base + il;
+        const bool live = item < items;
+        int unit = 0, h0 = 0, c_lo = 0, c_hi = -1;
+        if (live) {
+            unit = item / groups;
+            h0 = (item - unit * groups) * kMergeHeads;
+            const int b = unit / a.Hkv, hk = unit - b * a.Hkv;
+            const int np = a.prefix[b + 1] - a.prefix[b];
+            if (np > 0) {
+                const long first = (long)a.Hkv * a.prefix[b] + (long)hk * np, last = first + np - 1;
+                c_lo = (int)(((first + 1) * grid - 1) / total);
+                c_hi = (int)(((last + 1) * grid - 1) / total);
+            }
         }
-        {
-            const int h = h0 + hl;
-            const bool active = h < a.G;
-            float M = -INFINITY, Lsum = 0.f, A = 0.f;
-            if (active) {  // unrolled: a long sequence spreads over tens of slots
-#pragma unroll 8
-                for (int c = c_lo; c <= c_hi; ++c)
-                    M = fmaxf(M, a.partial[(((size_t)unit + c) * a.G + h) * kPartStride]);
-                if (M != -INFINITY)
-#pragma unroll 8
-                    for (int c = c_lo; c <= c_hi; ++c) {
-                        const float* pp = a.partial + (((size_t)unit + c) * a.G + h) * kPartStride;
-                        const float ms = pp[0];
-                        const float wt = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
-                        Lsum = fmaf(wt, pp[1], Lsum);
-                        A = fmaf(wt, pp[2 + i], A);
-                    }
+        // online log-sum-exp over the slots, all heads at once: the loads of several
+        // slots are in flight together
+        float M[kMergeHeads], Lsum[kMergeHeads], A[kMergeHeads];
+#pragma unroll
+        for (int e = 0; e < kMergeHeads; ++e) M[e] = -INFINITY, Lsum[e] = 0.f, A[e] = 0.f;
+        const int nh = a.G - h0 < kMergeHeads ? a.G - h0 : kMergeHeads;
+#pragma unroll 4
+        for (int c = c_lo; c <= c_hi; ++c) {
+            const float* pp = a.partial + (((size_t)unit + c) * a.G + h0) * kPartStride;
+            float ms[kMergeHeads], ls[kMergeHeads], as[kMergeHeads];
+#pragma unroll
+            for (int e = 0; e < kMergeHeads; ++e) {
+                const bool on = e < nh;
+                ms[e] = on ? pp[e * kPartStride] : -INFINITY;
+                ls[e] = on ? pp[e * kPartStride + 1] : 0.f;
+                as[e] = on ? pp[e * kPartStride + 2 + i] : 0.f;
             }
-            __syncthreads();  // the previous heads' un-rotation is done with orot
-            orot[hl * kDim + i] = Lsum > 0.f ? A / Lsum : 0.f;
-            __syncthreads();
-            if (active) {
-                float y = 0.f;
-                const float* orh = orot + hl * kDim;
-#pragma unroll 8
-                for (int j = 0; j < kDim; ++j) y = fmaf(rts[j * kDim + i], orh[j], y);  // o_i = sum_j R[i][j] orot_j
-                const size_t oi = ((size_t)unit * a.G + h) * kDim + i;
-                if (a.out_fp32)
-                    static_cast<float*>(a.out)[oi] = y;
-                else
-                    static_cast<__half*>(a.out)[oi] = __float2half_rn(y);
+#pragma unroll
+            for (int e = 0; e < kMergeHeads; ++e) {
+                const float mn = fmaxf(M[e], ms[e]);
+                const float sa = (M[e] == -INFINITY) ? 0.f : exp2f(M[e] - mn);
+                const float sb = (ms[e] == -INFINITY) ? 0.f : exp2f(ms[e] - mn);
+                Lsum[e] = fmaf(Lsum[e], sa, ls[e] * sb);
+                A[e] = fmaf(A[e], sa, as[e] * sb);
+                M[e] = mn;
             }
+        }
+        float o[kMergeHeads];
+#pragma unroll
+        for (int e = 0; e < kMergeHeads; ++e) o[e] = (live && Lsum[e] > 0.f) ? A[e] / Lsum[e] : 0.f;
+        __syncthreads();  // the previous items' un-rotation is done with orot
+        orot[i] = make_float4(o[0], o[1], o[2], o[3]);
+        __syncthreads();
+        if (!live) continue;
+        float y[kMergeHeads] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int j = 0; j < kDim; ++j) {  // o_i = sum_j R[i][j] orot_j, for the 4 heads at once
+            const float r = rts[j * kDim + i];
+            const float4 v = orot[j];
+            y[0] = fmaf(r, v.x, y[0]);
+            y[1] = fmaf(r, v.y, y[1]);
+            y[2] = fmaf(r, v.z, y[2]);
+            y[3] = fmaf(r, v.w, y[3]);
+        }
+#pragma unroll
+        for (int e = 0; e < kMergeHeads; ++e) {
+            const int h = h0 + e;
+            if (h >= a.G) break;
+            const size_t oi = ((size_t)unit * a.G + h) * kDim + i;
+            if (a.out_fp32)
+                static_cast<float*>(a.out)[oi] = y[e];
+            else
+                static_cast<__half*>(a.out)[oi] = __float2half_rn(y[e]);
         }
     }
 }
@@ -888,8 +917,9 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
 #undef TQ_DEC_CASE
     if (e != cudaSuccess) return e;
     const int mitems = B * Hkv * ((a.G + kMergeHeads - 1) / kMergeHeads);
-    const dim3 mgrid(mitems < ctx->sm_count ? mitems : ctx->sm_count);
-    const size_t msmem = sizeof(float) * (kDim * kDim + kDim * kMergeHeads);
+    const int mctas = (mitems + kMergeItems - 1) / kMergeItems;
+    const dim3 mgrid(mctas < ctx->sm_count ? mctas : ctx->sm_count);
+    const size_t msmem = sizeof(float) * (kDim * kDim + kDim * kMergeHeads * kMergeItems);
     e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
     if (e != cudaSuccess) return e;
     e = launch_dependent(decode_merge_kernel, mgrid, dim3(kMergeThreads), msmem, stream, a);
