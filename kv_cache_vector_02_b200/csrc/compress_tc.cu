@@ -26,7 +26,9 @@
 // registers (acc = A + B), and ||x|| = ||acc|| / (acc / y).
 // In both cases v = sqrt(d) y / ||x||; the epilogue works in cell units u = v * scale of a shared-memory
 // table of uniform cells (each holds at most one boundary): round(u) addresses
-// the cell, one fp32 compare with its boundary gives the code.
+// the cell, one fp32 compare with its boundary gives the code (values: of
+// u - round(u) with the boundary's offset in the cell, from one 4-byte read;
+// keys: of u with the boundary, from one 16-byte read that also holds the levels).
 // Keys (prod mode): the residual d = u - c[code] (cell units) gives
 // gamma = ||x - x_hat|| and rho = 32 (v - c[code]), and the sign sketch
 //   S (x - x_hat) = (S R) (y - y_hat)
@@ -139,15 +141,17 @@ __device__ __forceinline__ float rsqrt_refined(float x) {
 }
 
 // Table reads at a 32-bit shared-memory address.
-__device__ __forceinline__ void lds_v2(uint32_t addr, uint32_t& x, uint32_t& y) {
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(x), "=r"(y) : "r"(addr));
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+    uint32_t x;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(x) : "r"(addr));
+    return x;
+}
+__device__ __forceinline__ void lds_v4(uint32_t addr, uint32_t& x, uint32_t& y, uint32_t& z, uint32_t& w) {
+    asm("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(x), "=r"(y), "=r"(z), "=r"(w) : "r"(addr));
 }
 // in program order with the other volatile accesses (bounds how far loads are hoisted)
 __device__ __forceinline__ void lds_v4_ordered(uint32_t addr, uint32_t& x, uint32_t& y, uint32_t& z, uint32_t& w) {
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(x), "=r"(y), "=r"(z), "=r"(w) : "r"(addr));
-}
-__device__ __forceinline__ void lds_v4(uint32_t addr, uint32_t& x, uint32_t& y, uint32_t& z, uint32_t& w) {
-    asm("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(x), "=r"(y), "=r"(z), "=r"(w) : "r"(addr));
 }
 
 // s0 += lo^2, s1 += hi^2 for the two fp16 halves of w (exact squares, fp32 sums).
@@ -240,26 +244,30 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_f16(128, 128);
-            const uint32_t img = sbase + C::kOffImg;
             bool ok = mbar_wait(bar(kBarConst), 0, abort, kWaitNs);
-            auto kdesc = [](uint32_t base, int step) {  // K-step of 16 elements inside a 128x128 operand
-                return smem_desc_sw128(base + (uint32_t)(step >> 2) * kHalf + (uint32_t)(step & 3) * 32u);
+            // descriptors as low halves: operand i of the images, stage s of x, and
+            // the offset of K-step st (16 elements) inside a 128x128 operand
+            constexpr uint32_t kTileU = kTile >> 4;
+            const uint32_t img = sw128_desc_lo(sbase + C::kOffImg);
+            const uint32_t x0 = sw128_desc_lo(sbase + C::kOffX);
+            auto kdesc = [](uint32_t lo, int step) {
+                return sw128_desc(lo + (((uint32_t)(step >> 2) * kHalf + (uint32_t)(step & 3) * 32u) >> 4));
             };
             // rotation of local tile k into its team's buffer; false when not ready yet
             auto try_rot = [&](int k) -> bool {
                 const int s = k % C::kStages;
                 const int t = k % C::kTeams;
                 const uint32_t use = (uint32_t)(k / C::kTeams);
-                if (!mbar_try_wait(bar(kBarXFull + s), (uint32_t)(k / C::kStages) & 1u)) return false;
-                if (!mbar_try_wait(bar(kBarRotEmpty + t), (use & 1u) ^ 1u)) return false;
+                if (!mbar_test_wait(bar(kBarXFull + s), (uint32_t)(k / C::kStages) & 1u)) return false;
+                if (!mbar_test_wait(bar(kBarRotEmpty + t), (use & 1u) ^ 1u)) return false;
                 tc_fence_after();
                 const uint32_t dA = tmem + C::kBufCols * (uint32_t)t, dB = PROD ? dA + kColB : dA;
-                const uint32_t xs = sbase + C::kOffX + s * kTile;
+                const uint32_t xs = x0 + (uint32_t)s * kTileU;
                 uint32_t accA = 0u;
                 if (ROT == 0) {  // the small lo pass first, then K-steps 0-3 of the hi pass
 #pragma unroll
                     for (int st = 0; st < 8; ++st) {
-                        umma_ss(dA, kdesc(xs, st), kdesc(img + kTile, st), idesc, accA);
+                        umma_ss(dA, kdesc(xs, st), kdesc(img + kTileU, st), idesc, accA);
                         accA = 1u;
                     }
                 }
@@ -278,11 +286,11 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
             // sketch of local tile k (keys); false when its rho is not written yet
             auto try_qjl = [&](int k) -> bool {
                 const int t = k & 1;
-                if (!mbar_try_wait(bar(kBarRhoFull + t), (uint32_t)(k >> 1) & 1u)) return false;
+                if (!mbar_test_wait(bar(kBarRhoFull + t), (uint32_t)(k >> 1) & 1u)) return false;
                 tc_fence_after();
                 const uint32_t buf = tmem + C::kBufCols * (uint32_t)t;
                 const uint32_t d = buf + kColB;
-                const uint32_t m0 = img + C::kRotImages * kTile;
+                const uint32_t m0 = img + C::kRotImages * kTileU;
                 // rho of K-step st: columns 16 st (hi pairs) and 16 st + 8 (lo pairs)
                 auto rho_col = [&](int st) { return buf + 16u * (uint32_t)st; };
                 uint32_t acc2 = 0u;
@@ -294,7 +302,7 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 }
                 if (ROT == 0) {
 #pragma unroll
-                    for (int st = 0; st < 8; ++st) umma_ts(d, rho_col(st), kdesc(m0 + kTile, st), idesc, 1u);
+                    for (int st = 0; st < 8; ++st) umma_ts(d, rho_col(st), kdesc(m0 + kTileU, st), idesc, 1u);
                 }
 #pragma unroll
                 for (int st = 0; st < 8; ++st) umma_ts(d, rho_col(st), kdesc(m0, st), idesc, 1u);
@@ -346,13 +354,15 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
         const int row = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         const uint32_t buf = tmem + lane_addr + C::kBufCols * (uint32_t)team;
-        // table entry of u: bits(u + magic) * 128 + lut_off, in this lane's replica
+        // table entry of u: bits(u + magic) * 128 + lut_off, in this lane's copy
         // (bits(u + magic) = bits(1.5 * 2^23) + cells / 2 + round(u), see tc_params.h)
         const uint32_t lut_off = sbase + C::kOffLut +
-                                 (PROD ? 16u * (uint32_t)(lane & (kLutReplProd - 1))
-                                       : 8u * (uint32_t)(lane & (kLutReplMse - 1))) -
+                                 (PROD ? 16u * (uint32_t)(lane & (kLutReplProd - 1)) : 4u * (uint32_t)lane) -
                                  __float_as_uint(12582912.0f) * 128u;
         const float2 magic2 = make_float2(a.lut_magic, a.lut_magic);
+        const float2 mone2 = make_float2(-1.f, -1.f);
+        // code of u from its cell's entry e and fr = u - round(u) (exact)
+        auto code_of = [](uint32_t e, float fr) -> uint32_t { return (e & 15u) + (__uint_as_float(e) < fr ? 1u : 0u); };
         const float2 rho_k = make_float2(a.rho_scale, a.rho_scale);
         constexpr int kPer = 32 / W;       // codes per 32-bit word
         constexpr int kQW = 32 / kPer;     // words of 32 columns' codes
@@ -555,11 +565,9 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 for (int i = 0; i < 8; ++i) {
                     const float2 u = __fmul2_rn(av[i], s2);
                     const float2 gg = __fadd2_rn(u, magic2);
-                    uint32_t b0, base0, b1, base1;
-                    lds_v2(__float_as_uint(gg.x) * 128u + lut_off, b0, base0);
-                    lds_v2(__float_as_uint(gg.y) * 128u + lut_off, b1, base1);
-                    const uint32_t code0 = base0 + (__uint_as_float(b0) < u.x ? 1u : 0u);
-                    const uint32_t code1 = base1 + (__uint_as_float(b1) < u.y ? 1u : 0u);
+                    const float2 fr = __fadd2_rn(u, __ffma2_rn(gg, mone2, magic2));  // u - round(u)
+                    const uint32_t code0 = code_of(lds_u32(__float_as_uint(gg.x) * 128u + lut_off), fr.x);
+                    const uint32_t code1 = code_of(lds_u32(__float_as_uint(gg.y) * 128u + lut_off), fr.y);
                     const int j = 16 * sub + 2 * i;  // column within the 32
                     words[j / kPer] += code0 << (W * (j % kPer));
                     words[(j + 1) / kPer] += code1 << (W * ((j + 1) % kPer));

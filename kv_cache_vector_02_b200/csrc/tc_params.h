@@ -11,16 +11,23 @@ namespace tq {
 struct HostParams;
 
 // Bucketize tables: uniform cells over v = sqrt(d) y / ||x|| in [-V, V]; a cell
-// holds at most one interior boundary, far from its edges.  Entries hold the
-// boundary (+inf if none) and the levels in cell units u = v * scale.
-// Each entry is stored once per lane group, interleaved, so that the lanes of
-// one shared-memory phase (16 for 8-byte loads, 8 for 16-byte loads) always hit
-// distinct banks: byte offset = cell * 128 + replica * entry_size.
-constexpr int kLutCellsMse = 256;   // entry {float bnd; int base}
-constexpr int kLutCellsProd = 128;  // entry {float bnd; int base; float c_lo; float c_hi}
-constexpr int kLutReplMse = 16;
+// holds at most one interior boundary, at least 5% of a cell from its edges.  In
+// cell units u = v * scale, cell r covers [r - 1/2, r + 1/2).
+//   MSE (values and MSE keys): a 32-bit entry per cell, the fp32 offset
+//     f = bnd - r of the boundary (1.0 if none) whose 4 low mantissa bits are
+//     replaced by the code of the cell's lower side (base), the value rounded up
+//     so that it never falls below f: code = base + [u - r > f'].  Stored once
+//     per lane (32 copies, interleaved: byte offset = cell * 128 + lane * 4), so
+//     a warp's 32 lookups never share a bank.
+//   Product keys: a 16-byte entry {float bnd; int base; float c_lo; float c_hi}
+//     (bnd = +inf if none; levels in cell units), one read gives the code and its
+//     level: code = base + [u > bnd].  Stored once per 8 lanes (byte offset =
+//     cell * 128 + (lane % 8) * 16), so a quarter-warp phase never shares a bank.
+constexpr int kLutCellsMse = 256;
+constexpr int kLutCellsProd = 128;
+constexpr int kLutReplMse = 32;
 constexpr int kLutReplProd = 8;
-constexpr int kLutBytesMse = kLutCellsMse * 8 * kLutReplMse;
+constexpr int kLutBytesMse = kLutCellsMse * 4 * kLutReplMse;
 constexpr int kLutBytesProd = kLutCellsProd * 16 * kLutReplProd;
 
 // u = v * scale; cell = bits(u + magic) - bits(1.5 * 2^23), magic = 1.5 * 2^23 + cells / 2

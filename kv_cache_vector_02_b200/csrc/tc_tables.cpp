@@ -73,33 +73,42 @@ bool build_lut(const std::vector<double>& t, const std::vector<double>& c, int c
         lp.magic = float(12582912.0 + cells / 2);
         const int L = int(c.size());
         for (int cell = 0; cell < cells; ++cell) {
-            // cell covers u in [cell - cells/2 - 0.5, cell - cells/2 + 0.5)
-            const double ulo = cell - cells / 2 - 0.5, uhi = ulo + 1.0;
+            // cell covers u in [r - 0.5, r + 0.5), r = cell - cells/2
+            const int r = cell - cells / 2;
             int base = 0;
-            float bnd = INFINITY;
+            float bnd = INFINITY;  // the boundary inside the cell, as the kernel compares it
             for (double tk : t) {
-                const double u = double(float(tk)) * double(scale);
-                if (u < ulo) ++base;
-                else if (u < uhi) bnd = float(tk * double(scale));
+                const float ub = float(tk * double(scale));
+                if (double(ub) < r - 0.5) ++base;
+                else if (double(ub) < r + 0.5) bnd = ub;
             }
             if (base > L - 1) base = L - 1;
             if (prod) {
                 const float clo = float(c[base] * double(scale));
                 const float chi = float(c[base + 1 < L ? base + 1 : base] * double(scale));
-                for (int r = 0; r < kLutReplProd; ++r) {
-                    uint8_t* e = dst + 128 * cell + 16 * r;
+                for (int l = 0; l < kLutReplProd; ++l) {
+                    uint8_t* e = dst + 128 * cell + 16 * l;
                     std::memcpy(e + 0, &bnd, 4);
                     std::memcpy(e + 4, &base, 4);
                     std::memcpy(e + 8, &clo, 4);
                     std::memcpy(e + 12, &chi, 4);
                 }
-            } else {
-                for (int r = 0; r < kLutReplMse; ++r) {
-                    uint8_t* e = dst + 128 * cell + 8 * r;
-                    std::memcpy(e + 0, &bnd, 4);
-                    std::memcpy(e + 4, &base, 4);
-                }
+                continue;
             }
+            // offset in the cell (exact: |bnd - r| < 1/2); none: 1.0 > any u - r
+            const float f = std::isfinite(bnd) ? bnd - float(r) : 1.0f;
+            // the smallest float >= f whose 4 low mantissa bits are base
+            uint32_t fb;
+            std::memcpy(&fb, &f, 4);
+            float best = INFINITY;
+            for (int k = -2; k <= 2; ++k) {
+                const uint32_t cand = uint32_t(int64_t(fb & ~15u) + 16 * k) | uint32_t(base);
+                float cf;
+                std::memcpy(&cf, &cand, 4);
+                if (std::isfinite(cf) && cf >= f && cf < best && std::signbit(cf) == std::signbit(f)) best = cf;
+            }
+            if (!std::isfinite(best)) return false;
+            for (int l = 0; l < kLutReplMse; ++l) std::memcpy(dst + 128 * cell + 4 * l, &best, 4);
         }
         return true;
     }
