@@ -372,9 +372,16 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
         // slot of this thread's row of a tile, and the row's destination: the chunk
         // pointer with the row inside the page in its low 4 bits (chunks are
         // 16-byte aligned), or null
+        // row vi = tile * 128 + row is (token vi / H, head vi % H); when H divides 128
+        // a tile holds 128 / H whole tokens and this thread's token offset and head
+        // are the same in every tile
+        const bool hdiv = (128 % a.H) == 0;
+        const int tok_per_tile = hdiv ? 128 / a.H : 0;
+        const int row_tok = hdiv ? row / a.H : 0, row_head = hdiv ? row % a.H : 0;
+        auto token_of = [&](int tile, int vi) -> int { return hdiv ? tile * tok_per_tile + row_tok : vi / a.H; };
         auto slot_of = [&](int tile) -> int {
             const int vi = tile * 128 + row;
-            return vi < a.N ? __ldg(a.slots + vi / a.H) : -1;
+            return vi < a.N ? __ldg(a.slots + token_of(tile, vi)) : -1;
         };
         auto dest = [&](int tile, int slot) -> uint8_t* {
             const int vi = tile * 128 + row;
@@ -383,8 +390,8 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 atomicOr(a.err, TQ_DEVERR_SLOT);
                 return nullptr;
             }
-            const int head = vi % a.H;
-            return a.cache + ((size_t)(slot / kPage) * a.H + head) * (size_t)a.lay.bytes + (size_t)(slot % kPage);
+            const int head = hdiv ? row_head : vi % a.H;
+            return a.cache + ((size_t)(slot >> 4) * a.H + head) * (size_t)a.lay.bytes + (size_t)(slot & (kPage - 1));
         };
         // codes of columns [32 q, 32 q + 32) of the row
         auto store_codes = [&](uint8_t* d, int q, const uint32_t (&w)[kQW]) {
