@@ -157,6 +157,14 @@ __global__ void __launch_bounds__(kPrepThreads) decode_prep_kernel(DecodeArgs a)
     }
 }
 
+// Transpose of an 8x8 fp16 matrix held as m8n8 fragments (thread 4 g + c holds row g,
+// columns 2c, 2c + 1): afterwards it holds row g of the transpose.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t h2bits(__half lo, __half hi) {
     return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
 }
@@ -314,7 +322,6 @@ template <int KM, int VM, bool PROD, int NT>
 struct SplitCtx {
     uint32_t klo0, klo1, khi0, khi1;
     const uint8_t* smem;
-    __half* pt;
     int lane, lane4, g, c;
 };
 
@@ -328,8 +335,9 @@ __device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, 
     const bool valid0 = g < ntok, valid1 = g + 8 < ntok;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-        // ---- scores: 8 K-steps of 16 coordinates
-        float d1[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- scores: 8 K-steps of 16 coordinates, even and odd K-steps in separate
+        // accumulators (two independent MMA chains)
+        float d1[2][4] = {}, d2[2][4] = {};
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
             uint32_t ak[2][2];  // [row g / g+8][coords (4ks,4ks+1) / (4ks+2,4ks+3)]
@@ -366,13 +374,13 @@ __device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, 
                     ak[i][1] = e.y;
                 }
             }
-            mma16816(d1, ak[0][0], ak[1][0], ak[0][1], ak[1][1], bq[nt][ks][0], bq[nt][ks][1]);
+            mma16816(d1[ks & 1], ak[0][0], ak[1][0], ak[0][1], ak[1][1], bq[nt][ks][0], bq[nt][ks][1]);
             if (PROD) {
                 const uint32_t oa = nib_off8<0>(cur.s[0] >> (4 * ks));
                 const uint32_t ob = nib_off8<0>(cur.s[1] >> (4 * ks));
                 const uint2 s0 = *reinterpret_cast<const uint2*>(x.smem + L::kOffS + oa);
                 const uint2 s1 = *reinterpret_cast<const uint2*>(x.smem + L::kOffS + ob);
-                mma16816(d2, s0.x, s1.x, s0.y, s1.y, bs[nt][ks][0], bs[nt][ks][1]);
+                mma16816(d2[ks & 1], s0.x, s1.x, s0.y, s1.y, bs[nt][ks][0], bs[nt][ks][1]);
             }
         }
         // ---- base-2 logits of tokens g, g+8 for heads nt*8 + 2c + e
@@ -381,58 +389,48 @@ __device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, 
         for (int i = 0; i < 2; ++i)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                float s = cur.kn[i] * d1[2 * i + e];
-                if (PROD) s = fmaf(cur.kg[i], d2[2 * i + e], s);
+                float s = cur.kn[i] * (d1[0][2 * i + e] + d1[1][2 * i + e]);
+                if (PROD) s = fmaf(cur.kg[i], d2[0][2 * i + e] + d2[1][2 * i + e], s);
                 sc[i][e] = (i == 0 ? valid0 : valid1) ? s : -INFINITY;
             }
+        // Lazy maximum: each lane checks its own two logits per column against
+        // m + kSlack; only when one exceeds it is the page maximum reduced over the
+        // column's lanes and the state rescaled.  l holds this lane's partial sum
+        // (its rows), reduced over the column's lanes once per item.
         float pw[2][2];
-        bool need = false;
-        float mnew[2];
+        bool over = false;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            float mx = fmaxf(sc[0][e], sc[1][e]);
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-            const bool up = mx > m[nt][e] + kSlack;
-            mnew[e] = up ? mx : m[nt][e];
-            need |= up;
-        }
-        if (__any_sync(0xffffffffu, need)) {
+        for (int e = 0; e < 2; ++e) over |= fmaxf(sc[0][e], sc[1][e]) > m[nt][e] + kSlack;
+        if (__any_sync(0xffffffffu, over)) {
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const float corr = exp2f(m[nt][e] - mnew[e]);  // 1 when unchanged, 0 from -inf
+                float mx = fmaxf(sc[0][e], sc[1][e]);
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                const float mnew = mx > m[nt][e] + kSlack ? mx : m[nt][e];
+                const float corr = exp2f(m[nt][e] - mnew);  // 1 when unchanged, 0 from -inf
                 l[nt][e] *= corr;
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
                     acc[nt][mt][e] *= corr;
                     acc[nt][mt][2 + e] *= corr;
                 }
-                m[nt][e] = mnew[e];
+                m[nt][e] = mnew;
             }
         }
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const float p0v = exp2f(sc[0][e] - m[nt][e]), p1v = exp2f(sc[1][e] - m[nt][e]);
-            float ps = p0v + p1v;
-            ps += __shfl_xor_sync(0xffffffffu, ps, 4);
-            ps += __shfl_xor_sync(0xffffffffu, ps, 8);
-            ps += __shfl_xor_sync(0xffffffffu, ps, 16);
-            l[nt][e] += ps;
+            l[nt][e] += p0v + p1v;
             pw[0][e] = valid0 ? p0v * cur.vn[0] : 0.f;
             pw[1][e] = valid1 ? p1v * cur.vn[1] : 0.f;
         }
-        // ---- P' to the B-operand layout through shared memory: ptn[head][token]
-        __half* ptn = x.pt + nt * 8 * 16;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            ptn[(2 * c + e) * 16 + g] = __float2half_rn(pw[0][e]);
-            ptn[(2 * c + e) * 16 + g + 8] = __float2half_rn(pw[1][e]);
-        }
-        __syncwarp();
-        const uint32_t pb0 = *reinterpret_cast<const uint32_t*>(ptn + g * 16 + 2 * c);
-        const uint32_t pb1 = *reinterpret_cast<const uint32_t*>(ptn + g * 16 + 2 * c + 8);
-        __syncwarp();
+        // ---- P' to the B-operand layout: each 8-token half of the C fragment
+        // (token row g, heads 2c, 2c + 1) transposed in registers to (tokens 2c,
+        // 2c + 1, head g)
+        const uint32_t pb0 = movmatrix_trans(h2bits(__float2half_rn(pw[0][0]), __float2half_rn(pw[0][1])));
+        const uint32_t pb1 = movmatrix_trans(h2bits(__float2half_rn(pw[1][0]), __float2half_rn(pw[1][1])));
         // ---- values: m-tile mt, row g -> coord 16g + 2mt (nibbles), row g+8 -> +1
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
@@ -490,7 +488,6 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
     build_tables<KM, VM, PROD>(smem, a);
     SplitCtx<KM, VM, PROD, NT> x{};
     x.smem = smem;
-    x.pt = reinterpret_cast<__half*>(smem + L::kOffP) + warp * 2 * 8 * 16;
     x.lane = lane;
     x.lane4 = lane << 2;
     x.g = g;
@@ -650,6 +647,14 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
         }
 
         // ---- merge the warps of the CTA (coordinates back in natural order)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {  // l over the column's lanes
+                l[nt][e] += __shfl_xor_sync(0xffffffffu, l[nt][e], 4);
+                l[nt][e] += __shfl_xor_sync(0xffffffffu, l[nt][e], 8);
+                l[nt][e] += __shfl_xor_sync(0xffffffffu, l[nt][e], 16);
+            }
         __syncthreads();
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
