@@ -697,14 +697,15 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
 }
 
 // ------------------------------------------------------------------ merge
-// Persistent: CTA i takes the (unit, group of kMergeHeads heads) items
-// i * kMergeItems .. + kMergeItems - 1, then + grid * kMergeItems, ...; 128 threads
-// per item, thread = coordinate, computing all the group's heads so that each
-// element of R is read once per item.  R^T is staged once per CTA (while the split
+// Persistent: with n = blockDim.x / 128 items per CTA (chosen at launch so that
+// the CTAs cover the SMs), CTA i takes the (unit, group of kMergeHeads heads)
+// items i n .. i n + n - 1, then + grid n, ...; 128 threads per item, thread =
+// coordinate, computing all the group's heads so that each element of R is read
+// once per item.  R^T is staged once per CTA (while the split
 // kernel runs).  Unit u's pieces sit in slots u + c for the split CTAs c whose
 // page range meets it: c(p) = ((p + 1) grid - 1) / total is the CTA of page p.
 constexpr int kMergeHeads = 4;
-constexpr int kMergeItems = 4;
+constexpr int kMergeItems = 4;  // most items per CTA
 constexpr int kMergeThreads = kDim * kMergeItems;
 __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs a) {
     extern __shared__ __align__(16) float sm[];  // RT [128*128] | orot [items][128][kMergeHeads]
@@ -721,7 +722,8 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs 
     const long grid = a.split_grid;
     const int groups = (a.G + kMergeHeads - 1) / kMergeHeads;
     const int items = a.B * a.Hkv * groups;
-    for (int base = blockIdx.x * kMergeItems; base < items; base += gridDim.x * kMergeItems) {
+    const int ipc = (int)blockDim.x / kDim;
+    for (int base = blockIdx.x * ipc; base < items; base += gridDim.x * ipc) {
         const int item = base + il;
         const bool live = item < items;
         int unit = 0, h0 = 0, c_lo = 0, c_hi = -1;
@@ -922,12 +924,16 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
 #undef TQ_DEC_CASE
     if (e != cudaSuccess) return e;
     const int mitems = B * Hkv * ((a.G + kMergeHeads - 1) / kMergeHeads);
-    const int mctas = (mitems + kMergeItems - 1) / kMergeItems;
+    // items per CTA: as few as keep the CTAs within one per SM (at most kMergeItems)
+    int ipc = (mitems + ctx->sm_count - 1) / ctx->sm_count;
+    ipc = ipc < 1 ? 1 : (ipc > kMergeItems ? kMergeItems : ipc);
+    const int mctas = (mitems + ipc - 1) / ipc;
     const dim3 mgrid(mctas < ctx->sm_count ? mctas : ctx->sm_count);
-    const size_t msmem = sizeof(float) * (kDim * kDim + kDim * kMergeHeads * kMergeItems);
-    e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+    const size_t msmem = sizeof(float) * (kDim * kDim + kDim * kMergeHeads * ipc);
+    e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(sizeof(float) * (kDim * kDim + kDim * kMergeHeads * kMergeItems)));
     if (e != cudaSuccess) return e;
-    e = launch_dependent(decode_merge_kernel, mgrid, dim3(kMergeThreads), msmem, stream, a);
+    e = launch_dependent(decode_merge_kernel, mgrid, dim3(kDim * ipc), msmem, stream, a);
     if (e != cudaSuccess) return e;
     count_launches(3);
     return cudaGetLastError();
