@@ -202,6 +202,11 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
         mbar_init(bar(kBarDrain), 1);
         *abort = 0;
         fence_mbar_init();
+        // the operand images and the table (set up by tq_init, not by the kernel before)
+        mbar_arrive_expect_tx(bar(kBarConst), C::kImages * kTile + C::kLutBytes);
+        for (int i = 0; i < C::kImages; ++i)
+            bulk_g2s(sbase + C::kOffImg + i * kTile, a.images + (size_t)i * kTile, kTile, bar(kBarConst));
+        bulk_g2s(sbase + C::kOffLut, a.lut, C::kLutBytes, bar(kBarConst));
     }
     if (warp == C::kWarpMma) {
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
@@ -211,14 +216,12 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    griddep_wait();  // the inputs, the slot mapping and the cache may come from the kernel before
+    griddep_launch_dependents();
 
     if (warp == C::kWarpProducer) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(bar(kBarConst), C::kImages * kTile + C::kLutBytes);
-            for (int i = 0; i < C::kImages; ++i)
-                bulk_g2s(sbase + C::kOffImg + i * kTile, a.images + (size_t)i * kTile, kTile, bar(kBarConst));
-            bulk_g2s(sbase + C::kOffLut, a.lut, C::kLutBytes, bar(kBarConst));
             int issued = 0;
             for (int k = 0; k < my_tiles; ++k) {
                 const int s = k % C::kStages;
@@ -631,8 +634,19 @@ cudaError_t launch_tc(const CUtensorMap& tmap, const TcArgs& a, int grid, cudaSt
     auto k = compress_tc_kernel<ROT, PROD, W>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
     if (e != cudaSuccess) return e;
-    k<<<grid, C::kThreads, C::kSmem, stream>>>(tmap, a);
-    return cudaGetLastError();
+    // programmatic stream serialization: the setup above griddep_wait overlaps the
+    // end of the kernel before
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, tmap, a);
 }
 
 }  // namespace

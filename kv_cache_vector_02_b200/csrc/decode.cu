@@ -73,11 +73,8 @@ __device__ __forceinline__ bool seq_len_ok(const DecodeArgs& a, int L) {
 }
 
 // ------------------------------------------------------------------ helpers
-// Programmatic dependent launch: a kernel launched with programmatic stream
-// serialization may start before its predecessor ends; it reads nothing that the
-// predecessor (or anything before it) writes until griddep_wait() returns.
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+using sm100::griddep_wait;
+using sm100::griddep_launch_dependents;
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -94,6 +91,7 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // computes output columns 8 (8 y + w) .. +7 of the 256 (q' then s).
 constexpr int kPrepThreads = 256;
 __global__ void __launch_bounds__(kPrepThreads) decode_prep_kernel(DecodeArgs a) {
+    griddep_wait();  // q and seq_lens may come from the kernel before
     const int NQ = a.B * a.Hq;
     const int h0 = blockIdx.x * 16;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
@@ -904,13 +902,14 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
     a.out_fp32 = out_fp32;
     a.err = ctx->dev_error;
 
-    decode_prep_kernel<<<dim3((B * Hq + 15) / 16, 4), kPrepThreads, 0, stream>>>(a);
+    cudaError_t e = launch_dependent(decode_prep_kernel, dim3((B * Hq + 15) / 16, 4), dim3(kPrepThreads), 0, stream, a);
+    if (e != cudaSuccess) return e;
     const int KM = kmode_of(ctx);
     const int VM = ctx->cb_value.width == 4 ? kVByte4 : kVByte2;
     const bool prod = ctx->lay_key.prod;
     const int NT = a.G <= 8 ? 1 : 2;
     const int grid = plan.grid;
-    cudaError_t e = cudaErrorInvalidValue;
+    e = cudaErrorInvalidValue;
 #define TQ_DEC_CASE(K_, V_, P_, N_) \
     if (KM == K_ && VM == V_ && prod == P_ && NT == N_) e = launch_split<K_, V_, P_, N_>(a, grid, stream);
 #define TQ_DEC_NT(K_, V_, P_) TQ_DEC_CASE(K_, V_, P_, 1) TQ_DEC_CASE(K_, V_, P_, 2)

@@ -92,6 +92,15 @@ __device__ __forceinline__ void mbar_arrive_warp(uint32_t bar) {
     if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start before its
+// predecessor in the stream ends; it reads nothing that the predecessor (or
+// anything before it) writes until griddep_wait() returns.  griddep_launch_dependents()
+// lets the next such kernel start launching.  Both are no-ops without the launch
+// attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- proxies
 __device__ __forceinline__ void fence_proxy_async_shared() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
