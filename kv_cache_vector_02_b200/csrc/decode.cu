@@ -25,6 +25,7 @@
 //          are contiguous packed bytes.  The warps of a CTA merge their states;
 //          each item's partial (m, l, acc) goes to the workspace.
 //   merge  log-sum-exp combination of the splits, division by l, un-rotation.
+#include <algorithm>
 #include <cmath>
 #include <mutex>
 
@@ -56,6 +57,7 @@ struct DecodeArgs {
     float* partial;    // [slots][G][130]: m, l, acc (rotated domain)
     int* prefix;       // [B + 1] pages of the sequences before b (prep writes it)
     int split_grid;    // CTAs of the split kernel
+    int merge_sg;      // merge: groups of 128 threads per item, each on every merge_sg-th slot
     const float* RT;       // row-major R^T (fp32)
     const uint16_t* RTh;   // fp16 R^T hi / lo, S (row-major)
     const uint16_t* RTl;
@@ -695,21 +697,35 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
 }
 
 // ------------------------------------------------------------------ merge
-// Persistent: with n = blockDim.x / 128 items per CTA (chosen at launch so that
-// the CTAs cover the SMs), CTA i takes the (unit, group of kMergeHeads heads)
-// items i n .. i n + n - 1, then + grid n, ...; 128 threads per item, thread =
-// coordinate, computing all the group's heads so that each element of R is read
-// once per item.  R^T is staged once per CTA (while the split
+// Persistent: with n items per CTA (chosen at launch so that the CTAs cover the
+// SMs), CTA i takes the (unit, group of kMergeHeads heads) items i n .. i n + n - 1,
+// then + grid n, ...; thread = coordinate, computing all the group's heads so that
+// each element of R is read once per item.  An item has sg groups of 128 threads
+// (sg > 1 when a unit spans many split CTAs, as in one long sequence): group g
+// folds every sg-th slot from the g-th, and the first group combines the sg
+// partial states and un-rotates.  R^T is staged once per CTA (while the split
 // kernel runs).  Unit u's pieces sit in slots u + c for the split CTAs c whose
 // page range meets it: c(p) = ((p + 1) grid - 1) / total is the CTA of page p.
 constexpr int kMergeHeads = 4;
 constexpr int kMergeItems = 4;  // most items per CTA
-constexpr int kMergeThreads = kDim * kMergeItems;
+constexpr int kMergeGroups = 8; // most slot groups per item
+constexpr int kMergeThreads = 1024;
+size_t merge_smem(int ipc, int sg) {
+    return sizeof(float) * (kDim * kDim + (size_t)ipc * kDim * kMergeHeads +
+                            (sg > 1 ? (size_t)ipc * sg * (kDim * kMergeHeads + 2 * kMergeHeads) : 0));
+}
 __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs a) {
-    extern __shared__ __align__(16) float sm[];  // RT [128*128] | orot [items][128][kMergeHeads]
-    const int i = threadIdx.x % kDim, il = threadIdx.x / kDim;
+    // RT [128*128] | orot [items][128][kMergeHeads] | group states A [items][sg][128][kMergeHeads],
+    // (M, L) [items][sg][kMergeHeads][2]
+    extern __shared__ __align__(16) float sm[];
+    const int sg = a.merge_sg;
+    const int ipc = (int)blockDim.x / (kDim * sg);
+    const int i = threadIdx.x % kDim, gi = (threadIdx.x / kDim) % sg, il = threadIdx.x / (kDim * sg);
     float* rts = sm;
     float4* orot = reinterpret_cast<float4*>(sm + kDim * kDim) + il * kDim;  // this item's [j] of 4 heads
+    float4* gA = reinterpret_cast<float4*>(sm + kDim * kDim + ipc * kDim * kMergeHeads) + (il * sg) * kDim;
+    float* gML = sm + kDim * kDim + ipc * kDim * kMergeHeads + ipc * sg * kDim * kMergeHeads +
+                 (il * sg) * 2 * kMergeHeads;
     {
         const float4* src = reinterpret_cast<const float4*>(a.RT);
         float4* dst = reinterpret_cast<float4*>(rts);
@@ -720,7 +736,6 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs 
     const long grid = a.split_grid;
     const int groups = (a.G + kMergeHeads - 1) / kMergeHeads;
     const int items = a.B * a.Hkv * groups;
-    const int ipc = (int)blockDim.x / kDim;
     for (int base = blockIdx.x * ipc; base < items; base += gridDim.x * ipc) {
         const int item = base + il;
         const bool live = item < items;
@@ -743,7 +758,7 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs 
         for (int e = 0; e < kMergeHeads; ++e) M[e] = -INFINITY, Lsum[e] = 0.f, A[e] = 0.f;
         const int nh = a.G - h0 < kMergeHeads ? a.G - h0 : kMergeHeads;
 #pragma unroll 4
-        for (int c = c_lo; c <= c_hi; ++c) {
+        for (int c = c_lo + gi; c <= c_hi; c += sg) {
             const float* pp = a.partial + (((size_t)unit + c) * a.G + h0) * kPartStride;
             float ms[kMergeHeads], ls[kMergeHeads], as[kMergeHeads];
 #pragma unroll
@@ -763,13 +778,37 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs 
                 M[e] = mn;
             }
         }
+        __syncthreads();  // the previous items' un-rotation is done with orot and the group states
+        if (sg > 1) {  // the first group combines the groups' states
+            if (i == 0)
+#pragma unroll
+                for (int e = 0; e < kMergeHeads; ++e) gML[gi * 2 * kMergeHeads + 2 * e] = M[e], gML[gi * 2 * kMergeHeads + 2 * e + 1] = Lsum[e];
+            gA[gi * kDim + i] = make_float4(A[0], A[1], A[2], A[3]);
+            __syncthreads();
+            if (gi == 0) {
+#pragma unroll
+                for (int e = 0; e < kMergeHeads; ++e) {
+                    float Mx = -INFINITY;
+                    for (int g = 0; g < sg; ++g) Mx = fmaxf(Mx, gML[g * 2 * kMergeHeads + 2 * e]);
+                    float L2 = 0.f, A2 = 0.f;
+                    for (int g = 0; g < sg; ++g) {
+                        const float mg = gML[g * 2 * kMergeHeads + 2 * e];
+                        if (mg == -INFINITY) continue;
+                        const float w = exp2f(mg - Mx);
+                        const float4 ag = gA[g * kDim + i];
+                        L2 = fmaf(gML[g * 2 * kMergeHeads + 2 * e + 1], w, L2);
+                        A2 = fmaf(e == 0 ? ag.x : e == 1 ? ag.y : e == 2 ? ag.z : ag.w, w, A2);
+                    }
+                    M[e] = Mx, Lsum[e] = L2, A[e] = A2;
+                }
+            }
+        }
         float o[kMergeHeads];
 #pragma unroll
         for (int e = 0; e < kMergeHeads; ++e) o[e] = (live && Lsum[e] > 0.f) ? A[e] / Lsum[e] : 0.f;
-        __syncthreads();  // the previous items' un-rotation is done with orot
-        orot[i] = make_float4(o[0], o[1], o[2], o[3]);
+        if (gi == 0) orot[i] = make_float4(o[0], o[1], o[2], o[3]);
         __syncthreads();
-        if (!live) continue;
+        if (!live || gi != 0) continue;
         float y[kMergeHeads] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
         for (int j = 0; j < kDim; ++j) {  // o_i = sum_j R[i][j] orot_j, for the 4 heads at once
@@ -923,16 +962,27 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
 #undef TQ_DEC_CASE
     if (e != cudaSuccess) return e;
     const int mitems = B * Hkv * ((a.G + kMergeHeads - 1) / kMergeHeads);
-    // items per CTA: as few as keep the CTAs within one per SM (at most kMergeItems)
-    int ipc = (mitems + ctx->sm_count - 1) / ctx->sm_count;
-    ipc = ipc < 1 ? 1 : (ipc > kMergeItems ? kMergeItems : ipc);
+    // slot groups per item: a unit of the longest sequence meets about grid / units
+    // + 1 split CTAs when all sequences are that long; one group per 4 such slots
+    const long units = (long)B * Hkv;
+    const long est_slots = units > 0 ? (grid + units - 1) / units + 1 : 1;
+    int sg = (int)(est_slots / 4);
+    sg = sg < 1 ? 1 : (sg > kMergeGroups ? kMergeGroups : sg);
+    // items per CTA: as few as keep the CTAs within one per SM (at most kMergeItems; one
+    // when an item has several groups)
+    int ipc = 1;
+    if (sg == 1) {
+        ipc = (mitems + ctx->sm_count - 1) / ctx->sm_count;
+        ipc = ipc < 1 ? 1 : (ipc > kMergeItems ? kMergeItems : ipc);
+    }
+    a.merge_sg = sg;
     const int mctas = (mitems + ipc - 1) / ipc;
     const dim3 mgrid(mctas < ctx->sm_count ? mctas : ctx->sm_count);
-    const size_t msmem = sizeof(float) * (kDim * kDim + kDim * kMergeHeads * ipc);
+    const size_t msmem = merge_smem(ipc, sg);
     e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(sizeof(float) * (kDim * kDim + kDim * kMergeHeads * kMergeItems)));
+                             (int)std::max(merge_smem(kMergeItems, 1), merge_smem(1, kMergeGroups)));
     if (e != cudaSuccess) return e;
-    e = launch_dependent(decode_merge_kernel, mgrid, dim3(kDim * ipc), msmem, stream, a);
+    e = launch_dependent(decode_merge_kernel, mgrid, dim3(kDim * ipc * sg), msmem, stream, a);
     if (e != cudaSuccess) return e;
     count_launches(3);
     return cudaGetLastError();
