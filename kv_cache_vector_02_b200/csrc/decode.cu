@@ -731,26 +731,34 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs 
         float4* dst = reinterpret_cast<float4*>(rts);
         for (int k = threadIdx.x; k < kDim * kDim / 4; k += blockDim.x) dst[k] = src[k];
     }
-    griddep_wait();  // the split partials
+    // The items' units and slot ranges depend on the page prefix sums only, which the
+    // prep kernel wrote before the split kernel could start (and so before this
+    // kernel was launched): they are read before waiting for the split partials.
     const long total = (long)a.Hkv * a.prefix[a.B];
     const long grid = a.split_grid;
     const int groups = (a.G + kMergeHeads - 1) / kMergeHeads;
     const int items = a.B * a.Hkv * groups;
+    auto item_info = [&](int item, int& unit, int& h0, int& c_lo, int& c_hi) {
+        unit = 0, h0 = 0, c_lo = 0, c_hi = -1;
+        if (item >= items) return;
+        unit = item / groups;
+        h0 = (item - unit * groups) * kMergeHeads;
+        const int b = unit / a.Hkv, hk = unit - b * a.Hkv;
+        const int np = a.prefix[b + 1] - a.prefix[b];
+        if (np > 0) {
+            const long first = (long)a.Hkv * a.prefix[b] + (long)hk * np, last = first + np - 1;
+            c_lo = (int)(((first + 1) * grid - 1) / total);
+            c_hi = (int)(((last + 1) * grid - 1) / total);
+        }
+    };
+    int n_unit, n_h0, n_clo, n_chi;  // the first item's
+    item_info(blockIdx.x * ipc + il, n_unit, n_h0, n_clo, n_chi);
+    griddep_wait();  // the split partials
     for (int base = blockIdx.x * ipc; base < items; base += gridDim.x * ipc) {
         const int item = base + il;
         const bool live = item < items;
-        int unit = 0, h0 = 0, c_lo = 0, c_hi = -1;
-        if (live) {
-            unit = item / groups;
-            h0 = (item - unit * groups) * kMergeHeads;
-            const int b = unit / a.Hkv, hk = unit - b * a.Hkv;
-            const int np = a.prefix[b + 1] - a.prefix[b];
-            if (np > 0) {
-                const long first = (long)a.Hkv * a.prefix[b] + (long)hk * np, last = first + np - 1;
-                c_lo = (int)(((first + 1) * grid - 1) / total);
-                c_hi = (int)(((last + 1) * grid - 1) / total);
-            }
-        }
+        int unit = n_unit, h0 = n_h0, c_lo = n_clo, c_hi = n_chi;
+        if (base + gridDim.x * ipc < items) item_info(item + gridDim.x * ipc, n_unit, n_h0, n_clo, n_chi);
         // online log-sum-exp over the slots, all heads at once: the loads of several
         // slots are in flight together
         float M[kMergeHeads], Lsum[kMergeHeads], A[kMergeHeads];
