@@ -231,7 +231,6 @@ __device__ __forceinline__ void load_page(PageRegs<KM, VM, PROD>& r, const uint8
 //   K    key byte table (same layouts) when keys are not byte-permuted
 //   S    sign nibble table [16] 2 x half2 of +-1 (bit set -> +1)
 //   K1   1-bit key nibble table [16] 2 x half2 of c[bit]
-//   P    per warp P' transpose [2 n-tiles][8 heads][16 tokens] fp16
 //   M    per warp m[16], l[16]
 //   Bar  per warp kStagesD mbarriers of the page ring
 //   Ring per warp kStagesD stages of one page (key chunk, then value chunk), filled
@@ -248,8 +247,7 @@ struct SmemLayout {
     static constexpr uint32_t kOffK = kOffV + kTabBytes;
     static constexpr uint32_t kOffS = kOffK + (kKTab ? kTabBytes : 0);
     static constexpr uint32_t kOffK1 = kOffS + 128;
-    static constexpr uint32_t kOffP = kOffK1 + 128;
-    static constexpr uint32_t kOffM = kOffP + kWarps * 2 * 8 * 16 * 2;
+    static constexpr uint32_t kOffM = kOffK1 + 128;
     static constexpr uint32_t kOffBar = kOffM + kWarps * 2 * kMaxG * 4;
     static constexpr uint32_t kOffRing = (kOffBar + kWarps * kStagesD * 8 + 127) & ~127u;
     static constexpr uint32_t kRingBytes = kWarps * kStagesD * kStageBytes;
