@@ -58,11 +58,11 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kSmemMax = 232448;
 
 // TMEM (512 columns): buffer t holds team t's tile.  Values: 128-column
-// accumulators at 128 t.  Keys: at 256 t the rotation accumulators A [0,128) and
-// B [128,256); A is then reused for rho: the 16 coordinates of K-step st
-// (A columns [16 st, 16 st + 16)) become 8 columns of rho_hi pairs followed by 8
-// of rho_lo pairs, written by the thread that has just read those A columns, and
-// the sketch accumulates over B.
+// accumulators at 128 t.  Keys: at 256 t the rotation accumulator A [0,128) and
+// the sketch accumulator B [128,256); A is reused for rho: the 16 coordinates of
+// K-step st (A columns [16 st, 16 st + 16)) become 8 columns of rho_hi pairs
+// followed by 8 of rho_lo pairs, written by the thread that has just read those
+// A columns.
 constexpr uint32_t kColB = 128;
 
 template <int ROT, bool PROD>
@@ -162,11 +162,6 @@ __device__ __forceinline__ void sq_acc2(uint32_t w, float& s0, float& s1) {
         : "r"(w));
 }
 
-__device__ __forceinline__ float2 ld_sum(const uint32_t (&r0)[32], const uint32_t (&r1)[32], int i) {
-    return __fadd2_rn(make_float2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1])),
-                      make_float2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1])));
-}
-
 template <int ROT, bool PROD, int W>
 __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs a) {
     using C = Cfg<ROT, PROD>;
@@ -264,10 +259,10 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 if (!mbar_test_wait(bar(kBarXFull + s), (uint32_t)(k / C::kStages) & 1u)) return false;
                 if (!mbar_test_wait(bar(kBarRotEmpty + t), (use & 1u) ^ 1u)) return false;
                 tc_fence_after();
-                const uint32_t dA = tmem + C::kBufCols * (uint32_t)t, dB = PROD ? dA + kColB : dA;
+                const uint32_t dA = tmem + C::kBufCols * (uint32_t)t;
                 const uint32_t xs = x0 + (uint32_t)s * kTileU;
                 uint32_t accA = 0u;
-                if (ROT == 0) {  // the small lo pass first, then K-steps 0-3 of the hi pass
+                if (ROT == 0) {  // the small lo pass first, then the hi pass
 #pragma unroll
                     for (int st = 0; st < 8; ++st) {
                         umma_ss(dA, kdesc(xs, st), kdesc(img + kTileU, st), idesc, accA);
@@ -275,13 +270,10 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                     }
                 }
 #pragma unroll
-                for (int st = 0; st < 4; ++st) {
+                for (int st = 0; st < 8; ++st) {
                     umma_ss(dA, kdesc(xs, st), kdesc(img, st), idesc, accA);
                     accA = 1u;
                 }
-#pragma unroll
-                for (int st = 4; st < 8; ++st)
-                    umma_ss(dB, kdesc(xs, st), kdesc(img, st), idesc, (PROD && st == 4) ? 0u : 1u);
                 umma_commit(bar(kBarXEmpty + s));
                 umma_commit(bar(kBarRotFull + t));
                 return true;
@@ -463,19 +455,18 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                     break;
                 }
                 tc_fence_after();
-                // ---- ||acc||^2 of the row, acc = A + B
+                // ---- ||acc||^2 of the row
                 float2 q2[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) q2[i] = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    uint32_t r0[32], r1[32];
+                    uint32_t r0[32];
                     tmem_ld32(buf + 32 * c, r0);
-                    tmem_ld32(buf + kColB + 32 * c, r1);
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float2 v = ld_sum(r0, r1, i);
+                        const float2 v = make_float2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
                         q2[i & 3] = __ffma2_rn(v, v, q2[i & 3]);
                     }
                 }
@@ -504,12 +495,11 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 const uint32_t col = buf + 32 * q;
                 float2 av[16];
                 {
-                    uint32_t r0[32], r1[32];
+                    uint32_t r0[32];
                     tmem_ld32(col, r0);
-                    tmem_ld32(col + kColB, r1);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) av[i] = ld_sum(r0, r1, i);
+                    for (int i = 0; i < 16; ++i) av[i] = make_float2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
                 }
                 if (any_bad && !finite) {
 #pragma unroll
