@@ -57,13 +57,13 @@ constexpr uint32_t kHalf = kTile / 2;      // one 128-byte-swizzled K-half
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kSmemMax = 232448;
 
-// TMEM (512 columns): buffer t holds team t's tile.  Values: 128-column
-// accumulators at 128 t.  Keys: at 256 t the rotation accumulator A [0,128) and
-// the sketch accumulator B [128,256); A is reused for rho: the 16 coordinates of
-// K-step st (A columns [16 st, 16 st + 16)) become 8 columns of rho_hi pairs
-// followed by 8 of rho_lo pairs, written by the thread that has just read those
-// A columns.
-constexpr uint32_t kColB = 128;
+// TMEM (512 columns): buffer t (columns [128 t, 128 t + 128)) holds team t's tile.
+// Values: four teams, each buffer a rotation accumulator.  Keys: three teams; the
+// buffer holds the rotation accumulator, then rho: the 16 coordinates of K-step st
+// (columns [16 st, 16 st + 16)) become 8 columns of rho_hi pairs followed by 8 of
+// rho_lo pairs, written by the thread that has just read those columns.  The
+// sketches, issued in tile order, share the accumulator at column kColSketch.
+constexpr uint32_t kColSketch = 384;
 
 template <int ROT, bool PROD>
 struct Cfg {
@@ -83,15 +83,14 @@ struct Cfg {
     static constexpr uint32_t kOffBar = kOffPart + kPartBytes;
     static constexpr uint32_t kSmem = kOffBar + kBarBytes;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr int kTeams = PROD ? 2 : 4;
+    static constexpr int kTeams = PROD ? 3 : 4;
     static constexpr int kEpiWarps = 4 * kTeams;
     static constexpr int kWarpProducer = kEpiWarps;
     static constexpr int kWarpMma = kEpiWarps + 1;
     static constexpr int kThreads = kEpiWarps * 32 + 64;
-    // registers: keys 10 warps, three on the busiest SM sub-partition, 3 x 32 x 168
-    // <= 16384 (the bound of 384 threads gives 168); values 18 warps at 96
-    static constexpr int kBound = PROD ? 384 : kThreads;
-    static constexpr uint32_t kBufCols = PROD ? 256 : 128;
+    // registers: keys 14 warps at 144, values 18 warps at 96
+    static constexpr int kBound = kThreads;
+    static constexpr uint32_t kBufCols = 128;
     static_assert(kStages >= 1, "shared memory budget");
     static_assert(kSmem <= kSmemMax, "shared memory budget");
 };
@@ -103,10 +102,11 @@ enum : int {
     kBarXEmpty = 5,    // +stage (4)
     kBarRotFull = 9,    // +team (4): rotation accumulators ready
     kBarRotEmpty = 13,  // +team (4): the team is done with its buffer
-    kBarRhoFull = 17,   // +team (2): rho written (keys)
-    kBarQjlFull = 19,   // +team (2): sketch ready (keys)
-    kBarDrain = 21,
-    kNumBars = 22
+    kBarRhoFull = 17,   // +team (3): rho written (keys)
+    kBarQjlFull = 20,   // +team (3): sketch ready (keys)
+    kBarSketchEmpty = 23,  // the sketch accumulator has been read (keys)
+    kBarDrain = 24,
+    kNumBars = 25
 };
 
 struct TcArgs {
@@ -194,6 +194,7 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 mbar_init(bar(kBarQjlFull + t), 1);
             }
         }
+        mbar_init(bar(kBarSketchEmpty), kTeamWarps);
         mbar_init(bar(kBarDrain), 1);
         *abort = 0;
         fence_mbar_init();
@@ -278,13 +279,15 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 umma_commit(bar(kBarRotFull + t));
                 return true;
             };
-            // sketch of local tile k (keys); false when its rho is not written yet
+            // sketch of local tile k (keys); false when its rho is not written yet or
+            // the sketch of tile k - 1 has not been read
             auto try_qjl = [&](int k) -> bool {
-                const int t = k & 1;
-                if (!mbar_test_wait(bar(kBarRhoFull + t), (uint32_t)(k >> 1) & 1u)) return false;
+                const int t = k % C::kTeams;
+                if (!mbar_test_wait(bar(kBarRhoFull + t), (uint32_t)(k / C::kTeams) & 1u)) return false;
+                if (!mbar_test_wait(bar(kBarSketchEmpty), ((uint32_t)k & 1u) ^ 1u)) return false;
                 tc_fence_after();
                 const uint32_t buf = tmem + C::kBufCols * (uint32_t)t;
-                const uint32_t d = buf + kColB;
+                const uint32_t d = tmem + kColSketch;
                 const uint32_t m0 = img + C::kRotImages * kTileU;
                 // rho of K-step st: columns 16 st (hi pairs) and 16 st + 8 (lo pairs)
                 auto rho_col = [&](int st) { return buf + 16u * (uint32_t)st; };
@@ -304,29 +307,22 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 umma_commit(bar(kBarQjlFull + t));
                 return true;
             };
-            // Rotations go in tile order (the stage ring); each team's sketch goes
-            // as soon as its rho is in.  Polls with a bound on time without progress.
-            int next_rot = 0;
-            int qjl_next[2] = {0, 1};
+            // Rotations and sketches each go in tile order.  Polls with a bound on
+            // time without progress.
+            int next_rot = 0, next_qjl = 0;
             uint64_t t_last = globaltimer_ns();
             uint32_t spins = 0;
             while (ok) {
                 bool progress = false;
-                if (PROD) {
-#pragma unroll
-                    for (int t = 0; t < 2; ++t) {
-                        const int k = qjl_next[t];
-                        if (k < next_rot && try_qjl(k)) {
-                            qjl_next[t] = k + 2;
-                            progress = true;
-                        }
-                    }
+                if (PROD && next_qjl < next_rot && try_qjl(next_qjl)) {
+                    ++next_qjl;
+                    progress = true;
                 }
-                if (next_rot < my_tiles && (!PROD || qjl_next[next_rot & 1] >= next_rot - 1) && try_rot(next_rot)) {
+                if (next_rot < my_tiles && try_rot(next_rot)) {
                     ++next_rot;
                     progress = true;
                 }
-                const bool done = next_rot >= my_tiles && (!PROD || (qjl_next[0] >= my_tiles && qjl_next[1] >= my_tiles));
+                const bool done = next_rot >= my_tiles && (!PROD || next_qjl >= my_tiles);
                 if (done) break;
                 if (progress) {
                     spins = 0;
@@ -349,6 +345,7 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
         const int row = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         const uint32_t buf = tmem + lane_addr + C::kBufCols * (uint32_t)team;
+        const uint32_t sketch = tmem + lane_addr + kColSketch;  // keys
         // table entry of u: bits(u + magic) * 128 + lut_off, in this lane's copy
         // (bits(u + magic) = bits(1.5 * 2^23) + cells / 2 + round(u), see tc_params.h)
         const uint32_t lut_off = sbase + C::kOffLut +
@@ -594,12 +591,14 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 set_abort(abort, a.err);
                 break;
             }
+            // the sketch is done with rho: the buffer is free for the team's next rotation
             tc_fence_after();
+            mbar_arrive_warp(bar(kBarRotEmpty + team));
             uint32_t sg[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t q[32];
-                tmem_ld32(buf + kColB + 32 * c, q);
+                tmem_ld32(sketch + 32 * c, q);
                 tmem_ld_wait();
                 uint32_t neg = 0u;  // bit j = sign bit of column 32 c + j
 #pragma unroll
@@ -607,7 +606,7 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 sg[c] = live ? ~neg : 0xffffffffu;
             }
             tc_fence_before();
-            mbar_arrive_warp(bar(kBarRotEmpty + team));
+            mbar_arrive_warp(bar(kBarSketchEmpty));
             store_tail(dst, norm, gamma, sg);
         }
     }
