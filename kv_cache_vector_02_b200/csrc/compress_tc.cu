@@ -65,19 +65,22 @@ constexpr uint32_t kSmemMax = 232448;
 // sketches, issued in tile order, share the accumulator at column kColSketch.
 constexpr uint32_t kColSketch = 384;
 
-template <int ROT, bool PROD>
+template <int ROT, bool PROD, bool PAIR>
 struct Cfg {
     static constexpr int kRotImages = ROT == 0 ? 2 : 1;
     static constexpr int kQjlImages = PROD ? (ROT == 0 ? 2 : 1) : 0;
     static constexpr int kImages = kRotImages + kQjlImages;
+    // this CTA's part of an operand image: all 128 rows, or (pair) 64 of them
+    static constexpr uint32_t kImgBytes = PAIR ? kTile / 2 : kTile;
+    static constexpr uint32_t kImgHalf = kImgBytes / 2;  // K-half stride inside an image
     static constexpr int kLutBytes = PROD ? kLutBytesProd : kLutBytesMse;
     static constexpr uint32_t kPartBytes = 0;
     static constexpr uint32_t kBarBytes = 512;
-    static constexpr uint32_t kFixed = kImages * kTile + kLutBytes + kPartBytes + kBarBytes;
+    static constexpr uint32_t kFixed = kImages * kImgBytes + kLutBytes + kPartBytes + kBarBytes;
     static constexpr int kStagesFit = (int)((kSmemMax - kFixed) / kTile);
     static constexpr int kStages = kStagesFit > 4 ? 4 : kStagesFit;
     static constexpr uint32_t kOffImg = 0;
-    static constexpr uint32_t kOffX = kOffImg + kImages * kTile;
+    static constexpr uint32_t kOffX = kOffImg + kImages * kImgBytes;
     static constexpr uint32_t kOffLut = kOffX + kStages * kTile;
     static constexpr uint32_t kOffPart = kOffLut + kLutBytes;
     static constexpr uint32_t kOffBar = kOffPart + kPartBytes;
@@ -86,9 +89,10 @@ struct Cfg {
     static constexpr int kTeams = PROD ? 3 : 4;
     static constexpr int kEpiWarps = 4 * kTeams;
     static constexpr int kWarpProducer = kEpiWarps;
-    static constexpr int kWarpMma = kEpiWarps + 1;
-    static constexpr int kThreads = kEpiWarps * 32 + 64;
-    // registers: keys 14 warps at 144, values 18 warps at 96
+    static constexpr int kWarpMma = kEpiWarps + 1;     // rotations
+    static constexpr int kWarpSketch = kEpiWarps + 2;  // keys: the sketches, from a second thread
+    static constexpr int kThreads = kEpiWarps * 32 + (PROD ? 96 : 64);
+    // registers: keys 15 warps at 136, values 18 warps at 112
     static constexpr int kBound = kThreads;
     static constexpr uint32_t kBufCols = 128;
     static_assert(kStages >= 1, "shared memory budget");
@@ -105,8 +109,9 @@ enum : int {
     kBarRhoFull = 17,   // +team (3): rho written (keys)
     kBarQjlFull = 20,   // +team (3): sketch ready (keys)
     kBarSketchEmpty = 23,  // the sketch accumulator has been read (keys)
-    kBarDrain = 24,
-    kNumBars = 25
+    kBarDrain = 24,      // +issuer (2): the issuer's MMAs are complete
+    kBarPeerConst = 26,  // pair: the odd CTA's operand images are in (arrived from it)
+    kNumBars = 27
 };
 
 struct TcArgs {
@@ -162,9 +167,9 @@ __device__ __forceinline__ void sq_acc2(uint32_t w, float& s0, float& s1) {
         : "r"(w));
 }
 
-template <int ROT, bool PROD, int W>
-__global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs a) {
-    using C = Cfg<ROT, PROD>;
+template <int ROT, bool PROD, int W, bool PAIR>
+__global__ void __launch_bounds__(Cfg<ROT, PROD, PAIR>::kBound, 1) compress_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs a) {
+    using C = Cfg<ROT, PROD, PAIR>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -176,40 +181,63 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
     auto bar = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + 8 * kNumBars);
     volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffBar + 8 * kNumBars + 4);
-    const int ntiles = (a.N + 127) / 128;
-    const int my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    // Tiles: 128 rows per CTA, or (pair) 256 rows per 2-CTA cluster, the even CTA taking
+    // the first 128; worker u (CTA or cluster) takes tiles u, u + workers, ...
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const bool lead = rank == 0;
+    const int workers = PAIR ? (int)gridDim.x / 2 : (int)gridDim.x;
+    const int uid = PAIR ? (int)blockIdx.x / 2 : (int)blockIdx.x;
+    constexpr int kTileRows = PAIR ? 256 : 128;
+    const int ntiles = (a.N + kTileRows - 1) / kTileRows;
+    const int my_tiles = uid < ntiles ? (ntiles - 1 - uid) / workers + 1 : 0;
+    auto row0_of = [&](int k) -> int { return (uid + k * workers) * kTileRows + (int)rank * 128; };
+    // barriers that the odd CTA of a pair also arrives on count both CTAs' arrivals
+    constexpr int kBoth = PAIR ? 2 : 1;
 
     if (threadIdx.x == 0) {
         mbar_init(bar(kBarConst), 1);
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(bar(kBarXFull + s), 1);
+            // pair: the even CTA's stage is full once its own copy landed and the odd CTA
+            // has reported its copy (an arrival forwarded by its MMA warp)
+            mbar_init(bar(kBarXFull + s), PAIR && lead ? 2 : 1);
             // released by the rotation MMAs and, for values, by the team that reads ||x||
             mbar_init(bar(kBarXEmpty + s), PROD ? 1 : 1 + kTeamWarps);
         }
         for (int t = 0; t < C::kTeams; ++t) {
             mbar_init(bar(kBarRotFull + t), 1);
-            mbar_init(bar(kBarRotEmpty + t), kTeamWarps);
+            mbar_init(bar(kBarRotEmpty + t), kBoth * kTeamWarps);
             if (PROD) {
-                mbar_init(bar(kBarRhoFull + t), kTeamWarps);
+                mbar_init(bar(kBarRhoFull + t), kBoth * kTeamWarps);
                 mbar_init(bar(kBarQjlFull + t), 1);
             }
         }
-        mbar_init(bar(kBarSketchEmpty), kTeamWarps);
+        mbar_init(bar(kBarSketchEmpty), kBoth * kTeamWarps);
         mbar_init(bar(kBarDrain), 1);
+        mbar_init(bar(kBarDrain + 1), 1);
+        mbar_init(bar(kBarPeerConst), 1);
         *abort = 0;
         fence_mbar_init();
-        // the operand images and the table (set up by tq_init, not by the kernel before)
-        mbar_arrive_expect_tx(bar(kBarConst), C::kImages * kTile + C::kLutBytes);
+        // the operand images (pair: this CTA's 64 rows of each K-half) and the table (set
+        // up by tq_init, not by the kernel before)
+        mbar_arrive_expect_tx(bar(kBarConst), C::kImages * C::kImgBytes + C::kLutBytes);
         for (int i = 0; i < C::kImages; ++i)
-            bulk_g2s(sbase + C::kOffImg + i * kTile, a.images + (size_t)i * kTile, kTile, bar(kBarConst));
+            for (int h = 0; h < 2; ++h)
+                bulk_g2s(sbase + C::kOffImg + i * C::kImgBytes + h * C::kImgHalf,
+                         a.images + (size_t)i * kTile + h * kHalf + rank * C::kImgHalf, C::kImgHalf, bar(kBarConst));
         bulk_g2s(sbase + C::kOffLut, a.lut, C::kLutBytes, bar(kBarConst));
     }
     if (warp == C::kWarpMma) {
-        tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();  // both CTAs' barriers are initialised before either signals the other
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     griddep_wait();  // the inputs, the slot mapping and the cache may come from the kernel before
@@ -226,7 +254,7 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                     set_abort(abort, a.err);
                     break;
                 }
-                const int row0 = ((int)blockIdx.x + k * (int)gridDim.x) * 128;
+                const int row0 = row0_of(k);
                 mbar_arrive_expect_tx(bar(kBarXFull + s), kTile);
                 tma_load_2d(sbase + C::kOffX + s * kTile, &tmap, 0, row0, bar(kBarXFull + s));
                 tma_load_2d(sbase + C::kOffX + s * kTile + kHalf, &tmap, 64, row0, bar(kBarXFull + s));
@@ -239,26 +267,74 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 mbar_wait(bar(kBarXFull + k % C::kStages), (uint32_t)(k / C::kStages) & 1u, &never, kWaitNs);
         }
         __syncwarp();
-    } else if (warp == C::kWarpMma) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == C::kWarpMma && PAIR && !lead) {
+        // ------------------------------------------------------------ odd CTA of a pair
+        // Forwards to the even CTA that this CTA's operand images are in and, stage by
+        // stage, that the x tile it loaded is full.
         if (lane == 0) {
-            const uint32_t idesc = idesc_f16(128, 128);
             bool ok = mbar_wait(bar(kBarConst), 0, abort, kWaitNs);
+            if (ok) mbar_arrive_remote(bar(kBarPeerConst), 0);
+            for (int k = 0; ok && k < my_tiles; ++k) {
+                const int s = k % C::kStages;
+                ok = mbar_wait(bar(kBarXFull + s), (uint32_t)(k / C::kStages) & 1u, abort, kWaitNs);
+                if (ok) mbar_arrive_remote(bar(kBarXFull + s), 0);
+            }
+            if (!ok) set_abort(abort, a.err);
+        }
+        __syncwarp();
+    } else if ((warp == C::kWarpMma || (PROD && warp == C::kWarpSketch)) && (!PAIR || lead)) {
+        // ------------------------------------------------------------ MMA issuers
+        // Rotations from one thread, the keys' sketches from another (on another SM
+        // sub-partition), so that neither waits for the other's MMA issue.
+        const bool rot_issuer = warp == C::kWarpMma;
+        if (lane == 0) {
+            // pair: M = 256 (each CTA's 128 rows of x), each CTA holding 64 of the image rows
+            const uint32_t idesc = idesc_f16(PAIR ? 256 : 128, 128);
+            // barriers that the odd CTA also arrives on are tested at cluster scope
+            auto test = [](uint32_t b, uint32_t parity) -> bool {
+                return PAIR ? mbar_test_wait_cluster(b, parity) : mbar_test_wait(b, parity);
+            };
+            bool ok = mbar_wait(bar(kBarConst), 0, abort, kWaitNs);
+            if (PAIR && ok) {  // the odd CTA's images
+                const uint64_t t0 = globaltimer_ns();
+                for (uint32_t it = 0; !test(bar(kBarPeerConst), 0); ++it)
+                    if ((it & 31u) == 31u && (*abort || globaltimer_ns() - t0 > kWaitNs)) {
+                        ok = false;
+                        break;
+                    }
+            }
+            auto mma_ss = [](uint32_t d, uint64_t ad, uint64_t bd, uint32_t id, uint32_t acc) {
+                if (PAIR) umma_ss_pair(d, ad, bd, id, acc);
+                else umma_ss(d, ad, bd, id, acc);
+            };
+            auto mma_ts = [](uint32_t d, uint32_t at, uint64_t bd, uint32_t id, uint32_t acc) {
+                if (PAIR) umma_ts_pair(d, at, bd, id, acc);
+                else umma_ts(d, at, bd, id, acc);
+            };
+            auto commit_both = [](uint32_t b) {  // on this CTA's barrier and (pair) the odd CTA's
+                if (PAIR) umma_commit_pair_both(b);
+                else umma_commit(b);
+            };
             // descriptors as low halves: operand i of the images, stage s of x, and
-            // the offset of K-step st (16 elements) inside a 128x128 operand
+            // the offset of K-step st (16 elements) inside an operand (x: 128 rows, K-halves
+            // 16 KB apart; images: this CTA's rows, K-halves kImgHalf apart)
             constexpr uint32_t kTileU = kTile >> 4;
+            constexpr uint32_t kImgU = C::kImgBytes >> 4;
             const uint32_t img = sw128_desc_lo(sbase + C::kOffImg);
             const uint32_t x0 = sw128_desc_lo(sbase + C::kOffX);
             auto kdesc = [](uint32_t lo, int step) {
                 return sw128_desc(lo + (((uint32_t)(step >> 2) * kHalf + (uint32_t)(step & 3) * 32u) >> 4));
+            };
+            auto bdesc = [](uint32_t lo, int step) {
+                return sw128_desc(lo + (((uint32_t)(step >> 2) * C::kImgHalf + (uint32_t)(step & 3) * 32u) >> 4));
             };
             // rotation of local tile k into its team's buffer; false when not ready yet
             auto try_rot = [&](int k) -> bool {
                 const int s = k % C::kStages;
                 const int t = k % C::kTeams;
                 const uint32_t use = (uint32_t)(k / C::kTeams);
-                if (!mbar_test_wait(bar(kBarXFull + s), (uint32_t)(k / C::kStages) & 1u)) return false;
-                if (!mbar_test_wait(bar(kBarRotEmpty + t), (use & 1u) ^ 1u)) return false;
+                if (!test(bar(kBarXFull + s), (uint32_t)(k / C::kStages) & 1u)) return false;
+                if (!test(bar(kBarRotEmpty + t), (use & 1u) ^ 1u)) return false;
                 tc_fence_after();
                 const uint32_t dA = tmem + C::kBufCols * (uint32_t)t;
                 const uint32_t xs = x0 + (uint32_t)s * kTileU;
@@ -266,65 +342,54 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 if (ROT == 0) {  // the small lo pass first, then the hi pass
 #pragma unroll
                     for (int st = 0; st < 8; ++st) {
-                        umma_ss(dA, kdesc(xs, st), kdesc(img + kTileU, st), idesc, accA);
+                        mma_ss(dA, kdesc(xs, st), bdesc(img + kImgU, st), idesc, accA);
                         accA = 1u;
                     }
                 }
 #pragma unroll
                 for (int st = 0; st < 8; ++st) {
-                    umma_ss(dA, kdesc(xs, st), kdesc(img, st), idesc, accA);
+                    mma_ss(dA, kdesc(xs, st), bdesc(img, st), idesc, accA);
                     accA = 1u;
                 }
-                umma_commit(bar(kBarXEmpty + s));
-                umma_commit(bar(kBarRotFull + t));
+                commit_both(bar(kBarXEmpty + s));
+                commit_both(bar(kBarRotFull + t));
                 return true;
             };
             // sketch of local tile k (keys); false when its rho is not written yet or
             // the sketch of tile k - 1 has not been read
             auto try_qjl = [&](int k) -> bool {
                 const int t = k % C::kTeams;
-                if (!mbar_test_wait(bar(kBarRhoFull + t), (uint32_t)(k / C::kTeams) & 1u)) return false;
-                if (!mbar_test_wait(bar(kBarSketchEmpty), ((uint32_t)k & 1u) ^ 1u)) return false;
+                if (!test(bar(kBarRhoFull + t), (uint32_t)(k / C::kTeams) & 1u)) return false;
+                if (!test(bar(kBarSketchEmpty), ((uint32_t)k & 1u) ^ 1u)) return false;
                 tc_fence_after();
                 const uint32_t buf = tmem + C::kBufCols * (uint32_t)t;
                 const uint32_t d = tmem + kColSketch;
-                const uint32_t m0 = img + C::kRotImages * kTileU;
+                const uint32_t m0 = img + C::kRotImages * kImgU;
                 // rho of K-step st: columns 16 st (hi pairs) and 16 st + 8 (lo pairs)
                 auto rho_col = [&](int st) { return buf + 16u * (uint32_t)st; };
                 uint32_t acc2 = 0u;
                 // the small terms first: rho_lo M_hi (+ rho_hi M_lo for Haar), then rho_hi M_hi
 #pragma unroll
                 for (int st = 0; st < 8; ++st) {
-                    umma_ts(d, rho_col(st) + 8u, kdesc(m0, st), idesc, acc2);
+                    mma_ts(d, rho_col(st) + 8u, bdesc(m0, st), idesc, acc2);
                     acc2 = 1u;
                 }
                 if (ROT == 0) {
 #pragma unroll
-                    for (int st = 0; st < 8; ++st) umma_ts(d, rho_col(st), kdesc(m0 + kTileU, st), idesc, 1u);
+                    for (int st = 0; st < 8; ++st) mma_ts(d, rho_col(st), bdesc(m0 + kImgU, st), idesc, 1u);
                 }
 #pragma unroll
-                for (int st = 0; st < 8; ++st) umma_ts(d, rho_col(st), kdesc(m0, st), idesc, 1u);
-                umma_commit(bar(kBarQjlFull + t));
+                for (int st = 0; st < 8; ++st) mma_ts(d, rho_col(st), bdesc(m0, st), idesc, 1u);
+                commit_both(bar(kBarQjlFull + t));
                 return true;
             };
-            // Rotations and sketches each go in tile order.  Polls with a bound on
-            // time without progress.
-            int next_rot = 0, next_qjl = 0;
+            // Each issuer goes in tile order.  Polls with a bound on time without progress.
+            int next = 0;
             uint64_t t_last = globaltimer_ns();
             uint32_t spins = 0;
-            while (ok) {
-                bool progress = false;
-                if (PROD && next_qjl < next_rot && try_qjl(next_qjl)) {
-                    ++next_qjl;
-                    progress = true;
-                }
-                if (next_rot < my_tiles && try_rot(next_rot)) {
-                    ++next_rot;
-                    progress = true;
-                }
-                const bool done = next_rot >= my_tiles && (!PROD || next_qjl >= my_tiles);
-                if (done) break;
-                if (progress) {
+            while (ok && next < my_tiles) {
+                if (rot_issuer ? try_rot(next) : try_qjl(next)) {
+                    ++next;
                     spins = 0;
                     t_last = globaltimer_ns();
                 } else if ((++spins & 31u) == 0) {
@@ -332,13 +397,15 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 }
             }
             if (!ok) set_abort(abort, a.err);
-            // all MMAs of this CTA complete before its tensor memory is released
-            umma_commit(bar(kBarDrain));
+            // this thread's MMAs (pair: of both CTAs) complete before the tensor memory is released
+            const int drain = kBarDrain + (rot_issuer ? 0 : 1);
+            if (PAIR) umma_commit_pair_local(bar(drain));
+            else umma_commit(bar(drain));
             const volatile int never = 0;
-            mbar_wait(bar(kBarDrain), 0, &never, kWaitNs);
+            mbar_wait(bar(drain), 0, &never, kWaitNs);
         }
         __syncwarp();
-    } else {
+    } else if (warp < C::kEpiWarps) {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int team = warp >> 2;    // tiles k with k % kTeams == team, buffer team
@@ -364,19 +431,20 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
         // slot of this thread's row of a tile, and the row's destination: the chunk
         // pointer with the row inside the page in its low 4 bits (chunks are
         // 16-byte aligned), or null
-        // row vi = tile * 128 + row is (token vi / H, head vi % H); when H divides 128
-        // a tile holds 128 / H whole tokens and this thread's token offset and head
-        // are the same in every tile
+        // row vi = row0 + row of this CTA's 128 rows from row0 (a multiple of 128) is
+        // (token vi / H, head vi % H); when H divides 128 a block of 128 rows holds
+        // 128 / H whole tokens and this thread's token offset and head are the same in
+        // every block
         const bool hdiv = (128 % a.H) == 0;
-        const int tok_per_tile = hdiv ? 128 / a.H : 0;
+        const int tok_per_block = hdiv ? 128 / a.H : 0;
         const int row_tok = hdiv ? row / a.H : 0, row_head = hdiv ? row % a.H : 0;
-        auto token_of = [&](int tile, int vi) -> int { return hdiv ? tile * tok_per_tile + row_tok : vi / a.H; };
-        auto slot_of = [&](int tile) -> int {
-            const int vi = tile * 128 + row;
-            return vi < a.N ? __ldg(a.slots + token_of(tile, vi)) : -1;
+        auto token_of = [&](int row0, int vi) -> int { return hdiv ? (row0 >> 7) * tok_per_block + row_tok : vi / a.H; };
+        auto slot_of = [&](int row0) -> int {
+            const int vi = row0 + row;
+            return vi < a.N ? __ldg(a.slots + token_of(row0, vi)) : -1;
         };
-        auto dest = [&](int tile, int slot) -> uint8_t* {
-            const int vi = tile * 128 + row;
+        auto dest = [&](int row0, int slot) -> uint8_t* {
+            const int vi = row0 + row;
             if (vi >= a.N || slot < 0) return nullptr;
             if (slot >= a.num_blocks * kPage) {
                 atomicOr(a.err, TQ_DEVERR_SLOT);
@@ -403,13 +471,18 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
             if (PROD) reinterpret_cast<float*>(chunk + a.lay.gamma_off)[pr] = gamma;
         };
 
-        int slot_next = team < my_tiles ? slot_of((int)blockIdx.x + team * (int)gridDim.x) : -1;
+        // the buffer-release arrivals of both CTAs of a pair go to the even CTA's issuer
+        auto release = [&](int b) {
+            if (PAIR) mbar_arrive_remote_warp(bar(b), 0);
+            else mbar_arrive_warp(bar(b));
+        };
+        int slot_next = team < my_tiles ? slot_of(row0_of(team)) : -1;
         for (int k = team; k < my_tiles; k += C::kTeams) {
-            const int tile = (int)blockIdx.x + k * (int)gridDim.x;
+            const int row0 = row0_of(k);
             const uint32_t use = (uint32_t)(k / C::kTeams);
             const int slot = slot_next;
-            if (k + C::kTeams < my_tiles) slot_next = slot_of(tile + C::kTeams * (int)gridDim.x);
-            uint8_t* dst = dest(tile, slot);
+            if (k + C::kTeams < my_tiles) slot_next = slot_of(row0_of(k + C::kTeams));
+            uint8_t* dst = dest(row0, slot);
             float nsq;
             if (!PROD) {
                 // ---- ||x||^2 of the row from the swizzled fp16 tile (logical 16-byte
@@ -575,7 +648,7 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
             }
             if (!PROD) {
                 tc_fence_before();
-                mbar_arrive_warp(bar(kBarRotEmpty + team));
+                release(kBarRotEmpty + team);
                 const uint32_t none[4] = {0u, 0u, 0u, 0u};
                 store_tail(dst, norm, 0.f, none);
                 continue;
@@ -583,7 +656,7 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
             // ---- keys: release rho; gamma; then the sketch as sign bits
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive_warp(bar(kBarRhoFull + team));
+            release(kBarRhoFull + team);
             const float gsq = (gs[0].x + gs[0].y) + (gs[1].x + gs[1].y);
             const float gamma = (live && gsq > 0.f) ? gsq * rsqrt_refined(gsq) * nacc * a.gamma_scale : 0.f;
             const bool sk = mbar_wait_warp(bar(kBarQjlFull + team), use & 1u, abort, kWaitNs);
@@ -593,7 +666,7 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
             }
             // the sketch is done with rho: the buffer is free for the team's next rotation
             tc_fence_after();
-            mbar_arrive_warp(bar(kBarRotEmpty + team));
+            release(kBarRotEmpty + team);
             uint32_t sg[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -606,35 +679,59 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD>::kBound, 1) compress_tc_kernel(
                 sg[c] = live ? ~neg : 0xffffffffu;
             }
             tc_fence_before();
-            mbar_arrive_warp(bar(kBarSketchEmpty));
+            release(kBarSketchEmpty);
             store_tail(dst, norm, gamma, sg);
         }
     }
     __syncthreads();
+    // pair: neither CTA leaves, or frees tensor memory the even CTA's MMAs write, while
+    // the other may still signal it
+    if (PAIR) cluster_sync();
     if (warp == C::kWarpMma) {
         tc_fence_after();
-        tmem_dealloc(tmem, C::kTmemCols);
+        if (PAIR) tmem_dealloc_pair(tmem, C::kTmemCols);
+        else tmem_dealloc(tmem, C::kTmemCols);
     }
 }
 
-template <int ROT, bool PROD, int W>
-cudaError_t launch_tc(const CUtensorMap& tmap, const TcArgs& a, int grid, cudaStream_t stream) {
-    using C = Cfg<ROT, PROD>;
-    auto k = compress_tc_kernel<ROT, PROD, W>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
-    if (e != cudaSuccess) return e;
-    // programmatic stream serialization: the setup above griddep_wait overlaps the
-    // end of the kernel before
+// One launch over N rows: 2-CTA clusters (pair) or single CTAs, as many as are
+// resident at once and no more than there are tiles; programmatic stream
+// serialization lets the setup above griddep_wait overlap the end of the kernel before.
+template <int ROT, bool PROD, int W, bool PAIR>
+cudaError_t launch_tc(const CUtensorMap& tmap, const TcArgs& a, int sm_count, cudaStream_t stream) {
+    using C = Cfg<ROT, PROD, PAIR>;
+    auto k = compress_tc_kernel<ROT, PROD, W, PAIR>;
+    static int resident = 0;  // CTAs (pair: clusters) resident at once, for this kernel
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(C::kThreads);
     cfg.dynamicSmemBytes = C::kSmem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = PAIR ? 2 : 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
+    if (resident == 0) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+        if (e != cudaSuccess) return e;
+        int n = PAIR ? sm_count / 2 : sm_count;
+        if (PAIR) {
+            cfg.gridDim = dim3(2 * (unsigned)n);
+            int clusters = 0;
+            e = cudaOccupancyMaxActiveClusters(&clusters, k, &cfg);
+            if (e != cudaSuccess) return e;
+            if (clusters > 0 && clusters < n) n = clusters;
+        }
+        resident = n > 0 ? n : 1;
+    }
+    const int rows = PAIR ? 256 : 128;
+    const int ntiles = (a.N + rows - 1) / rows;
+    const int workers = ntiles < resident ? (ntiles > 0 ? ntiles : 1) : resident;
+    cfg.gridDim = dim3((unsigned)(PAIR ? 2 * workers : workers));
     return cudaLaunchKernelEx(&cfg, k, tmap, a);
 }
 
@@ -669,12 +766,11 @@ cudaError_t launch_compress_tc(const tq_ctx* ctx, int kind, const uint16_t* x, i
     a.gamma_scale = (float)(n_scale / (std::sqrt((double)kDim) * (double)lp.scale));
     a.lay = lay;
     a.err = ctx->dev_error;
-    const int ntiles = (N + 127) / 128;
-    const int grid = ntiles < ctx->sm_count ? ntiles : ctx->sm_count;
     const int W = container_width(value ? ctx->host.vbits : ctx->host.kbits);
     cudaError_t e = cudaErrorInvalidValue;
+    // every kind runs as MMA pairs on the two SMs of 2-CTA clusters, 256 rows a tile
 #define TQ_TC_CASE(R, P, WW) \
-    if (rot == R && prod == P && W == WW) e = launch_tc<R, P, WW>(tmap, a, grid, stream);
+    if (rot == R && prod == P && W == WW) e = launch_tc<R, P, WW, true>(tmap, a, ctx->sm_count, stream);
     TQ_TC_CASE(0, false, 4)
     TQ_TC_CASE(0, false, 2)
     TQ_TC_CASE(1, false, 4)
