@@ -6,24 +6,26 @@
 // [TQ-RS] "TurboQuant : compresser le KV-cache…", "Couche 1" (randomized
 // Walsh-Hadamard rotation).
 //
-// One CTA per SM walks 128-vector tiles of the flattened [T*Hkv, 128] input:
+// 2-CTA clusters (one CTA per SM) walk 256-vector tiles of the flattened
+// [T*Hkv, 128] input, 128 rows per CTA; every MMA is a cta_group::2 pair issued
+// by the even CTA (M = 256, each CTA holding its own x rows and half of the
+// operand image rows, each CTA's tensor memory receiving its own 128 rows):
 //   warps 0..4n-1  epilogue, n teams of four warps (one per TMEM lane quarter,
-//                  one thread per row); team t takes the CTA's tiles k with
+//                  one thread per row); team t takes the cluster's tiles k with
 //                  k % n == t in TMEM buffer t, so one team's waits overlap the
-//                  other teams' arithmetic (values n = 4, keys n = 2)
-//   warp 4n        TMA producer: 128x128 fp16 tiles (two 128-byte-swizzled boxes)
-//   warp 4n+1      TMEM owner and single-thread MMA issuer
+//                  other teams' arithmetic (values n = 4, keys n = 3)
+//   warp 4n        TMA producer: this CTA's 128 x 128 fp16 rows of the tile
+//   warp 4n+1      TMEM owner; even CTA: rotation issuer; odd CTA: forwards its
+//                  stage-full and operands-ready events to the even CTA
+//   warp 4n+2      keys, even CTA: sketch issuer (a second issuing thread)
 // Rotation: D[v][n] = sum_k x[v][k] B[n][k] with B the rotation split into
 // fp16 parts held in shared memory for the whole kernel:
 //   Haar      B = 16 R^T = hi + lo (two passes, x is exact in fp16, products are
-//             exact, fp32 accumulation)  -> acc = 16 y
+//             exact, fp32 accumulation, the small lo pass first)  -> acc = 16 y
 //   Hadamard  B = H D (entries +-1, exact, one pass)  -> acc = sqrt(d) y
-// Values: one accumulator; ||x|| comes from the fp16 tile in shared memory
-// (exact squares, fp32 sums), and the codes only need acc within the 1e-6 window.
-// Keys: gamma needs the residual to ~1e-7 of ||x||, and the tensor core rounds
-// each accumulation step, so the rotation goes to two accumulators,
-// A = (lo pass) + K-steps 0-3 of the hi pass and B = K-steps 4-7, summed in
-// registers (acc = A + B), and ||x|| = ||acc|| / (acc / y).
+// Values: ||x|| comes from the fp16 tile in shared memory (exact squares, fp32
+// sums), read while the rotation runs; the codes only need acc within the 1e-6
+// window.  Keys: ||x|| = ||acc|| / (acc / y) from the accumulator itself.
 // In both cases v = sqrt(d) y / ||x||; the epilogue works in cell units u = v * scale of a shared-memory
 // table of uniform cells (each holds at most one boundary): round(u) addresses
 // the cell, one fp32 compare with its boundary gives the code (values: of
@@ -34,7 +36,7 @@
 //   S (x - x_hat) = (S R) (y - y_hat)
 // is a second contraction whose A operand rho (split into fp16 hi + lo) the
 // epilogue writes back into tensor memory over the accumulator columns it has
-// just read; the sketch accumulates over the tile's B accumulator:
+// just read; the sketches, in tile order, share one accumulator:
 //   Haar      acc2 = rho_lo M_hi + rho_hi M_lo + rho_hi M_hi   (M = S R)
 //   Hadamard  acc2 = (rho_lo + rho_hi) M',   M' = S D H integer, exact in fp16
 // sign bit j = [acc2_j >= 0].  Every wait is bounded (TQ_DEVERR_TIMEOUT).
