@@ -147,6 +147,13 @@ __device__ __forceinline__ float rsqrt_refined(float x) {
     return fmaf(0.5f * r, e, r);
 }
 
+// A read-only global load that stays where it is written (not sunk to its use).
+__device__ __forceinline__ int ldg_early(const int32_t* p) {
+    int v;
+    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
 // Table reads at a 32-bit shared-memory address.
 __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
     uint32_t x;
@@ -441,9 +448,10 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD, PAIR>::kBound, 1) compress_tc_k
         const int tok_per_block = hdiv ? 128 / a.H : 0;
         const int row_tok = hdiv ? row / a.H : 0, row_head = hdiv ? row % a.H : 0;
         auto token_of = [&](int row0, int vi) -> int { return hdiv ? (row0 >> 7) * tok_per_block + row_tok : vi / a.H; };
+        // (a volatile load: issued where it is written, a tile before its use)
         auto slot_of = [&](int row0) -> int {
             const int vi = row0 + row;
-            return vi < a.N ? __ldg(a.slots + token_of(row0, vi)) : -1;
+            return vi < a.N ? ldg_early(a.slots + token_of(row0, vi)) : -1;
         };
         auto dest = [&](int row0, int slot) -> uint8_t* {
             const int vi = row0 + row;
@@ -478,13 +486,18 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD, PAIR>::kBound, 1) compress_tc_k
             if (PAIR) mbar_arrive_remote_warp(bar(b), 0);
             else mbar_arrive_warp(bar(b));
         };
-        int slot_next = team < my_tiles ? slot_of(row0_of(team)) : -1;
+        // the destination of the team's current tile and the slot of its next one; the
+        // next tile's destination and the slot of the one after it are worked out while
+        // the team waits for the rotation (values) or after the tile's stores (keys)
+        int slot_next = team + C::kTeams < my_tiles ? slot_of(row0_of(team + C::kTeams)) : -1;
+        uint8_t* dst = team < my_tiles ? dest(row0_of(team), slot_of(row0_of(team))) : nullptr;
+        uint8_t* dst_next = nullptr;
+        auto advance = [&](int k) {
+            dst_next = k + C::kTeams < my_tiles ? dest(row0_of(k + C::kTeams), slot_next) : nullptr;
+            if (k + 2 * C::kTeams < my_tiles) slot_next = slot_of(row0_of(k + 2 * C::kTeams));
+        };
         for (int k = team; k < my_tiles; k += C::kTeams) {
-            const int row0 = row0_of(k);
             const uint32_t use = (uint32_t)(k / C::kTeams);
-            const int slot = slot_next;
-            if (k + C::kTeams < my_tiles) slot_next = slot_of(row0_of(k + C::kTeams));
-            uint8_t* dst = dest(row0, slot);
             float nsq;
             if (!PROD) {
                 // ---- ||x||^2 of the row from the swizzled fp16 tile (logical 16-byte
@@ -513,6 +526,7 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD, PAIR>::kBound, 1) compress_tc_k
                 fence_proxy_async_shared();  // these reads before the next TMA write of the stage
                 mbar_arrive_warp(bar(kBarXEmpty + stg));
                 nsq = (sq[0] + sq[1]) + (sq[2] + sq[3]);
+                advance(k);
                 good = mbar_wait_warp(bar(kBarRotFull + team), use & 1u, abort, kWaitNs);
                 if (!good) {
                     set_abort(abort, a.err);
@@ -577,46 +591,44 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD, PAIR>::kBound, 1) compress_tc_k
 #pragma unroll
                     for (int i = 0; i < 16; ++i) av[i] = make_float2(0.f, 0.f);
                 }
-                uint32_t rho_hi[16], rho_lo[16];
+                // K-step 2 q + h: its rho goes over its A columns (already read), hi pairs
+                // at the first 8 and lo pairs at the next 8, as soon as they are known
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float2 u = __fmul2_rn(av[i], s2);
-                    const float2 gg = __fadd2_rn(u, magic2);
-                    uint32_t b0, base0, lo0, hi0, b1, base1, lo1, hi1;
-                    lds_v4(__float_as_uint(gg.x) * 128u + lut_off, b0, base0, lo0, hi0);
-                    lds_v4(__float_as_uint(gg.y) * 128u + lut_off, b1, base1, lo1, hi1);
-                    const bool p0 = __uint_as_float(b0) < u.x;
-                    const bool p1 = __uint_as_float(b1) < u.y;
-                    const uint32_t code0 = base0 + (p0 ? 1u : 0u);
-                    const uint32_t code1 = base1 + (p1 ? 1u : 0u);
-                    const float c0 = __uint_as_float(p0 ? hi0 : lo0);
-                    const float c1 = __uint_as_float(p1 ? hi1 : lo1);
-                    const float2 d = __ffma2_rn(av[i], s2, make_float2(-c0, -c1));  // residual, cell units
-                    gs[i & 1] = __ffma2_rn(d, d, gs[i & 1]);
-                    // rho = 32 (v - c) = hi + lo in fp16: hi keeps the top 11 significant bits
-                    // (exact in fp16 for |rho| < 65504), lo = rho - hi exactly
-                    const float2 rho = __fmul2_rn(d, rho_k);
-                    const float2 hf = make_float2(__uint_as_float(__float_as_uint(rho.x) & 0xffffe000u),
-                                                  __uint_as_float(__float_as_uint(rho.y) & 0xffffe000u));
-                    const float2 rem = __fadd2_rn(rho, make_float2(-hf.x, -hf.y));
-                    const __half2 hi = __floats2half2_rn(hf.x, hf.y);
-                    const __half2 lo = __floats2half2_rn(rem.x, rem.y);
-                    rho_hi[i] = *reinterpret_cast<const uint32_t*>(&hi);
-                    rho_lo[i] = *reinterpret_cast<const uint32_t*>(&lo);
-                    const int j = 2 * i;  // column within the 32
-                    words[j / kPer] += code0 << (W * (j % kPer));
-                    words[(j + 1) / kPer] += code1 << (W * ((j + 1) % kPer));
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t rho_hi[8], rho_lo[8];
+#pragma unroll
+                    for (int ii = 0; ii < 8; ++ii) {
+                        const int i = 8 * h + ii;
+                        const float2 u = __fmul2_rn(av[i], s2);
+                        const float2 gg = __fadd2_rn(u, magic2);
+                        uint32_t b0, base0, lo0, hi0, b1, base1, lo1, hi1;
+                        lds_v4(__float_as_uint(gg.x) * 128u + lut_off, b0, base0, lo0, hi0);
+                        lds_v4(__float_as_uint(gg.y) * 128u + lut_off, b1, base1, lo1, hi1);
+                        const bool p0 = __uint_as_float(b0) < u.x;
+                        const bool p1 = __uint_as_float(b1) < u.y;
+                        const uint32_t code0 = base0 + (p0 ? 1u : 0u);
+                        const uint32_t code1 = base1 + (p1 ? 1u : 0u);
+                        const float c0 = __uint_as_float(p0 ? hi0 : lo0);
+                        const float c1 = __uint_as_float(p1 ? hi1 : lo1);
+                        const float2 d = __ffma2_rn(av[i], s2, make_float2(-c0, -c1));  // residual, cell units
+                        gs[i & 1] = __ffma2_rn(d, d, gs[i & 1]);
+                        // rho = 32 (v - c) = hi + lo in fp16: hi keeps the top 11 significant bits
+                        // (exact in fp16 for |rho| < 65504), lo = rho - hi exactly
+                        const float2 rho = __fmul2_rn(d, rho_k);
+                        const float2 hf = make_float2(__uint_as_float(__float_as_uint(rho.x) & 0xffffe000u),
+                                                      __uint_as_float(__float_as_uint(rho.y) & 0xffffe000u));
+                        const float2 rem = __fadd2_rn(rho, make_float2(-hf.x, -hf.y));
+                        const __half2 hi = __floats2half2_rn(hf.x, hf.y);
+                        const __half2 lo = __floats2half2_rn(rem.x, rem.y);
+                        rho_hi[ii] = *reinterpret_cast<const uint32_t*>(&hi);
+                        rho_lo[ii] = *reinterpret_cast<const uint32_t*>(&lo);
+                        const int j = 2 * i;  // column within the 32
+                        words[j / kPer] += code0 << (W * (j % kPer));
+                        words[(j + 1) / kPer] += code1 << (W * ((j + 1) % kPer));
+                    }
+                    tmem_st8(col + 16 * h, rho_hi);
+                    tmem_st8(col + 16 * h + 8, rho_lo);
                 }
-                // over the K-steps' A columns, already read: K-step st -> hi at 16 st, lo at 16 st + 8
-                uint32_t h8[8], l8[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) h8[i] = rho_hi[i], l8[i] = rho_lo[i];
-                tmem_st8(col, h8);
-                tmem_st8(col + 8, l8);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) h8[i] = rho_hi[8 + i], l8[i] = rho_lo[8 + i];
-                tmem_st8(col + 16, h8);
-                tmem_st8(col + 24, l8);
               } else {
 #pragma unroll
               for (int sub = 0; sub < 2; ++sub) {
@@ -653,6 +665,7 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD, PAIR>::kBound, 1) compress_tc_k
                 release(kBarRotEmpty + team);
                 const uint32_t none[4] = {0u, 0u, 0u, 0u};
                 store_tail(dst, norm, 0.f, none);
+                dst = dst_next;
                 continue;
             }
             // ---- keys: release rho; gamma; then the sketch as sign bits
@@ -683,6 +696,8 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD, PAIR>::kBound, 1) compress_tc_k
             tc_fence_before();
             release(kBarSketchEmpty);
             store_tail(dst, norm, gamma, sg);
+            advance(k);
+            dst = dst_next;
         }
     }
     __syncthreads();
