@@ -39,7 +39,9 @@ def test_tiny_workload_full(orc, rot, bits, km):
 
 
 @pytest.mark.parametrize("rot,bits,km", SETTINGS[:3])
-@pytest.mark.parametrize("T,H", [(37, 3), (16, 8), (1, 1), (300, 5)])
+# rows T * H: below one 128-row block, exactly one, one and a half (the odd CTA of a
+# 2-CTA cluster partly filled), and several 256-row cluster tiles with a ragged tail
+@pytest.mark.parametrize("T,H", [(37, 3), (16, 8), (1, 1), (25, 8), (300, 5)])
 def test_ragged_shapes(orc, rot, bits, km, T, H):
     import torch
     rng = np.random.default_rng(T * 31 + H)
