@@ -97,6 +97,7 @@ class Context:
     def __init__(self, handle: int, head_dim: int, bits: int, seed: int, rotation: int, key_mode: int):
         self.handle = handle
         self.head_dim, self.bits, self.seed, self.rotation, self.key_mode = head_dim, bits, seed, rotation, key_mode
+        self._chunk = {}  # chunk bytes by kind, asked of the library once
 
     def __del__(self):
         h = getattr(self, "handle", None)
@@ -131,7 +132,10 @@ def tq_destroy(ctx: Context):
 
 
 def tq_chunk_bytes(ctx: Context, kind: int) -> int:
-    return int(_lib.tq_chunk_bytes(ctx.handle, kind))
+    n = ctx._chunk.get(kind)
+    if n is None:
+        n = ctx._chunk[kind] = int(_lib.tq_chunk_bytes(ctx.handle, kind))
+    return n
 
 
 def tq_code_bits(ctx: Context, kind: int) -> int:
@@ -159,9 +163,11 @@ def tq_export_params(ctx: Context) -> dict:
 def _expect(t, shape, dtypes, what: str, name: str):
     """The C ABI takes raw pointers plus sizes: every tensor must hold exactly what
     those sizes promise (shape, dtype, dense row-major), or the call is refused here."""
-    import torch
-    ok = t is not None and t.dim() == len(shape) and t.is_contiguous() and t.dtype in dtypes
-    ok = ok and all(want is None or int(got) == want for got, want in zip(t.shape, shape))
+    ok = t is not None and t.dtype in dtypes and t.is_contiguous()
+    if ok:
+        got = t.shape
+        ok = got == shape if None not in shape else (
+            len(got) == len(shape) and all(w is None or g == w for g, w in zip(got, shape)))
     if not ok:
         desc = "None" if t is None else "%s %s" % (tuple(t.shape), t.dtype)
         raise TQError(TQ_ERR_INVALID_ARG, "%s: %s must be %s of %s, got %s" % (what, name, list(shape), dtypes, desc))
