@@ -718,7 +718,11 @@ template <int ROT, bool PROD, int W, bool PAIR>
 cudaError_t launch_tc(const CUtensorMap& tmap, const TcArgs& a, int sm_count, cudaStream_t stream) {
     using C = Cfg<ROT, PROD, PAIR>;
     auto k = compress_tc_kernel<ROT, PROD, W, PAIR>;
-    static int resident = 0;  // CTAs (pair: clusters) resident at once, for this kernel
+    // CTAs (pair: clusters) of this kernel resident at once, per device
+    static int resident_of[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    int& resident = resident_of[dev];
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(C::kThreads);
     cfg.dynamicSmemBytes = C::kSmem;
