@@ -94,7 +94,8 @@ struct Cfg {
     static constexpr int kWarpMma = kEpiWarps + 1;     // rotations
     static constexpr int kWarpSketch = kEpiWarps + 2;  // keys: the sketches, from a second thread
     static constexpr int kThreads = kEpiWarps * 32 + (PROD ? 96 : 64);
-    // registers: keys 15 warps at 136, values 18 warps at 112
+    // registers: warps get them in fours (one per SM sub-partition), so keys (15 warps)
+    // run at up to 128 and values (18 warps) at up to 112
     static constexpr int kBound = kThreads;
     static constexpr uint32_t kBufCols = 128;
     static_assert(kStages >= 1, "shared memory budget");
@@ -106,7 +107,7 @@ enum : int {
     kBarConst = 0,
     kBarXFull = 1,     // +stage (4)
     kBarXEmpty = 5,    // +stage (4)
-    kBarRotFull = 9,    // +team (4): rotation accumulators ready
+    kBarRotFull = 9,    // +team (4): rotation accumulator ready
     kBarRotEmpty = 13,  // +team (4): the team is done with its buffer
     kBarRhoFull = 17,   // +team (3): rho written (keys)
     kBarQjlFull = 20,   // +team (3): sketch ready (keys)
