@@ -82,6 +82,7 @@ def _declare(L):
         "orc_read_paged": (None, [_P, _I, _P, _I, _I, _P, _P, _P, _P, _P]),
         "orc_decompress_paged": (None, [_P, _I, _P, _I, _I, _P, _P, _I]),
         "orc_decode": (_I, [_P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _D, _I, _P, _I]),
+        "orc_decode_window": (_I, [_P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _P, _P, _P, _I, _D, _I, _P, _I]),
         "orc_max_threads": (_I, []),
     }
     for name, (res, args) in sig.items():
@@ -289,7 +290,14 @@ class Oracle:
         lib().orc_decompress_paged(self._h, kind, _ptr(cache), T, H, _ptr(sm), _ptr(out), self.nthreads)
         return out
 
-    def decode(self, q, kcache, vcache, block_table, seq_lens, Hkv: int, scale=None, form: int = 1):
+    def decode(self, q, kcache, vcache, block_table, seq_lens, Hkv: int, scale=None, form: int = 1,
+               tail_k=None, tail_v=None, tail_lens=None):
+        """Decode attention over the paged cache; with tail_k / tail_v [B, W, Hkv, d]
+        and tail_lens [B], the last tail_lens[b] tokens of sequence b are uncompressed
+        (the residual window) and join the same softmax."""
+        if tail_k is not None:
+            return self._decode_window(q, kcache, vcache, block_table, seq_lens, Hkv, scale, form,
+                                       tail_k, tail_v, tail_lens)
         q = _f64(q)
         B, Hq, d = q.shape
         assert d == self.d and Hq % Hkv == 0
@@ -304,4 +312,26 @@ class Oracle:
                               bt.shape[1], _ptr(sl), B, Hq, Hkv, float(scale), form, _ptr(out), self.nthreads)
         if rc != 0:
             raise ValueError("block id or sequence length out of range")
+        return out
+
+    def _decode_window(self, q, kcache, vcache, block_table, seq_lens, Hkv, scale, form, tail_k, tail_v, tail_lens):
+        q = _f64(q)
+        B, Hq, d = q.shape
+        assert d == self.d and Hq % Hkv == 0
+        tk = _f64(tail_k)
+        tv = _f64(tail_v)
+        assert tk.shape == tv.shape and tk.shape[0] == B and tk.shape[2] == Hkv and tk.shape[3] == d
+        kcache = np.ascontiguousarray(kcache, np.uint8)
+        vcache = np.ascontiguousarray(vcache, np.uint8)
+        bt = np.ascontiguousarray(block_table, np.int32)
+        sl = np.ascontiguousarray(seq_lens, np.int32)
+        tl = np.ascontiguousarray(tail_lens, np.int32)
+        if scale is None:
+            scale = 1.0 / np.sqrt(d)
+        out = np.empty((B, Hq, d), np.float64)
+        rc = lib().orc_decode_window(self._h, _ptr(q), _ptr(kcache), _ptr(vcache), kcache.shape[0], _ptr(bt),
+                                     bt.shape[1], _ptr(sl), B, Hq, Hkv, _ptr(tk), _ptr(tv), _ptr(tl), tk.shape[1],
+                                     float(scale), form, _ptr(out), self.nthreads)
+        if rc != 0:
+            raise ValueError("block id, sequence length or window length out of range")
         return out

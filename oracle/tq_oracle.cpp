@@ -600,11 +600,19 @@ void orc_decompress_paged(void* h, int kind, const uint8_t* cache, int T, int H,
 //   p = softmax(s) (max-subtracted), o = sum_t p_t v_hat_t.
 // form 0: explicit dequantize-then-dot in the original domain.
 // form 1: rotated domain, <q, k_hat> = n/sqrt(d) <R^T q, c[idx]>, o = R sum_t p_t n_t c[idx_t]/sqrt(d).
-// q: [B, Hq, d] fp64; out: [B, Hq, d] fp64.  Returns 0, or -1 on a block id or
-// sequence length that falls outside the cache / table.
-int orc_decode(void* h, const double* q, const uint8_t* kcache, const uint8_t* vcache, int num_blocks,
-               const int32_t* block_table, int max_blocks, const int32_t* seq_lens, int B, int Hq, int Hkv,
-               double scale, int form, double* out, int nthreads) {
+// Residual window ([TQ-RS] "Couche 5 — Fenêtre résiduelle" and "Couche 7"
+// (residual_window=128); the KIVI page's FP16 residual of the most recent tokens):
+// the last tail_lens[b] tokens of sequence b are not compressed; their fp16 keys
+// and values tail_k / tail_v [B, tail_cap, Hkv, d] join the same softmax with the
+// exact score s_u = scale * <q, k_u> and contribute p_u v_u.  READING: the pages
+// only name the window and its size, so the plainest reading is one softmax over
+// the compressed tokens and the window's tokens together.  tail_k = NULL: no window.
+// q: [B, Hq, d] fp64; out: [B, Hq, d] fp64.  Returns 0, or -1 on a block id,
+// sequence length or window length that falls outside the cache / table / window.
+int orc_decode_window(void* h, const double* q, const uint8_t* kcache, const uint8_t* vcache, int num_blocks,
+                      const int32_t* block_table, int max_blocks, const int32_t* seq_lens, int B, int Hq, int Hkv,
+                      const double* tail_k, const double* tail_v, const int32_t* tail_lens, int tail_cap,
+                      double scale, int form, double* out, int nthreads) {
     Params* P = (Params*)h;
     const int d = P->d;
     const bool prod = P->key_mode == 0;
@@ -614,6 +622,7 @@ int orc_decode(void* h, const double* q, const uint8_t* kcache, const uint8_t* v
     const double qjl = std::sqrt(3.14159265358979323846 / 2.0) / d;
     for (int b = 0; b < B; ++b) {
         if (seq_lens[b] < 0 || seq_lens[b] > max_blocks * 16) return -1;
+        if (tail_k && (tail_lens[b] < 0 || tail_lens[b] > tail_cap)) return -1;
         for (int p = 0; p < (seq_lens[b] + 15) / 16; ++p) {
             int blk = block_table[(size_t)b * max_blocks + p];
             if (blk < 0 || blk >= num_blocks) return -1;
@@ -626,8 +635,9 @@ int orc_decode(void* h, const double* q, const uint8_t* kcache, const uint8_t* v
         const double* qv = q + bh * d;
         double* ov = out + bh * d;
         const int Tn = seq_lens[b];
+        const int Un = tail_k ? tail_lens[b] : 0;
         for (int i = 0; i < d; ++i) ov[i] = 0.0;
-        if (Tn == 0) continue;   // READING: an empty sequence attends to nothing -> zeros
+        if (Tn + Un == 0) continue;   // READING: an empty sequence attends to nothing -> zeros
         std::vector<double> sq(d, 0.0), qr(d, 0.0);
         for (int j = 0; j < d; ++j) {
             double s = 0.0;
@@ -639,7 +649,7 @@ int orc_decode(void* h, const double* q, const uint8_t* kcache, const uint8_t* v
             for (int i = 0; i < d; ++i) s += P->R[(size_t)i * d + j] * qv[i];
             qr[j] = s;
         }
-        std::vector<double> sc(Tn);
+        std::vector<double> sc(Tn + Un);
         std::vector<int> codes(d), signs(d, 0);
         std::vector<double> kv(d);
         for (int t = 0; t < Tn; ++t) {
@@ -662,11 +672,18 @@ int orc_decode(void* h, const double* q, const uint8_t* kcache, const uint8_t* v
             }
             sc[t] = scale * dot;
         }
+        // the window's tokens: exact fp16 keys (widened), exact scores
+        for (int u = 0; u < Un; ++u) {
+            const double* ku = tail_k + (((size_t)b * tail_cap + u) * Hkv + hk) * d;
+            double dot = 0.0;
+            for (int i = 0; i < d; ++i) dot += qv[i] * ku[i];
+            sc[Tn + u] = scale * dot;
+        }
         double m = sc[0];
-        for (int t = 1; t < Tn; ++t)
+        for (int t = 1; t < Tn + Un; ++t)
             if (sc[t] > m) m = sc[t];
         double den = 0.0;
-        for (int t = 0; t < Tn; ++t) {
+        for (int t = 0; t < Tn + Un; ++t) {
             sc[t] = std::exp(sc[t] - m);
             den += sc[t];
         }
@@ -690,8 +707,20 @@ int orc_decode(void* h, const double* q, const uint8_t* kcache, const uint8_t* v
                 for (int j = 0; j < d; ++j) s += P->R[(size_t)i * d + j] * acc[j];
                 ov[i] = s;
             }
+        for (int u = 0; u < Un; ++u) {
+            const double* vu = tail_v + (((size_t)b * tail_cap + u) * Hkv + hk) * d;
+            const double p = sc[Tn + u] / den;
+            for (int i = 0; i < d; ++i) ov[i] += p * vu[i];
+        }
     }
     return 0;
+}
+
+int orc_decode(void* h, const double* q, const uint8_t* kcache, const uint8_t* vcache, int num_blocks,
+               const int32_t* block_table, int max_blocks, const int32_t* seq_lens, int B, int Hq, int Hkv,
+               double scale, int form, double* out, int nthreads) {
+    return orc_decode_window(h, q, kcache, vcache, num_blocks, block_table, max_blocks, seq_lens, B, Hq, Hkv,
+                             nullptr, nullptr, nullptr, 0, scale, form, out, nthreads);
 }
 
 int orc_max_threads(void) {
