@@ -69,6 +69,8 @@ def _declare(L):
         "orc_pack": (None, [_P, _I, _I, _P]),
         "orc_unpack": (None, [_P, _I, _I, _P]),
         "orc_create": (_P, [_I, _I, _U64, _I, _I]),
+        "orc_create_ex": (_P, [_I, _I, _U64, _I, _I, _I, _I]),
+        "orc_lloyd_max_beta": (None, [_I, _I, _P, _P]),
         "orc_destroy": (None, [_P]),
         "orc_get_rotation": (None, [_P, _P]),
         "orc_get_S": (None, [_P, _P]),
@@ -153,6 +155,15 @@ def lloyd_max(bits: int):
     return c, t[: L - 1]
 
 
+def lloyd_max_beta(d: int, bits: int):
+    """Exact-d Lloyd-Max codebook of v = sqrt(d) u_1, u uniform on the sphere."""
+    L = 1 << bits
+    c = np.empty(L, np.float64)
+    t = np.empty(max(L - 1, 1), np.float64)
+    lib().orc_lloyd_max_beta(d, bits, _ptr(c), _ptr(t))
+    return c, t[: L - 1]
+
+
 def pack(codes, width: int) -> np.ndarray:
     codes = np.ascontiguousarray(codes, np.int32)
     n = codes.size
@@ -177,10 +188,11 @@ class Oracle:
     """Parameters of one compressor instance (R, S, codebooks) and its operations."""
 
     def __init__(self, d: int = 128, bits: int = 4, seed: int = 0, rot: int = ROT_HAAR,
-                 key_mode: int = KEY_PROD, nthreads: int = 0):
+                 key_mode: int = KEY_PROD, nthreads: int = 0, beta: bool = False, dense3: bool = False):
         self.d, self.bits, self.seed, self.rot, self.key_mode = d, bits, seed, rot, key_mode
+        self.beta, self.dense3 = bool(beta), bool(dense3)
         self.nthreads = nthreads
-        self._h = lib().orc_create(d, bits, seed, rot, key_mode)
+        self._h = lib().orc_create_ex(d, bits, seed, rot, key_mode, int(beta), int(dense3))
         if not self._h:
             raise ValueError("unsupported oracle parameters")
 

@@ -213,6 +213,94 @@ void lloyd_max_gaussian(int bits, double* c, double* t) {
 }
 
 // ---------------------------------------------------------------------------
+// Exact-d codebook ([TQ-RS] "Étape 2" and "Couche 2": after the rotation each
+// coordinate of a unit vector follows the spherical Beta law, and the Lloyd-Max
+// quantizer is computed for that law).  The coordinate compared with the
+// boundaries is v = sqrt(d) u_1, u uniform on the unit sphere of R^d, whose
+// density is proportional to (1 - v^2/d)^((d-3)/2) on (-sqrt(d), sqrt(d)).
+// Lloyd's two conditions, as for the Gaussian codebook:
+//   c_j = int_{t_j}^{t_{j+1}} v f(v) dv / int_{t_j}^{t_{j+1}} f(v) dv,
+//   t_j = (c_{j-1} + c_j) / 2,
+// the numerator in closed form, -d/(d-1) (1 - v^2/d)^((d-1)/2) / Z between the
+// cell's ends, the denominator through the law's CDF, a regularized incomplete
+// beta function: (u_1 + 1) / 2 ~ Beta((d-1)/2, (d-1)/2).  READING: the page's "50 iterations" do not converge in
+// fp64; iterated, like the Gaussian codebook, until nothing moves by 1e-15.
+// ---------------------------------------------------------------------------
+// Regularized incomplete beta I_x(p, q) by its continued fraction (DLMF 8.17.22,
+// evaluated with the modified Lentz method), for x < (p + 1) / (p + q + 2).
+double ibeta_cf(double x, double p, double q) {
+    const double lead = std::exp(p * std::log(x) + q * std::log1p(-x) -
+                                 (std::lgamma(p) + std::lgamma(q) - std::lgamma(p + q))) / p;
+    const double tiny = 1e-300;
+    double f = 1.0, C = 1.0, Dn = 0.0;
+    for (int i = 0; i <= 4000; ++i) {
+        double num;
+        if (i == 0) {
+            num = 1.0;
+        } else {
+            const int m = i / 2;
+            num = (i & 1) ? -((p + m) * (p + q + m) * x) / ((p + 2.0 * m) * (p + 2.0 * m + 1.0))
+                          : (m * (q - m) * x) / ((p + 2.0 * m - 1.0) * (p + 2.0 * m));
+        }
+        Dn = 1.0 + num * Dn;
+        if (std::fabs(Dn) < tiny) Dn = tiny;
+        Dn = 1.0 / Dn;
+        C = 1.0 + num / C;
+        if (std::fabs(C) < tiny) C = tiny;
+        const double delta = C * Dn;
+        f *= delta;
+        if (std::fabs(delta - 1.0) < 1e-16) break;
+    }
+    return lead * (f - 1.0);
+}
+// P(V > v) for v >= 0: V = sqrt(d) u_1, (u_1 + 1) / 2 ~ Beta((d-1)/2, (d-1)/2)
+double beta_upper_tail(int d, double v) {
+    const double p = 0.5 * (d - 1);
+    const double x = 0.5 * (1.0 - v / std::sqrt((double)d));   // P(V > v) = I_x(p, p)
+    if (x <= 0.0) return 0.0;
+    return ibeta_cf(x, p, p);   // x <= 1/2 < (p + 1) / (2p + 2)
+}
+// int_a^b of the density (normalised), on the side of 0 that keeps precision
+double beta_mass(int d, double a, double b) {
+    if (a >= 0.0) return beta_upper_tail(d, a) - beta_upper_tail(d, b);
+    if (b <= 0.0) return beta_upper_tail(d, -b) - beta_upper_tail(d, -a);
+    return 1.0 - beta_upper_tail(d, -a) - beta_upper_tail(d, b);
+}
+// int_a^b v f(v) dv for the normalised density f(v) = (1 - v^2/d)^((d-3)/2) / Z,
+// Z = sqrt(d) B(1/2, (d-1)/2); the antiderivative is -d/(d-1) (1 - v^2/d)^((d-1)/2) / Z
+double beta_first_moment(int d, double a, double b) {
+    const double k1 = 0.5 * (d - 1);
+    const double logZ = 0.5 * std::log((double)d) + std::lgamma(0.5) + std::lgamma(k1) - std::lgamma(0.5 + k1);
+    auto F = [&](double v) {
+        const double w = 1.0 - v * v / d;
+        return w <= 0.0 ? 0.0 : -(double)d / (d - 1) * std::exp(k1 * std::log(w) - logZ);
+    };
+    return F(b) - F(a);
+}
+
+void lloyd_max_beta(int d, int bits, double* c, double* t) {
+    const int L = 1 << bits;
+    const double vmax = std::sqrt((double)d);
+    std::vector<double> cc(L), tt(L + 1);
+    for (int j = 0; j < L; ++j) cc[j] = (L == 1) ? 0.0 : -2.0 + 4.0 * (j + 0.5) / L;
+    for (int it = 0; it < 200000; ++it) {
+        tt[0] = -vmax;
+        tt[L] = vmax;
+        for (int j = 1; j < L; ++j) tt[j] = 0.5 * (cc[j - 1] + cc[j]);
+        double moved = 0.0;
+        for (int j = 0; j < L; ++j) {
+            const double nc = beta_first_moment(d, tt[j], tt[j + 1]) / beta_mass(d, tt[j], tt[j + 1]);
+            const double dm = std::fabs(nc - cc[j]);
+            if (dm > moved) moved = dm;
+            cc[j] = nc;
+        }
+        if (moved < 1e-15) break;
+    }
+    for (int j = 0; j < L; ++j) c[j] = cc[j];
+    for (int j = 1; j < L; ++j) t[j - 1] = 0.5 * (cc[j - 1] + cc[j]);
+}
+
+// ---------------------------------------------------------------------------
 // Packed layout of one 16-token page chunk (READING: the pages fix only the
 // nibble / 2-bit packing and the separate fp32 norm; byte and bit order, the
 // 1-bit container and the per-chunk arrangement are this design's):
@@ -222,24 +310,34 @@ void lloyd_max_gaussian(int bits, double* c, double* t) {
 //   nibble: byte i = c[2i] | c[2i+1] << 4; crumb: byte i = sum_k c[4i+k] << 2k;
 //   bit:    byte i = sum_k c[8i+k] << k
 // ---------------------------------------------------------------------------
+// Dense 3-bit option ([TQ-RS] "Couche 3" packs indices into bytes; the dense form
+// is this design's): 3-bit codes as a bit string, code i in bits [3i, 3i + 3),
+// least significant bit first -- 48 B per 128 codes instead of 64 B of nibbles.
 int container_width(int b) { return b >= 3 ? 4 : (b == 2 ? 2 : 1); }
+int code_width(int b, bool dense3) { return (dense3 && b == 3) ? 3 : container_width(b); }
 
+// codes as a bit string: code i occupies bits [w i, w i + w) of out, LSB first
+// (for w = 1, 2, 4 this is byte i = sum_k c[(8/w) i + k] << k w)
 void pack_codes(const int* codes, int n, int w, uint8_t* out) {
-    const int per = 8 / w;
-    for (int i = 0; i < n / per; ++i) {
-        unsigned byte = 0;
-        for (int k = 0; k < per; ++k) byte |= ((unsigned)codes[i * per + k] & ((1u << w) - 1u)) << (k * w);
-        out[i] = (uint8_t)byte;
-    }
+    const int nbytes = n * w / 8;
+    for (int i = 0; i < nbytes; ++i) out[i] = 0;
+    for (int i = 0; i < n; ++i)
+        for (int k = 0; k < w; ++k)
+            if ((codes[i] >> k) & 1) out[(i * w + k) / 8] |= (uint8_t)(1u << ((i * w + k) % 8));
 }
 
 void unpack_codes(const uint8_t* in, int n, int w, int* codes) {
-    const int per = 8 / w;
-    for (int i = 0; i < n; ++i) codes[i] = (in[i / per] >> ((i % per) * w)) & ((1 << w) - 1);
+    for (int i = 0; i < n; ++i) {
+        int c = 0;
+        for (int k = 0; k < w; ++k) c |= ((in[(i * w + k) / 8] >> ((i * w + k) % 8)) & 1) << k;
+        codes[i] = c;
+    }
 }
 
 struct Params {
     int d, bits, rot, key_mode;   // rot: 0 Haar, 1 Hadamard; key_mode: 0 prod (QJL), 1 MSE
+    int beta = 0;                 // codebooks: 0 Gaussian Lloyd-Max, 1 exact-d (spherical Beta) Lloyd-Max
+    int dense3 = 0;               // 3-bit codes: 0 nibble containers, 1 dense bit string
     std::vector<double> R;        // row-major, y = R^T x
     std::vector<int8_t> S;        // row-major, (S r)_j = sum_i S[j][i] r_i
     std::vector<int8_t> D;        // Hadamard signs (rot == 1)
@@ -252,9 +350,9 @@ size_t chunk_bytes(const Params& P, int kind /*0 key, 1 value*/) {
     const int d = P.d;
     if (kind == 1 || P.key_mode == 1) {
         int b = (kind == 1) ? P.vbits : P.kbits;
-        return (size_t)16 * d * container_width(b) / 8 + 64;
+        return (size_t)16 * d * code_width(b, P.dense3) / 8 + 64;
     }
-    return (size_t)16 * d * container_width(P.kbits) / 8 + (size_t)16 * d / 8 + 128;
+    return (size_t)16 * d * code_width(P.kbits, P.dense3) / 8 + (size_t)16 * d / 8 + 128;
 }
 
 // One vector through the compress step [FQ-TQ steps 1-4, QJL section].
@@ -369,7 +467,7 @@ void read_row(const Params& P, int kind, const uint8_t* chunk, int row, int* cod
     const bool value = (kind == 1);
     const bool prod = !value && P.key_mode == 0;
     const int b = value ? P.vbits : P.kbits;
-    const int w = container_width(b);
+    const int w = code_width(b, P.dense3);
     const size_t code_row = (size_t)d * w / 8;
     unpack_codes(chunk + row * code_row, d, w, codes);
     size_t off = 16 * code_row;
@@ -390,7 +488,7 @@ void write_row(const Params& P, int kind, uint8_t* chunk, int row, const int* co
     const bool value = (kind == 1);
     const bool prod = !value && P.key_mode == 0;
     const int b = value ? P.vbits : P.kbits;
-    const int w = container_width(b);
+    const int w = code_width(b, P.dense3);
     const size_t code_row = (size_t)d * w / 8;
     pack_codes(codes, d, w, chunk + row * code_row);
     size_t off = 16 * code_row;
@@ -439,7 +537,16 @@ void orc_unpack(const uint8_t* in, int n, int w, int* codes) { unpack_codes(in, 
 // ---- parameters ------------------------------------------------------------
 // rot: 0 = Haar, 1 = randomized Hadamard.  key_mode: 0 = prod (b-1 bit MSE code
 // + 1-bit QJL), 1 = MSE at b bits.  d must be a power of two >= 8.
+void orc_lloyd_max_beta(int d, int bits, double* c, double* t) { lloyd_max_beta(d, bits, c, t); }
+
+void* orc_create_ex(int d, int bits, uint64_t seed, int rot, int key_mode, int beta, int dense3);
 void* orc_create(int d, int bits, uint64_t seed, int rot, int key_mode) {
+    return orc_create_ex(d, bits, seed, rot, key_mode, 0, 0);
+}
+
+// beta: exact-d codebooks instead of the Gaussian ones; dense3: 3-bit codes as a
+// dense bit string instead of nibbles (both READINGS of [TQ-RS] "Couche 2" / "Couche 3").
+void* orc_create_ex(int d, int bits, uint64_t seed, int rot, int key_mode, int beta, int dense3) {
     if (d < 8 || (d & (d - 1)) != 0 || bits < 1 || bits > 8) return nullptr;
     if (key_mode == 0 && bits < 2) return nullptr;
     Params* P = new Params();
@@ -460,12 +567,19 @@ void* orc_create(int d, int bits, uint64_t seed, int rot, int key_mode) {
     sign_fill(seed, 1, (long)d * d, P->S.data());
     P->vbits = bits;
     P->kbits = (key_mode == 0) ? bits - 1 : bits;
+    P->beta = beta;
+    P->dense3 = dense3;
     P->cv.resize(1 << P->vbits);
     P->tv.resize((1 << P->vbits) - 1);
-    lloyd_max_gaussian(P->vbits, P->cv.data(), P->tv.data());
     P->ck.resize(1 << P->kbits);
     P->tk.resize((1 << P->kbits) - 1);
-    lloyd_max_gaussian(P->kbits, P->ck.data(), P->tk.data());
+    if (beta) {
+        lloyd_max_beta(d, P->vbits, P->cv.data(), P->tv.data());
+        lloyd_max_beta(d, P->kbits, P->ck.data(), P->tk.data());
+    } else {
+        lloyd_max_gaussian(P->vbits, P->cv.data(), P->tv.data());
+        lloyd_max_gaussian(P->kbits, P->ck.data(), P->tk.data());
+    }
     return P;
 }
 void orc_destroy(void* h) { delete (Params*)h; }
