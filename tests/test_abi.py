@@ -78,3 +78,22 @@ def test_host_only_context_refuses_device_work(tq):
 def test_chunk_bytes(tq, bits, km, ck, cv):
     ctx = tq.tq_init_host(128, bits, 0, 0, km)
     assert tq.tq_chunk_bytes(ctx, tq.KIND_KEY) == ck and tq.tq_chunk_bytes(ctx, tq.KIND_VALUE) == cv
+
+
+def test_noalloc_size_constant_matches_header(tq):
+    src = open(os.path.join(ROOT, "include", "tq.h")).read()
+    m = re.search(r"#define\s+TQ_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", src)
+    assert m, "TQ_NOALLOC_SCRATCH_BYTES not found in tq.h"
+    assert int(m.group(1)) << int(m.group(2)) == tq.NOALLOC_SCRATCH_BYTES
+
+
+def test_noalloc_raw_call_refuses_bad_arguments(tq):
+    """The allocation-free entry point through the raw symbol: a null or host-only
+    context is refused on the host before any device is touched."""
+    L = tq._lib
+    f = L.tq_decode_attention_noalloc
+    args = (16, 16, 16, 1, 16, 1, 16, 1, 1, 1, 16, 0.0, 16, 1, None)
+    assert f(None, *args) == tq.TQ_ERR_INVALID_ARG
+    ctx = tq.tq_init_host(128, 4, 0)
+    assert f(ctx.handle, *args) == tq.TQ_ERR_INVALID_ARG
+    tq.tq_destroy(ctx)

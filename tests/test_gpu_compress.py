@@ -7,7 +7,8 @@ from parity import compare_compress, gpu_compress, gpu_ctx
 
 pytestmark = pytest.mark.gpu
 
-SETTINGS = [(0, 4, 0), (1, 4, 0), (0, 2, 0), (1, 3, 0), (0, 3, 1), (1, 2, 1)]  # (rot, bits, key_mode)
+# (rot, bits, key_mode): every (rotation, code width) pair of the compress kernels, both key modes
+SETTINGS = [(0, 4, 0), (1, 4, 0), (0, 2, 0), (1, 3, 0), (0, 3, 0), (0, 3, 1), (1, 2, 1)]
 
 
 def _read(orc_obj, kind, cache, slots, H):
@@ -35,7 +36,7 @@ def test_tiny_workload_full(orc, rot, bits, km):
     slots = W.prefill_slots(w, bt)
     o = orc.Oracle(128, bits, w.param_seed, rot=rot, key_mode=km, nthreads=0)
     ctx = gpu_ctx(bits, w.param_seed, rot, km)
-    _check_all(orc, o, ctx, k, v, slots, w.num_blocks, w.Hkv, "tiny")
+    _check_all(orc, o, ctx, k, v, slots, w.num_blocks, w.Hkv, "tiny rot%d b%d km%d" % (rot, bits, km))
 
 
 @pytest.mark.parametrize("rot,bits,km", SETTINGS[:3])
@@ -52,7 +53,7 @@ def test_ragged_shapes(orc, rot, bits, km, T, H):
     slots = (perm[np.arange(T) // 16] * 16 + np.arange(T) % 16).astype(np.int32)
     o = orc.Oracle(128, bits, 3, rot=rot, key_mode=km)
     ctx = gpu_ctx(bits, 3, rot, km)
-    _check_all(orc, o, ctx, k, v, slots, nb, H, "ragged T=%d H=%d" % (T, H))
+    _check_all(orc, o, ctx, k, v, slots, nb, H, "ragged T=%d H=%d rot%d b%d km%d" % (T, H, rot, bits, km))
 
 
 @pytest.mark.parametrize("rot", [0, 1])
@@ -64,7 +65,7 @@ def test_llama8b_prefill_full(orc, rot):
     slots = W.prefill_slots(w, bt)
     o = orc.Oracle(128, 4, w.param_seed, rot=rot)
     ctx = gpu_ctx(4, w.param_seed, rot, 0)
-    _check_all(orc, o, ctx, k, v, slots, w.num_blocks, w.Hkv, "llama8b")
+    _check_all(orc, o, ctx, k, v, slots, w.num_blocks, w.Hkv, "llama8b rot%d" % rot)
 
 
 def _sampled(orc, w, n_sample, seed):
@@ -96,7 +97,8 @@ def _sampled(orc, w, n_sample, seed):
         got = o.read_paged(kind, sub, sub_slots, w.Hkv)
         got = {kk: (vv.reshape(xs.shape[0], -1) if vv is not None and vv.ndim == 3 else
                     (vv.reshape(-1) if vv is not None else None)) for kk, vv in got.items()}
-        res[kind] = compare_compress(o, kind, xs, got, label="%s kind %d" % (w.name, kind))
+        res[kind] = compare_compress(o, kind, xs, got, label="%s rot%d b%d km%d kind %d (sampled)"
+                                     % (w.name, w.rotation, w.bits, w.key_mode, kind))
     del k, v, kc, vc
     torch.cuda.empty_cache()
     return res
@@ -114,7 +116,7 @@ def test_long70b_prefill_sampled(orc, rot, bits):
     _sampled(orc, W.WORKLOADS["long70b"].with_(rotation=rot, bits=bits), 1024, 6)
 
 
-@pytest.mark.parametrize("rot,bits", [(0, 4), (1, 3), (0, 2)])
+@pytest.mark.parametrize("rot,bits", [(0, 4), (1, 3), (0, 3), (0, 2)])
 def test_prefill80_sampled(orc, rot, bits):
     from kv_cache_vector_02_b200 import workloads as W
     _sampled(orc, W.WORKLOADS["prefill80"].with_(rotation=rot, bits=bits), 1024, 7)

@@ -4,7 +4,7 @@ import math
 import numpy as np
 import pytest
 
-from parity import DECODE_ATOL, gpu_compress, gpu_ctx
+from parity import DECODE_ATOL, check_decode, gpu_compress, gpu_ctx, record, zero_gamma
 
 pytestmark = pytest.mark.gpu
 
@@ -57,7 +57,7 @@ def test_tiny_decode_on_oracle_cache(orc, rot, bits, km):
     ctx = gpu_ctx(bits, w.param_seed, rot, km)
     got, err = _decode_gpu(ctx, q, kc, vc, bt, seq, w.T, w.Hkv)
     assert err == 0
-    assert np.abs(got - want).max() <= DECODE_ATOL
+    check_decode(got, want, "decode tiny rot%d b%d km%d" % (rot, bits, km))
 
 
 @pytest.mark.parametrize("B,T,Hkv,G,maxlen", [(3, 45, 2, 3, 64), (2, 1, 1, 16, 16), (4, 300, 2, 4, 300),
@@ -81,7 +81,7 @@ def test_ragged_decode_on_oracle_cache(orc, B, T, Hkv, G, maxlen):
     ctx = gpu_ctx(4, 9, 0, 0)
     got, err = _decode_gpu(ctx, q, kc, vc, bt, seq, maxlen, Hkv)
     assert err == 0
-    assert np.abs(got - want).max() <= DECODE_ATOL
+    check_decode(got, want, "decode ragged B%d T%d Hkv%d G%d" % (B, T, Hkv, G))
 
 
 def test_llama8b_compress_append_decode_end_to_end(orc):
@@ -119,6 +119,7 @@ def test_llama8b_compress_append_decode_end_to_end(orc):
             want = o.decode(q.numpy().astype(np.float64), kc_o, vc_o, bt, seq, w.Hkv)
             worst = max(worst, float(np.abs(out.cpu().numpy() - want).max()))
     assert tq.tq_get_device_error(ctx) == 0
+    record("decode llama8b 64 appended steps (worst)", {"decode_max_abs": worst, "outputs": w.B * w.Hq * 128 * 5})
     assert worst <= DECODE_ATOL, worst
 
 
@@ -142,7 +143,7 @@ def test_full_size_decode(orc, name, bits, rot, nseq):
     assert err == 0
     sel = rng.choice(w.B, size=nseq, replace=False)
     want = o.decode(q[sel].astype(np.float64), kc, vc, bt[sel], seq[sel], w.Hkv)
-    assert np.abs(got[sel] - want).max() <= DECODE_ATOL
+    check_decode(got[sel], want, "decode %s b%d rot%d (%d seqs)" % (name, bits, rot, nseq))
     torch.cuda.empty_cache()
 
 
@@ -184,3 +185,105 @@ def test_decompress_matches_oracle(orc, rot, bits, km):
         got = out.cpu().numpy()
         scale = np.linalg.norm(x.astype(np.float64), axis=-1, keepdims=True)
         assert np.abs(got - want).max() <= 1e-5 * scale.max()
+
+
+# Every instantiation of the split kernel: (key code mode, value code mode, QJL or not)
+# x (one or two tiles of 8 query heads).  bits 4 / 3 / 2 with prod keys (3-, 2-, 1-bit
+# key codes + signs) and with MSE keys (4-, 3-, 2-bit key codes).
+DECODE_MODES = [(0, 4, 0), (1, 3, 0), (1, 2, 0), (0, 4, 1), (1, 3, 1), (0, 2, 1)]
+
+
+@pytest.mark.parametrize("rot,bits,km", DECODE_MODES)
+@pytest.mark.parametrize("G", [4, 16])
+def test_every_decode_mode(orc, rot, bits, km, G):
+    o = orc.Oracle(128, bits, 21, rot=rot, key_mode=km)
+    rng = np.random.default_rng(100 * bits + 10 * km + G)
+    B, T, Hkv, maxlen = 3, 211, 2, 224
+    nbps = (maxlen + 15) // 16
+    nb = B * nbps + 2
+    bt = rng.permutation(nb)[: B * nbps].reshape(B, nbps).astype(np.int32)
+    seq = np.array([T, 17, 160], np.int32)
+    kc, vc = o.new_cache(0, nb, Hkv), o.new_cache(1, nb, Hkv)
+    for b in range(B):
+        t = np.arange(T)
+        sl = (bt[b][t // 16] * 16 + t % 16).astype(np.int32)
+        o.compress_paged(0, (rng.standard_normal((T, Hkv, 128)) * 2).astype(np.float16), sl, kc)
+        o.compress_paged(1, rng.standard_normal((T, Hkv, 128)).astype(np.float16), sl, vc)
+    q = (rng.standard_normal((B, G * Hkv, 128)) * 3 / math.sqrt(128)).astype(np.float16)
+    want = o.decode(q.astype(np.float64), kc, vc, bt, seq, Hkv)
+    ctx = gpu_ctx(bits, 21, rot, km)
+    got, err = _decode_gpu(ctx, q, kc, vc, bt, seq, maxlen, Hkv)
+    assert err == 0
+    check_decode(got, want, "decode mode rot%d b%d km%d G%d" % (rot, bits, km, G))
+
+
+def _logit_spread(q, k, scale=1 / math.sqrt(128)):
+    """Spread (max - min over tokens, smallest over heads) of the exact logits
+    q.k * scale: how far the softmax is from uniform."""
+    lg = np.einsum("hd,td->ht", q.astype(np.float64), k.astype(np.float64)) * scale
+    return float((lg.max(1) - lg.min(1)).min())
+
+
+def _power_check(o, got, want, kc, vc, bt, seq, Hkv, q, label):
+    """The GPU output is within the bar of the oracle, and at least 10x its own error
+    away from the oracle without the QJL term (gamma zeroed): a decode that dropped
+    or mangled that term could not pass."""
+    err = check_decode(got, want, label)
+    want0 = o.decode(q.astype(np.float64), zero_gamma(o, kc), vc, bt, seq, Hkv)
+    gap = float(np.abs(np.asarray(got, np.float64) - want0).max())
+    record(label + " [no-QJL gap]", {"decode_max_abs": gap, "outputs": int(want0.size),
+                                     "ratio": gap / max(err, 1e-30)})
+    assert gap >= 10 * err, "%s: no-QJL oracle only %.2e away, GPU error %.2e" % (label, gap, err)
+
+
+@pytest.mark.parametrize("rot", [0, 1])
+def test_peaked_tiny_decode_power(orc, rot):
+    """Tiny workload with q scaled x8 (logits spread over several units)."""
+    from kv_cache_vector_02_b200 import workloads as W
+    w = W.WORKLOADS["tiny"].with_(rotation=rot)
+    o = orc.Oracle(128, w.bits, w.param_seed, rot=rot)
+    bt = W.block_table(w)
+    slots = W.prefill_slots(w, bt)
+    k, v = W.gen_kv(w, 0).numpy(), W.gen_kv(w, 1).numpy()
+    kc, vc = o.new_cache(0, w.num_blocks, 1), o.new_cache(1, w.num_blocks, 1)
+    o.compress_paged(0, k, slots, kc)
+    o.compress_paged(1, v, slots, vc)
+    q = (W.gen_q(w).numpy().astype(np.float32) * 8).astype(np.float16)
+    spread = _logit_spread(q[0], k[:, 0])
+    assert spread >= 3.0, spread
+    seq = np.array([w.T], np.int32)
+    want = o.decode(q.astype(np.float64), kc, vc, bt, seq, 1)
+    ctx = gpu_ctx(w.bits, w.param_seed, rot, 0)
+    got, err = _decode_gpu(ctx, q, kc, vc, bt, seq, w.T, 1)
+    assert err == 0
+    _power_check(o, got, want, kc, vc, bt, seq, 1, q, "decode tiny peaked x8 rot%d (spread %.1f)" % (rot, spread))
+
+
+def test_peaked_batched_decode_power(orc):
+    """Batched workload (32 x 4096 tokens, 8 kv / 32 q heads) with q scaled x4, on a
+    cache that libtq compressed from the workload's own K and V; the oracle decodes
+    three sequences of it."""
+    import torch
+    from kv_cache_vector_02_b200 import tq, workloads as W
+    w = W.WORKLOADS["batched"]
+    o = orc.Oracle(128, w.bits, w.param_seed)
+    ctx = gpu_ctx(w.bits, w.param_seed, 0, 0)
+    bt = W.block_table(w)
+    slots = W.prefill_slots(w, bt)
+    k = W.gen_kv(w, 0, device="cuda")
+    v = W.gen_kv(w, 1, device="cuda")
+    kc, vc = gpu_compress(ctx, k, v, slots, w.num_blocks, w.Hkv)
+    q = (W.gen_q(w).numpy().astype(np.float32) * 4).astype(np.float16)
+    seq = np.full(w.B, w.T, np.int32)
+    got, err = _decode_gpu(ctx, q, kc, vc, bt, seq, w.T, w.Hkv)
+    assert err == 0
+    sel = np.array([0, 13, 31])
+    k0 = k[: w.T, 0].float().cpu().numpy()   # sequence 0, kv head 0
+    spread = _logit_spread(q[0, :4], k0)
+    assert spread >= 3.0, spread
+    kc_h, vc_h = kc.cpu().numpy(), vc.cpu().numpy()
+    want = o.decode(q[sel].astype(np.float64), kc_h, vc_h, bt[sel], seq[sel], w.Hkv)
+    _power_check(o, got[sel], want, kc_h, vc_h, bt[sel], seq[sel], w.Hkv, q[sel],
+                 "decode batched peaked x4 (3 seqs, spread %.1f)" % spread)
+    del k, v, kc, vc
+    torch.cuda.empty_cache()
