@@ -103,6 +103,23 @@ typedef enum { TQ_KIND_KEY = 0, TQ_KIND_VALUE = 1 } tq_kind;
  */
 TQ_API tq_status tq_init(int head_dim, int bits, uint64_t seed, int rotation, int key_mode, tq_ctx** out);
 
+/* tq_init_ex flags. */
+#define TQ_FLAG_SPHERE_CODEBOOK 0x1  /* exact-d Lloyd-Max codebooks instead of the Gaussian ones */
+#define TQ_FLAG_HOST_ONLY       0x4  /* build the parameters on the host only (as tq_init_host) */
+
+/*
+ * tq_init_ex -- tq_init with options (tq_init = tq_init_ex with flags 0).
+ *   TQ_FLAG_SPHERE_CODEBOOK: both codebooks are the Lloyd-Max quantizers of the
+ *     exact law of a rotated unit vector's coordinate, v = sqrt(d) u_1 with u uniform
+ *     on the sphere ((u_1 + 1)/2 ~ Beta((d-1)/2, (d-1)/2)), instead of its large-d
+ *     limit N(0, 1) [TQ-RS "Étape 2" and "Couche 2": the spherical Beta law].  Only
+ *     the codebooks and bucketize tables change; every call works as with tq_init.
+ *   TQ_FLAG_HOST_ONLY: as tq_init_host.
+ * Unknown flags give TQ_ERR_UNSUPPORTED.
+ */
+TQ_API tq_status tq_init_ex(int head_dim, int bits, uint64_t seed, int rotation, int key_mode, int flags,
+                            tq_ctx** out);
+
 /*
  * tq_init_host -- the same parameters as tq_init, built on the host only: no
  * device is touched and nothing is allocated on one.  Such a context serves
@@ -111,8 +128,9 @@ TQ_API tq_status tq_init(int head_dim, int bits, uint64_t seed, int rotation, in
  */
 TQ_API tq_status tq_init_host(int head_dim, int bits, uint64_t seed, int rotation, int key_mode, tq_ctx** out);
 
-/* tq_destroy -- free a context (NULL is accepted).  Synchronizes the device of a
- * device context first. */
+/* tq_destroy -- free a context (NULL is accepted).  First waits for the work this
+ * context has queued (on every stream it was given, up to each stream's latest
+ * call), not for the whole device; the CUDA runtime's free may still wait for more. */
 TQ_API tq_status tq_destroy(tq_ctx* ctx);
 
 /* Bytes of one chunk (16 tokens, one kv head) for kind (tq_kind); 0 on error. */
@@ -166,9 +184,9 @@ TQ_API tq_status tq_decompress(const tq_ctx* ctx, int kind, const uint8_t* cache
  * tq_decode_workspace_bytes -- device scratch needed by tq_decode_attention for
  * B sequences, Hq query heads over Hkv kv heads and sequences of at most
  * max_seq_len tokens (0 on invalid arguments).
- * The workspace must be zero-filled once when it is allocated; the decode
- * leaves it zero-filled where that matters, so it can be reused without
- * clearing.  Two decodes that run at the same time need separate workspaces.
+ * Nothing in the workspace has to start at zero and it needs no clearing between
+ * calls: every byte a decode reads is written earlier in the same call.  Two
+ * decodes that run at the same time need separate workspaces.
  */
 TQ_API size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_seq_len);
 
@@ -191,13 +209,38 @@ TQ_API size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hk
  *   scale          : softmax scale; pass 0 for the default 1/sqrt(d).
  *   out_dev        : [B][Hq][128], fp16 (out_fp32 = 0) or fp32 (out_fp32 = 1).
  *   workspace_dev  : >= tq_decode_workspace_bytes(ctx, B, Hq, Hkv, max_seq_len) bytes,
- *                    zero-filled at allocation (see above).
+ *                    any contents (see above).
  */
 TQ_API tq_status tq_decode_attention(const tq_ctx* ctx, const uint16_t* q_dev, const uint8_t* k_cache_dev,
                               const uint8_t* v_cache_dev, int num_blocks, const int32_t* block_table_dev,
                               int max_blocks, const int32_t* seq_lens_dev, int B, int Hq, int Hkv, int max_seq_len,
                               float scale, void* out_dev, int out_fp32, void* workspace_dev, size_t workspace_bytes,
                               void* stream);
+
+/*
+ * tq_decode_attention_window -- tq_decode_attention with an fp16 residual window
+ * [TQ-RS "Couche 5 — Fenêtre résiduelle" and "Couche 7" (residual_window=128); the
+ * KIVI page's FP16 residual of the most recent tokens].  The last tail_lens[b]
+ * tokens of sequence b are kept uncompressed; they join the same softmax as its
+ * seq_lens[b] compressed tokens:
+ *   s_u = scale * <q, k_u>,   o = sum_t p_t v_hat_t + sum_u p_u v_u,
+ * p the softmax over both sets (reading: one softmax over the compressed and the
+ * window tokens; the pages give only the window's name and size).
+ *   tail_k_dev, tail_v_dev : [B][tail_cap][Hkv][128] fp16, device, 16-byte aligned;
+ *                            row u < tail_lens[b] of sequence b is window token u.
+ *   tail_lens_dev          : [B] int32, device; a length outside [0, tail_cap] is
+ *                            taken as 0 and sets TQ_DEVERR_SEQLEN.
+ *   tail_cap               : 1 .. 256 (TQ_ERR_INVALID_ARG otherwise).
+ * Every other argument, the workspace size and the results are those of
+ * tq_decode_attention (which is this call without a window).
+ */
+TQ_API tq_status tq_decode_attention_window(const tq_ctx* ctx, const uint16_t* q_dev, const uint8_t* k_cache_dev,
+                                            const uint8_t* v_cache_dev, int num_blocks,
+                                            const int32_t* block_table_dev, int max_blocks,
+                                            const int32_t* seq_lens_dev, int B, int Hq, int Hkv, int max_seq_len,
+                                            const uint16_t* tail_k_dev, const uint16_t* tail_v_dev,
+                                            const int32_t* tail_lens_dev, int tail_cap, float scale, void* out_dev,
+                                            int out_fp32, void* workspace_dev, size_t workspace_bytes, void* stream);
 
 /*
  * Size of the device array behind tq_decode_attention_noalloc.  Every GPU that
@@ -237,6 +280,19 @@ TQ_API tq_status tq_decode_attention_noalloc(const tq_ctx* ctx, const uint16_t* 
  * the word was non-zero, TQ_OK otherwise.
  */
 TQ_API tq_status tq_get_device_error(const tq_ctx* ctx, void* stream, uint32_t* code);
+
+/*
+ * tq_debug_stall -- test hook for the failure-detection path (no counterpart on
+ * the pages).  The next `launches` kernels of this context that stream their
+ * inputs through asynchronous copies (the compress kernels; the decode page
+ * kernel) skip issuing those copies, so the waits that expect them run out after
+ * their bounded limit (about 2 s): the kernel sets TQ_DEVERR_TIMEOUT in the device
+ * error word, abandons its work (its outputs are then undefined), releases what it
+ * holds and returns.  Nothing faults or hangs, and the context stays usable.
+ * launches = 0 cancels a pending stall.  Returns TQ_ERR_INVALID_ARG for a null or
+ * host-only context or a negative count.
+ */
+TQ_API tq_status tq_debug_stall(tq_ctx* ctx, int launches);
 
 /* Number of kernels libtq has launched in this process so far (all contexts,
  * all devices).  Lets a caller count the library's launches in a region. */

@@ -40,6 +40,7 @@
 //   Haar      acc2 = rho_lo M_hi + rho_hi M_lo + rho_hi M_hi   (M = S R)
 //   Hadamard  acc2 = (rho_lo + rho_hi) M',   M' = S D H integer, exact in fp16
 // sign bit j = [acc2_j >= 0].  Every wait is bounded (TQ_DEVERR_TIMEOUT).
+#include <atomic>
 #include <cmath>
 
 #include <cuda.h>
@@ -133,6 +134,7 @@ struct TcArgs {
     float n_scale;     // ||x|| = n_scale * ||acc||
     float gamma_scale; // n_scale / (sqrt(d) * table scale): gamma = ||d|| ||acc|| gamma_scale
     uint32_t* err;
+    int stall;         // test hook: load no x tile (every wait for one runs out)
 };
 
 __device__ __forceinline__ void set_abort(volatile int* abort, uint32_t* err) {
@@ -257,7 +259,8 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD, PAIR>::kBound, 1) compress_tc_k
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             int issued = 0;
-            for (int k = 0; k < my_tiles; ++k) {
+            const int to_load = a.stall ? 0 : my_tiles;
+            for (int k = 0; k < to_load; ++k) {
                 const int s = k % C::kStages;
                 const uint32_t ph = (uint32_t)(k / C::kStages) & 1u;
                 if (!mbar_wait(bar(kBarXEmpty + s), ph ^ 1u, abort, kWaitNs)) {
@@ -719,11 +722,12 @@ template <int ROT, bool PROD, int W, bool PAIR>
 cudaError_t launch_tc(const CUtensorMap& tmap, const TcArgs& a, int sm_count, cudaStream_t stream) {
     using C = Cfg<ROT, PROD, PAIR>;
     auto k = compress_tc_kernel<ROT, PROD, W, PAIR>;
-    // CTAs (pair: clusters) of this kernel resident at once, per device
-    static int resident_of[64] = {};
+    // CTAs (pair: clusters) of this kernel resident at once, per device; computed once
+    // and published atomically (two threads computing it at once store the same value)
+    static std::atomic<int> resident_of[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    int& resident = resident_of[dev];
+    int resident = resident_of[dev].load(std::memory_order_relaxed);
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(C::kThreads);
     cfg.dynamicSmemBytes = C::kSmem;
@@ -749,6 +753,7 @@ cudaError_t launch_tc(const CUtensorMap& tmap, const TcArgs& a, int sm_count, cu
             if (clusters > 0 && clusters < n) n = clusters;
         }
         resident = n > 0 ? n : 1;
+        resident_of[dev].store(resident, std::memory_order_relaxed);
     }
     const int rows = PAIR ? 256 : 128;
     const int ntiles = (a.N + rows - 1) / rows;
@@ -788,6 +793,7 @@ cudaError_t launch_compress_tc(const tq_ctx* ctx, int kind, const uint16_t* x, i
     a.gamma_scale = (float)(n_scale / (std::sqrt((double)kDim) * (double)lp.scale));
     a.lay = lay;
     a.err = ctx->dev_error;
+    a.stall = take_stall(ctx) ? 1 : 0;
     const int W = container_width(value ? ctx->host.vbits : ctx->host.kbits);
     cudaError_t e = cudaErrorInvalidValue;
     // every kind runs as MMA pairs on the two SMs of 2-CTA clusters, 256 rows a tile

@@ -9,22 +9,33 @@
 // once per query head (o = R acc / l).
 //
 // Kernels:
-//   prep   one CTA per (sequence, kv head): q' = R^T q and s = S q for its G query
-//          heads, stored fp16.
-//   split  persistent CTAs over items (sequence, kv head, page range); each warp
-//          takes one 16-token page at a time:
+//   prep   q' = R^T q and s = S q for every query head (fp32), and the page prefix
+//          sums of the sequences.
+//   split  one persistent CTA per SM over an equal range of the pages of all
+//          (sequence, kv head) units; page p of a unit's piece goes to warp p % kNW.
+//          Each warp streams its own pages (one bulk copy each of the key and the
+//          value chunk) into its ring of shared-memory stages, its issue cursor
+//          running ahead across pieces, and per 16-token page:
 //            scores  D[16 tok x 8 heads] = sum_k Khat[tok][k] q'[k][h]   (mma m16n8k16)
 //                    plus the sign term with +-1 fragments against s
 //            softmax online, base 2, per head column
 //            values  D[16 coords x 8 heads] += Vhat^T[coord][tok] P'[tok][h]
-//          Packed codes become fp16 fragments in registers: key codes (<= 8 levels)
-//          through byte permutes of an 8-entry table, sign nibbles and value bytes
-//          through small shared-memory tables (the value table is replicated per
-//          lane so a warp's 32 lookups never share a bank).  Coordinates are
-//          permuted inside each contraction so that a thread's fragment elements
-//          are contiguous packed bytes.  The warps of a CTA merge their states;
-//          each item's partial (m, l, acc) goes to the workspace.
-//   merge  log-sum-exp combination of the splits, division by l, un-rotation.
+//          The warps of the CTA merge their states per piece; each piece's partial
+//          (m, l, acc) goes to the workspace.
+//   merge  log-sum-exp combination of a unit's pieces, division by l, un-rotation.
+//
+// Packed codes become fp16 MMA fragments in registers:
+//   - 3-bit key codes (nibbles): byte permutes of an 8-entry register table;
+//   - value codes: two tokens' codes of one coordinate are merged into one "pair
+//     byte" (two ALU ops per 4 or 8 pair bytes), and one PRMT builds the full
+//     shared-memory address of the pair byte's entry in a lane-replicated table
+//     (tables sit at shared address 64 KiB, 256 bytes per entry, so the address is
+//     0x10000 | byte << 8 | lane offset); one LDS then gives the fragment register;
+//   - sign bits (and 1- or 2-bit key codes, taken as +-1 bit planes): one LDS.128
+//     per sign byte from an 8-fold replicated table gives four +-1 fragment
+//     registers.
+// Inside a page the token order is permuted (row r holds token r ^ ((r >> 1) & 1))
+// so that a warp's loads of four tokens' value bytes meet at most two to a bank.
 #include <algorithm>
 #include <cmath>
 #include <mutex>
@@ -35,17 +46,32 @@
 namespace tq {
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kThreads = kWarps * 32;
-constexpr int kMaxG = 16;
-constexpr int kPartStride = kDim + 2;  // m, l, acc[128]
+constexpr int kNW = 12;                       // warps per split CTA (one CTA per SM, three per scheduler)
+constexpr int kSplitThreads = kNW * 32;
+constexpr int kPartStride = kDim + 2;         // m, l, acc[128]
+constexpr int kStages = 3;                    // page stages per warp
+constexpr uint32_t kStageBytes = 2496;        // >= key chunk + value chunk at every bit width (16-byte multiple)
+constexpr uint32_t kTabAddr = 65536;          // shared-window address of the lookup tables
+constexpr uint32_t kTabBytes = 65536;         // 256 entries x 256 bytes
+constexpr uint32_t kRingAddr = kTabAddr + kTabBytes;
+constexpr uint32_t kRingBytes = kNW * kStages * kStageBytes;
+constexpr uint32_t kSplitSmem = kRingAddr + kRingBytes;  // dynamic bytes: enough for any window base >= 0
+// Below the tables, from the window base: barriers, per-stage valid flags, the abort
+// flag, the warps' (m, l) and the CTA merge area (one tile of 8 heads at a time).
+constexpr uint32_t kOffFull = 0;                                // [kNW][kStages] mbarrier: page landed
+constexpr uint32_t kOffValid = kOffFull + kNW * kStages * 8;    // [kNW][kStages] int: the block id was valid
+constexpr uint32_t kOffAbort = kOffValid + kNW * kStages * 4;   // int
+constexpr uint32_t kOffML = (kOffAbort + 4 + 15) & ~15u;        // [kNW][2][8] float: m, l
+constexpr uint32_t kOffMerge = kOffML + kNW * 2 * 8 * 4;        // [kNW][8][128] float
+constexpr uint32_t kLowBytes = kOffMerge + kNW * 8 * kDim * 4;
+constexpr uint64_t kWaitNs = 2000000000ull;
 
 enum KMode { kKPrmt = 0, kKByte4 = 1, kKByte2 = 2, kKBit1 = 3 };
 enum VMode { kVByte4 = 0, kVByte2 = 1 };
 
 struct DecodeArgs {
     const uint16_t* q;
-    __half* qf;  // [B][Hq][2][128] fp16: q' then s
+    float* qf;  // [B][Hq][2][128] fp32: q' then s
     const uint8_t* kc;
     const uint8_t* vc;
     int num_blocks;
@@ -53,7 +79,6 @@ struct DecodeArgs {
     int max_blocks;
     const int32_t* seq_lens;
     int B, Hq, Hkv, G, max_seq_len;
-    float scale_log2;  // softmax scale * log2(e)
     float* partial;    // [slots][G][130]: m, l, acc (rotated domain)
     int* prefix;       // [B + 1] pages of the sequences before b (prep writes it)
     int split_grid;    // CTAs of the split kernel
@@ -63,10 +88,20 @@ struct DecodeArgs {
     const uint16_t* RTl;
     const uint16_t* Sh;
     float qscale, sscale;  // scale*log2(e)/sqrt(d), scale*log2(e)*sqrt(pi/2)/d
+    float kscale;          // 1-bit keys: the level c[1] (key term = c1 <q', 2b - 1>)
+    float kalpha, kbeta;   // 2-bit keys: c[code] = alpha (2 b1 - 1) + beta (2 b0 - 1)
     Codebook cbk, cbv;
     ChunkLayout lk, lv;
     void* out;
     int out_fp32;
+    int stall;             // test hook: the producer copies no page
+    // residual window: fp16 keys / values [B][tail_cap][Hkv][128] of the last tail_lens[b]
+    // tokens of each sequence, uncompressed (tail_k == NULL: none)
+    const uint16_t* tail_k;
+    const uint16_t* tail_v;
+    const int32_t* tail_lens;
+    int tail_cap;
+    float scale_log2;      // softmax scale * log2(e)
     uint32_t* err;
 };
 
@@ -87,10 +122,67 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Transpose of an 8x8 fp16 matrix held as m8n8 fragments (thread 4 g + c holds row g,
+// columns 2c, 2c + 1): afterwards it holds row g of the transpose.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t h2bits(__half lo, __half hi) {
+    return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+}
+__device__ __forceinline__ uint32_t f2h2(float lo, float hi) { return h2bits(__float2half_rn(lo), __float2half_rn(hi)); }
+
+__device__ __forceinline__ __half cb_half(const Codebook& cb, int code) {
+    float v = 0.f;
+#pragma unroll
+    for (int k = 0; k < kMaxLevels; ++k) v = (k == code) ? cb.c[k] : v;
+    return __float2half_rn(v);
+}
+
+// Table reads at 32-bit shared-window addresses (the table is written once, before
+// a CTA barrier, and never again).
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t x;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(x) : "r"(addr));
+    return x;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 x;
+    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(x.x), "=r"(x.y) : "r"(addr));
+    return x;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 x;
+    asm("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w) : "r"(addr));
+    return x;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+
+// Shared-window address of the table entry of byte K of p: 0x10000 | p.byte[K] << 8 |
+// L.byte[X], where L holds this lane's offsets inside an entry in bytes 0 and 1 and
+// 0x01, 0x00 in bytes 2 and 3 (one PRMT).
+template <int K, int X>
+__device__ __forceinline__ uint32_t taddr(uint32_t p, uint32_t L) {
+    return __byte_perm(p, L, 0x7600u | (K << 4) | (4 + X));
+}
+
+// Lazy softmax rescaling: the running maximum only moves when a page exceeds it by
+// more than 2^kSlack (log2 units), so exponentials stay <= 2^kSlack in fp32 / fp16.
+constexpr float kSlack = 8.f;
+
+// Token of page row r (see the file comment).
+__host__ __device__ constexpr int row_token(int r) { return r ^ ((r >> 1) & 1); }
+
 // ------------------------------------------------------------------ prep
 // [q' | s] = q [R | S^T] for 16 query heads per CTA, on mma.sync (fp16 inputs, fp32
-// accumulation; R^T enters as fp16 hi + lo, S is exact).  CTA (x, y), warp w
-// computes output columns 8 (8 y + w) .. +7 of the 256 (q' then s).
+// accumulation; R^T enters as fp16 hi + lo, S is exact); fp32 results.  CTA (x, y),
+// warp w computes output columns 8 (8 y + w) .. +7 of the 256 (q' then s).  CTA (0, 0)
+// also writes the page prefix sums of the sequences.
 constexpr int kPrepThreads = 256;
 __global__ void __launch_bounds__(kPrepThreads) decode_prep_kernel(DecodeArgs a) {
     griddep_wait();  // q and seq_lens may come from the kernel before
@@ -136,66 +228,169 @@ __global__ void __launch_bounds__(kPrepThreads) decode_prep_kernel(DecodeArgs a)
         A[ks][2] = r0 ? q0[8 * ks + c + 4] : 0u;
         A[ks][3] = r1 ? q1[8 * ks + c + 4] : 0u;
     }
-    {
-        const int nt = blockIdx.y * 8 + warp;  // 0..15 -> q', 16..31 -> s
-        const bool isq = nt < 16;
-        const int n = (nt & 15) * 8 + g;
-        const uint32_t* bh = reinterpret_cast<const uint32_t*>((isq ? a.RTh : a.Sh) + (size_t)n * kDim);
-        const uint32_t* bl = reinterpret_cast<const uint32_t*>(a.RTl + (size_t)n * kDim);
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
+    const int nt = blockIdx.y * 8 + warp;  // 0..15 -> q', 16..31 -> s
+    const bool isq = nt < 16;
+    const int n = (nt & 15) * 8 + g;
+    const uint32_t* bh = reinterpret_cast<const uint32_t*>((isq ? a.RTh : a.Sh) + (size_t)n * kDim);
+    const uint32_t* bl = reinterpret_cast<const uint32_t*>(a.RTl + (size_t)n * kDim);
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            mma16816(d, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bh[8 * ks + c], bh[8 * ks + c + 4]);
-            if (isq) mma16816(d, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bl[8 * ks + c], bl[8 * ks + c + 4]);
-        }
-        const int col = (nt & 15) * 8 + 2 * c, which = isq ? 0 : 1;
-        if (r0)
-            *reinterpret_cast<__half2*>(a.qf + ((size_t)(h0 + g) * 2 + which) * kDim + col) = __floats2half2_rn(d[0], d[1]);
-        if (r1)
-            *reinterpret_cast<__half2*>(a.qf + ((size_t)(h0 + g + 8) * 2 + which) * kDim + col) =
-                __floats2half2_rn(d[2], d[3]);
+    for (int ks = 0; ks < 8; ++ks) {
+        if (isq) mma16816(d, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bl[8 * ks + c], bl[8 * ks + c + 4]);
+        mma16816(d, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bh[8 * ks + c], bh[8 * ks + c + 4]);
+    }
+    const int col = (nt & 15) * 8 + 2 * c, which = isq ? 0 : 1;
+    if (r0) *reinterpret_cast<float2*>(a.qf + ((size_t)(h0 + g) * 2 + which) * kDim + col) = make_float2(d[0], d[1]);
+    if (r1) *reinterpret_cast<float2*>(a.qf + ((size_t)(h0 + g + 8) * 2 + which) * kDim + col) = make_float2(d[2], d[3]);
+}
+
+// ------------------------------------------------------------------ split: tables
+// Entry e (a byte) of the 64 KiB table at kTabAddr is 256 bytes:
+//   bytes   0..127  region A, values:
+//                     nibble pair bytes (low nibble: token t, high: token t + 1):
+//                       half2(c[e & 15], c[e >> 4]), 32 copies (lane * 4);
+//                     crumb pair bytes (crumbs: tokens t, t + 1 of a coordinate j,
+//                     then of coordinate j + 2): {half2 of j, half2 of j + 2}, 16
+//                     copies ((lane % 16) * 8)
+//   bytes 128..255  region B, keys:
+//                     sign bytes (bit = 1 -> +1): four half2 {bits 0,1 | 2,3 | 4,5 |
+//                     6,7}, 8 copies (128 + (lane % 8) * 16) -- the QJL signs and the
+//                     bit planes of 1- and 2-bit key codes;
+//                     or (4-bit MSE keys) nibble pair bytes of one token:
+//                     half2(c[e & 15], c[e >> 4]), 32 copies (128 + lane * 4)
+template <int KM, int VM, bool PROD>
+__device__ void build_tables(const DecodeArgs& a, int e) {
+    const uint32_t row = kTabAddr + 256u * (uint32_t)e;
+    if (VM == kVByte4) {
+        const uint32_t w = h2bits(cb_half(a.cbv, e & 15), cb_half(a.cbv, e >> 4));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sts128(row + 16 * i, w, w, w, w);
+    } else {
+        const uint32_t x = h2bits(cb_half(a.cbv, e & 3), cb_half(a.cbv, (e >> 2) & 3));
+        const uint32_t y = h2bits(cb_half(a.cbv, (e >> 4) & 3), cb_half(a.cbv, e >> 6));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sts128(row + 16 * i, x, y, x, y);
+    }
+    constexpr bool kSignTab = PROD || KM == kKByte2 || KM == kKBit1;
+    if (kSignTab) {
+        const __half one = __float2half_rn(1.f), mone = __float2half_rn(-1.f);
+        auto pm = [&](int bit) { return ((e >> bit) & 1) ? one : mone; };
+        const uint32_t x = h2bits(pm(0), pm(1)), y = h2bits(pm(2), pm(3));
+        const uint32_t z = h2bits(pm(4), pm(5)), w = h2bits(pm(6), pm(7));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sts128(row + 128 + 16 * i, x, y, z, w);
+    } else if (KM == kKByte4) {
+        const uint32_t w = h2bits(cb_half(a.cbk, e & 15), cb_half(a.cbk, e >> 4));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sts128(row + 128 + 16 * i, w, w, w, w);
     }
 }
 
-// Transpose of an 8x8 fp16 matrix held as m8n8 fragments (thread 4 g + c holds row g,
-// columns 2c, 2c + 1): afterwards it holds row g of the transpose.
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
-    uint32_t d;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
-    return d;
-}
+// ------------------------------------------------------------------ split: pieces
+// The CTA's range [pos, end) of the pages of all units in order (unit u = b Hkv + h
+// holds the pages of sequence b), cut into pieces by unit.
+struct Pieces {
+    long pos, end;
+    int b;
+    __device__ void init(const DecodeArgs& a, long p, long e) {
+        pos = p;
+        end = e;
+        b = 0;
+        if (pos < end) {  // the last sequence b with Hkv * prefix[b] <= pos
+            int lo = 0, hi = a.B - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if ((long)a.Hkv * a.prefix[mid] <= pos) lo = mid;
+                else hi = mid - 1;
+            }
+            b = lo;
+        }
+    }
+    // next piece: sequence bb, kv head hk, pages [p0, p1) of the sequence
+    __device__ bool next(const DecodeArgs& a, int& bb, int& hk, int& p0, int& p1) {
+        while (pos < end && b < a.B) {
+            const int np = a.prefix[b + 1] - a.prefix[b];
+            const long off = pos - (long)a.Hkv * a.prefix[b];
+            if (np == 0 || off >= (long)a.Hkv * np) {
+                ++b;
+                continue;
+            }
+            hk = (int)(off / np);
+            p0 = (int)(off - (long)hk * np);
+            p1 = (int)min((long)np, p0 + (end - pos));
+            pos += p1 - p0;
+            bb = b;
+            return true;
+        }
+        return false;
+    }
+};
 
-__device__ __forceinline__ uint32_t h2bits(__half lo, __half hi) {
-    return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
-}
+// The pages of one warp (p0 + warp, + kNW, ...) of every piece of the CTA, in
+// order, with their block ids: lane l holds the block id of the warp's page
+// wbase + l of the piece, and the next 32 are loaded 16 pages ahead of their use.
+struct PageCursor {
+    Pieces it;
+    int b, hk, p0, p1, ji, nj;
+    bool live;
+    int win, win_next, wbase;
+    __device__ int load_win(const DecodeArgs& a, int warp, int lane, int base) const {
+        const int jj = base + lane;
+        return jj < nj ? a.block_table[(size_t)b * a.max_blocks + p0 + warp + jj * kNW] : -1;
+    }
+    __device__ void enter(const DecodeArgs& a, int warp, int lane) {  // the next piece with pages for this warp
+        live = false;
+        while (it.next(a, b, hk, p0, p1)) {
+            nj = p0 + warp < p1 ? (p1 - p0 - warp + kNW - 1) / kNW : 0;
+            if (nj == 0) continue;
+            ji = 0;
+            wbase = 0;
+            win = load_win(a, warp, lane, 0);
+            win_next = -1;
+            live = true;
+            return;
+        }
+    }
+    __device__ void init(const DecodeArgs& a, long pos, long end, int warp, int lane) {
+        it.init(a, pos, end);
+        enter(a, warp, lane);
+    }
+    // block id of the current page (warp-uniform; every lane calls it)
+    __device__ int block() const { return __shfl_sync(0xffffffffu, win, ji - wbase); }
+    __device__ void advance(const DecodeArgs& a, int warp, int lane) {
+        ++ji;
+        if (ji >= nj) {
+            enter(a, warp, lane);
+            return;
+        }
+        if (ji - wbase == 16 && wbase + 32 < nj) win_next = load_win(a, warp, lane, wbase + 32);
+        if (ji - wbase == 32) {
+            wbase = ji;
+            win = win_next;
+        }
+    }
+};
 
-__device__ __forceinline__ __half cb_half(const Codebook& cb, int code) {
-    float v = 0.f;
-#pragma unroll
-    for (int k = 0; k < kMaxLevels; ++k) v = (k == code) ? cb.c[k] : v;
-    return __float2half_rn(v);
-}
-
-// Raw bytes of one page that one thread needs (lane = 4 g + c), with the per-token
-// scalars already multiplied by the constants of the score and of P'.
+// ------------------------------------------------------------------ split: one page
 template <int KM, int VM, bool PROD>
 struct PageRegs {
     uint32_t k[2][4];    // key code bytes of token rows g, g+8 (coords 32c .. 32c+31)
     uint32_t s[2];       // sign word c of rows g, g+8
-    float kn[2], kg[2];  // key norm * qscale, gamma * sscale of tokens g, g+8
-    uint32_t v[4][2];    // value code bytes of token rows 2c, 2c+1, 2c+8, 2c+9 (coords 16g .. 16g+15)
-    float vn[2];         // value norm / sqrt(d) of tokens g, g+8
+    float kn[2], kg[2];  // key norm * qscale, gamma * sscale of rows g, g+8
+    uint32_t v[4][2];    // value code bytes of rows 2c, 2c+1, 2c+8, 2c+9 (coords 16g .. 16g+15)
+    float vn[2];         // value norm / sqrt(d) of rows g, g+8
 };
 
-// Fragment bytes of one page from its shared-memory stage (key chunk at kst, value
-// chunk at vst).
+// Fragment bytes of one page from its stage (key chunk at kst, value chunk at vst);
+// krow[i], vrow[i]: byte offsets of this thread's rows' tokens (see row_token).
 template <int KM, int VM, bool PROD>
 __device__ __forceinline__ void load_page(PageRegs<KM, VM, PROD>& r, const uint8_t* kst, const uint8_t* vst,
-                                          const DecodeArgs& a, int g, int c) {
+                                          const DecodeArgs& a, const int (&tk)[2], const int (&tv)[4], int g,
+                                          int c) {
     constexpr int kBytes = KM == kKBit1 ? 4 : (KM == kKByte2 ? 8 : 16);  // per key row per thread
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-        const uint8_t* row = kst + (g + 8 * i) * a.lk.code_row + kBytes * c;
+        const uint8_t* row = kst + tk[i] * a.lk.code_row + kBytes * c;
         if (kBytes == 16) {
             const uint4 w = *reinterpret_cast<const uint4*>(row);
             r.k[i][0] = w.x, r.k[i][1] = w.y, r.k[i][2] = w.z, r.k[i][3] = w.w;
@@ -206,17 +401,16 @@ __device__ __forceinline__ void load_page(PageRegs<KM, VM, PROD>& r, const uint8
             r.k[i][0] = *reinterpret_cast<const uint32_t*>(row);
         }
         if (PROD) {
-            r.s[i] = reinterpret_cast<const uint32_t*>(kst + a.lk.signs_off + (g + 8 * i) * 16)[c];
-            r.kg[i] = reinterpret_cast<const float*>(kst + a.lk.gamma_off)[g + 8 * i] * a.sscale;
+            r.s[i] = reinterpret_cast<const uint32_t*>(kst + a.lk.signs_off + tk[i] * 16)[c];
+            r.kg[i] = reinterpret_cast<const float*>(kst + a.lk.gamma_off)[tk[i]] * a.sscale;
         }
-        r.kn[i] = reinterpret_cast<const float*>(kst + a.lk.norm_off)[g + 8 * i] * a.qscale;
-        r.vn[i] = reinterpret_cast<const float*>(vst + a.lv.norm_off)[g + 8 * i] * 0.08838834764831845f;
+        r.kn[i] = reinterpret_cast<const float*>(kst + a.lk.norm_off)[tk[i]] * a.qscale;
+        r.vn[i] = reinterpret_cast<const float*>(vst + a.lv.norm_off)[tk[i]] * 0.08838834764831845f;
     }
     constexpr int vBytes = VM == kVByte4 ? 8 : 4;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int tok = 2 * c + (i & 1) + 8 * (i >> 1);
-        const uint8_t* row = vst + tok * a.lv.code_row + vBytes * g;
+        const uint8_t* row = vst + tv[i] * a.lv.code_row + vBytes * g;
         if (vBytes == 8) {
             const uint2 w = *reinterpret_cast<const uint2*>(row);
             r.v[i][0] = w.x, r.v[i][1] = w.y;
@@ -226,176 +420,122 @@ __device__ __forceinline__ void load_page(PageRegs<KM, VM, PROD>& r, const uint8
     }
 }
 
-// Shared memory of the split kernel (byte offsets; V at offset 0).
-//   V    value byte table, lane-replicated: [256][32] half2 (nibbles) or [256][16] 2 x half2 (crumbs)
-//   K    key byte table (same layouts) when keys are not byte-permuted
-//   S    sign nibble table [16] 2 x half2 of +-1 (bit set -> +1)
-//   K1   1-bit key nibble table [16] 2 x half2 of c[bit]
-//   M    per warp m[16], l[16]
-//   Bar  per warp kStagesD mbarriers of the page ring
-//   Ring per warp kStagesD stages of one page (key chunk, then value chunk), filled
-//        by bulk copies; after the page loop the same bytes hold the warps'
-//        accumulators for the CTA merge (Acc: per warp acc[16 heads][128])
-constexpr int kTabBytes = 32768;
-constexpr int kStagesD = 4;
-constexpr int kStageBytes = 2496;  // >= key chunk + value chunk for every bit width (16-byte multiple)
-
-template <int KM, int VM, bool PROD>
-struct SmemLayout {
-    static constexpr bool kKTab = (KM == kKByte4 || KM == kKByte2);
-    static constexpr uint32_t kOffV = 0;
-    static constexpr uint32_t kOffK = kOffV + kTabBytes;
-    static constexpr uint32_t kOffS = kOffK + (kKTab ? kTabBytes : 0);
-    static constexpr uint32_t kOffK1 = kOffS + 128;
-    static constexpr uint32_t kOffM = kOffK1 + 128;
-    static constexpr uint32_t kOffBar = kOffM + kWarps * 2 * kMaxG * 4;
-    static constexpr uint32_t kOffRing = (kOffBar + kWarps * kStagesD * 8 + 127) & ~127u;
-    static constexpr uint32_t kRingBytes = kWarps * kStagesD * kStageBytes;
-    static constexpr uint32_t kAccBytes = kWarps * kMaxG * kDim * 4;
-    static constexpr uint32_t kOffAcc = kOffRing;
-    static constexpr uint32_t kBytes = kOffRing + (kRingBytes > kAccBytes ? kRingBytes : kAccBytes);
+template <int KM>
+struct KeyTerm {
+    static constexpr int kSteps = KM == kKByte2 ? 16 : 8;  // 2-bit codes: 128 coordinates x 2 bit planes
 };
 
-template <int KM, int VM, bool PROD>
-__device__ void build_tables(uint8_t* smem, const DecodeArgs& a) {
-    using L = SmemLayout<KM, VM, PROD>;
-    const int tid = threadIdx.x;
-    for (int e = tid; e < 256; e += kThreads) {
-        if (VM == kVByte4) {
-            const uint32_t w = h2bits(cb_half(a.cbv, e & 15), cb_half(a.cbv, e >> 4));
-            uint32_t* t = reinterpret_cast<uint32_t*>(smem + L::kOffV) + e * 32;
-#pragma unroll
-            for (int l = 0; l < 32; ++l) t[l] = w;
-        } else {
-            const uint2 w = make_uint2(h2bits(cb_half(a.cbv, e & 3), cb_half(a.cbv, (e >> 2) & 3)),
-                                       h2bits(cb_half(a.cbv, (e >> 4) & 3), cb_half(a.cbv, e >> 6)));
-            uint2* t = reinterpret_cast<uint2*>(smem + L::kOffV) + e * 16;
-#pragma unroll
-            for (int l = 0; l < 16; ++l) t[l] = w;
-        }
-        if (KM == kKByte4) {
-            const uint32_t w = h2bits(cb_half(a.cbk, e & 15), cb_half(a.cbk, e >> 4));
-            uint32_t* t = reinterpret_cast<uint32_t*>(smem + L::kOffK) + e * 32;
-#pragma unroll
-            for (int l = 0; l < 32; ++l) t[l] = w;
-        } else if (KM == kKByte2) {
-            const uint2 w = make_uint2(h2bits(cb_half(a.cbk, e & 3), cb_half(a.cbk, (e >> 2) & 3)),
-                                       h2bits(cb_half(a.cbk, (e >> 4) & 3), cb_half(a.cbk, e >> 6)));
-            uint2* t = reinterpret_cast<uint2*>(smem + L::kOffK) + e * 16;
-#pragma unroll
-            for (int l = 0; l < 16; ++l) t[l] = w;
-        }
-    }
-    if (tid < 16) {
-        const __half one = __float2half_rn(1.f), mone = __float2half_rn(-1.f);
-        auto pm = [&](int bit) { return ((tid >> bit) & 1) ? one : mone; };
-        reinterpret_cast<uint2*>(smem + L::kOffS)[tid] = make_uint2(h2bits(pm(0), pm(1)), h2bits(pm(2), pm(3)));
-        const __half lo = cb_half(a.cbk, 0), hi = cb_half(a.cbk, 1);
-        auto pk = [&](int bit) { return ((tid >> bit) & 1) ? hi : lo; };
-        reinterpret_cast<uint2*>(smem + L::kOffK1)[tid] = make_uint2(h2bits(pk(0), pk(1)), h2bits(pk(2), pk(3)));
-    }
-}
-
-// byte k (0..3) of w, times `scale` (a power of two), as a shared-memory byte offset
-template <int K, int LOG2SCALE>
-__device__ __forceinline__ uint32_t byte_off(uint32_t w) {
-    constexpr int sh = 8 * K - LOG2SCALE;
-    const uint32_t x = sh >= 0 ? (w >> sh) : (w << (-sh));
-    return x & (0xffu << LOG2SCALE);
-}
-// nibble k (0..7) of w, times 8 (a uint2 table index as a byte offset)
-template <int K>
-__device__ __forceinline__ uint32_t nib_off8(uint32_t w) {
-    constexpr int sh = 4 * K - 3;
-    const uint32_t x = sh >= 0 ? (w >> sh) : (w << (-sh));
-    return x & 0x78u;
-}
-
-// Lazy softmax rescaling: the running maximum only moves when a page exceeds it by
-// more than 2^kSlack (log2 units), so exponentials stay <= 2^kSlack in fp32 / fp16.
-constexpr float kSlack = 8.f;
-
-// ------------------------------------------------------------------ split
+// Scores, online softmax and the value accumulation of one page (ntok valid rows).
 template <int KM, int VM, bool PROD, int NT>
-struct SplitCtx {
-    uint32_t klo0, klo1, khi0, khi1;
-    const uint8_t* smem;
-    int lane, lane4, g, c;
-};
-
-template <int KM, int VM, bool PROD, int NT>
-__device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, int ntok,
-                                             const SplitCtx<KM, VM, PROD, NT>& x, const uint32_t (&bq)[NT][8][2],
+__device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, int ntok, const int (&tk)[2],
+                                             uint32_t klo0, uint32_t klo1, uint32_t khi0, uint32_t khi1,
+                                             uint32_t LA, uint32_t LB,
+                                             const uint32_t (&bq)[NT][KeyTerm<KM>::kSteps][2],
                                              const uint32_t (&bs)[NT][8][2], float (&m)[NT][2], float (&l)[NT][2],
                                              float (&acc)[NT][8][4]) {
-    using L = SmemLayout<KM, VM, PROD>;
-    const int g = x.g, c = x.c;
-    const bool valid0 = g < ntok, valid1 = g + 8 < ntok;
+    // ---- scores: the key term (even and odd K-steps in separate accumulators) and the sign term
+    float d1[NT][2][4], d2[NT][2][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        // ---- scores: 8 K-steps of 16 coordinates, even and odd K-steps in separate
-        // accumulators (two independent MMA chains)
-        float d1[2][4] = {}, d2[2][4] = {};
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d1[nt][h][e] = d2[nt][h][e] = 0.f;
+    if (KM == kKPrmt || KM == kKByte4) {
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-            uint32_t ak[2][2];  // [row g / g+8][coords (4ks,4ks+1) / (4ks+2,4ks+3)]
+            uint32_t ak[2][2];  // [row g / g+8][coords 32c+4ks+{0,1} / +{2,3}]
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
+                const uint32_t w = cur.k[i][ks >> 1];
                 if (KM == kKPrmt) {
-                    const uint32_t w = cur.k[i][ks >> 1];
                     const uint32_t sel = (ks & 1) ? (w >> 16) : w;
-                    const uint32_t lo = __byte_perm(x.klo0, x.klo1, sel);
-                    const uint32_t hi = __byte_perm(x.khi0, x.khi1, sel);
+                    const uint32_t lo = __byte_perm(klo0, klo1, sel);
+                    const uint32_t hi = __byte_perm(khi0, khi1, sel);
                     ak[i][0] = __byte_perm(lo, hi, 0x5140);
                     ak[i][1] = __byte_perm(lo, hi, 0x7362);
-                } else if (KM == kKByte4) {
-                    const uint32_t w = cur.k[i][ks >> 1];
-                    const uint32_t o0 = (ks & 1) ? byte_off<2, 7>(w) : byte_off<0, 7>(w);
-                    const uint32_t o1 = (ks & 1) ? byte_off<3, 7>(w) : byte_off<1, 7>(w);
-                    ak[i][0] = *reinterpret_cast<const uint32_t*>(x.smem + L::kOffK + (o0 | x.lane4));
-                    ak[i][1] = *reinterpret_cast<const uint32_t*>(x.smem + L::kOffK + (o1 | x.lane4));
-                } else if (KM == kKByte2) {
-                    const uint32_t w = cur.k[i][ks >> 2];
-                    uint32_t o;
-                    switch (ks & 3) {
-                        case 0: o = byte_off<0, 7>(w); break;
-                        case 1: o = byte_off<1, 7>(w); break;
-                        case 2: o = byte_off<2, 7>(w); break;
-                        default: o = byte_off<3, 7>(w); break;
-                    }
-                    const uint2 e = *reinterpret_cast<const uint2*>(x.smem + L::kOffK + (o | ((x.lane & 15) << 3)));
-                    ak[i][0] = e.x;
-                    ak[i][1] = e.y;
+                } else if (ks & 1) {
+                    ak[i][0] = lds32(taddr<2, 1>(w, LA));
+                    ak[i][1] = lds32(taddr<3, 1>(w, LA));
                 } else {
-                    const uint2 e = reinterpret_cast<const uint2*>(x.smem + L::kOffK1)[(cur.k[i][0] >> (4 * ks)) & 0xfu];
-                    ak[i][0] = e.x;
-                    ak[i][1] = e.y;
+                    ak[i][0] = lds32(taddr<0, 1>(w, LA));
+                    ak[i][1] = lds32(taddr<1, 1>(w, LA));
                 }
             }
-            mma16816(d1[ks & 1], ak[0][0], ak[1][0], ak[0][1], ak[1][1], bq[nt][ks][0], bq[nt][ks][1]);
-            if (PROD) {
-                const uint32_t oa = nib_off8<0>(cur.s[0] >> (4 * ks));
-                const uint32_t ob = nib_off8<0>(cur.s[1] >> (4 * ks));
-                const uint2 s0 = *reinterpret_cast<const uint2*>(x.smem + L::kOffS + oa);
-                const uint2 s1 = *reinterpret_cast<const uint2*>(x.smem + L::kOffS + ob);
-                mma16816(d2[ks & 1], s0.x, s1.x, s0.y, s1.y, bs[nt][ks][0], bs[nt][ks][1]);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                mma16816(d1[nt][ks & 1], ak[0][0], ak[1][0], ak[0][1], ak[1][1], bq[nt][ks][0], bq[nt][ks][1]);
+        }
+    } else {
+        // +-1 bit planes: byte b of the thread's key bytes -> K-steps 2b, 2b+1
+        constexpr int kB = KM == kKByte2 ? 8 : 4;
+#pragma unroll
+        for (int b = 0; b < kB; ++b) {
+            uint4 t[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const uint32_t w = cur.k[i][b >> 2];
+                switch (b & 3) {
+                    case 0: t[i] = lds128(taddr<0, 0>(w, LB)); break;
+                    case 1: t[i] = lds128(taddr<1, 0>(w, LB)); break;
+                    case 2: t[i] = lds128(taddr<2, 0>(w, LB)); break;
+                    default: t[i] = lds128(taddr<3, 0>(w, LB)); break;
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                mma16816(d1[nt][0], t[0].x, t[1].x, t[0].y, t[1].y, bq[nt][2 * b][0], bq[nt][2 * b][1]);
+                mma16816(d1[nt][1], t[0].z, t[1].z, t[0].w, t[1].w, bq[nt][2 * b + 1][0], bq[nt][2 * b + 1][1]);
             }
         }
-        // ---- base-2 logits of tokens g, g+8 for heads nt*8 + 2c + e
+    }
+    if (PROD) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            uint4 t[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const uint32_t w = cur.s[i];
+                switch (b) {
+                    case 0: t[i] = lds128(taddr<0, 0>(w, LB)); break;
+                    case 1: t[i] = lds128(taddr<1, 0>(w, LB)); break;
+                    case 2: t[i] = lds128(taddr<2, 0>(w, LB)); break;
+                    default: t[i] = lds128(taddr<3, 0>(w, LB)); break;
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                mma16816(d2[nt][0], t[0].x, t[1].x, t[0].y, t[1].y, bs[nt][2 * b][0], bs[nt][2 * b][1]);
+                mma16816(d2[nt][1], t[0].z, t[1].z, t[0].w, t[1].w, bs[nt][2 * b + 1][0], bs[nt][2 * b + 1][1]);
+            }
+        }
+    }
+    const bool full = ntok >= kPage;
+    const bool valid0 = full || tk[0] < ntok, valid1 = full || tk[1] < ntok;
+    uint32_t pb[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        // ---- base-2 logits of rows g, g+8 for heads nt*8 + 2c + e
         float sc[2][2];
 #pragma unroll
         for (int i = 0; i < 2; ++i)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                float s = cur.kn[i] * (d1[0][2 * i + e] + d1[1][2 * i + e]);
-                if (PROD) s = fmaf(cur.kg[i], d2[0][2 * i + e] + d2[1][2 * i + e], s);
-                sc[i][e] = (i == 0 ? valid0 : valid1) ? s : -INFINITY;
+                float s = cur.kn[i] * (d1[nt][0][2 * i + e] + d1[nt][1][2 * i + e]);
+                if (PROD) s = fmaf(cur.kg[i], d2[nt][0][2 * i + e] + d2[nt][1][2 * i + e], s);
+                sc[i][e] = s;
             }
+        if (!full) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                sc[0][e] = valid0 ? sc[0][e] : -INFINITY;
+                sc[1][e] = valid1 ? sc[1][e] : -INFINITY;
+            }
+        }
         // Lazy maximum: each lane checks its own two logits per column against
         // m + kSlack; only when one exceeds it is the page maximum reduced over the
         // column's lanes and the state rescaled.  l holds this lane's partial sum
-        // (its rows), reduced over the column's lanes once per item.
-        float pw[2][2];
+        // (its rows), reduced over the column's lanes once per piece.
         bool over = false;
 #pragma unroll
         for (int e = 0; e < 2; ++e) over |= fmaxf(sc[0][e], sc[1][e]) > m[nt][e] + kSlack;
@@ -417,159 +557,211 @@ __device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, 
                 m[nt][e] = mnew;
             }
         }
+        float pw[2][2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const float p0v = exp2f(sc[0][e] - m[nt][e]), p1v = exp2f(sc[1][e] - m[nt][e]);
             l[nt][e] += p0v + p1v;
-            pw[0][e] = valid0 ? p0v * cur.vn[0] : 0.f;
-            pw[1][e] = valid1 ? p1v * cur.vn[1] : 0.f;
+            pw[0][e] = p0v * cur.vn[0];
+            pw[1][e] = p1v * cur.vn[1];
         }
-        // ---- P' to the B-operand layout: each 8-token half of the C fragment
-        // (token row g, heads 2c, 2c + 1) transposed in registers to (tokens 2c,
-        // 2c + 1, head g)
-        const uint32_t pb0 = movmatrix_trans(h2bits(__float2half_rn(pw[0][0]), __float2half_rn(pw[0][1])));
-        const uint32_t pb1 = movmatrix_trans(h2bits(__float2half_rn(pw[1][0]), __float2half_rn(pw[1][1])));
-        // ---- values: m-tile mt, row g -> coord 16g + 2mt (nibbles), row g+8 -> +1
+        // ---- P' to the B-operand layout: each 8-row half of the C fragment (row g,
+        // heads 2c, 2c + 1) transposed in registers to (rows 2c, 2c + 1, head g)
+        pb[nt][0] = movmatrix_trans(f2h2(pw[0][0], pw[0][1]));
+        pb[nt][1] = movmatrix_trans(f2h2(pw[1][0], pw[1][1]));
+    }
+    // ---- values: m-tile mt, row g -> coordinate c0(mt) of the thread's 16, row g+8 -> c0 + 1
+    if (VM == kVByte4) {
+        // pair bytes of rows (2c, 2c+1) and (2c+8, 2c+9): lo -> even coordinates, hi -> odd
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-            uint32_t av[4];
-            if (VM == kVByte4) {
-                uint32_t t[4];
+        for (int hf = 0; hf < 2; ++hf) {
+            constexpr uint32_t M4 = 0x0F0F0F0Fu;
+            const uint32_t A = cur.v[0][hf], B = cur.v[1][hf], C = cur.v[2][hf], D = cur.v[3][hf];
+            const uint32_t pl0 = (A & M4) | ((B << 4) & ~M4), ph0 = ((A >> 4) & M4) | (B & ~M4);
+            const uint32_t pl1 = (C & M4) | ((D << 4) & ~M4), ph1 = ((C >> 4) & M4) | (D & ~M4);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t w = cur.v[i][mt >> 2];
-                    uint32_t o;
-                    switch (mt & 3) {
-                        case 0: o = byte_off<0, 7>(w); break;
-                        case 1: o = byte_off<1, 7>(w); break;
-                        case 2: o = byte_off<2, 7>(w); break;
-                        default: o = byte_off<3, 7>(w); break;
-                    }
-                    t[i] = *reinterpret_cast<const uint32_t*>(x.smem + L::kOffV + (o | x.lane4));
+            for (int k = 0; k < 4; ++k) {
+                uint32_t a0, a1, a2, a3;
+                switch (k) {
+                    case 0: a0 = lds32(taddr<0, 0>(pl0, LA)), a1 = lds32(taddr<0, 0>(ph0, LA)),
+                            a2 = lds32(taddr<0, 0>(pl1, LA)), a3 = lds32(taddr<0, 0>(ph1, LA)); break;
+                    case 1: a0 = lds32(taddr<1, 0>(pl0, LA)), a1 = lds32(taddr<1, 0>(ph0, LA)),
+                            a2 = lds32(taddr<1, 0>(pl1, LA)), a3 = lds32(taddr<1, 0>(ph1, LA)); break;
+                    case 2: a0 = lds32(taddr<2, 0>(pl0, LA)), a1 = lds32(taddr<2, 0>(ph0, LA)),
+                            a2 = lds32(taddr<2, 0>(pl1, LA)), a3 = lds32(taddr<2, 0>(ph1, LA)); break;
+                    default: a0 = lds32(taddr<3, 0>(pl0, LA)), a1 = lds32(taddr<3, 0>(ph0, LA)),
+                             a2 = lds32(taddr<3, 0>(pl1, LA)), a3 = lds32(taddr<3, 0>(ph1, LA)); break;
                 }
-                av[0] = __byte_perm(t[0], t[1], 0x5410);  // lower coord, tokens 2c, 2c+1
-                av[1] = __byte_perm(t[0], t[1], 0x7632);  // upper coord
-                av[2] = __byte_perm(t[2], t[3], 0x5410);  // tokens 2c+8, 2c+9
-                av[3] = __byte_perm(t[2], t[3], 0x7632);
-            } else {
-                uint2 t[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t w = cur.v[i][0];
-                    uint32_t o;
-                    switch (mt >> 1) {
-                        case 0: o = byte_off<0, 7>(w); break;
-                        case 1: o = byte_off<1, 7>(w); break;
-                        case 2: o = byte_off<2, 7>(w); break;
-                        default: o = byte_off<3, 7>(w); break;
-                    }
-                    t[i] = *reinterpret_cast<const uint2*>(x.smem + L::kOffV + (o | ((x.lane & 15) << 3)));
-                }
-                const uint32_t x0 = (mt & 1) ? t[0].y : t[0].x, x1 = (mt & 1) ? t[1].y : t[1].x;
-                const uint32_t x2 = (mt & 1) ? t[2].y : t[2].x, x3 = (mt & 1) ? t[3].y : t[3].x;
-                av[0] = __byte_perm(x0, x1, 0x5410);
-                av[1] = __byte_perm(x0, x1, 0x7632);
-                av[2] = __byte_perm(x2, x3, 0x5410);
-                av[3] = __byte_perm(x2, x3, 0x7632);
+                for (int nt = 0; nt < NT; ++nt) mma16816(acc[nt][4 * hf + k], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
             }
-            mma16816(acc[nt][mt], av[0], av[1], av[2], av[3], pb0, pb1);
+        }
+    } else {
+        // crumb pair bytes: X -> coordinates 4m, 4m+2 of the 16, Y -> 4m+1, 4m+3
+        constexpr uint32_t M2 = 0x33333333u;
+        const uint32_t A = cur.v[0][0], B = cur.v[1][0], C = cur.v[2][0], D = cur.v[3][0];
+        const uint32_t x0 = (A & M2) | ((B << 2) & ~M2), y0 = ((A >> 2) & M2) | (B & ~M2);
+        const uint32_t x1 = (C & M2) | ((D << 2) & ~M2), y1 = ((C >> 2) & M2) | (D & ~M2);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            uint2 tx0, ty0, tx1, ty1;
+            switch (k) {
+                case 0: tx0 = lds64(taddr<0, 1>(x0, LB)), ty0 = lds64(taddr<0, 1>(y0, LB)),
+                        tx1 = lds64(taddr<0, 1>(x1, LB)), ty1 = lds64(taddr<0, 1>(y1, LB)); break;
+                case 1: tx0 = lds64(taddr<1, 1>(x0, LB)), ty0 = lds64(taddr<1, 1>(y0, LB)),
+                        tx1 = lds64(taddr<1, 1>(x1, LB)), ty1 = lds64(taddr<1, 1>(y1, LB)); break;
+                case 2: tx0 = lds64(taddr<2, 1>(x0, LB)), ty0 = lds64(taddr<2, 1>(y0, LB)),
+                        tx1 = lds64(taddr<2, 1>(x1, LB)), ty1 = lds64(taddr<2, 1>(y1, LB)); break;
+                default: tx0 = lds64(taddr<3, 1>(x0, LB)), ty0 = lds64(taddr<3, 1>(y0, LB)),
+                         tx1 = lds64(taddr<3, 1>(x1, LB)), ty1 = lds64(taddr<3, 1>(y1, LB)); break;
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                mma16816(acc[nt][2 * k], tx0.x, ty0.x, tx1.x, ty1.x, pb[nt][0], pb[nt][1]);
+                mma16816(acc[nt][2 * k + 1], tx0.y, ty0.y, tx1.y, ty1.y, pb[nt][0], pb[nt][1]);
+            }
         }
     }
 }
 
+// Coordinate of row g of m-tile mt among the thread's 16 (16 g + c0; row g+8 -> c0 + 1).
+template <int VM>
+__device__ __forceinline__ int coord_of(int mt) {
+    return VM == kVByte4 ? 2 * mt : 4 * (mt >> 1) + 2 * (mt & 1);
+}
+
+// ------------------------------------------------------------------ split kernel
 template <int KM, int VM, bool PROD, int NT>
-__global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
-    using L = SmemLayout<KM, VM, PROD>;
+__global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, c = lane & 3;
-    build_tables<KM, VM, PROD>(smem, a);
-    SplitCtx<KM, VM, PROD, NT> x{};
-    x.smem = smem;
-    x.lane = lane;
-    x.lane4 = lane << 2;
-    x.g = g;
-    x.c = c;
-    if (KM == kKPrmt) {  // 8-entry key tables: low / high bytes of the fp16 levels
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const uint32_t hb = __half_as_ushort(cb_half(a.cbk, k));
-            if (k < 4) {
-                x.klo0 |= (hb & 0xffu) << (8 * k);
-                x.khi0 |= (hb >> 8) << (8 * k);
-            } else {
-                x.klo1 |= (hb & 0xffu) << (8 * (k - 4));
-                x.khi1 |= (hb >> 8) << (8 * (k - 4));
-            }
-        }
+    const uint32_t base = sm100::smem_u32(smem);
+    if (base + kLowBytes > kTabAddr) {  // the window leaves no room below the tables
+        if (tid == 0) atomicOr(a.err, TQ_DEVERR_INTERNAL);
+        return;
     }
-    const uint32_t ring = sm100::smem_u32(smem + L::kOffRing) + warp * kStagesD * kStageBytes;
-    const uint32_t bars = sm100::smem_u32(smem + L::kOffBar) + warp * kStagesD * 8;
-    if (lane == 0) {
-        for (int st = 0; st < kStagesD; ++st) sm100::mbar_init(bars + 8 * st, 1);
+    const uint32_t full_bar = base + kOffFull;
+    int* valid = reinterpret_cast<int*>(smem + kOffValid);
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffAbort);
+    if (tid < 256) build_tables<KM, VM, PROD>(a, tid);
+    if (tid == 0) {
+        for (int i = 0; i < kNW * kStages; ++i) sm100::mbar_init(full_bar + 8 * i, 1);
+        *abort = 0;
         sm100::fence_mbar_init();
     }
     __syncthreads();
     griddep_wait();  // q', s and the page prefix sums from the prep kernel; the caller's inputs
     griddep_launch_dependents();  // the merge kernel may stage its rotation meanwhile
-    float* wm = reinterpret_cast<float*>(smem + L::kOffM);      // [warp][2][16]: m then l
-    float* wacc = reinterpret_cast<float*>(smem + L::kOffAcc);  // [warp][16 heads][128]
-    const volatile int never = 0;
-    uint32_t issued = 0, consumed = 0;  // pages this warp has requested / processed (all items)
-    bool dead = false;                  // a page copy never arrived: this warp stops working
-
-    // this CTA's range [pos, end) of the pages of all units in order (unit
-    // u = b Hkv + h holds the pages of sequence b), cut into pieces by unit
     const long total = (long)a.Hkv * a.prefix[a.B];
-    long pos = total * (long)blockIdx.x / gridDim.x;
+    const long pos0 = total * (long)blockIdx.x / gridDim.x;
     const long end = total * (long)(blockIdx.x + 1) / gridDim.x;
-    int b = 0;
-    if (pos < end) {  // the last sequence b with Hkv * prefix[b] <= pos
-        int lo = 0, hi = a.B - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if ((long)a.Hkv * a.prefix[mid] <= pos) lo = mid;
-            else hi = mid - 1;
-        }
-        b = lo;
-    }
-    while (pos < end && b < a.B) {
-        const int np = a.prefix[b + 1] - a.prefix[b];  // pages of sequence b (the same for each kv head)
-        const long off = pos - (long)a.Hkv * a.prefix[b];
-        if (np == 0 || off >= (long)a.Hkv * np) {  // past sequence b
-            ++b;
-            continue;
-        }
-        const int hk = (int)(off / np);
-        const int p0 = (int)(off - (long)hk * np);
-        const int p1 = (int)min((long)np, p0 + (end - pos));
-        pos += p1 - p0;
-        const int unit = b * a.Hkv + hk;
-        const int Ls = a.seq_lens[b];  // valid: np > 0
+    const uint32_t kb = (uint32_t)a.lk.bytes, vb = (uint32_t)a.lv.bytes;
 
-        // query fragments (B operand): head nt*8 + g, coords 32c .. 32c+31; K-step ks
-        // uses coords 32c + 4ks + {0,1} (b0) and {2,3} (b1)
-        uint32_t bq[NT][8][2], bs[NT][8][2];
+    // ---- this warp's page stream: issue cursor (runs kStages pages ahead) and the
+    // copies of page number `k` of the warp into stage k % kStages
+    PageCursor icur;
+    icur.init(a, pos0, end, warp, lane);
+    uint32_t issued = 0, landed = 0;  // pages issued; pages whose copies were started (for the drain)
+    auto issue_next = [&]() {
+        if (!icur.live) return;
+        const int blk = icur.block();
+        const uint32_t st = warp * kStages + issued % kStages;
+        if (lane == 0) {
+            const bool v = blk >= 0 && blk < a.num_blocks;
+            valid[st] = v ? 1 : 0;
+            if (a.stall) {
+                // test hook: nothing arrives on the stage
+            } else if (v) {
+                const size_t chunk = (size_t)blk * a.Hkv + icur.hk;
+                const uint32_t dst = kRingAddr + st * kStageBytes;
+                sm100::mbar_arrive_expect_tx(full_bar + 8 * st, kb + vb);
+                sm100::bulk_g2s(dst, a.kc + chunk * kb, kb, full_bar + 8 * st);
+                sm100::bulk_g2s(dst + kb, a.vc + chunk * vb, vb, full_bar + 8 * st);
+            } else {
+                atomicOr(a.err, TQ_DEVERR_BLOCK);
+                sm100::mbar_arrive(full_bar + 8 * st);  // nothing to copy: the stage completes at once
+            }
+        }
+        if (!a.stall) ++landed;
+        ++issued;
+        icur.advance(a, warp, lane);
+    };
+    for (int i = 0; i < kStages; ++i) issue_next();
+
+    // ---------------------------------------------------------------- pages
+    const int g = lane >> 2, c = lane & 3;
+    // rows of this thread in the page: score rows g, g+8; value rows 2c, 2c+1, 2c+8, 2c+9
+    const int tk[2] = {row_token(g), row_token(g + 8)};
+    const int tv[4] = {row_token(2 * c), row_token(2 * c + 1), row_token(2 * c + 8), row_token(2 * c + 9)};
+    // lane offsets inside a table entry: LA = {lane*4 (A), 128 + lane*4 (B)}, LB = {128 +
+    // (lane%8)*16 (B, 16-byte entries), (lane%16)*8 (A, 8-byte entries)}; bytes 2, 3 = 0x01, 0x00
+    const uint32_t LA = (uint32_t)(lane * 4) | ((uint32_t)(128 + lane * 4) << 8) | 0x10000u;
+    const uint32_t LB = (uint32_t)(128 + (lane & 7) * 16) | ((uint32_t)((lane & 15) * 8) << 8) | 0x10000u;
+    // 3-bit key codes: low / high bytes of the 8 fp16 levels
+    uint32_t klo0 = 0, klo1 = 0, khi0 = 0, khi1 = 0;
+    if (KM == kKPrmt) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const uint32_t hb = __half_as_ushort(cb_half(a.cbk, k));
+            if (k < 4) {
+                klo0 |= (hb & 0xffu) << (8 * k);
+                khi0 |= (hb >> 8) << (8 * k);
+            } else {
+                klo1 |= (hb & 0xffu) << (8 * (k - 4));
+                khi1 |= (hb >> 8) << (8 * (k - 4));
+            }
+        }
+    }
+    float* wml = reinterpret_cast<float*>(smem + kOffML);      // [warp][2][8]: m then l
+    float* wacc = reinterpret_cast<float*>(smem + kOffMerge);  // [warp][8 heads][128]
+    uint32_t cnt = 0;   // pages this warp has consumed (all pieces)
+    bool dead = false;  // a page never arrived: this warp stops working
+    Pieces it;
+    it.init(a, pos0, end);
+    int b, hk, p0, p1;
+    constexpr int KS = KeyTerm<KM>::kSteps;
+    while (it.next(a, b, hk, p0, p1)) {
+        const int unit = b * a.Hkv + hk;
+        const int Ls = a.seq_lens[b];  // valid: the sequence has pages
+        // query fragments (B operand) of heads nt*8 + g: key term and sign term
+        uint32_t bq[NT][KS][2], bs[NT][8][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int h = nt * 8 + g;
             if (h < a.G) {
-                const uint4* src =
-                    reinterpret_cast<const uint4*>(a.qf + (((size_t)unit * a.G + h) * 2) * kDim + 32 * c);
+                const float4* src = reinterpret_cast<const float4*>(a.qf + (((size_t)unit * a.G + h) * 2) * kDim + 32 * c);
+                float4 x[8];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint4 w = src[i];
-                    bq[nt][2 * i][0] = w.x, bq[nt][2 * i][1] = w.y;
-                    bq[nt][2 * i + 1][0] = w.z, bq[nt][2 * i + 1][1] = w.w;
-                    if (PROD) {
-                        const uint4 u = src[i + kDim / 8];
-                        bs[nt][2 * i][0] = u.x, bs[nt][2 * i][1] = u.y;
-                        bs[nt][2 * i + 1][0] = u.z, bs[nt][2 * i + 1][1] = u.w;
+                for (int i = 0; i < 8; ++i) x[i] = src[i];
+                if (KM == kKByte2) {
+#pragma unroll
+                    for (int ks = 0; ks < 16; ++ks) {
+                        const float4 v = x[ks >> 1];
+                        const float q0 = (ks & 1) ? v.z : v.x, q1 = (ks & 1) ? v.w : v.y;
+                        bq[nt][ks][0] = f2h2(a.kbeta * q0, a.kalpha * q0);
+                        bq[nt][ks][1] = f2h2(a.kbeta * q1, a.kalpha * q1);
+                    }
+                } else {
+                    const float ksc = a.kscale;
+#pragma unroll
+                    for (int ks = 0; ks < KS && ks < 8; ++ks) {
+                        bq[nt][ks][0] = f2h2(ksc * x[ks].x, ksc * x[ks].y);
+                        bq[nt][ks][1] = f2h2(ksc * x[ks].z, ksc * x[ks].w);
+                    }
+                }
+                if (PROD) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 v = src[i + kDim / 4];
+                        bs[nt][i][0] = f2h2(v.x, v.y);
+                        bs[nt][i][1] = f2h2(v.z, v.w);
                     }
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) bq[nt][i][0] = bq[nt][i][1] = bs[nt][i][0] = bs[nt][i][1] = 0u;
+                for (int i = 0; i < KS; ++i) bq[nt][i][0] = bq[nt][i][1] = 0u;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) bs[nt][i][0] = bs[nt][i][1] = 0u;
             }
         }
         float m[NT][2], l[NT][2], acc[NT][8][4];
@@ -581,70 +773,36 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
             for (int mt = 0; mt < 8; ++mt) acc[nt][mt][0] = acc[nt][mt][1] = acc[nt][mt][2] = acc[nt][mt][3] = 0.f;
         }
 
-        // ---- page loop: the warp takes pages first, first + 4, ...; a ring of
-        // kStagesD shared-memory stages keeps the next pages' bulk copies in flight
-        const int first = p0 + warp;
-        const int nj = first < p1 ? (p1 - first + kWarps - 1) / kWarps : 0;
-        const int* btab = a.block_table + (size_t)b * a.max_blocks + first;
-        const int win = (lane < nj) ? btab[lane * kWarps] : -1;  // block ids of the first 32 pages
-        auto blk_of = [&](int j) -> int {
-            int v = __shfl_sync(0xffffffffu, win, j & 31);
-            if (j >= 32) {
-                v = lane == 0 ? btab[j * kWarps] : 0;
-                v = __shfl_sync(0xffffffffu, v, 0);
-            }
-            return v;
-        };
-        const uint32_t kb = (uint32_t)a.lk.bytes, vb = (uint32_t)a.lv.bytes;
-        auto issue = [&](int j) {
-            const int blk = blk_of(j);
-            const uint32_t st = ring + (issued % kStagesD) * kStageBytes;
-            const uint32_t bar = bars + 8 * (issued % kStagesD);
-            if (lane == 0) {
-                if (blk >= 0 && blk < a.num_blocks) {
-                    const size_t chunk = (size_t)blk * a.Hkv + hk;
-                    sm100::mbar_arrive_expect_tx(bar, kb + vb);
-                    sm100::bulk_g2s(st, a.kc + chunk * kb, kb, bar);
-                    sm100::bulk_g2s(st + kb, a.vc + chunk * vb, vb, bar);
-                } else {
-                    sm100::mbar_arrive(bar);  // nothing to copy: the stage completes at once
+        // ---- the warp's pages of the piece: p0 + warp, + kNW, ...
+        const int nj = p0 + warp < p1 ? (p1 - p0 - warp + kNW - 1) / kNW : 0;
+        for (int j = 0; j < nj; ++j) {
+            const uint32_t st = warp * kStages + cnt % kStages;
+            if (!dead) {
+                const bool ok = sm100::mbar_wait(full_bar + 8 * st, (cnt / kStages) & 1u, abort, kWaitNs);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    if (lane == 0 && !*abort) {
+                        *abort = 1;
+                        atomicOr(a.err, TQ_DEVERR_TIMEOUT);
+                    }
+                    dead = true;
                 }
             }
-            ++issued;
-        };
-        if (!dead)
-            for (int j = 0; j < nj && j < kStagesD; ++j) issue(j);
-        for (int j = 0; j < nj && !dead; ++j) {
-            const uint32_t sidx = consumed % kStagesD;
-            const bool ok = sm100::mbar_wait_warp(bars + 8 * sidx, (consumed / kStagesD) & 1u, &never, 2000000000ull);
-            const int blk = blk_of(j);
-            if (!ok) {
-                if (lane == 0) atomicOr(a.err, TQ_DEVERR_TIMEOUT);
-                dead = true;
-                break;
-            }
-            ++consumed;
-            const int page = first + j * kWarps;
-            if (blk < 0 || blk >= a.num_blocks) {
-                if (lane == 0) atomicOr(a.err, TQ_DEVERR_BLOCK);
-            } else {
-                const uint8_t* st = smem + L::kOffRing + (size_t)(warp * kStagesD + sidx) * kStageBytes;
+            if (dead) continue;  // this warp stops: no more pages are consumed or issued
+            const int page = p0 + warp + j * kNW;
+            if (valid[st]) {
+                const uint8_t* sp = smem + (kRingAddr - base) + st * kStageBytes;
                 PageRegs<KM, VM, PROD> r;
-                load_page<KM, VM, PROD>(r, st, st + kb, a, g, c);
-                process_page<KM, VM, PROD, NT>(r, min(kPage, Ls - page * kPage), x, bq, bs, m, l, acc);
+                load_page<KM, VM, PROD>(r, sp, sp + kb, a, tk, tv, g, c);
+                process_page<KM, VM, PROD, NT>(r, min(kPage, Ls - page * kPage), tk, klo0, klo1, khi0, khi1, LA, LB,
+                                               bq, bs, m, l, acc);
             }
             sm100::fence_proxy_async_shared();  // this lane's reads before the refill's bulk copy
-            __syncwarp();  // every lane is done with the stage before it is refilled
-            if (j + kStagesD < nj) issue(j + kStagesD);
-        }
-        if (dead) {  // let copies already in flight land before the stages are reused
-            while (consumed < issued) {
-                sm100::mbar_wait(bars + 8 * (consumed % kStagesD), (consumed / kStagesD) & 1u, &never, 2000000000ull);
-                ++consumed;
-            }
+            __syncwarp();                       // every lane is done with the stage before it is refilled
+            ++cnt;
+            issue_next();
         }
 
-        // ---- merge the warps of the CTA (coordinates back in natural order)
+        // ---- merge the CTA's warps (one tile of 8 heads at a time; coordinates back in order)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -653,44 +811,54 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
                 l[nt][e] += __shfl_xor_sync(0xffffffffu, l[nt][e], 8);
                 l[nt][e] += __shfl_xor_sync(0xffffffffu, l[nt][e], 16);
             }
-        __syncthreads();
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < NT; ++nt) {
+            __syncthreads();  // the previous merge is done with the area
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const int h = nt * 8 + 2 * c + e;
+                const int hh = 2 * c + e;
                 if (g == 0) {
-                    wm[(warp * 2 + 0) * kMaxG + h] = m[nt][e];
-                    wm[(warp * 2 + 1) * kMaxG + h] = l[nt][e];
+                    wml[(warp * 2 + 0) * 8 + hh] = m[nt][e];
+                    wml[(warp * 2 + 1) * 8 + hh] = l[nt][e];
                 }
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
-                    const int c0 = (VM == kVByte4) ? 16 * g + 2 * mt : 16 * g + 4 * (mt >> 1) + 2 * (mt & 1);
-                    wacc[(warp * kMaxG + h) * kDim + c0] = acc[nt][mt][e];
-                    wacc[(warp * kMaxG + h) * kDim + c0 + 1] = acc[nt][mt][2 + e];
+                    const int c0 = 16 * g + coord_of<VM>(mt);
+                    wacc[(warp * 8 + hh) * kDim + c0] = acc[nt][mt][e];
+                    wacc[(warp * 8 + hh) * kDim + c0 + 1] = acc[nt][mt][2 + e];
                 }
             }
-        __syncthreads();
-        for (int h = 0; h < a.G; ++h) {  // thread = coordinate
-            float M = -INFINITY;
+            __syncthreads();
+            // thread = (head hh = warp, coordinates 4 lane .. 4 lane + 3) for the first 8 warps
+            const int hh = warp, h = nt * 8 + hh;
+            if (hh < 8 && h < a.G) {
+                float M = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wm[(w * 2) * kMaxG + h]);
-            float Lsum = 0.f, A = 0.f;
+                for (int w = 0; w < kNW; ++w) M = fmaxf(M, wml[(w * 2) * 8 + hh]);
+                float Lsum = 0.f;
+                float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) {
-                const float mw = wm[(w * 2) * kMaxG + h];
-                const float wt = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-                Lsum = fmaf(wt, wm[(w * 2 + 1) * kMaxG + h], Lsum);
-                A = fmaf(wt, wacc[(w * kMaxG + h) * kDim + tid], A);
+                for (int w = 0; w < kNW; ++w) {
+                    const float mw = wml[(w * 2) * 8 + hh];
+                    const float wt = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+                    Lsum = fmaf(wt, wml[(w * 2 + 1) * 8 + hh], Lsum);
+                    const float4 v = reinterpret_cast<const float4*>(wacc + (w * 8 + hh) * kDim)[lane];
+                    A.x = fmaf(wt, v.x, A.x);
+                    A.y = fmaf(wt, v.y, A.y);
+                    A.z = fmaf(wt, v.z, A.z);
+                    A.w = fmaf(wt, v.w, A.w);
+                }
+                float* part = a.partial + (((size_t)unit + blockIdx.x) * a.G + h) * kPartStride;
+                if (lane == 0) *reinterpret_cast<float2*>(part) = make_float2(M, Lsum);
+                reinterpret_cast<float2*>(part + 2)[2 * lane] = make_float2(A.x, A.y);
+                reinterpret_cast<float2*>(part + 2)[2 * lane + 1] = make_float2(A.z, A.w);
             }
-            float* part = a.partial + (((size_t)unit + blockIdx.x) * a.G + h) * kPartStride;
-            if (tid == 0) {
-                part[0] = M;
-                part[1] = Lsum;
-            }
-            part[2 + tid] = A;
         }
-        __syncthreads();
+    }
+    if (dead && landed > cnt) {  // the copies this warp started land before the CTA exits
+        const volatile int never = 0;
+        for (uint32_t k = cnt; k < landed; ++k)
+            sm100::mbar_wait(full_bar + 8 * (warp * kStages + k % kStages), (k / kStages) & 1u, &never, kWaitNs);
     }
 }
 
@@ -704,13 +872,19 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
 // partial states and un-rotates.  R^T is staged once per CTA (while the split
 // kernel runs).  Unit u's pieces sit in slots u + c for the split CTAs c whose
 // page range meets it: c(p) = ((p + 1) grid - 1) / total is the CTA of page p.
+// With a residual window, the first group of an item also attends to the window's
+// fp16 tokens (scores with a thread per token, values with a thread per coordinate)
+// and combines that partial state with the compressed one in the original domain.
 constexpr int kMergeHeads = 4;
 constexpr int kMergeItems = 4;  // most items per CTA
 constexpr int kMergeGroups = 8; // most slot groups per item
 constexpr int kMergeThreads = 1024;
-size_t merge_smem(int ipc, int sg) {
+constexpr int kTailMax = 256;   // most window tokens per sequence
+constexpr size_t kTailFloats = kMergeHeads * kDim + kTailMax * kMergeHeads + 2 * 4 * kMergeHeads;  // per item
+size_t merge_smem(int ipc, int sg, bool tail) {
     return sizeof(float) * (kDim * kDim + (size_t)ipc * kDim * kMergeHeads +
-                            (sg > 1 ? (size_t)ipc * sg * (kDim * kMergeHeads + 2 * kMergeHeads) : 0));
+                            (sg > 1 ? (size_t)ipc * sg * (kDim * kMergeHeads + 2 * kMergeHeads) : 0) +
+                            (tail ? (size_t)ipc * kTailFloats : 0));
 }
 __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs a) {
     // RT [128*128] | orot [items][128][kMergeHeads] | group states A [items][sg][128][kMergeHeads],
@@ -724,6 +898,12 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs 
     float4* gA = reinterpret_cast<float4*>(sm + kDim * kDim + ipc * kDim * kMergeHeads) + (il * sg) * kDim;
     float* gML = sm + kDim * kDim + ipc * kDim * kMergeHeads + ipc * sg * kDim * kMergeHeads +
                  (il * sg) * 2 * kMergeHeads;
+    // window: q of the item's heads [4][128], scores / probabilities [kTailMax][4], warp maxima
+    // and sums [2][4 warps][4]
+    float* tq_s = sm + kDim * kDim + ipc * kDim * kMergeHeads +
+                  (sg > 1 ? ipc * sg * (kDim * kMergeHeads + 2 * kMergeHeads) : 0) + il * kTailFloats;
+    float* ts_s = tq_s + kMergeHeads * kDim;
+    float* red_s = ts_s + kTailMax * kMergeHeads;
     {
         const float4* src = reinterpret_cast<const float4*>(a.RT);
         float4* dst = reinterpret_cast<float4*>(rts);
@@ -813,6 +993,86 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs 
 #pragma unroll
         for (int e = 0; e < kMergeHeads; ++e) o[e] = (live && Lsum[e] > 0.f) ? A[e] / Lsum[e] : 0.f;
         if (gi == 0) orot[i] = make_float4(o[0], o[1], o[2], o[3]);
+        // residual window of the item's sequence: (tM, tL, tA) of its fp16 tokens, base 2
+        float tM[kMergeHeads], tL[kMergeHeads], tA[kMergeHeads];
+#pragma unroll
+        for (int e = 0; e < kMergeHeads; ++e) tM[e] = -INFINITY, tL[e] = 0.f, tA[e] = 0.f;
+        if (a.tail_k) {
+            const int b = unit / a.Hkv, hk = unit - b * a.Hkv;
+            int tl = 0;
+            if (live && gi == 0) {
+                tl = a.tail_lens[b];
+                if (tl < 0 || tl > a.tail_cap) {
+                    if (i == 0 && h0 == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
+                    tl = 0;
+                }
+#pragma unroll
+                for (int e = 0; e < kMergeHeads; ++e)
+                    tq_s[e * kDim + i] = h0 + e < a.G ? __half2float(__ushort_as_half(
+                                                            a.q[((size_t)b * a.Hq + hk * a.G + h0 + e) * kDim + i]))
+                                                      : 0.f;
+            }
+            __syncthreads();
+            const int wi = i >> 5, ln = i & 31;  // warp of the item's first group, lane
+            float mx[kMergeHeads] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            for (int u = i; u < tl; u += kDim) {  // scores: a thread per token
+                const uint4* kr = reinterpret_cast<const uint4*>(
+                    a.tail_k + (((size_t)b * a.tail_cap + u) * a.Hkv + hk) * kDim);
+                float sc[kMergeHeads] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                for (int c8 = 0; c8 < kDim / 8; ++c8) {
+                    const uint4 w = kr[c8];
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const float2 kk = __half22float2(*reinterpret_cast<const __half2*>(&ww[jj]));
+#pragma unroll
+                        for (int e = 0; e < kMergeHeads; ++e) {
+                            sc[e] = fmaf(tq_s[e * kDim + 8 * c8 + 2 * jj], kk.x, sc[e]);
+                            sc[e] = fmaf(tq_s[e * kDim + 8 * c8 + 2 * jj + 1], kk.y, sc[e]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < kMergeHeads; ++e) {
+                    sc[e] *= a.scale_log2;
+                    ts_s[u * kMergeHeads + e] = sc[e];
+                    mx[e] = fmaxf(mx[e], sc[e]);
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < kMergeHeads; ++e) {
+                for (int off = 16; off > 0; off >>= 1) mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], off));
+                if (gi == 0 && ln == 0) red_s[wi * kMergeHeads + e] = mx[e];
+            }
+            __syncthreads();
+            float sm4[kMergeHeads] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int e = 0; e < kMergeHeads; ++e)
+                tM[e] = fmaxf(fmaxf(red_s[e], red_s[kMergeHeads + e]), fmaxf(red_s[2 * kMergeHeads + e], red_s[3 * kMergeHeads + e]));
+            for (int u = i; u < tl; u += kDim)
+#pragma unroll
+                for (int e = 0; e < kMergeHeads; ++e) {
+                    const float p = exp2f(ts_s[u * kMergeHeads + e] - tM[e]);
+                    ts_s[u * kMergeHeads + e] = p;
+                    sm4[e] += p;
+                }
+#pragma unroll
+            for (int e = 0; e < kMergeHeads; ++e) {
+                for (int off = 16; off > 0; off >>= 1) sm4[e] += __shfl_xor_sync(0xffffffffu, sm4[e], off);
+                if (gi == 0 && ln == 0) red_s[4 * kMergeHeads + wi * kMergeHeads + e] = sm4[e];
+            }
+            __syncthreads();
+#pragma unroll
+            for (int e = 0; e < kMergeHeads; ++e)
+                tL[e] = (red_s[4 * kMergeHeads + e] + red_s[5 * kMergeHeads + e]) +
+                        (red_s[6 * kMergeHeads + e] + red_s[7 * kMergeHeads + e]);
+            for (int u = 0; u < tl; ++u) {  // values: a thread per coordinate
+                const float v = __half2float(__ushort_as_half(a.tail_v[(((size_t)b * a.tail_cap + u) * a.Hkv + hk) * kDim + i]));
+#pragma unroll
+                for (int e = 0; e < kMergeHeads; ++e) tA[e] = fmaf(ts_s[u * kMergeHeads + e], v, tA[e]);
+            }
+        }
         __syncthreads();
         if (!live || gi != 0) continue;
         float y[kMergeHeads] = {0.f, 0.f, 0.f, 0.f};
@@ -824,6 +1084,16 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs 
             y[1] = fmaf(r, v.y, y[1]);
             y[2] = fmaf(r, v.z, y[2]);
             y[3] = fmaf(r, v.w, y[3]);
+        }
+        if (a.tail_k) {  // o = (Wc R acc / Lc + Wt tA / tL) with the weights of both parts
+#pragma unroll
+            for (int e = 0; e < kMergeHeads; ++e) {
+                const float Mx = fmaxf(M[e], tM[e]);
+                const float wc = Lsum[e] > 0.f ? exp2f(M[e] - Mx) * Lsum[e] : 0.f;
+                const float et = tL[e] > 0.f ? exp2f(tM[e] - Mx) : 0.f;
+                const float den = wc + et * tL[e];
+                y[e] = den > 0.f ? (wc * y[e] + et * tA[e]) / den : 0.f;
+            }
         }
 #pragma unroll
         for (int e = 0; e < kMergeHeads; ++e) {
@@ -845,18 +1115,6 @@ int kmode_of(const tq_ctx* ctx) {
     return kKBit1;
 }
 
-size_t split_smem(int km) {
-    return (km == kKByte4 || km == kKByte2) ? SmemLayout<kKByte4, kVByte4, true>::kBytes
-                                            : SmemLayout<kKPrmt, kVByte4, true>::kBytes;
-}
-
-int ctas_per_sm_for(size_t smem) {
-    int n = (int)(233472 / (smem + 1024));  // 228 KB of shared memory per SM, 1 KB reserved per CTA
-    if (n > 4) n = 4;
-    return n < 1 ? 1 : n;
-}
-
-
 // Launch with programmatic stream serialization (see griddep_wait).
 template <typename K>
 cudaError_t launch_dependent(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, const DecodeArgs& a) {
@@ -875,11 +1133,10 @@ cudaError_t launch_dependent(K kernel, dim3 grid, dim3 block, size_t smem, cudaS
 
 template <int KM, int VM, bool PROD, int NT>
 cudaError_t launch_split(const DecodeArgs& a, int grid, cudaStream_t stream) {
-    using L = SmemLayout<KM, VM, PROD>;
     auto k = decode_split_kernel<KM, VM, PROD, NT>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSplitSmem);
     if (e != cudaSuccess) return e;
-    return launch_dependent(k, dim3(grid), dim3(kThreads), L::kBytes, stream, a);
+    return launch_dependent(k, dim3(grid), dim3(kSplitThreads), kSplitSmem, stream, a);
 }
 
 }  // namespace
@@ -887,10 +1144,10 @@ cudaError_t launch_split(const DecodeArgs& a, int grid, cudaStream_t stream) {
 DecodePlan plan_decode(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_seq_len) {
     DecodePlan p{};
     p.max_pages = (max_seq_len + kPage - 1) / kPage;
-    const long resident = (long)ctx->sm_count * ctas_per_sm_for(split_smem(kmode_of(ctx)));
+    const long resident = (long)ctx->sm_count;  // one split CTA per SM
     const long units = (long)B * Hkv;
-    // every resident CTA, but at least 16 pages (4 per warp) per CTA for small batches
-    long grid = (units * p.max_pages + 4 * kWarps - 1) / (4 * kWarps);
+    // every SM, but at least 4 pages per consumer warp for small batches
+    long grid = (units * p.max_pages + 4 * kNW - 1) / (4 * kNW);
     if (grid > resident) grid = resident;
     if (grid < 1) grid = 1;
     p.grid = (int)grid;
@@ -898,7 +1155,7 @@ DecodePlan plan_decode(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_seq_le
     const int G = Hkv > 0 ? Hq / Hkv : 0;
     size_t off = 0;
     p.qprep_off = off;
-    off += (size_t)B * Hq * 2 * kDim * sizeof(__half);
+    off += (size_t)B * Hq * 2 * kDim * sizeof(float);
     off = (off + 255) & ~size_t(255);
     p.partial_off = off;
     off += (size_t)p.slots * G * kPartStride * sizeof(float);
@@ -912,12 +1169,12 @@ DecodePlan plan_decode(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_seq_le
 
 cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint16_t* q, const uint8_t* kc,
                           const uint8_t* vc, int num_blocks, const int32_t* block_table, int max_blocks,
-                          const int32_t* seq_lens, int B, int Hq, int Hkv, int max_seq_len, float scale, void* out,
-                          int out_fp32, void* workspace, cudaStream_t stream) {
+                          const int32_t* seq_lens, int B, int Hq, int Hkv, int max_seq_len, const DecodeTail& tail,
+                          float scale, void* out, int out_fp32, void* workspace, cudaStream_t stream) {
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     DecodeArgs a{};
     a.q = q;
-    a.qf = reinterpret_cast<__half*>(ws + plan.qprep_off);
+    a.qf = reinterpret_cast<float*>(ws + plan.qprep_off);
     a.kc = kc;
     a.vc = vc;
     a.num_blocks = num_blocks;
@@ -929,9 +1186,14 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
     a.Hkv = Hkv;
     a.G = Hq / Hkv;
     a.max_seq_len = max_seq_len;
-    a.scale_log2 = scale * 1.4426950408889634f;
-    a.qscale = a.scale_log2 / sqrtf((float)kDim);
-    a.sscale = a.scale_log2 * 1.2533141373155003f / (float)kDim;
+    const float scale_log2 = scale * 1.4426950408889634f;
+    a.scale_log2 = scale_log2;
+    a.tail_k = tail.k;
+    a.tail_v = tail.v;
+    a.tail_lens = tail.lens;
+    a.tail_cap = tail.cap;
+    a.qscale = scale_log2 / sqrtf((float)kDim);
+    a.sscale = scale_log2 * 1.2533141373155003f / (float)kDim;
     a.partial = reinterpret_cast<float*>(ws + plan.partial_off);
     a.prefix = reinterpret_cast<int*>(ws + plan.prefix_off);
     a.split_grid = plan.grid;
@@ -946,10 +1208,17 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
     a.out = out;
     a.out_fp32 = out_fp32;
     a.err = ctx->dev_error;
+    const int KM = kmode_of(ctx);
+    // +-1 bit planes of low-bit key codes (symmetric codebooks, exact up to rounding):
+    // 1 bit: c[b] = c1 (2b - 1); 2 bits: c[2 b1 + b0] = alpha (2 b1 - 1) + beta (2 b0 - 1)
+    const float* ck = ctx->cb_key.c;
+    a.kscale = KM == kKBit1 ? 0.5f * (ck[1] - ck[0]) : 1.f;
+    a.kalpha = KM == kKByte2 ? 0.25f * (ck[3] + ck[2] - ck[1] - ck[0]) : 0.f;
+    a.kbeta = KM == kKByte2 ? 0.25f * (ck[3] - ck[2] + ck[1] - ck[0]) : 0.f;
+    a.stall = take_stall(ctx) ? 1 : 0;
 
     cudaError_t e = launch_dependent(decode_prep_kernel, dim3((B * Hq + 15) / 16, 4), dim3(kPrepThreads), 0, stream, a);
     if (e != cudaSuccess) return e;
-    const int KM = kmode_of(ctx);
     const int VM = ctx->cb_value.width == 4 ? kVByte4 : kVByte2;
     const bool prod = ctx->lay_key.prod;
     const int NT = a.G <= 8 ? 1 : 2;
@@ -984,9 +1253,9 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
     a.merge_sg = sg;
     const int mctas = (mitems + ipc - 1) / ipc;
     const dim3 mgrid(mctas < ctx->sm_count ? mctas : ctx->sm_count);
-    const size_t msmem = merge_smem(ipc, sg);
+    const size_t msmem = merge_smem(ipc, sg, a.tail_k != nullptr);
     e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)std::max(merge_smem(kMergeItems, 1), merge_smem(1, kMergeGroups)));
+                             (int)std::max(merge_smem(kMergeItems, 1, true), merge_smem(1, kMergeGroups, true)));
     if (e != cudaSuccess) return e;
     e = launch_dependent(decode_merge_kernel, mgrid, dim3(kDim * ipc * sg), msmem, stream, a);
     if (e != cudaSuccess) return e;

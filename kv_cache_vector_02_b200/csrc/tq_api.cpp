@@ -1,6 +1,7 @@
 // C ABI of libtq: validation, parameter upload, dispatch.  The arithmetic of
 // the hot path runs in the CUDA translation units; this file only checks
 // arguments, owns the context and launches.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -18,6 +19,13 @@ std::atomic<uint64_t> g_launches{0};
 }
 
 void tq::count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+bool tq::take_stall(const tq_ctx* ctx) {
+    int n = ctx->debug_stall.load(std::memory_order_relaxed);
+    while (n > 0)
+        if (ctx->debug_stall.compare_exchange_weak(n, n - 1, std::memory_order_relaxed)) return true;
+    return false;
+}
 
 namespace {
 
@@ -58,11 +66,40 @@ tq::Codebook make_codebook(const std::vector<double>& c, const std::vector<doubl
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Records that ctx's parameters are in use by work queued on `stream` up to now.
+// Returns false if the event could not be created or recorded.
+bool note_use(const tq_ctx* ctx, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lock(ctx->use_mu);
+    for (auto& u : ctx->uses)
+        if (u.stream == stream) return cudaEventRecord(u.done, stream) == cudaSuccess;
+    if (ctx->uses.size() >= 32) {  // many streams: the oldest one's work is waited for and its slot reused
+        tq_ctx::StreamUse& old = ctx->uses.front();
+        if (cudaEventSynchronize(old.done) != cudaSuccess) return false;
+        old.stream = stream;
+        std::rotate(ctx->uses.begin(), ctx->uses.begin() + 1, ctx->uses.end());
+        return cudaEventRecord(ctx->uses.back().done, stream) == cudaSuccess;
+    }
+    tq_ctx::StreamUse u{stream, nullptr};
+    if (cudaEventCreateWithFlags(&u.done, cudaEventDisableTiming) != cudaSuccess) return false;
+    if (cudaEventRecord(u.done, stream) != cudaSuccess) {
+        cudaEventDestroy(u.done);
+        return false;
+    }
+    ctx->uses.push_back(u);
+    return true;
+}
+
 }  // namespace
 
 extern "C" {
 
 uint64_t tq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+tq_status tq_debug_stall(tq_ctx* ctx, int launches) {
+    if (!ctx || ctx->host_only || launches < 0) return TQ_ERR_INVALID_ARG;
+    ctx->debug_stall.store(launches, std::memory_order_relaxed);
+    return TQ_OK;
+}
 
 const char* tq_status_string(tq_status s) {
     switch (s) {
@@ -76,16 +113,17 @@ const char* tq_status_string(tq_status s) {
     return "TQ_ERR_UNKNOWN";
 }
 
-static tq_status validate_init(int head_dim, int bits, int rotation, int key_mode) {
+static tq_status validate_init(int head_dim, int bits, int rotation, int key_mode, int flags) {
     if (head_dim != kDim) return TQ_ERR_UNSUPPORTED;
     if (bits < 2 || bits > 4) return TQ_ERR_UNSUPPORTED;
     if (rotation != TQ_ROT_HAAR && rotation != TQ_ROT_HADAMARD) return TQ_ERR_UNSUPPORTED;
     if (key_mode != TQ_KEY_PROD && key_mode != TQ_KEY_MSE) return TQ_ERR_UNSUPPORTED;
+    if (flags & ~(TQ_FLAG_SPHERE_CODEBOOK | TQ_FLAG_HOST_ONLY)) return TQ_ERR_UNSUPPORTED;
     return TQ_OK;
 }
 
-static void fill_host(tq_ctx* ctx, int head_dim, int bits, uint64_t seed, int rotation, int key_mode) {
-    ctx->host = tq::make_host_params(head_dim, bits, seed, rotation, key_mode);
+static void fill_host(tq_ctx* ctx, int head_dim, int bits, uint64_t seed, int rotation, int key_mode, int flags) {
+    ctx->host = tq::make_host_params(head_dim, bits, seed, rotation, key_mode, flags & TQ_FLAG_SPHERE_CODEBOOK);
     const tq::HostParams& H = ctx->host;
     ctx->cb_value = make_codebook(H.cv, H.tv, H.vbits);
     ctx->cb_key = make_codebook(H.ck, H.tk, H.kbits);
@@ -93,15 +131,12 @@ static void fill_host(tq_ctx* ctx, int head_dim, int bits, uint64_t seed, int ro
     ctx->lay_key = make_layout(H.kbits, key_mode == TQ_KEY_PROD);
 }
 
-tq_status tq_init_host(int head_dim, int bits, uint64_t seed, int rotation, int key_mode, tq_ctx** out) {
-    if (!out) return TQ_ERR_INVALID_ARG;
-    *out = nullptr;
-    const tq_status v = validate_init(head_dim, bits, rotation, key_mode);
-    if (v != TQ_OK) return v;
+static tq_status init_host_only(int head_dim, int bits, uint64_t seed, int rotation, int key_mode, int flags,
+                                tq_ctx** out) {
     tq_ctx* ctx = new (std::nothrow) tq_ctx();
     if (!ctx) return TQ_ERR_OOM;
     ctx->host_only = true;
-    fill_host(ctx, head_dim, bits, seed, rotation, key_mode);
+    fill_host(ctx, head_dim, bits, seed, rotation, key_mode, flags);
     tq::TcBlob tcb;  // same tables as a device context, built to surface any failure here too
     if (!tq::build_tc_blob(ctx->host, tcb)) {
         delete ctx;
@@ -111,11 +146,20 @@ tq_status tq_init_host(int head_dim, int bits, uint64_t seed, int rotation, int 
     return TQ_OK;
 }
 
+tq_status tq_init_host(int head_dim, int bits, uint64_t seed, int rotation, int key_mode, tq_ctx** out) {
+    return tq_init_ex(head_dim, bits, seed, rotation, key_mode, TQ_FLAG_HOST_ONLY, out);
+}
+
 tq_status tq_init(int head_dim, int bits, uint64_t seed, int rotation, int key_mode, tq_ctx** out) {
+    return tq_init_ex(head_dim, bits, seed, rotation, key_mode, 0, out);
+}
+
+tq_status tq_init_ex(int head_dim, int bits, uint64_t seed, int rotation, int key_mode, int flags, tq_ctx** out) {
     if (!out) return TQ_ERR_INVALID_ARG;
     *out = nullptr;
-    const tq_status v = validate_init(head_dim, bits, rotation, key_mode);
+    const tq_status v = validate_init(head_dim, bits, rotation, key_mode, flags);
     if (v != TQ_OK) return v;
+    if (flags & TQ_FLAG_HOST_ONLY) return init_host_only(head_dim, bits, seed, rotation, key_mode, flags, out);
 
     tq_ctx* ctx = new (std::nothrow) tq_ctx();
     if (!ctx) return TQ_ERR_OOM;
@@ -125,24 +169,21 @@ tq_status tq_init(int head_dim, int bits, uint64_t seed, int rotation, int key_m
         cudaGetLastError();
         return TQ_ERR_CUDA;
     }
-    fill_host(ctx, head_dim, bits, seed, rotation, key_mode);
+    fill_host(ctx, head_dim, bits, seed, rotation, key_mode, flags);
     const tq::HostParams& H = ctx->host;
 
-    // device copies: R, R^T, S, S^T (fp32), R^T hi / lo and S (fp16); then the tensor-core blob
+    // device copies: R^T and S (fp32; decode merge and decompress), R^T hi / lo and S
+    // (fp16; decode prep); then the tensor-core blob
     const size_t n = size_t(kDim) * kDim;
-    std::vector<float> blob(4 * n);
+    std::vector<float> blob(2 * n);
     std::vector<__half> blob16(3 * n);
-    float* R = blob.data();
-    float* RT = R + n;
+    float* RT = blob.data();
     float* S = RT + n;
-    float* ST = S + n;
     for (int i = 0; i < kDim; ++i)
         for (int j = 0; j < kDim; ++j) {
             const double r = H.R[size_t(i) * kDim + j];
-            R[i * kDim + j] = float(r);
             RT[j * kDim + i] = float(r);
             S[i * kDim + j] = float(H.S[size_t(i) * kDim + j]);
-            ST[j * kDim + i] = float(H.S[size_t(i) * kDim + j]);
             const __half hi = __double2half(r);
             blob16[size_t(j) * kDim + i] = hi;
             blob16[n + size_t(j) * kDim + i] = __double2half(r - double(__half2float(hi)));
@@ -181,10 +222,8 @@ tq_status tq_init(int head_dim, int bits, uint64_t seed, int rotation, int key_m
         return TQ_ERR_CUDA;
     }
     const float* base = static_cast<const float*>(ctx->dev_block);
-    ctx->dev.R = base;
-    ctx->dev.RT = base + n;
-    ctx->dev.S = base + 2 * n;
-    ctx->dev.ST = base + 3 * n;
+    ctx->dev.RT = base;
+    ctx->dev.S = base + n;
     const uint16_t* base16 = reinterpret_cast<const uint16_t*>(base8 + f16_off);
     ctx->dev.RTh = base16;
     ctx->dev.RTl = base16 + n;
@@ -204,7 +243,16 @@ tq_status tq_destroy(tq_ctx* ctx) {
         delete ctx;
         return TQ_OK;
     }
-    cudaDeviceSynchronize();
+    // the context's own work: every stream it launched on, up to its latest launch
+    // (cudaFree below may still wait for the device as the runtime sees fit)
+    {
+        std::lock_guard<std::mutex> lock(ctx->use_mu);
+        for (auto& u : ctx->uses) {
+            cudaEventSynchronize(u.done);
+            cudaEventDestroy(u.done);
+        }
+        ctx->uses.clear();
+    }
     cudaFree(ctx->dev_block);
     cudaFree(ctx->dev_error);
     cudaGetLastError();
@@ -255,7 +303,7 @@ tq_status tq_compress(const tq_ctx* ctx, const uint16_t* k, const uint16_t* v, i
         return TQ_ERR_CUDA;
     if (v && tq::launch_compress(ctx, TQ_KIND_VALUE, v, T, Hkv, slot_mapping, v_cache, num_blocks, s) != cudaSuccess)
         return TQ_ERR_CUDA;
-    return TQ_OK;
+    return note_use(ctx, s) ? TQ_OK : TQ_ERR_CUDA;
 }
 
 tq_status tq_decompress(const tq_ctx* ctx, int kind, const uint8_t* cache, int num_blocks,
@@ -268,7 +316,7 @@ tq_status tq_decompress(const tq_ctx* ctx, int kind, const uint8_t* cache, int n
     if (tq::launch_decompress(ctx, kind, cache, num_blocks, slot_mapping, T, Hkv, out, out_fp32,
                               static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return TQ_ERR_CUDA;
-    return TQ_OK;
+    return note_use(ctx, static_cast<cudaStream_t>(stream)) ? TQ_OK : TQ_ERR_CUDA;
 }
 
 size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_seq_len) {
@@ -276,10 +324,11 @@ size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int 
     return tq::plan_decode(ctx, B, Hq, Hkv, max_seq_len).bytes;
 }
 
-tq_status tq_decode_attention(const tq_ctx* ctx, const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
-                              int num_blocks, const int32_t* block_table, int max_blocks, const int32_t* seq_lens,
-                              int B, int Hq, int Hkv, int max_seq_len, float scale, void* out, int out_fp32,
-                              void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+tq_status decode_common(const tq_ctx* ctx, const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                        int num_blocks, const int32_t* block_table, int max_blocks, const int32_t* seq_lens, int B,
+                        int Hq, int Hkv, int max_seq_len, const tq::DecodeTail& tail, float scale, void* out,
+                        int out_fp32, void* workspace, size_t workspace_bytes, void* stream) {
     if (!ctx || ctx->host_only || B < 0 || Hq < 1 || Hkv < 1 || max_blocks < 0 || num_blocks < 0 || max_seq_len < 0)
         return TQ_ERR_INVALID_ARG;
     if (Hq % Hkv != 0 || Hq / Hkv > 16) return TQ_ERR_INVALID_ARG;
@@ -287,15 +336,44 @@ tq_status tq_decode_attention(const tq_ctx* ctx, const uint16_t* q, const uint8_
     if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !out || !workspace) return TQ_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(workspace))
         return TQ_ERR_INVALID_ARG;
+    if (tail.k) {
+        if (!tail.v || !tail.lens || tail.cap < 1 || tail.cap > tq::kDecodeTailMax) return TQ_ERR_INVALID_ARG;
+        if (!aligned16(tail.k) || !aligned16(tail.v)) return TQ_ERR_INVALID_ARG;
+    }
     if (!(scale >= 0.f) || !std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
     const tq::DecodePlan plan = tq::plan_decode(ctx, B, Hq, Hkv, max_seq_len);
     if (workspace_bytes < plan.bytes) return TQ_ERR_INVALID_ARG;
     if (scale == 0.f) scale = 1.0f / std::sqrt(float(kDim));
     if (tq::launch_decode(ctx, plan, q, k_cache, v_cache, num_blocks, block_table, max_blocks, seq_lens, B, Hq, Hkv,
-                          max_seq_len, scale, out, out_fp32, workspace, static_cast<cudaStream_t>(stream)) !=
+                          max_seq_len, tail, scale, out, out_fp32, workspace, static_cast<cudaStream_t>(stream)) !=
         cudaSuccess)
         return TQ_ERR_CUDA;
-    return TQ_OK;
+    return note_use(ctx, static_cast<cudaStream_t>(stream)) ? TQ_OK : TQ_ERR_CUDA;
+}
+}  // namespace
+
+tq_status tq_decode_attention(const tq_ctx* ctx, const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                              int num_blocks, const int32_t* block_table, int max_blocks, const int32_t* seq_lens,
+                              int B, int Hq, int Hkv, int max_seq_len, float scale, void* out, int out_fp32,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    return decode_common(ctx, q, k_cache, v_cache, num_blocks, block_table, max_blocks, seq_lens, B, Hq, Hkv,
+                         max_seq_len, tq::DecodeTail{}, scale, out, out_fp32, workspace, workspace_bytes, stream);
+}
+
+tq_status tq_decode_attention_window(const tq_ctx* ctx, const uint16_t* q, const uint8_t* k_cache,
+                                     const uint8_t* v_cache, int num_blocks, const int32_t* block_table,
+                                     int max_blocks, const int32_t* seq_lens, int B, int Hq, int Hkv,
+                                     int max_seq_len, const uint16_t* tail_k, const uint16_t* tail_v,
+                                     const int32_t* tail_lens, int tail_cap, float scale, void* out, int out_fp32,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+    if (!tail_k) return TQ_ERR_INVALID_ARG;
+    tq::DecodeTail tail;
+    tail.k = tail_k;
+    tail.v = tail_v;
+    tail.lens = tail_lens;
+    tail.cap = tail_cap;
+    return decode_common(ctx, q, k_cache, v_cache, num_blocks, block_table, max_blocks, seq_lens, B, Hq, Hkv,
+                         max_seq_len, tail, scale, out, out_fp32, workspace, workspace_bytes, stream);
 }
 
 tq_status tq_get_device_error(const tq_ctx* ctx, void* stream, uint32_t* code) {

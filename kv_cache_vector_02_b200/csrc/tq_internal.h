@@ -2,7 +2,9 @@
 #pragma once
 
 #include <cstddef>
+#include <atomic>
 #include <cstdint>
+#include <mutex>
 #include <vector>
 
 #include <cuda_runtime.h>
@@ -20,6 +22,7 @@ constexpr int kMaxLevels = 16;  // up to 4-bit codebooks
 struct HostParams {
     int d = 0, bits = 0, rotation = 0, key_mode = 0;
     int vbits = 0, kbits = 0;
+    int flags = 0;                // TQ_FLAG_* of tq_init_ex
     std::vector<double> R;        // [d*d] row-major, y = R^T x
     std::vector<int8_t> S;        // [d*d] row-major, (S r)_j = sum_i S[j][i] r_i
     std::vector<int8_t> hsigns;   // [d] Hadamard signs (rotation == 1)
@@ -28,7 +31,7 @@ struct HostParams {
     std::vector<double> ck, tk;   // key codebook / interior boundaries
 };
 
-HostParams make_host_params(int d, int bits, uint64_t seed, int rotation, int key_mode);
+HostParams make_host_params(int d, int bits, uint64_t seed, int rotation, int key_mode, int flags);
 
 // Codebook of one kind as the kernels see it (by value, kernel parameter space).
 struct Codebook {
@@ -51,10 +54,8 @@ struct ChunkLayout {
 
 // Device copies of the parameters (one allocation owned by the context).
 struct DeviceParams {
-    const float* R;       // [d*d] R[i][j] row-major
     const float* RT;      // [d*d] R^T row-major
     const float* S;       // [d*d] S row-major as +-1.0f
-    const float* ST;      // [d*d] S^T row-major
     const uint16_t* RTh;  // [d*d] fp16 R^T, high part
     const uint16_t* RTl;  // [d*d] fp16 R^T - RTh
     const uint16_t* Sh;   // [d*d] fp16 S (+-1, exact)
@@ -65,6 +66,18 @@ inline int container_width(int b) { return b >= 3 ? 4 : (b == 2 ? 2 : 1); }
 }  // namespace tq
 
 struct tq_ctx {
+    // Streams this context has launched work on, each with an event recorded after
+    // its latest launches; tq_destroy waits for these (not for the whole device).
+    struct StreamUse {
+        cudaStream_t stream;
+        cudaEvent_t done;
+    };
+    mutable std::mutex use_mu;
+    mutable std::vector<StreamUse> uses;
+
+    // Test hook (tq_debug_stall): launches left that skip their input copies.
+    mutable std::atomic<int> debug_stall{0};
+
     bool host_only = false;         // built by tq_init_host: no device state
     int device = 0;
     int sm_count = 0;
@@ -81,6 +94,10 @@ namespace tq {
 
 // Adds n to the process-wide launch counter (tq_launch_count).
 void count_launches(unsigned n);
+
+// Test hook: true (once per pending stall) if this launch must skip its input
+// copies so that its bounded waits run out (tq_debug_stall).
+bool take_stall(const tq_ctx* ctx);
 
 // Kernel launchers (CUDA translation units).  Each returns cudaSuccess or the
 // launch error.
@@ -105,9 +122,18 @@ struct DecodePlan {
     size_t bytes;        // total workspace
 };
 DecodePlan plan_decode(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_seq_len);
+// Residual window of the decode: fp16 [B][cap][Hkv][128] keys and values, lengths [B]
+// (k == nullptr: none).
+struct DecodeTail {
+    const uint16_t* k = nullptr;
+    const uint16_t* v = nullptr;
+    const int32_t* lens = nullptr;
+    int cap = 0;
+};
+constexpr int kDecodeTailMax = 256;
 cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint16_t* q, const uint8_t* kc,
                           const uint8_t* vc, int num_blocks, const int32_t* block_table, int max_blocks,
-                          const int32_t* seq_lens, int B, int Hq, int Hkv, int max_seq_len, float scale, void* out,
-                          int out_fp32, void* workspace, cudaStream_t stream);
+                          const int32_t* seq_lens, int B, int Hq, int Hkv, int max_seq_len, const DecodeTail& tail,
+                          float scale, void* out, int out_fp32, void* workspace, cudaStream_t stream);
 
 }  // namespace tq

@@ -132,9 +132,65 @@ void gaussian_lloyd_max(int bits, std::vector<double>& levels, std::vector<doubl
     bounds[m - 1] = 0.0;
 }
 
+// Exact-d Lloyd-Max codebook ([TQ-RS] "Étape 2" / "Couche 2": the rotated
+// coordinate of a unit vector follows the spherical Beta law).  The quantized
+// value is v = sqrt(d) cos(theta), where the angle theta of a uniform unit vector
+// to an axis has density proportional to sin^n(theta), n = d - 2, on (0, pi).
+// With J(alpha) = int_0^alpha sin^n, by the reduction formula
+//   J_k(alpha) = -sin^(k-1)(alpha) cos(alpha) / k + (k-1)/k J_(k-2)(alpha),
+//   P(v > x)   = J(acos(x / sqrt(d))) / J(pi),
+//   E[v; v > x] = sqrt(d) sin^(n+1)(acos(x / sqrt(d))) / ((n+1) J(pi)).
+// (The recursion loses relative accuracy in the far tail, beyond the largest
+// boundary a 4-bit codebook has; the last cell's mass is dominated by its start.)
+// Solved on the positive half like the Gaussian codebook.
+double sin_power_integral(int n, double alpha) {
+    const double s = std::sin(alpha), c = std::cos(alpha);
+    double j = (n % 2 == 0) ? alpha : 1.0 - c;
+    double sp = (n % 2 == 0) ? s : s * s;  // sin^(k-1) for the first k
+    for (int k = (n % 2 == 0) ? 2 : 3; k <= n; k += 2) {
+        j = -sp * c / k + double(k - 1) / k * j;
+        sp *= s * s;
+    }
+    return j;
+}
+
+void sphere_lloyd_max(int d, int bits, std::vector<double>& levels, std::vector<double>& bounds) {
+    const int L = 1 << bits, m = L / 2, n = d - 2;
+    const double rd = std::sqrt(double(d)), total = sin_power_integral(n, M_PI);
+    auto tail = [&](double x) { return sin_power_integral(n, std::acos(std::fmin(x / rd, 1.0))) / total; };
+    auto tail_moment = [&](double x) {
+        const double th = std::acos(std::fmin(x / rd, 1.0));
+        return rd * std::pow(std::sin(th), n + 1) / ((n + 1) * total);
+    };
+    std::vector<double> a(m), e(m + 1);
+    for (int k = 0; k < m; ++k) a[k] = 3.0 * (k + 0.5) / m;
+    for (int iter = 0; iter < 400000; ++iter) {
+        e[0] = 0.0;
+        for (int k = 1; k < m; ++k) e[k] = 0.5 * (a[k - 1] + a[k]);
+        double delta = 0.0;
+        for (int k = 0; k < m; ++k) {
+            const bool last = (k == m - 1);
+            const double num = tail_moment(e[k]) - (last ? 0.0 : tail_moment(e[k + 1]));
+            const double den = tail(e[k]) - (last ? 0.0 : tail(e[k + 1]));
+            const double nv = num / den;
+            delta = std::fmax(delta, std::fabs(nv - a[k]));
+            a[k] = nv;
+        }
+        if (delta < 1e-16) break;
+    }
+    levels.assign(L, 0.0);
+    for (int k = 0; k < m; ++k) {
+        levels[m + k] = a[k];
+        levels[m - 1 - k] = -a[k];
+    }
+    bounds.assign(L - 1, 0.0);
+    for (int j = 0; j + 1 < L; ++j) bounds[j] = 0.5 * (levels[j] + levels[j + 1]);
+    bounds[m - 1] = 0.0;
+}
+
 }  // namespace
 
-HostParams make_host_params(int d, int bits, uint64_t seed, int rotation, int key_mode) {
+HostParams make_host_params(int d, int bits, uint64_t seed, int rotation, int key_mode, int flags) {
     HostParams P;
     P.d = d;
     P.bits = bits;
@@ -152,8 +208,14 @@ HostParams make_host_params(int d, int bits, uint64_t seed, int rotation, int ke
             for (int j = 0; j < d; ++j) P.R[size_t(i) * d + j] = P.hsigns[i] * hadamard_entry(i, j) * s;
     }
     P.S = rademacher(seed, 1, size_t(d) * d);
-    gaussian_lloyd_max(P.vbits, P.cv, P.tv);
-    gaussian_lloyd_max(P.kbits, P.ck, P.tk);
+    P.flags = flags;
+    if (flags & TQ_FLAG_SPHERE_CODEBOOK) {
+        sphere_lloyd_max(d, P.vbits, P.cv, P.tv);
+        sphere_lloyd_max(d, P.kbits, P.ck, P.tk);
+    } else {
+        gaussian_lloyd_max(P.vbits, P.cv, P.tv);
+        gaussian_lloyd_max(P.kbits, P.ck, P.tk);
+    }
     // M = S R: the QJL sketch taken in the rotated domain, S r = S R (R^T r).
     P.M.assign(size_t(d) * d, 0.0);
     for (int j = 0; j < d; ++j)

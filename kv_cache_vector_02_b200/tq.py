@@ -23,9 +23,12 @@ KEY_PROD, KEY_MSE = 0, 1
 KIND_KEY, KIND_VALUE = 0, 1
 DEVERR_SLOT, DEVERR_BLOCK, DEVERR_SEQLEN, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 
-EXPORTED = ("tq_init", "tq_init_host", "tq_destroy", "tq_chunk_bytes", "tq_code_bits", "tq_export_params", "tq_compress",
-            "tq_decompress", "tq_decode_workspace_bytes", "tq_decode_attention", "tq_decode_attention_noalloc",
-            "tq_get_device_error", "tq_launch_count", "tq_status_string")
+FLAG_SPHERE_CODEBOOK, FLAG_HOST_ONLY = 0x1, 0x4
+
+EXPORTED = ("tq_init", "tq_init_ex", "tq_init_host", "tq_destroy", "tq_chunk_bytes", "tq_code_bits", "tq_export_params", "tq_compress",
+            "tq_decompress", "tq_decode_workspace_bytes", "tq_decode_attention", "tq_decode_attention_window",
+            "tq_decode_attention_noalloc",
+            "tq_get_device_error", "tq_debug_stall", "tq_launch_count", "tq_status_string")
 
 
 class TQError(RuntimeError):
@@ -42,6 +45,7 @@ def _load():
     sig = {
         "tq_init": (I, [I, I, U64, I, I, ctypes.POINTER(P)]),
         "tq_init_host": (I, [I, I, U64, I, I, ctypes.POINTER(P)]),
+        "tq_init_ex": (I, [I, I, U64, I, I, I, ctypes.POINTER(P)]),
         "tq_destroy": (I, [P]),
         "tq_chunk_bytes": (Z, [P, I]),
         "tq_code_bits": (I, [P, I]),
@@ -50,8 +54,10 @@ def _load():
         "tq_decompress": (I, [P, I, P, I, P, I, I, P, I, P]),
         "tq_decode_workspace_bytes": (Z, [P, I, I, I, I]),
         "tq_decode_attention": (I, [P, P, P, P, I, P, I, P, I, I, I, I, F, P, I, P, Z, P]),
+        "tq_decode_attention_window": (I, [P, P, P, P, I, P, I, P, I, I, I, I, P, P, P, I, F, P, I, P, Z, P]),
         "tq_decode_attention_noalloc": (I, [P, P, P, P, I, P, I, P, I, I, I, I, F, P, I, P]),
         "tq_get_device_error": (I, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
+        "tq_debug_stall": (I, [P, I]),
         "tq_launch_count": (ctypes.c_uint64, []),
         "tq_status_string": (ctypes.c_char_p, [I]),
     }
@@ -114,6 +120,14 @@ def tq_init(head_dim: int = 128, bits: int = 4, seed: int = 0, rotation: int = R
             key_mode: int = KEY_PROD) -> Context:
     h = ctypes.c_void_p()
     _check(_lib.tq_init(head_dim, bits, seed, rotation, key_mode, ctypes.byref(h)), "tq_init")
+    return Context(h.value, head_dim, bits, seed, rotation, key_mode)
+
+
+def tq_init_ex(head_dim: int = 128, bits: int = 4, seed: int = 0, rotation: int = ROT_HAAR,
+               key_mode: int = KEY_PROD, flags: int = 0) -> Context:
+    """tq_init with TQ_FLAG_* options (see tq.h)."""
+    h = ctypes.c_void_p()
+    _check(_lib.tq_init_ex(head_dim, bits, seed, rotation, key_mode, flags, ctypes.byref(h)), "tq_init_ex")
     return Context(h.value, head_dim, bits, seed, rotation, key_mode)
 
 
@@ -214,7 +228,7 @@ def tq_decode_workspace_bytes(ctx: Context, B: int, Hq: int, Hkv: int, max_seq_l
 def tq_decode_attention(ctx: Context, q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int, out,
                         workspace, scale: float = 0.0, Hkv: int | None = None, stream=None):
     """q: [B, Hq, 128] fp16; caches [num_blocks, Hkv, chunk] uint8; block_table [B, max_blocks] int32;
-    seq_lens [B] int32; out [B, Hq, 128] fp16 or fp32; workspace uint8 tensor (zeroed once)."""
+    seq_lens [B] int32; out [B, Hq, 128] fp16 or fp32; workspace uint8 tensor (any contents)."""
     import torch
     B, Hq = int(q.shape[0]), int(q.shape[1])
     if Hkv is None:
@@ -226,6 +240,30 @@ def tq_decode_attention(ctx: Context, q, k_cache, v_cache, block_table, seq_lens
                                     int(max_seq_len), float(scale), _ptr(out), 1 if out.dtype == torch.float32 else 0,
                                     _ptr(workspace), int(workspace.numel() * workspace.element_size()),
                                     _stream(stream)), "tq_decode_attention")
+
+
+def tq_decode_attention_window(ctx: Context, q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int,
+                               tail_k, tail_v, tail_lens, out, workspace, scale: float = 0.0,
+                               Hkv: int | None = None, stream=None):
+    """tq_decode_attention plus an fp16 residual window: tail_k, tail_v [B, W, Hkv, 128]
+    fp16 (W <= 256), tail_lens [B] int32 (see tq.h)."""
+    import torch
+    B, Hq = int(q.shape[0]), int(q.shape[1])
+    if Hkv is None:
+        Hkv = int(k_cache.shape[1])
+    what = "tq_decode_attention_window"
+    _check_decode_args(ctx, q, k_cache, v_cache, block_table, seq_lens, out, Hkv, what)
+    _expect(workspace, (None,), (torch.uint8,), what, "workspace")
+    W = int(tail_k.shape[1]) if tail_k is not None and tail_k.dim() == 4 else 0
+    _expect(tail_k, (B, W, Hkv, ctx.head_dim), (torch.float16,), what, "tail_k")
+    _expect(tail_v, (B, W, Hkv, ctx.head_dim), (torch.float16,), what, "tail_v")
+    _expect(tail_lens, (B,), (torch.int32,), what, "tail_lens")
+    _check(_lib.tq_decode_attention_window(ctx.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache), int(k_cache.shape[0]),
+                                           _ptr(block_table), int(block_table.shape[1]), _ptr(seq_lens), B, Hq, Hkv,
+                                           int(max_seq_len), _ptr(tail_k), _ptr(tail_v), _ptr(tail_lens), W,
+                                           float(scale), _ptr(out), 1 if out.dtype == torch.float32 else 0,
+                                           _ptr(workspace), int(workspace.numel() * workspace.element_size()),
+                                           _stream(stream)), what)
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -265,6 +303,12 @@ def tq_get_device_error(ctx: Context, stream=None) -> int:
     if st not in (TQ_OK, TQ_ERR_DEVICE):
         raise TQError(st, "tq_get_device_error")
     return int(code.value)
+
+
+def tq_debug_stall(ctx: Context, launches: int):
+    """Test hook: the next `launches` streaming kernels of ctx skip their input
+    copies, so their bounded waits run out and TQ_DEVERR_TIMEOUT is set (see tq.h)."""
+    _check(_lib.tq_debug_stall(ctx.handle, int(launches)), "tq_debug_stall")
 
 
 def tq_launch_count() -> int:
