@@ -37,3 +37,24 @@ def test_fp32_rotation_is_orthogonal(tq):
     p = tq.tq_export_params(tq.tq_init_host(128, 4, 0))
     R32 = p["R"].astype(np.float32).astype(np.float64)
     assert np.abs(R32.T @ R32 - np.eye(128)).max() < 1e-5
+
+
+@pytest.mark.parametrize("bits,km", [(4, 0), (3, 1), (2, 0)])
+def test_sphere_codebook_matches_oracle(tq, orc, bits, km):
+    """libtq's exact-d codebook (angle form: reduction formula of the sine power)
+    against the oracle's (incomplete beta continued fraction)."""
+    ctx = tq.tq_init_ex(128, bits, 0, 0, km, tq.FLAG_SPHERE_CODEBOOK | tq.FLAG_HOST_ONLY)
+    p = tq.tq_export_params(ctx)
+    o = orc.Oracle(128, bits, 0, key_mode=km, beta=True)
+    cv, tv = o.codebook(orc.KIND_VALUE)
+    ck, tk = o.codebook(orc.KIND_KEY)
+    assert np.abs(p["cv"] - cv).max() < 1e-11 and np.abs(p["tv"] - tv).max() < 1e-11
+    assert np.abs(p["ck"] - ck).max() < 1e-11 and np.abs(p["tk"] - tk).max() < 1e-11
+    g = tq.tq_export_params(tq.tq_init_host(128, bits, 0, 0, km))
+    assert np.abs(p["cv"] - g["cv"]).max() > 1e-4   # really another codebook
+
+
+def test_unknown_init_flag_is_refused(tq):
+    import ctypes
+    h = ctypes.c_void_p()
+    assert tq._lib.tq_init_ex(128, 4, 0, 0, 0, 0x100, ctypes.byref(h)) == tq.TQ_ERR_UNSUPPORTED
