@@ -9,10 +9,14 @@ prefill (K and V of every token and kv head) and tq_decode_attention of one
 decode query per sequence over the cache the previous step compressed (two
 caches alternate, so the decode reads pages that 700 MB of compress traffic
 has since pushed out of L2).  Inputs are resident in HBM before the timed
-region.  `value` = algorithmic bytes of the step (compress: fp16 K+V in, packed
-pages out; decode: packed K+V pages read, q in, out) / step time, summed over
-ranks.  Under torchrun every rank runs its own batch (weak scaling, no
-collective on the data path); times are the max over ranks.
+region.
+
+`value` is the headline metric: decode-attention KV GB/s = the decode's
+algorithmic bytes (packed K+V pages of every attended token, q in, out, block
+table) / the decode's device time, summed over ranks.  Compress Mtokens/s and
+both kernels' fractions of the measured HBM bandwidth sit beside it.  Under
+torchrun every rank runs its own batch (weak scaling, no collective on the data
+path); times are the max over ranks.
 
 --impl reference times the CPU oracle (the plain fp64 restatement of the
 method) on a bounded sample of the same workload, in the same unit.
@@ -24,6 +28,7 @@ import hashlib
 import json
 import math
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -47,7 +52,7 @@ def parse():
     ap.add_argument("--workload", default="batched")
     ap.add_argument("--bits", type=int, default=4)
     ap.add_argument("--rotation", default="haar", choices=["haar", "hadamard"])
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -196,22 +201,36 @@ def whole_job_gbs(ws: int, bytes_per_rank_step: float, ms_step_max: float) -> fl
 
 
 # ---------------------------------------------------------------- oracle (CPU) leg
-def oracle_sample(w, target_s: float = 15.0, min_seqs: int = 1):
-    """Run the CPU oracle on whole sequences of the workload (compress K and V of
-    the sequence, then one decode of all its query heads) until about target_s
-    seconds have passed.  Returns (seconds, compress_bytes, decode_bytes, seqs, threads)."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+def oracle_sample(w, target_s: float = 10.0, threads: int = 0, min_seqs: int = 1, max_seqs: int | None = None):
+    """The CPU oracle on whole sequences of the workload: compress K and V of the
+    sequence (timed separately), then decode all its query heads (timed), until
+    about target_s seconds of decode time have passed.  threads = 0: every core.
+    Returns dict(decode_s, decode_bytes, compress_s, compress_bytes, seqs, threads)."""
     import numpy as np
 
     import oracle
     from kv_cache_vector_02_b200 import workloads as W
-    o = oracle.Oracle(D, w.bits, w.param_seed, rot=w.rotation, key_mode=w.key_mode)
+    nth = threads if threads > 0 else oracle.max_threads()
+    o = oracle.Oracle(D, w.bits, w.param_seed, rot=w.rotation, key_mode=w.key_mode, nthreads=nth)
     one = w.with_(B=1, layers=1, decode_steps=0)
     bt = np.arange(one.max_blocks, dtype=np.int32)[None]
     slots = W.prefill_slots(one, bt)
     cb, db = step_bytes(one)
-    elapsed = 0.0
-    n = 0
+    r = {"decode_s": 0.0, "decode_bytes": 0.0, "compress_s": 0.0, "compress_bytes": 0.0, "seqs": 0, "threads": nth}
+    cap = max_seqs if max_seqs is not None else w.B * w.layers
     while True:
+        n = r["seqs"]
         wi = one.with_(data_seed=w.data_seed + 1000 + n)
         k, v = W.gen_kv(wi, 0).numpy(), W.gen_kv(wi, 1).numpy()
         q = W.gen_q(wi).numpy().astype(np.float64)
@@ -219,42 +238,51 @@ def oracle_sample(w, target_s: float = 15.0, min_seqs: int = 1):
         kc, vc = o.new_cache(0, one.num_blocks, one.Hkv), o.new_cache(1, one.num_blocks, one.Hkv)
         o.compress_paged(0, k, slots, kc)
         o.compress_paged(1, v, slots, vc)
+        r["compress_s"] += time.perf_counter() - ts
+        r["compress_bytes"] += cb
+        ts = time.perf_counter()
         o.decode(q, kc, vc, bt, np.array([one.T], np.int32), one.Hkv)
-        elapsed += time.perf_counter() - ts
-        n += 1
-        if (n >= min_seqs and elapsed >= target_s) or n >= w.B * w.layers:
+        r["decode_s"] += time.perf_counter() - ts
+        r["decode_bytes"] += db
+        r["seqs"] = n + 1
+        if (r["seqs"] >= min_seqs and r["decode_s"] >= target_s) or r["seqs"] >= cap:
             break
-    return elapsed, cb * n, db * n, n, oracle.max_threads()
+    return r
 
 
 def run_reference(args):
-    """Reference arm: the oracle as it stands, timed on the host cores."""
+    """Reference arm: the oracle as it stands, timed on the host cores, on the same
+    metric (decode-attention KV GB/s) over bounded samples of the workload."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     from kv_cache_vector_02_b200 import workloads as W
     w = W.WORKLOADS[args.workload].with_(bits=args.bits, rotation=1 if args.rotation == "hadamard" else 0)
-    per_step = max(2.0, 120.0 / max(1, args.steps + args.warmup))
+    per_step = max(1.0, 90.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         oracle_sample(w, target_s=0.0)
-    tot_s = tot_b = 0.0
+    dec_s = dec_b = comp_s = comp_b = 0.0
     seqs = 0
     threads = 1
     for _ in range(args.steps):
-        s, cb, db, n, threads = oracle_sample(w, target_s=per_step)
-        tot_s += s
-        tot_b += cb + db
-        seqs += n
-    gbs = tot_b / tot_s / 1e9
+        r = oracle_sample(w, target_s=per_step)
+        dec_s += r["decode_s"]
+        dec_b += r["decode_bytes"]
+        comp_s += r["compress_s"]
+        comp_b += r["compress_bytes"]
+        seqs += r["seqs"]
+        threads = r["threads"]
+    gbs = dec_b / dec_s / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": 1e3 * (dec_s + comp_s) / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w),
-        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
-                         "sample": "%d whole sequences (%d tokens x %d kv heads: compress K+V, decode %d q heads)"
-                                   % (seqs, w.T, w.Hkv, w.Hq)},
+        "compress": {"mtokens_per_s": seqs * w.T / comp_s / 1e6, "gbs": comp_b / comp_s / 1e9},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "cpu": cpu_model(),
+                         "sample": "%d whole sequences (%d tokens x %d kv heads): compress K+V untimed for the "
+                                   "metric, decode of %d query heads timed" % (seqs, w.T, w.Hkv, w.Hq)},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -369,76 +397,100 @@ def main():
 
     cbytes, dbytes = step_bytes(w)
     ms_step = ms_total / args.steps
-    value = whole_job_gbs(ws, cbytes + dbytes, ms_step)
     peak, peak_kind = measured_peak()
     comp_avg = max_over_ranks(ws, sum(comp_ms) / len(comp_ms))
     dec_avg = max_over_ranks(ws, sum(dec_ms) / len(dec_ms))
     comp_gbs = cbytes / (comp_avg * 1e-3) / 1e9
     dec_gbs = dbytes / (dec_avg * 1e-3) / 1e9
+    value = whole_job_gbs(ws, dbytes, dec_avg)  # the headline: decode-attention KV GB/s
     tokens = w.B * w.T * w.layers
-    dominant = "compress" if comp_avg >= dec_avg else "decode"
-    rec = traffic_record(dominant)
-    roof = {
-        "kernel": "tq_compress (K and V launches)" if dominant == "compress" else "tq_decode_attention",
-        "bound": "hbm",
-        "achieved": comp_gbs if dominant == "compress" else dec_gbs,
-        "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-        "traffic": (rec["bytes_per_call"] if rec else None),
-    }
-    roof["frac"] = roof["achieved"] / peak
 
-    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    def roofline(kind):
+        rec = traffic_record(kind)
+        r = {"kernel": "tq_compress (K and V launches)" if kind == "compress" else
+             "tq_decode_attention (prep, page kernel, merge)",
+             "bound": "hbm", "achieved": comp_gbs if kind == "compress" else dec_gbs,
+             "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+             "traffic": (rec["bytes_per_call"] if rec else None)}
+        r["frac"] = r["achieved"] / peak
+        if rec and rec.get("tensor_pipe_pct") is not None:
+            r["tensor_pipe_pct"] = rec["tensor_pipe_pct"]
+        return r
+    dominant = "compress" if comp_avg >= dec_avg else "decode"
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region:
+    # decode (the metric's call): q host -> device, tq_decode_attention over the resident cache,
+    # out device -> host; compress: K, V and the slot mapping host -> device, tq_compress.
     hk = k.cpu().pin_memory()
     hv = v.cpu().pin_memory()
     hq = q.cpu().pin_memory()
     hslots = slots.cpu().pin_memory()
     hout = torch.empty_like(out, device="cpu").pin_memory()
     dk, dv, dq, dsl = torch.empty_like(k), torch.empty_like(v), torch.empty_like(q), torch.empty_like(slots)
-    h2d = hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 2 + hslots.numel() * 4
-    d2h = hout.numel() * 2
+    h2d_dec = hq.numel() * 2
+    d2h_dec = hout.numel() * 2
+    h2d_comp = hk.numel() * 2 + hv.numel() * 2 + hslots.numel() * 4
 
-    def e2e_step(i):
+    def e2e_decode(i):
         kc, vc = caches[i % 2]
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
         dq.copy_(hq, non_blocking=True)
-        dsl.copy_(hslots, non_blocking=True)
-        tq.tq_compress(ctx, dk, dv, dsl, kc, vc, stream=stream)
         tq.tq_decode_attention(ctx, dq, kc, vc, bt, seq, w.T, out, workspace, stream=stream)
         hout.copy_(out, non_blocking=True)
 
-    e2e_step(0)
-    torch.cuda.synchronize()
-    barrier(ws)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for i in range(args.e2e_steps):
-        e2e_step(i)
-    b.record(stream)
-    torch.cuda.synchronize()
-    barrier(ws)
-    e2e_ms = max_over_ranks(ws, a.elapsed_time(b)) / args.e2e_steps
-    e2e_val = whole_job_gbs(ws, cbytes + dbytes, e2e_ms)
+    def e2e_compress(i):
+        kc, vc = caches[i % 2]
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dsl.copy_(hslots, non_blocking=True)
+        tq.tq_compress(ctx, dk, dv, dsl, kc, vc, stream=stream)
+
+    def e2e_time(fn, n):
+        fn(0)
+        torch.cuda.synchronize()
+        barrier(ws)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(n):
+            fn(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+        return max_over_ranks(ws, a.elapsed_time(b)) / n
+
+    e2e_dec_ms = e2e_time(e2e_decode, max(1, args.e2e_steps))
+    e2e_comp_ms = e2e_time(e2e_compress, max(1, args.e2e_steps // 4))
+    if tq.tq_get_device_error(ctx) != 0:
+        raise RuntimeError("device error word set during the end-to-end steps")
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        s, cb1, db1, n, threads = oracle_sample(w, target_s=15.0)
-        cpu = {"value": (cb1 + db1) / s / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-               "sample": "%d whole sequences of the workload (%d tokens x %d kv heads: compress K+V, then decode "
-                         "of %d query heads), %.1f s" % (n, w.T, w.Hkv, w.Hq, s)}
+        ra = oracle_sample(w, target_s=8.0)   # every core first: the single-thread run lowers OpenMP's default
+        r1 = oracle_sample(w, target_s=3.0, threads=1, max_seqs=1)
+        cpu = {"value": ra["decode_bytes"] / ra["decode_s"] / 1e9, "unit": "GB/s", "cores": ra["threads"],
+               "kind": "oracle", "cpu": cpu_model(),
+               "single_thread": {"value": r1["decode_bytes"] / r1["decode_s"] / 1e9, "unit": "GB/s", "cores": 1},
+               "compress_mtokens_per_s": ra["seqs"] * w.T / ra["compress_s"] / 1e6,
+               "sample": "%d whole sequences of the workload (%d tokens x %d kv heads) compressed, then decode of "
+                         "their %d query heads timed: %.1f s on %d threads; single thread: %d sequence, %.1f s"
+                         % (ra["seqs"], w.T, w.Hkv, w.Hq, ra["decode_s"], ra["threads"], r1["seqs"],
+                            r1["decode_s"])}
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(w),
+            "vs_baseline": None, "dtype": "f16 operands, f32 accumulate", "data": "synthetic",
+            "config": workload_config(w),
+            "decode": {"gbs": dec_gbs, "ms": dec_avg, "frac_hbm": dec_gbs / peak, "bytes": dbytes},
             "compress": {"mtokens_per_s": ws * tokens / (comp_avg * 1e-3) / 1e6, "gbs": comp_gbs,
                          "ms": comp_avg, "frac_hbm": comp_gbs / peak, "bytes": cbytes},
-            "decode": {"gbs": dec_gbs, "ms": dec_avg, "frac_hbm": dec_gbs / peak, "bytes": dbytes},
-            "roofline": roof,
+            "roofline": roofline(dominant),
+            "roofline_decode": roofline("decode"),
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms},
+            "e2e": {"value": whole_job_gbs(ws, dbytes, e2e_dec_ms), "unit": "GB/s", "h2d_bytes_per_step": h2d_dec,
+                    "d2h_bytes_per_step": d2h_dec, "ms_per_step": e2e_dec_ms,
+                    "compress": {"mtokens_per_s": ws * tokens / (e2e_comp_ms * 1e-3) / 1e6,
+                                 "h2d_bytes_per_step": h2d_comp, "ms_per_step": e2e_comp_ms}},
             "gpu_launches": int(launches),
             "clocks": clk,
         }
