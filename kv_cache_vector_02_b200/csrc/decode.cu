@@ -49,21 +49,25 @@ namespace {
 constexpr int kNW = 12;                       // warps per split CTA (one CTA per SM, three per scheduler)
 constexpr int kSplitThreads = kNW * 32;
 constexpr int kPartStride = kDim + 2;         // m, l, acc[128]
-constexpr int kStages = 3;                    // page stages per warp
+constexpr int kStages = 4;                    // page stages per warp
 constexpr uint32_t kStageBytes = 2496;        // >= key chunk + value chunk at every bit width (16-byte multiple)
 constexpr uint32_t kTabAddr = 65536;          // shared-window address of the lookup tables
 constexpr uint32_t kTabBytes = 65536;         // 256 entries x 256 bytes
+// Stages: the first kLowStages below the tables (after the fields below), the rest
+// from kRingAddr on (see stage_addr).
+constexpr int kLowStages = 8;
 constexpr uint32_t kRingAddr = kTabAddr + kTabBytes;
-constexpr uint32_t kRingBytes = kNW * kStages * kStageBytes;
-constexpr uint32_t kSplitSmem = kRingAddr + kRingBytes;  // dynamic bytes: enough for any window base >= 0
+constexpr uint32_t kSplitSmem = kRingAddr + (kNW * kStages - kLowStages) * kStageBytes;  // any window base >= 0
 // Below the tables, from the window base: barriers, per-stage valid flags, the abort
-// flag, the warps' (m, l) and the CTA merge area (one tile of 8 heads at a time).
+// flag, the warps' (m, l), the CTA merge area (4 heads at a time), the low stages.
 constexpr uint32_t kOffFull = 0;                                // [kNW][kStages] mbarrier: page landed
 constexpr uint32_t kOffValid = kOffFull + kNW * kStages * 8;    // [kNW][kStages] int: the block id was valid
 constexpr uint32_t kOffAbort = kOffValid + kNW * kStages * 4;   // int
-constexpr uint32_t kOffML = (kOffAbort + 4 + 15) & ~15u;        // [kNW][2][8] float: m, l
-constexpr uint32_t kOffMerge = kOffML + kNW * 2 * 8 * 4;        // [kNW][8][128] float
-constexpr uint32_t kLowBytes = kOffMerge + kNW * 8 * kDim * 4;
+constexpr uint32_t kOffML = (kOffAbort + 4 + 15) & ~15u;        // [kNW][2][4] float: m, l
+constexpr uint32_t kOffMerge = kOffML + kNW * 2 * 4 * 4;        // [kNW][4][128] float
+constexpr uint32_t kOffLowStages = (kOffMerge + kNW * 4 * kDim * 4 + 127) & ~127u;
+constexpr uint32_t kLowBytes = kOffLowStages + kLowStages * kStageBytes;
+static_assert(kSplitSmem <= 232448, "shared memory budget");
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 enum KMode { kKPrmt = 0, kKByte4 = 1, kKByte2 = 2, kKBit1 = 3 };
@@ -82,11 +86,11 @@ struct DecodeArgs {
     float* partial;    // [slots][G][130]: m, l, acc (rotated domain)
     int* prefix;       // [B + 1] pages of the sequences before b (prep writes it)
     int split_grid;    // CTAs of the split kernel
-    int merge_sg;      // merge: groups of 128 threads per item, each on every merge_sg-th slot
-    const float* RT;       // row-major R^T (fp32)
     const uint16_t* RTh;   // fp16 R^T hi / lo, S (row-major)
     const uint16_t* RTl;
     const uint16_t* Sh;
+    const uint16_t* Rh;    // fp16 R hi / lo (row-major)
+    const uint16_t* Rl;
     float qscale, sscale;  // scale*log2(e)/sqrt(d), scale*log2(e)*sqrt(pi/2)/d
     float kscale;          // 1-bit keys: the level c[1] (key term = c1 <q', 2b - 1>)
     float kalpha, kbeta;   // 2-bit keys: c[code] = alpha (2 b1 - 1) + beta (2 b0 - 1)
@@ -171,6 +175,14 @@ __device__ __forceinline__ uint32_t taddr(uint32_t p, uint32_t L) {
     return __byte_perm(p, L, 0x7600u | (K << 4) | (4 + X));
 }
 
+// 2^x by the hardware approximation (flushes denormal results to 0; relative error
+// about 2^-22), for the softmax weights.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Lazy softmax rescaling: the running maximum only moves when a page exceeds it by
 // more than 2^kSlack (log2 units), so exponentials stay <= 2^kSlack in fp32 / fp16.
 constexpr float kSlack = 8.f;
@@ -185,10 +197,26 @@ __host__ __device__ constexpr int row_token(int r) { return r ^ ((r >> 1) & 1); 
 // also writes the page prefix sums of the sequences.
 constexpr int kPrepThreads = 256;
 __global__ void __launch_bounds__(kPrepThreads) decode_prep_kernel(DecodeArgs a) {
-    griddep_wait();  // q and seq_lens may come from the kernel before
     const int NQ = a.B * a.Hq;
     const int h0 = blockIdx.x * 16;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+    // B fragments of R^T (hi, lo) or S: parameters, loaded before waiting for the kernel before
+    const int nt = blockIdx.y * 8 + warp;  // 0..15 -> q', 16..31 -> s
+    const bool isq = nt < 16;
+    const int n = (nt & 15) * 8 + g;
+    uint32_t bh[8][2], bl[8][2];
+    {
+        const uint32_t* ph = reinterpret_cast<const uint32_t*>((isq ? a.RTh : a.Sh) + (size_t)n * kDim);
+        const uint32_t* pl = reinterpret_cast<const uint32_t*>(a.RTl + (size_t)n * kDim);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            bh[ks][0] = ph[8 * ks + c];
+            bh[ks][1] = ph[8 * ks + c + 4];
+            bl[ks][0] = isq ? pl[8 * ks + c] : 0u;
+            bl[ks][1] = isq ? pl[8 * ks + c + 4] : 0u;
+        }
+    }
+    griddep_wait();  // q and seq_lens may come from the kernel before
     const bool r0 = h0 + g < NQ, r1 = h0 + g + 8 < NQ;
     const uint32_t* q0 = reinterpret_cast<const uint32_t*>(a.q + (size_t)(r0 ? h0 + g : 0) * kDim);
     const uint32_t* q1 = reinterpret_cast<const uint32_t*>(a.q + (size_t)(r1 ? h0 + g + 8 : 0) * kDim);
@@ -228,16 +256,11 @@ __global__ void __launch_bounds__(kPrepThreads) decode_prep_kernel(DecodeArgs a)
         A[ks][2] = r0 ? q0[8 * ks + c + 4] : 0u;
         A[ks][3] = r1 ? q1[8 * ks + c + 4] : 0u;
     }
-    const int nt = blockIdx.y * 8 + warp;  // 0..15 -> q', 16..31 -> s
-    const bool isq = nt < 16;
-    const int n = (nt & 15) * 8 + g;
-    const uint32_t* bh = reinterpret_cast<const uint32_t*>((isq ? a.RTh : a.Sh) + (size_t)n * kDim);
-    const uint32_t* bl = reinterpret_cast<const uint32_t*>(a.RTl + (size_t)n * kDim);
     float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-        if (isq) mma16816(d, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bl[8 * ks + c], bl[8 * ks + c + 4]);
-        mma16816(d, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bh[8 * ks + c], bh[8 * ks + c + 4]);
+        if (isq) mma16816(d, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bl[ks][0], bl[ks][1]);
+        mma16816(d, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bh[ks][0], bh[ks][1]);
     }
     const int col = (nt & 15) * 8 + 2 * c, which = isq ? 0 : 1;
     if (r0) *reinterpret_cast<float2*>(a.qf + ((size_t)(h0 + g) * 2 + which) * kDim + col) = make_float2(d[0], d[1]);
@@ -381,37 +404,69 @@ struct PageRegs {
     float vn[2];         // value norm / sqrt(d) of rows g, g+8
 };
 
-// Fragment bytes of one page from its stage (key chunk at kst, value chunk at vst);
-// krow[i], vrow[i]: byte offsets of this thread's rows' tokens (see row_token).
+// Byte geometry of a page's key and value chunks (the same as the library's chunk
+// layouts, fixed by the code widths; checked against the context at launch).
 template <int KM, int VM, bool PROD>
-__device__ __forceinline__ void load_page(PageRegs<KM, VM, PROD>& r, const uint8_t* kst, const uint8_t* vst,
-                                          const DecodeArgs& a, const int (&tk)[2], const int (&tv)[4], int g,
-                                          int c) {
-    constexpr int kBytes = KM == kKBit1 ? 4 : (KM == kKByte2 ? 8 : 16);  // per key row per thread
+struct PageGeom {
+    static constexpr int kRow = KM == kKBit1 ? 16 : (KM == kKByte2 ? 32 : 64);  // key code bytes per token
+    static constexpr int kSigns = 16 * kRow;
+    static constexpr int kNorm = PROD ? kSigns + 16 * 16 : 16 * kRow;
+    static constexpr int kGamma = kNorm + 64;
+    static constexpr int kBytes = PROD ? kGamma + 64 : kNorm + 64;               // key chunk
+    static constexpr int vRow = VM == kVByte4 ? 64 : 32;
+    static constexpr int vNorm = 16 * vRow;
+    static constexpr int vBytes = vNorm + 64;                                   // value chunk
+    static constexpr int kPer = KM == kKBit1 ? 4 : (KM == kKByte2 ? 8 : 16);    // key bytes per thread per row
+    static constexpr int vPer = VM == kVByte4 ? 8 : 4;                          // value bytes per thread per token
+};
+
+// Per-thread byte offsets inside a stage (key chunk at 0, value chunk at kBytes):
+// rows g, g+8 of the scores are tokens tk0, tk0 + 8; the value rows are tokens tv0,
+// tv1 and tv0 + 8, tv1 + 8 (see row_token).
+struct PageOffs {
+    uint32_t key, sign, norm, val0, val1;
+};
+template <int KM, int VM, bool PROD>
+__device__ __forceinline__ PageOffs page_offsets(int tk0, int tv0, int tv1, int g, int c) {
+    using P = PageGeom<KM, VM, PROD>;
+    PageOffs o;
+    o.key = tk0 * P::kRow + P::kPer * c;
+    o.sign = P::kSigns + tk0 * 16 + 4 * c;
+    o.norm = 4 * tk0;
+    o.val0 = P::kBytes + tv0 * P::vRow + P::vPer * g;
+    o.val1 = P::kBytes + tv1 * P::vRow + P::vPer * g;
+    return o;
+}
+
+// Fragment bytes of one page from its stage st (a generic pointer to shared memory).
+template <int KM, int VM, bool PROD>
+__device__ __forceinline__ void load_page(PageRegs<KM, VM, PROD>& r, const uint8_t* st, const PageOffs& o,
+                                          float qscale, float sscale) {
+    using P = PageGeom<KM, VM, PROD>;
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-        const uint8_t* row = kst + tk[i] * a.lk.code_row + kBytes * c;
-        if (kBytes == 16) {
+        const uint8_t* row = st + o.key + i * 8 * P::kRow;
+        if (P::kPer == 16) {
             const uint4 w = *reinterpret_cast<const uint4*>(row);
             r.k[i][0] = w.x, r.k[i][1] = w.y, r.k[i][2] = w.z, r.k[i][3] = w.w;
-        } else if (kBytes == 8) {
+        } else if (P::kPer == 8) {
             const uint2 w = *reinterpret_cast<const uint2*>(row);
             r.k[i][0] = w.x, r.k[i][1] = w.y;
         } else {
             r.k[i][0] = *reinterpret_cast<const uint32_t*>(row);
         }
+        const uint8_t* nb = st + o.norm + i * 32;
         if (PROD) {
-            r.s[i] = reinterpret_cast<const uint32_t*>(kst + a.lk.signs_off + tk[i] * 16)[c];
-            r.kg[i] = reinterpret_cast<const float*>(kst + a.lk.gamma_off)[tk[i]] * a.sscale;
+            r.s[i] = *reinterpret_cast<const uint32_t*>(st + o.sign + i * 128);
+            r.kg[i] = *reinterpret_cast<const float*>(nb + P::kGamma) * sscale;
         }
-        r.kn[i] = reinterpret_cast<const float*>(kst + a.lk.norm_off)[tk[i]] * a.qscale;
-        r.vn[i] = reinterpret_cast<const float*>(vst + a.lv.norm_off)[tk[i]] * 0.08838834764831845f;
+        r.kn[i] = *reinterpret_cast<const float*>(nb + P::kNorm) * qscale;
+        r.vn[i] = *reinterpret_cast<const float*>(nb + P::kBytes + P::vNorm) * 0.08838834764831845f;
     }
-    constexpr int vBytes = VM == kVByte4 ? 8 : 4;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint8_t* row = vst + tv[i] * a.lv.code_row + vBytes * g;
-        if (vBytes == 8) {
+        const uint8_t* row = st + ((i & 1) ? o.val1 : o.val0) + (i >> 1) * 8 * P::vRow;
+        if (P::vPer == 8) {
             const uint2 w = *reinterpret_cast<const uint2*>(row);
             r.v[i][0] = w.x, r.v[i][1] = w.y;
         } else {
@@ -547,7 +602,7 @@ __device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, 
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
                 const float mnew = mx > m[nt][e] + kSlack ? mx : m[nt][e];
-                const float corr = exp2f(m[nt][e] - mnew);  // 1 when unchanged, 0 from -inf
+                const float corr = ex2(m[nt][e] - mnew);  // 1 when unchanged, 0 from -inf
                 l[nt][e] *= corr;
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
@@ -560,7 +615,7 @@ __device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, 
         float pw[2][2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            const float p0v = exp2f(sc[0][e] - m[nt][e]), p1v = exp2f(sc[1][e] - m[nt][e]);
+            const float p0v = ex2(sc[0][e] - m[nt][e]), p1v = ex2(sc[1][e] - m[nt][e]);
             l[nt][e] += p0v + p1v;
             pw[0][e] = p0v * cur.vn[0];
             pw[1][e] = p1v * cur.vn[1];
@@ -641,6 +696,11 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeAr
         return;
     }
     const uint32_t full_bar = base + kOffFull;
+    // shared-window address of stage st
+    auto stage_addr = [&](uint32_t st) -> uint32_t {
+        return st < (uint32_t)kLowStages ? base + kOffLowStages + st * kStageBytes
+                                         : kRingAddr + (st - kLowStages) * kStageBytes;
+    };
     int* valid = reinterpret_cast<int*>(smem + kOffValid);
     volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffAbort);
     if (tid < 256) build_tables<KM, VM, PROD>(a, tid);
@@ -655,13 +715,16 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeAr
     const long total = (long)a.Hkv * a.prefix[a.B];
     const long pos0 = total * (long)blockIdx.x / gridDim.x;
     const long end = total * (long)(blockIdx.x + 1) / gridDim.x;
-    const uint32_t kb = (uint32_t)a.lk.bytes, vb = (uint32_t)a.lv.bytes;
+    constexpr uint32_t kb = PageGeom<KM, VM, PROD>::kBytes, vb = PageGeom<KM, VM, PROD>::vBytes;
+    const size_t kstride = (size_t)a.Hkv * kb, vstride = (size_t)a.Hkv * vb;  // bytes per physical block
 
     // ---- this warp's page stream: issue cursor (runs kStages pages ahead) and the
     // copies of page number `k` of the warp into stage k % kStages
     PageCursor icur;
     icur.init(a, pos0, end, warp, lane);
     uint32_t issued = 0, landed = 0;  // pages issued; pages whose copies were started (for the drain)
+    // A page is two bulk copies (key chunk, value chunk) into the stage, completing on
+    // its barrier.  (Per-lane 16-byte cp.async copies measured slower.)
     auto issue_next = [&]() {
         if (!icur.live) return;
         const int blk = icur.block();
@@ -672,11 +735,10 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeAr
             if (a.stall) {
                 // test hook: nothing arrives on the stage
             } else if (v) {
-                const size_t chunk = (size_t)blk * a.Hkv + icur.hk;
-                const uint32_t dst = kRingAddr + st * kStageBytes;
+                const uint32_t dst = stage_addr(st);
                 sm100::mbar_arrive_expect_tx(full_bar + 8 * st, kb + vb);
-                sm100::bulk_g2s(dst, a.kc + chunk * kb, kb, full_bar + 8 * st);
-                sm100::bulk_g2s(dst + kb, a.vc + chunk * vb, vb, full_bar + 8 * st);
+                sm100::bulk_g2s(dst, a.kc + (size_t)blk * kstride + icur.hk * kb, kb, full_bar + 8 * st);
+                sm100::bulk_g2s(dst + kb, a.vc + (size_t)blk * vstride + icur.hk * vb, vb, full_bar + 8 * st);
             } else {
                 atomicOr(a.err, TQ_DEVERR_BLOCK);
                 sm100::mbar_arrive(full_bar + 8 * st);  // nothing to copy: the stage completes at once
@@ -692,7 +754,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeAr
     const int g = lane >> 2, c = lane & 3;
     // rows of this thread in the page: score rows g, g+8; value rows 2c, 2c+1, 2c+8, 2c+9
     const int tk[2] = {row_token(g), row_token(g + 8)};
-    const int tv[4] = {row_token(2 * c), row_token(2 * c + 1), row_token(2 * c + 8), row_token(2 * c + 9)};
+    const PageOffs po = page_offsets<KM, VM, PROD>(row_token(g), row_token(2 * c), row_token(2 * c + 1), g, c);
     // lane offsets inside a table entry: LA = {lane*4 (A), 128 + lane*4 (B)}, LB = {128 +
     // (lane%8)*16 (B, 16-byte entries), (lane%16)*8 (A, 8-byte entries)}; bytes 2, 3 = 0x01, 0x00
     const uint32_t LA = (uint32_t)(lane * 4) | ((uint32_t)(128 + lane * 4) << 8) | 0x10000u;
@@ -712,8 +774,8 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeAr
             }
         }
     }
-    float* wml = reinterpret_cast<float*>(smem + kOffML);      // [warp][2][8]: m then l
-    float* wacc = reinterpret_cast<float*>(smem + kOffMerge);  // [warp][8 heads][128]
+    float* wml = reinterpret_cast<float*>(smem + kOffML);      // [warp][2][4]: m then l
+    float* wacc = reinterpret_cast<float*>(smem + kOffMerge);  // [warp][4 heads][128]
     uint32_t cnt = 0;   // pages this warp has consumed (all pieces)
     bool dead = false;  // a page never arrived: this warp stops working
     Pieces it;
@@ -789,17 +851,18 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeAr
             }
             if (dead) continue;  // this warp stops: no more pages are consumed or issued
             const int page = p0 + warp + j * kNW;
-            if (valid[st]) {
-                const uint8_t* sp = smem + (kRingAddr - base) + st * kStageBytes;
-                PageRegs<KM, VM, PROD> r;
-                load_page<KM, VM, PROD>(r, sp, sp + kb, a, tk, tv, g, c);
-                process_page<KM, VM, PROD, NT>(r, min(kPage, Ls - page * kPage), tk, klo0, klo1, khi0, khi1, LA, LB,
-                                               bq, bs, m, l, acc);
-            }
+            // the page's bytes into registers, then the stage goes back to the stream
+            // before the page is worked, so every stage is in flight meanwhile
+            const bool vp = valid[st] != 0;
+            PageRegs<KM, VM, PROD> r;
+            if (vp) load_page<KM, VM, PROD>(r, smem + (stage_addr(st) - base), po, a.qscale, a.sscale);
             sm100::fence_proxy_async_shared();  // this lane's reads before the refill's bulk copy
             __syncwarp();                       // every lane is done with the stage before it is refilled
             ++cnt;
             issue_next();
+            if (vp)
+                process_page<KM, VM, PROD, NT>(r, min(kPage, Ls - page * kPage), tk, klo0, klo1, khi0, khi1, LA, LB,
+                                               bq, bs, m, l, acc);
         }
 
         // ---- merge the CTA's warps (one tile of 8 heads at a time; coordinates back in order)
@@ -812,48 +875,53 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeAr
                 l[nt][e] += __shfl_xor_sync(0xffffffffu, l[nt][e], 16);
             }
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            __syncthreads();  // the previous merge is done with the area
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int hh = 2 * c + e;
-                if (g == 0) {
-                    wml[(warp * 2 + 0) * 8 + hh] = m[nt][e];
-                    wml[(warp * 2 + 1) * 8 + hh] = l[nt][e];
+            for (int qq = 0; qq < 2; ++qq) {  // heads nt*8 + 4 qq + (0..3)
+                if (nt * 8 + 4 * qq >= a.G) break;
+                __syncthreads();  // the previous merge is done with the area
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int hh = 2 * c + e;
+                    if ((hh >> 2) != qq) continue;
+                    const int hl = hh & 3;
+                    if (g == 0) {
+                        wml[(warp * 2 + 0) * 4 + hl] = m[nt][e];
+                        wml[(warp * 2 + 1) * 4 + hl] = l[nt][e];
+                    }
+#pragma unroll
+                    for (int mt = 0; mt < 8; ++mt) {
+                        const int c0 = 16 * g + coord_of<VM>(mt);
+                        wacc[(warp * 4 + hl) * kDim + c0] = acc[nt][mt][e];
+                        wacc[(warp * 4 + hl) * kDim + c0 + 1] = acc[nt][mt][2 + e];
+                    }
                 }
+                __syncthreads();
+                // thread = (head hl = warp, coordinates 4 lane .. 4 lane + 3) for the first 4 warps
+                const int hl = warp, h = nt * 8 + 4 * qq + hl;
+                if (hl < 4 && h < a.G) {
+                    float M = -INFINITY;
 #pragma unroll
-                for (int mt = 0; mt < 8; ++mt) {
-                    const int c0 = 16 * g + coord_of<VM>(mt);
-                    wacc[(warp * 8 + hh) * kDim + c0] = acc[nt][mt][e];
-                    wacc[(warp * 8 + hh) * kDim + c0 + 1] = acc[nt][mt][2 + e];
+                    for (int w = 0; w < kNW; ++w) M = fmaxf(M, wml[(w * 2) * 4 + hl]);
+                    float Lsum = 0.f;
+                    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int w = 0; w < kNW; ++w) {
+                        const float mw = wml[(w * 2) * 4 + hl];
+                        const float wt = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+                        Lsum = fmaf(wt, wml[(w * 2 + 1) * 4 + hl], Lsum);
+                        const float4 v = reinterpret_cast<const float4*>(wacc + (w * 4 + hl) * kDim)[lane];
+                        A.x = fmaf(wt, v.x, A.x);
+                        A.y = fmaf(wt, v.y, A.y);
+                        A.z = fmaf(wt, v.z, A.z);
+                        A.w = fmaf(wt, v.w, A.w);
+                    }
+                    float* part = a.partial + (((size_t)unit + blockIdx.x) * a.G + h) * kPartStride;
+                    if (lane == 0) *reinterpret_cast<float2*>(part) = make_float2(M, Lsum);
+                    reinterpret_cast<float2*>(part + 2)[2 * lane] = make_float2(A.x, A.y);
+                    reinterpret_cast<float2*>(part + 2)[2 * lane + 1] = make_float2(A.z, A.w);
                 }
             }
-            __syncthreads();
-            // thread = (head hh = warp, coordinates 4 lane .. 4 lane + 3) for the first 8 warps
-            const int hh = warp, h = nt * 8 + hh;
-            if (hh < 8 && h < a.G) {
-                float M = -INFINITY;
-#pragma unroll
-                for (int w = 0; w < kNW; ++w) M = fmaxf(M, wml[(w * 2) * 8 + hh]);
-                float Lsum = 0.f;
-                float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int w = 0; w < kNW; ++w) {
-                    const float mw = wml[(w * 2) * 8 + hh];
-                    const float wt = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-                    Lsum = fmaf(wt, wml[(w * 2 + 1) * 8 + hh], Lsum);
-                    const float4 v = reinterpret_cast<const float4*>(wacc + (w * 8 + hh) * kDim)[lane];
-                    A.x = fmaf(wt, v.x, A.x);
-                    A.y = fmaf(wt, v.y, A.y);
-                    A.z = fmaf(wt, v.z, A.z);
-                    A.w = fmaf(wt, v.w, A.w);
-                }
-                float* part = a.partial + (((size_t)unit + blockIdx.x) * a.G + h) * kPartStride;
-                if (lane == 0) *reinterpret_cast<float2*>(part) = make_float2(M, Lsum);
-                reinterpret_cast<float2*>(part + 2)[2 * lane] = make_float2(A.x, A.y);
-                reinterpret_cast<float2*>(part + 2)[2 * lane + 1] = make_float2(A.z, A.w);
-            }
-        }
     }
     if (dead && landed > cnt) {  // the copies this warp started land before the CTA exits
         const volatile int never = 0;
@@ -863,248 +931,222 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeAr
 }
 
 // ------------------------------------------------------------------ merge
-// Persistent: with n items per CTA (chosen at launch so that the CTAs cover the
-// SMs), CTA i takes the (unit, group of kMergeHeads heads) items i n .. i n + n - 1,
-// then + grid n, ...; thread = coordinate, computing all the group's heads so that
-// each element of R is read once per item.  An item has sg groups of 128 threads
-// (sg > 1 when a unit spans many split CTAs, as in one long sequence): group g
-// folds every sg-th slot from the g-th, and the first group combines the sg
-// partial states and un-rotates.  R^T is staged once per CTA (while the split
-// kernel runs).  Unit u's pieces sit in slots u + c for the split CTAs c whose
-// page range meets it: c(p) = ((p + 1) grid - 1) / total is the CTA of page p.
-// With a residual window, the first group of an item also attends to the window's
-// fp16 tokens (scores with a thread per token, values with a thread per coordinate)
-// and combines that partial state with the compressed one in the original domain.
-constexpr int kMergeHeads = 4;
-constexpr int kMergeItems = 4;  // most items per CTA
-constexpr int kMergeGroups = 8; // most slot groups per item
-constexpr int kMergeThreads = 1024;
-constexpr int kTailMax = 256;   // most window tokens per sequence
-constexpr size_t kTailFloats = kMergeHeads * kDim + kTailMax * kMergeHeads + 2 * 4 * kMergeHeads;  // per item
-size_t merge_smem(int ipc, int sg, bool tail) {
-    return sizeof(float) * (kDim * kDim + (size_t)ipc * kDim * kMergeHeads +
-                            (sg > 1 ? (size_t)ipc * sg * (kDim * kMergeHeads + 2 * kMergeHeads) : 0) +
-                            (tail ? (size_t)ipc * kTailFloats : 0));
-}
+// One CTA of 8 warps per (unit, group of up to 8 query heads).  Unit u's pieces sit
+// in slots u + c for the split CTAs c whose page range meets it: c(p) = ((p + 1)
+// grid - 1) / total is the CTA of page p.
+//   1. log-sum-exp over the slots, thread = (head = warp, coordinates 4 lane ..
+//      4 lane + 3), into a = acc / l (rotated domain) in shared memory;
+//   2. with a residual window, the window's (m, l, acc) in the original domain:
+//      scores with a thread per token, values with the (head, 4 coordinates) layout;
+//   3. o = R a on mma.sync: A = a as fp16 hi + lo (heads on M), B = R as fp16 hi +
+//      lo (outputs on N; warp w takes the 8-output tiles w and w + 8), three passes
+//      (hi hi, hi lo, lo hi) into fp32; R's fragments are loaded before waiting for
+//      the page kernel (R is a parameter, not its output);
+//   4. o = (w_c R a + w_t acc_t) / (w_c + w_t l_t) with the two parts' log-sum-exp
+//      weights, stored fp16 or fp32.
+constexpr int kMergeWarps = 8;
+constexpr int kMergeThreads = kMergeWarps * 32;
+constexpr int kTailMax = 256;  // most window tokens per sequence
+struct MergeSmem {
+    float a[8][kDim];          // combined a = acc / l of each head (rotated), then o = R a
+    float ml[8][2];            // M, L of the compressed part per head
+    float q[8][kDim];          // window: q of the heads
+    float ts[kTailMax][8];     // window: scores, then probabilities
+    float red[2][kMergeWarps][8];
+};
 __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs a) {
-    // RT [128*128] | orot [items][128][kMergeHeads] | group states A [items][sg][128][kMergeHeads],
-    // (M, L) [items][sg][kMergeHeads][2]
-    extern __shared__ __align__(16) float sm[];
-    const int sg = a.merge_sg;
-    const int ipc = (int)blockDim.x / (kDim * sg);
-    const int i = threadIdx.x % kDim, gi = (threadIdx.x / kDim) % sg, il = threadIdx.x / (kDim * sg);
-    float* rts = sm;
-    float4* orot = reinterpret_cast<float4*>(sm + kDim * kDim) + il * kDim;  // this item's [j] of 4 heads
-    float4* gA = reinterpret_cast<float4*>(sm + kDim * kDim + ipc * kDim * kMergeHeads) + (il * sg) * kDim;
-    float* gML = sm + kDim * kDim + ipc * kDim * kMergeHeads + ipc * sg * kDim * kMergeHeads +
-                 (il * sg) * 2 * kMergeHeads;
-    // window: q of the item's heads [4][128], scores / probabilities [kTailMax][4], warp maxima
-    // and sums [2][4 warps][4]
-    float* tq_s = sm + kDim * kDim + ipc * kDim * kMergeHeads +
-                  (sg > 1 ? ipc * sg * (kDim * kMergeHeads + 2 * kMergeHeads) : 0) + il * kTailFloats;
-    float* ts_s = tq_s + kMergeHeads * kDim;
-    float* red_s = ts_s + kTailMax * kMergeHeads;
-    {
-        const float4* src = reinterpret_cast<const float4*>(a.RT);
-        float4* dst = reinterpret_cast<float4*>(rts);
-        for (int k = threadIdx.x; k < kDim * kDim / 4; k += blockDim.x) dst[k] = src[k];
+    __shared__ MergeSmem sm;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+    const int groups = (a.G + 7) / 8;
+    const int unit = blockIdx.x / groups, h0 = (blockIdx.x - unit * groups) * 8;
+    const int nh = min(8, a.G - h0);
+    const int b = unit / a.Hkv, hk = unit - b * a.Hkv;
+    // R fragments (B operand: column n = output i, K-pair = consecutive j of row i)
+    uint32_t rb[2][8][2][2];  // [tile][k-step][b0 / b1][hi / lo]
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int i = (warp + 8 * t) * 8 + g;
+        const uint32_t* rh = reinterpret_cast<const uint32_t*>(a.Rh + (size_t)i * kDim);
+        const uint32_t* rl = reinterpret_cast<const uint32_t*>(a.Rl + (size_t)i * kDim);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            rb[t][ks][0][0] = rh[8 * ks + c];
+            rb[t][ks][1][0] = rh[8 * ks + c + 4];
+            rb[t][ks][0][1] = rl[8 * ks + c];
+            rb[t][ks][1][1] = rl[8 * ks + c + 4];
+        }
     }
-    // The items' units and slot ranges depend on the page prefix sums only, which the
-    // prep kernel wrote before the split kernel could start (and so before this
-    // kernel was launched): they are read before waiting for the split partials.
+    griddep_wait();  // the split partials
+    // ---- 1. log-sum-exp over the unit's slots: head hh = warp, coordinates 4 lane ..
     const long total = (long)a.Hkv * a.prefix[a.B];
     const long grid = a.split_grid;
-    const int groups = (a.G + kMergeHeads - 1) / kMergeHeads;
-    const int items = a.B * a.Hkv * groups;
-    auto item_info = [&](int item, int& unit, int& h0, int& c_lo, int& c_hi) {
-        unit = 0, h0 = 0, c_lo = 0, c_hi = -1;
-        if (item >= items) return;
-        unit = item / groups;
-        h0 = (item - unit * groups) * kMergeHeads;
-        const int b = unit / a.Hkv, hk = unit - b * a.Hkv;
-        const int np = a.prefix[b + 1] - a.prefix[b];
-        if (np > 0) {
-            const long first = (long)a.Hkv * a.prefix[b] + (long)hk * np, last = first + np - 1;
-            c_lo = (int)(((first + 1) * grid - 1) / total);
-            c_hi = (int)(((last + 1) * grid - 1) / total);
-        }
-    };
-    int n_unit, n_h0, n_clo, n_chi;  // the first item's
-    item_info(blockIdx.x * ipc + il, n_unit, n_h0, n_clo, n_chi);
-    griddep_wait();  // the split partials
-    for (int base = blockIdx.x * ipc; base < items; base += gridDim.x * ipc) {
-        const int item = base + il;
-        const bool live = item < items;
-        int unit = n_unit, h0 = n_h0, c_lo = n_clo, c_hi = n_chi;
-        if (base + gridDim.x * ipc < items) item_info(item + gridDim.x * ipc, n_unit, n_h0, n_clo, n_chi);
-        // online log-sum-exp over the slots, all heads at once: the loads of several
-        // slots are in flight together
-        float M[kMergeHeads], Lsum[kMergeHeads], A[kMergeHeads];
-#pragma unroll
-        for (int e = 0; e < kMergeHeads; ++e) M[e] = -INFINITY, Lsum[e] = 0.f, A[e] = 0.f;
-        const int nh = a.G - h0 < kMergeHeads ? a.G - h0 : kMergeHeads;
+    const int np = a.prefix[b + 1] - a.prefix[b];
+    int c_lo = 0, c_hi = -1;
+    if (np > 0) {
+        const long first = (long)a.Hkv * a.prefix[b] + (long)hk * np, last = first + np - 1;
+        c_lo = (int)(((first + 1) * grid - 1) / total);
+        c_hi = (int)(((last + 1) * grid - 1) / total);
+    }
+    const int hh = warp;
+    float M = -INFINITY, L = 0.f;
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (hh < nh) {
 #pragma unroll 4
-        for (int c = c_lo + gi; c <= c_hi; c += sg) {
-            const float* pp = a.partial + (((size_t)unit + c) * a.G + h0) * kPartStride;
-            float ms[kMergeHeads], ls[kMergeHeads], as[kMergeHeads];
-#pragma unroll
-            for (int e = 0; e < kMergeHeads; ++e) {
-                const bool on = e < nh;
-                ms[e] = on ? pp[e * kPartStride] : -INFINITY;
-                ls[e] = on ? pp[e * kPartStride + 1] : 0.f;
-                as[e] = on ? pp[e * kPartStride + 2 + i] : 0.f;
-            }
-#pragma unroll
-            for (int e = 0; e < kMergeHeads; ++e) {
-                const float mn = fmaxf(M[e], ms[e]);
-                const float sa = (M[e] == -INFINITY) ? 0.f : exp2f(M[e] - mn);
-                const float sb = (ms[e] == -INFINITY) ? 0.f : exp2f(ms[e] - mn);
-                Lsum[e] = fmaf(Lsum[e], sa, ls[e] * sb);
-                A[e] = fmaf(A[e], sa, as[e] * sb);
-                M[e] = mn;
-            }
+        for (int cc = c_lo; cc <= c_hi; ++cc) {
+            const float* pp = a.partial + (((size_t)unit + cc) * a.G + h0 + hh) * kPartStride;
+            const float2 ml = *reinterpret_cast<const float2*>(pp);
+            const float2 x = reinterpret_cast<const float2*>(pp + 2)[2 * lane];
+            const float2 y = reinterpret_cast<const float2*>(pp + 2)[2 * lane + 1];
+            const float mn = fmaxf(M, ml.x);
+            const float sa = (M == -INFINITY) ? 0.f : exp2f(M - mn);
+            const float sb = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - mn);
+            L = fmaf(L, sa, ml.y * sb);
+            A.x = fmaf(A.x, sa, x.x * sb);
+            A.y = fmaf(A.y, sa, x.y * sb);
+            A.z = fmaf(A.z, sa, y.x * sb);
+            A.w = fmaf(A.w, sa, y.y * sb);
+            M = mn;
         }
-        __syncthreads();  // the previous items' un-rotation is done with orot and the group states
-        if (sg > 1) {  // the first group combines the groups' states
-            if (i == 0)
-#pragma unroll
-                for (int e = 0; e < kMergeHeads; ++e) gML[gi * 2 * kMergeHeads + 2 * e] = M[e], gML[gi * 2 * kMergeHeads + 2 * e + 1] = Lsum[e];
-            gA[gi * kDim + i] = make_float4(A[0], A[1], A[2], A[3]);
-            __syncthreads();
-            if (gi == 0) {
-#pragma unroll
-                for (int e = 0; e < kMergeHeads; ++e) {
-                    float Mx = -INFINITY;
-                    for (int g = 0; g < sg; ++g) Mx = fmaxf(Mx, gML[g * 2 * kMergeHeads + 2 * e]);
-                    float L2 = 0.f, A2 = 0.f;
-                    for (int g = 0; g < sg; ++g) {
-                        const float mg = gML[g * 2 * kMergeHeads + 2 * e];
-                        if (mg == -INFINITY) continue;
-                        const float w = exp2f(mg - Mx);
-                        const float4 ag = gA[g * kDim + i];
-                        L2 = fmaf(gML[g * 2 * kMergeHeads + 2 * e + 1], w, L2);
-                        A2 = fmaf(e == 0 ? ag.x : e == 1 ? ag.y : e == 2 ? ag.z : ag.w, w, A2);
-                    }
-                    M[e] = Mx, Lsum[e] = L2, A[e] = A2;
-                }
-            }
+    }
+    {
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        reinterpret_cast<float4*>(sm.a[hh])[lane] = make_float4(A.x * inv, A.y * inv, A.z * inv, A.w * inv);
+        if (lane == 0) sm.ml[hh][0] = M, sm.ml[hh][1] = L;
+    }
+    // ---- 2. the residual window of the unit's sequence (base 2, original domain)
+    float tM = -INFINITY, tL = 0.f;
+    float4 tA = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (a.tail_k) {
+        int tl = a.tail_lens[b];
+        if (tl < 0 || tl > a.tail_cap) {
+            if (threadIdx.x == 0 && h0 == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
+            tl = 0;
         }
-        float o[kMergeHeads];
-#pragma unroll
-        for (int e = 0; e < kMergeHeads; ++e) o[e] = (live && Lsum[e] > 0.f) ? A[e] / Lsum[e] : 0.f;
-        if (gi == 0) orot[i] = make_float4(o[0], o[1], o[2], o[3]);
-        // residual window of the item's sequence: (tM, tL, tA) of its fp16 tokens, base 2
-        float tM[kMergeHeads], tL[kMergeHeads], tA[kMergeHeads];
-#pragma unroll
-        for (int e = 0; e < kMergeHeads; ++e) tM[e] = -INFINITY, tL[e] = 0.f, tA[e] = 0.f;
-        if (a.tail_k) {
-            const int b = unit / a.Hkv, hk = unit - b * a.Hkv;
-            int tl = 0;
-            if (live && gi == 0) {
-                tl = a.tail_lens[b];
-                if (tl < 0 || tl > a.tail_cap) {
-                    if (i == 0 && h0 == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
-                    tl = 0;
-                }
-#pragma unroll
-                for (int e = 0; e < kMergeHeads; ++e)
-                    tq_s[e * kDim + i] = h0 + e < a.G ? __half2float(__ushort_as_half(
-                                                            a.q[((size_t)b * a.Hq + hk * a.G + h0 + e) * kDim + i]))
-                                                      : 0.f;
-            }
-            __syncthreads();
-            const int wi = i >> 5, ln = i & 31;  // warp of the item's first group, lane
-            float mx[kMergeHeads] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            for (int u = i; u < tl; u += kDim) {  // scores: a thread per token
-                const uint4* kr = reinterpret_cast<const uint4*>(
-                    a.tail_k + (((size_t)b * a.tail_cap + u) * a.Hkv + hk) * kDim);
-                float sc[kMergeHeads] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-                for (int c8 = 0; c8 < kDim / 8; ++c8) {
-                    const uint4 w = kr[c8];
-                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const float2 kk = __half22float2(*reinterpret_cast<const __half2*>(&ww[jj]));
-#pragma unroll
-                        for (int e = 0; e < kMergeHeads; ++e) {
-                            sc[e] = fmaf(tq_s[e * kDim + 8 * c8 + 2 * jj], kk.x, sc[e]);
-                            sc[e] = fmaf(tq_s[e * kDim + 8 * c8 + 2 * jj + 1], kk.y, sc[e]);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int e = 0; e < kMergeHeads; ++e) {
-                    sc[e] *= a.scale_log2;
-                    ts_s[u * kMergeHeads + e] = sc[e];
-                    mx[e] = fmaxf(mx[e], sc[e]);
-                }
-            }
-#pragma unroll
-            for (int e = 0; e < kMergeHeads; ++e) {
-                for (int off = 16; off > 0; off >>= 1) mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], off));
-                if (gi == 0 && ln == 0) red_s[wi * kMergeHeads + e] = mx[e];
-            }
-            __syncthreads();
-            float sm4[kMergeHeads] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int e = 0; e < kMergeHeads; ++e)
-                tM[e] = fmaxf(fmaxf(red_s[e], red_s[kMergeHeads + e]), fmaxf(red_s[2 * kMergeHeads + e], red_s[3 * kMergeHeads + e]));
-            for (int u = i; u < tl; u += kDim)
-#pragma unroll
-                for (int e = 0; e < kMergeHeads; ++e) {
-                    const float p = exp2f(ts_s[u * kMergeHeads + e] - tM[e]);
-                    ts_s[u * kMergeHeads + e] = p;
-                    sm4[e] += p;
-                }
-#pragma unroll
-            for (int e = 0; e < kMergeHeads; ++e) {
-                for (int off = 16; off > 0; off >>= 1) sm4[e] += __shfl_xor_sync(0xffffffffu, sm4[e], off);
-                if (gi == 0 && ln == 0) red_s[4 * kMergeHeads + wi * kMergeHeads + e] = sm4[e];
-            }
-            __syncthreads();
-#pragma unroll
-            for (int e = 0; e < kMergeHeads; ++e)
-                tL[e] = (red_s[4 * kMergeHeads + e] + red_s[5 * kMergeHeads + e]) +
-                        (red_s[6 * kMergeHeads + e] + red_s[7 * kMergeHeads + e]);
-            for (int u = 0; u < tl; ++u) {  // values: a thread per coordinate
-                const float v = __half2float(__ushort_as_half(a.tail_v[(((size_t)b * a.tail_cap + u) * a.Hkv + hk) * kDim + i]));
-#pragma unroll
-                for (int e = 0; e < kMergeHeads; ++e) tA[e] = fmaf(ts_s[u * kMergeHeads + e], v, tA[e]);
-            }
+        for (int k = threadIdx.x; k < 8 * kDim; k += kMergeThreads) {
+            const int e = k / kDim, i = k - e * kDim;
+            sm.q[e][i] = e < nh ? __half2float(__ushort_as_half(a.q[((size_t)b * a.Hq + hk * a.G + h0 + e) * kDim + i]))
+                                : 0.f;
         }
         __syncthreads();
-        if (!live || gi != 0) continue;
-        float y[kMergeHeads] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-        for (int j = 0; j < kDim; ++j) {  // o_i = sum_j R[i][j] orot_j, for the 4 heads at once
-            const float r = rts[j * kDim + i];
-            const float4 v = orot[j];
-            y[0] = fmaf(r, v.x, y[0]);
-            y[1] = fmaf(r, v.y, y[1]);
-            y[2] = fmaf(r, v.z, y[2]);
-            y[3] = fmaf(r, v.w, y[3]);
-        }
-        if (a.tail_k) {  // o = (Wc R acc / Lc + Wt tA / tL) with the weights of both parts
+        float mx[8];
 #pragma unroll
-            for (int e = 0; e < kMergeHeads; ++e) {
-                const float Mx = fmaxf(M[e], tM[e]);
-                const float wc = Lsum[e] > 0.f ? exp2f(M[e] - Mx) * Lsum[e] : 0.f;
-                const float et = tL[e] > 0.f ? exp2f(tM[e] - Mx) : 0.f;
-                const float den = wc + et * tL[e];
-                y[e] = den > 0.f ? (wc * y[e] + et * tA[e]) / den : 0.f;
+        for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+        for (int u = threadIdx.x; u < tl; u += kMergeThreads) {  // scores: a thread per token
+            const uint4* kr = reinterpret_cast<const uint4*>(a.tail_k + (((size_t)b * a.tail_cap + u) * a.Hkv + hk) * kDim);
+            float sc[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sc[e] = 0.f;
+#pragma unroll 2
+            for (int c8 = 0; c8 < kDim / 8; ++c8) {
+                const uint4 w = kr[c8];
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const float2 kk = __half22float2(*reinterpret_cast<const __half2*>(&ww[jj]));
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        sc[e] = fmaf(sm.q[e][8 * c8 + 2 * jj + 1], kk.y, fmaf(sm.q[e][8 * c8 + 2 * jj], kk.x, sc[e]));
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                sc[e] *= a.scale_log2;
+                sm.ts[u][e] = sc[e];
+                mx[e] = fmaxf(mx[e], sc[e]);
             }
         }
 #pragma unroll
-        for (int e = 0; e < kMergeHeads; ++e) {
-            const int h = h0 + e;
-            if (h >= a.G) break;
-            const size_t oi = ((size_t)unit * a.G + h) * kDim + i;
-            if (a.out_fp32)
-                static_cast<float*>(a.out)[oi] = y[e];
-            else
-                static_cast<__half*>(a.out)[oi] = __float2half_rn(y[e]);
+        for (int e = 0; e < 8; ++e) {
+            for (int off = 16; off > 0; off >>= 1) mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], off));
+            if (lane == 0) sm.red[0][warp][e] = mx[e];
         }
+        __syncthreads();
+        float gm[8], sm8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            gm[e] = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kMergeWarps; ++w) gm[e] = fmaxf(gm[e], sm.red[0][w][e]);
+            sm8[e] = 0.f;
+        }
+        for (int u = threadIdx.x; u < tl; u += kMergeThreads)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float p = exp2f(sm.ts[u][e] - gm[e]);
+                sm.ts[u][e] = p;
+                sm8[e] += p;
+            }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            for (int off = 16; off > 0; off >>= 1) sm8[e] += __shfl_xor_sync(0xffffffffu, sm8[e], off);
+            if (lane == 0) sm.red[1][warp][e] = sm8[e];
+        }
+        __syncthreads();
+        tM = gm[hh];
+#pragma unroll
+        for (int w = 0; w < kMergeWarps; ++w) tL += sm.red[1][w][hh];
+        for (int u = 0; u < tl; ++u) {  // values: (head hh, coordinates 4 lane ..)
+            const uint2 w = reinterpret_cast<const uint2*>(a.tail_v + (((size_t)b * a.tail_cap + u) * a.Hkv + hk) * kDim)[lane];
+            const float2 v0 = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
+            const float2 v1 = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
+            const float p = sm.ts[u][hh];
+            tA.x = fmaf(p, v0.x, tA.x);
+            tA.y = fmaf(p, v0.y, tA.y);
+            tA.z = fmaf(p, v1.x, tA.z);
+            tA.w = fmaf(p, v1.y, tA.w);
+        }
+    }
+    __syncthreads();  // a and ml complete
+    // ---- 3. o = R a for the (up to 8) heads: rows g (heads), columns = outputs
+    uint32_t ah[8][2], al[8][2];  // [k-step][k-cols 2c.. / 2c+8..] of head row g
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const float2 x = *reinterpret_cast<const float2*>(&sm.a[g][16 * ks + 8 * hf + 2 * c]);
+            const __half2 hi = __floats2half2_rn(x.x, x.y);
+            const float2 hif = __half22float2(hi);
+            const __half2 lo = __floats2half2_rn(x.x - hif.x, x.y - hif.y);
+            ah[ks][hf] = *reinterpret_cast<const uint32_t*>(&hi);
+            al[ks][hf] = *reinterpret_cast<const uint32_t*>(&lo);
+        }
+    float d[2][4];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) d[t][e] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            mma16816(d[t], al[ks][0], 0u, al[ks][1], 0u, rb[t][ks][0][0], rb[t][ks][1][0]);
+            mma16816(d[t], ah[ks][0], 0u, ah[ks][1], 0u, rb[t][ks][0][1], rb[t][ks][1][1]);
+            mma16816(d[t], ah[ks][0], 0u, ah[ks][1], 0u, rb[t][ks][0][0], rb[t][ks][1][0]);
+        }
+    }
+    __syncthreads();  // every warp has read a
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+        *reinterpret_cast<float2*>(&sm.a[g][(warp + 8 * t) * 8 + 2 * c]) = make_float2(d[t][0], d[t][1]);
+    __syncthreads();
+    // ---- 4. combine with the window and store: thread = (head hh, coordinates 4 lane ..)
+    if (hh >= nh) return;
+    float4 o = reinterpret_cast<const float4*>(sm.a[hh])[lane];
+    if (a.tail_k) {
+        const float Mc = sm.ml[hh][0], Lc = sm.ml[hh][1];
+        const float Mx = fmaxf(Mc, tM);
+        const float wc = Lc > 0.f ? exp2f(Mc - Mx) * Lc : 0.f;
+        const float et = tL > 0.f ? exp2f(tM - Mx) : 0.f;
+        const float den = wc + et * tL;
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        o = make_float4((wc * o.x + et * tA.x) * inv, (wc * o.y + et * tA.y) * inv, (wc * o.z + et * tA.z) * inv,
+                        (wc * o.w + et * tA.w) * inv);
+    }
+    const size_t oi = ((size_t)unit * a.G + h0 + hh) * kDim + 4 * lane;
+    if (a.out_fp32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(a.out) + oi) = o;
+    } else {
+        const __half2 lo = __floats2half2_rn(o.x, o.y), hi = __floats2half2_rn(o.z, o.w);
+        *reinterpret_cast<uint2*>(static_cast<__half*>(a.out) + oi) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
     }
 }
 
@@ -1133,6 +1175,11 @@ cudaError_t launch_dependent(K kernel, dim3 grid, dim3 block, size_t smem, cudaS
 
 template <int KM, int VM, bool PROD, int NT>
 cudaError_t launch_split(const DecodeArgs& a, int grid, cudaStream_t stream) {
+    using P = PageGeom<KM, VM, PROD>;
+    if (a.lk.bytes != P::kBytes || a.lv.bytes != P::vBytes || a.lk.code_row != P::kRow ||
+        a.lv.code_row != P::vRow || a.lk.norm_off != P::kNorm || a.lv.norm_off != P::vNorm ||
+        (PROD && (a.lk.signs_off != P::kSigns || a.lk.gamma_off != P::kGamma)))
+        return cudaErrorInvalidValue;  // the kernel's fixed geometry must be the context's
     auto k = decode_split_kernel<KM, VM, PROD, NT>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSplitSmem);
     if (e != cudaSuccess) return e;
@@ -1197,10 +1244,11 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
     a.partial = reinterpret_cast<float*>(ws + plan.partial_off);
     a.prefix = reinterpret_cast<int*>(ws + plan.prefix_off);
     a.split_grid = plan.grid;
-    a.RT = ctx->dev.RT;
     a.RTh = ctx->dev.RTh;
     a.RTl = ctx->dev.RTl;
     a.Sh = ctx->dev.Sh;
+    a.Rh = ctx->dev.Rh;
+    a.Rl = ctx->dev.Rl;
     a.cbk = ctx->cb_key;
     a.cbv = ctx->cb_value;
     a.lk = ctx->lay_key;
@@ -1236,28 +1284,8 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
 #undef TQ_DEC_NT
 #undef TQ_DEC_CASE
     if (e != cudaSuccess) return e;
-    const int mitems = B * Hkv * ((a.G + kMergeHeads - 1) / kMergeHeads);
-    // slot groups per item: a unit of the longest sequence meets about grid / units
-    // + 1 split CTAs when all sequences are that long; one group per 4 such slots
-    const long units = (long)B * Hkv;
-    const long est_slots = units > 0 ? (grid + units - 1) / units + 1 : 1;
-    int sg = (int)(est_slots / 4);
-    sg = sg < 1 ? 1 : (sg > kMergeGroups ? kMergeGroups : sg);
-    // items per CTA: as few as keep the CTAs within one per SM (at most kMergeItems; one
-    // when an item has several groups)
-    int ipc = 1;
-    if (sg == 1) {
-        ipc = (mitems + ctx->sm_count - 1) / ctx->sm_count;
-        ipc = ipc < 1 ? 1 : (ipc > kMergeItems ? kMergeItems : ipc);
-    }
-    a.merge_sg = sg;
-    const int mctas = (mitems + ipc - 1) / ipc;
-    const dim3 mgrid(mctas < ctx->sm_count ? mctas : ctx->sm_count);
-    const size_t msmem = merge_smem(ipc, sg, a.tail_k != nullptr);
-    e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)std::max(merge_smem(kMergeItems, 1, true), merge_smem(1, kMergeGroups, true)));
-    if (e != cudaSuccess) return e;
-    e = launch_dependent(decode_merge_kernel, mgrid, dim3(kDim * ipc * sg), msmem, stream, a);
+    const int mctas = B * Hkv * ((a.G + 7) / 8);
+    e = launch_dependent(decode_merge_kernel, dim3(mctas), dim3(kMergeThreads), 0, stream, a);
     if (e != cudaSuccess) return e;
     count_launches(3);
     return cudaGetLastError();

@@ -172,11 +172,11 @@ tq_status tq_init_ex(int head_dim, int bits, uint64_t seed, int rotation, int ke
     fill_host(ctx, head_dim, bits, seed, rotation, key_mode, flags);
     const tq::HostParams& H = ctx->host;
 
-    // device copies: R^T and S (fp32; decode merge and decompress), R^T hi / lo and S
-    // (fp16; decode prep); then the tensor-core blob
+    // device copies: R^T and S (fp32; decompress), R^T hi / lo and S (fp16; decode prep),
+    // R hi / lo (fp16; decode merge); then the tensor-core blob
     const size_t n = size_t(kDim) * kDim;
     std::vector<float> blob(2 * n);
-    std::vector<__half> blob16(3 * n);
+    std::vector<__half> blob16(5 * n);
     float* RT = blob.data();
     float* S = RT + n;
     for (int i = 0; i < kDim; ++i)
@@ -188,6 +188,8 @@ tq_status tq_init_ex(int head_dim, int bits, uint64_t seed, int rotation, int ke
             blob16[size_t(j) * kDim + i] = hi;
             blob16[n + size_t(j) * kDim + i] = __double2half(r - double(__half2float(hi)));
             blob16[2 * n + size_t(i) * kDim + j] = __double2half(double(H.S[size_t(i) * kDim + j]));
+            blob16[3 * n + size_t(i) * kDim + j] = hi;  // R row-major, hi / lo (decode merge)
+            blob16[4 * n + size_t(i) * kDim + j] = blob16[n + size_t(j) * kDim + i];
         }
     tq::TcBlob tcb;
     if (!tq::build_tc_blob(H, tcb)) {
@@ -228,6 +230,8 @@ tq_status tq_init_ex(int head_dim, int bits, uint64_t seed, int rotation, int ke
     ctx->dev.RTh = base16;
     ctx->dev.RTl = base16 + n;
     ctx->dev.Sh = base16 + 2 * n;
+    ctx->dev.Rh = base16 + 3 * n;
+    ctx->dev.Rl = base16 + 4 * n;
     ctx->tc.images = base8 + tc_off + tcb.off_images;
     ctx->tc.lut_value = base8 + tc_off + tcb.off_lut_value;
     ctx->tc.lut_key = base8 + tc_off + tcb.off_lut_key;

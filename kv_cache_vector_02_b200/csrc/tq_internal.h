@@ -59,6 +59,8 @@ struct DeviceParams {
     const uint16_t* RTh;  // [d*d] fp16 R^T, high part
     const uint16_t* RTl;  // [d*d] fp16 R^T - RTh
     const uint16_t* Sh;   // [d*d] fp16 S (+-1, exact)
+    const uint16_t* Rh;   // [d*d] fp16 R row-major, high part
+    const uint16_t* Rl;   // [d*d] fp16 R - Rh
 };
 
 inline int container_width(int b) { return b >= 3 ? 4 : (b == 2 ? 2 : 1); }
