@@ -185,8 +185,10 @@ TQ_API tq_status tq_decompress(const tq_ctx* ctx, int kind, const uint8_t* cache
  * B sequences, Hq query heads over Hkv kv heads and sequences of at most
  * max_seq_len tokens (0 on invalid arguments).
  * Nothing in the workspace has to start at zero and it needs no clearing between
- * calls: every byte a decode reads is written earlier in the same call.  Two
- * decodes that run at the same time need separate workspaces.
+ * calls: every byte a decode reads is written earlier in the same call, except the
+ * per-slot flags, which are compared against a 64-bit tag that no other launch in
+ * the process uses.  Two decodes that run at the same time need separate
+ * workspaces.
  */
 TQ_API size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_seq_len);
 
@@ -198,6 +200,11 @@ TQ_API size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hk
  *   o = sum_{t < seq_lens[b]} softmax(s)_t * v_hat_t.
  * Scores are taken in the rotated domain (<R^T q, c[idx]>), the value sum is
  * accumulated in the rotated domain and un-rotated once per head.
+ * One kernel launch, cooperative: a CTA per SM (at most), all resident at once,
+ * each over an equal share of the pages; the CTA that holds a (sequence, kv head)
+ * unit's first page merges the unit's partial results from the CTAs after it
+ * (waiting for them, bounded).  A device that cannot hold the grid at once (SMs
+ * taken by other work) makes the launch fail: TQ_ERR_CUDA.
  *   q_dev          : [B][Hq][128] fp16, device.
  *   block_table_dev: [B][max_blocks] int32, device; page p of sequence b lives in
  *                    physical block block_table[b][p].
@@ -283,12 +290,14 @@ TQ_API tq_status tq_get_device_error(const tq_ctx* ctx, void* stream, uint32_t* 
 
 /*
  * tq_debug_stall -- test hook for the failure-detection path (no counterpart on
- * the pages).  The next `launches` kernels of this context that stream their
- * inputs through asynchronous copies (the compress kernels; the decode page
- * kernel) skip issuing those copies, so the waits that expect them run out after
- * their bounded limit (about 2 s): the kernel sets TQ_DEVERR_TIMEOUT in the device
- * error word, abandons its work (its outputs are then undefined), releases what it
- * holds and returns.  Nothing faults or hangs, and the context stays usable.
+ * the pages).  The next `launches` kernels of this context that wait for other
+ * threads' work do not get it: the compress kernels skip issuing their input
+ * copies; the decode kernel's CTAs do not publish the partial results of units
+ * that another CTA merges.  The waits that expect them run out after their
+ * bounded limit (about 2 s): the kernel sets TQ_DEVERR_TIMEOUT in the device error
+ * word (its outputs are then undefined), releases what it holds and returns.
+ * Nothing faults or hangs, and the context stays usable.  (A decode whose units
+ * all fit one CTA each waits for nothing and is not affected.)
  * launches = 0 cancels a pending stall.  Returns TQ_ERR_INVALID_ARG for a null or
  * host-only context or a negative count.
  */

@@ -472,17 +472,18 @@ __global__ void __launch_bounds__(Cfg<ROT, PROD, PAIR>::kBound, 1) compress_tc_k
             if (!d) return;
             const int pr = (int)((uintptr_t)d & 15u);
             uint8_t* cp = d - pr + pr * a.lay.code_row + q * (4 * kQW);
-            if (kQW == 4) *reinterpret_cast<uint4*>(cp) = make_uint4(w[0], w[1 % kQW], w[2 % kQW], w[3 % kQW]);
-            else if (kQW == 2) *reinterpret_cast<uint2*>(cp) = make_uint2(w[0], w[1 % kQW]);
-            else *reinterpret_cast<uint32_t*>(cp) = w[0];
+            // streaming stores: the cache lines leave L2 first (nothing here reads them again)
+            if (kQW == 4) __stcs(reinterpret_cast<uint4*>(cp), make_uint4(w[0], w[1 % kQW], w[2 % kQW], w[3 % kQW]));
+            else if (kQW == 2) __stcs(reinterpret_cast<uint2*>(cp), make_uint2(w[0], w[1 % kQW]));
+            else __stcs(reinterpret_cast<unsigned int*>(cp), w[0]);
         };
         auto store_tail = [&](uint8_t* d, float norm, float gamma, const uint32_t (&sg)[4]) {
             if (!d) return;
             const int pr = (int)((uintptr_t)d & 15u);
             uint8_t* chunk = d - pr;
-            if (PROD) *reinterpret_cast<uint4*>(chunk + a.lay.signs_off + pr * (kDim / 8)) = make_uint4(sg[0], sg[1], sg[2], sg[3]);
-            reinterpret_cast<float*>(chunk + a.lay.norm_off)[pr] = norm;
-            if (PROD) reinterpret_cast<float*>(chunk + a.lay.gamma_off)[pr] = gamma;
+            if (PROD) __stcs(reinterpret_cast<uint4*>(chunk + a.lay.signs_off + pr * (kDim / 8)), make_uint4(sg[0], sg[1], sg[2], sg[3]));
+            __stcs(reinterpret_cast<float*>(chunk + a.lay.norm_off) + pr, norm);
+            if (PROD) __stcs(reinterpret_cast<float*>(chunk + a.lay.gamma_off) + pr, gamma);
         };
 
         // the buffer-release arrivals of both CTAs of a pair go to the even CTA's issuer

@@ -1,4 +1,5 @@
-// Split-K decode attention over the paged compressed cache, on tensor cores.
+// Split-K decode attention over the paged compressed cache, on tensor cores, in one
+// kernel launch.
 //
 // [FQ-TQ] "FlashQuant：生产级KV缓存压缩方案…":
 //   - section "注意力计算的特殊挑战与QJL校正": score estimator
@@ -8,21 +9,27 @@
 // the value sum is accumulated as sum_t p_t n_t c[idx_t]/sqrt(d) and un-rotated
 // once per query head (o = R acc / l).
 //
-// Kernels:
-//   prep   q' = R^T q and s = S q for every query head (fp32), and the page prefix
-//          sums of the sequences.
-//   split  one persistent CTA per SM over an equal range of the pages of all
-//          (sequence, kv head) units; page p of a unit's piece goes to warp p % kNW.
-//          Each warp streams its own pages (one bulk copy each of the key and the
-//          value chunk) into its ring of shared-memory stages, its issue cursor
-//          running ahead across pieces, and per 16-token page:
-//            scores  D[16 tok x 8 heads] = sum_k Khat[tok][k] q'[k][h]   (mma m16n8k16)
-//                    plus the sign term with +-1 fragments against s
-//            softmax online, base 2, per head column
-//            values  D[16 coords x 8 heads] += Vhat^T[coord][tok] P'[tok][h]
-//          The warps of the CTA merge their states per piece; each piece's partial
-//          (m, l, acc) goes to the workspace.
-//   merge  log-sum-exp combination of a unit's pieces, division by l, un-rotation.
+// One kernel (decode_attn_kernel), cooperative: one persistent CTA per SM over an
+// equal range of the pages of all (sequence, kv head) units, all CTAs resident.
+//   prologue  R^T (fp16 hi, lo) and S staged in shared memory; the CTA's own page
+//             prefix sums of the sequences; the lookup tables; q' = R^T q and s = S q
+//             of the units of the range (mma.sync) into the CTA's workspace slots.
+//   pages     page p of a unit's piece (the range's part of one unit) goes to warp
+//             p % kNW.  Each warp streams its own pages (16-byte async copies by
+//             every lane of the key and the value chunk, one commit group per page)
+//             into its ring of shared-memory stages, its issue cursor running ahead
+//             across pieces, and per 16-token page:
+//               scores  D[16 tok x 8 heads] = sum_k Khat[tok][k] q'[k][h]  (mma m16n8k16)
+//                       plus the sign term with +-1 fragments against s
+//               softmax online, base 2, per head column
+//               values  D[16 coords x 8 heads] += Vhat^T[coord][tok] P'[tok][h]
+//             The warps of the CTA merge their states per piece into the slot (unit
+//             + CTA); a piece that does not start its unit publishes the slot with
+//             the launch's tag.
+//   epilogue  the CTA that holds a unit's first page waits (bounded) for the later
+//             slots of the unit, combines them by log-sum-exp, adds the residual
+//             window, un-rotates (o = R a on mma.sync, R staged in shared memory) and
+//             stores, 16 query heads at a time.
 //
 // Packed codes become fp16 MMA fragments in registers:
 //   - 3-bit key codes (nibbles): byte permutes of an 8-entry register table;
@@ -37,6 +44,8 @@
 // Inside a page the token order is permuted (row r holds token r ^ ((r >> 1) & 1))
 // so that a warp's loads of four tokens' value bytes meet at most two to a bank.
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <cmath>
 #include <mutex>
 
@@ -58,24 +67,26 @@ constexpr uint32_t kTabBytes = 65536;         // 256 entries x 256 bytes
 constexpr int kLowStages = 8;
 constexpr uint32_t kRingAddr = kTabAddr + kTabBytes;
 constexpr uint32_t kSplitSmem = kRingAddr + (kNW * kStages - kLowStages) * kStageBytes;  // any window base >= 0
-// Below the tables, from the window base: barriers, per-stage valid flags, the abort
-// flag, the warps' (m, l), the CTA merge area (4 heads at a time), the low stages.
-constexpr uint32_t kOffFull = 0;                                // [kNW][kStages] mbarrier: page landed
-constexpr uint32_t kOffValid = kOffFull + kNW * kStages * 8;    // [kNW][kStages] int: the block id was valid
-constexpr uint32_t kOffAbort = kOffValid + kNW * kStages * 4;   // int
-constexpr uint32_t kOffML = (kOffAbort + 4 + 15) & ~15u;        // [kNW][2][4] float: m, l
+// Below the tables, from the window base: the warps' (m, l), the CTA merge area (4
+// heads at a time), the low stages.
+constexpr uint32_t kOffML = 0;                                  // [kNW][2][4] float: m, l
 constexpr uint32_t kOffMerge = kOffML + kNW * 2 * 4 * 4;        // [kNW][4][128] float
 constexpr uint32_t kOffLowStages = (kOffMerge + kNW * 4 * kDim * 4 + 127) & ~127u;
 constexpr uint32_t kLowBytes = kOffLowStages + kLowStages * kStageBytes;
+// The page prefix sums of up to kPreCap - 1 sequences sit in the rest of the window
+// below the tables (more sequences: the CTA's copy in the workspace).
+constexpr uint32_t kOffPre = kLowBytes;
+constexpr int kPreCap = 3840;
+static_assert(kOffPre + kPreCap * 4 + 1024 <= kTabAddr, "prefix sums below the tables");
 static_assert(kSplitSmem <= 232448, "shared memory budget");
-constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint64_t kWaitNs = 2000000000ull;  // bounded waits for another CTA's slot
 
 enum KMode { kKPrmt = 0, kKByte4 = 1, kKByte2 = 2, kKBit1 = 3 };
 enum VMode { kVByte4 = 0, kVByte2 = 1 };
 
 struct DecodeArgs {
     const uint16_t* q;
-    float* qf;  // [B][Hq][2][128] fp32: q' then s
+    float* qf;  // [slots][G][2][128] fp32: q' then s of unit u in slot u + CTA
     const uint8_t* kc;
     const uint8_t* vc;
     int num_blocks;
@@ -83,9 +94,10 @@ struct DecodeArgs {
     int max_blocks;
     const int32_t* seq_lens;
     int B, Hq, Hkv, G, max_seq_len;
-    float* partial;    // [slots][G][130]: m, l, acc (rotated domain)
-    int* prefix;       // [B + 1] pages of the sequences before b (prep writes it)
-    int split_grid;    // CTAs of the split kernel
+    float* partial;    // [slots][G][130]: m, l, acc (rotated domain) of unit u's piece in CTA c: slot u + c
+    unsigned long long* flags;  // [slots]: = epoch once the slot's partial is complete
+    unsigned long long epoch;   // this launch's tag (never repeats within the process)
+    int* prefix;       // [grid][B + 1]: each CTA's own page prefix sums (pages of sequences < b)
     const uint16_t* RTh;   // fp16 R^T hi / lo, S (row-major)
     const uint16_t* RTl;
     const uint16_t* Sh;
@@ -98,7 +110,7 @@ struct DecodeArgs {
     ChunkLayout lk, lv;
     void* out;
     int out_fp32;
-    int stall;             // test hook: the producer copies no page
+    int stall;             // test hook: no piece publishes its partial (the merges wait out their limit)
     // residual window: fp16 keys / values [B][tail_cap][Hkv][128] of the last tail_lens[b]
     // tokens of each sequence, uncompressed (tail_k == NULL: none)
     const uint16_t* tail_k;
@@ -114,8 +126,6 @@ __device__ __forceinline__ bool seq_len_ok(const DecodeArgs& a, int L) {
 }
 
 // ------------------------------------------------------------------ helpers
-using sm100::griddep_wait;
-using sm100::griddep_launch_dependents;
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -124,6 +134,16 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D = A B (no accumulator input).
+__device__ __forceinline__ void mma16816_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
 }
 
 // Transpose of an 8x8 fp16 matrix held as m8n8 fragments (thread 4 g + c holds row g,
@@ -190,83 +210,6 @@ constexpr float kSlack = 8.f;
 // Token of page row r (see the file comment).
 __host__ __device__ constexpr int row_token(int r) { return r ^ ((r >> 1) & 1); }
 
-// ------------------------------------------------------------------ prep
-// [q' | s] = q [R | S^T] for 16 query heads per CTA, on mma.sync (fp16 inputs, fp32
-// accumulation; R^T enters as fp16 hi + lo, S is exact); fp32 results.  CTA (x, y),
-// warp w computes output columns 8 (8 y + w) .. +7 of the 256 (q' then s).  CTA (0, 0)
-// also writes the page prefix sums of the sequences.
-constexpr int kPrepThreads = 256;
-__global__ void __launch_bounds__(kPrepThreads) decode_prep_kernel(DecodeArgs a) {
-    const int NQ = a.B * a.Hq;
-    const int h0 = blockIdx.x * 16;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-    // B fragments of R^T (hi, lo) or S: parameters, loaded before waiting for the kernel before
-    const int nt = blockIdx.y * 8 + warp;  // 0..15 -> q', 16..31 -> s
-    const bool isq = nt < 16;
-    const int n = (nt & 15) * 8 + g;
-    uint32_t bh[8][2], bl[8][2];
-    {
-        const uint32_t* ph = reinterpret_cast<const uint32_t*>((isq ? a.RTh : a.Sh) + (size_t)n * kDim);
-        const uint32_t* pl = reinterpret_cast<const uint32_t*>(a.RTl + (size_t)n * kDim);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            bh[ks][0] = ph[8 * ks + c];
-            bh[ks][1] = ph[8 * ks + c + 4];
-            bl[ks][0] = isq ? pl[8 * ks + c] : 0u;
-            bl[ks][1] = isq ? pl[8 * ks + c + 4] : 0u;
-        }
-    }
-    griddep_wait();  // q and seq_lens may come from the kernel before
-    const bool r0 = h0 + g < NQ, r1 = h0 + g + 8 < NQ;
-    const uint32_t* q0 = reinterpret_cast<const uint32_t*>(a.q + (size_t)(r0 ? h0 + g : 0) * kDim);
-    const uint32_t* q1 = reinterpret_cast<const uint32_t*>(a.q + (size_t)(r1 ? h0 + g + 8 : 0) * kDim);
-    if (blockIdx.x == 0 && blockIdx.y == 0) {
-        // pages per sequence (invalid lengths count as empty and raise the error
-        // word) and their exclusive prefix sum, in chunks of 256 sequences
-        __shared__ int sc[kPrepThreads];
-        int carry = 0;
-        for (int b0 = 0; b0 < a.B; b0 += kPrepThreads) {
-            const int b = b0 + (int)threadIdx.x;
-            int n = 0;
-            if (b < a.B) {
-                const int L = a.seq_lens[b];
-                if (seq_len_ok(a, L)) n = (L + kPage - 1) / kPage;
-                else atomicOr(a.err, TQ_DEVERR_SEQLEN);
-            }
-            sc[threadIdx.x] = n;
-            __syncthreads();
-            for (int off = 1; off < kPrepThreads; off <<= 1) {  // inclusive scan
-                const int v = threadIdx.x >= off ? sc[threadIdx.x - off] : 0;
-                __syncthreads();
-                sc[threadIdx.x] += v;
-                __syncthreads();
-            }
-            if (b < a.B) a.prefix[b] = carry + sc[threadIdx.x] - n;
-            carry += sc[kPrepThreads - 1];
-            __syncthreads();
-        }
-        if (threadIdx.x == 0) a.prefix[a.B] = carry;
-    }
-    griddep_launch_dependents();  // the split kernel may start its prologue
-    uint32_t A[8][4];
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-        A[ks][0] = r0 ? q0[8 * ks + c] : 0u;
-        A[ks][1] = r1 ? q1[8 * ks + c] : 0u;
-        A[ks][2] = r0 ? q0[8 * ks + c + 4] : 0u;
-        A[ks][3] = r1 ? q1[8 * ks + c + 4] : 0u;
-    }
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-        if (isq) mma16816(d, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bl[ks][0], bl[ks][1]);
-        mma16816(d, A[ks][0], A[ks][1], A[ks][2], A[ks][3], bh[ks][0], bh[ks][1]);
-    }
-    const int col = (nt & 15) * 8 + 2 * c, which = isq ? 0 : 1;
-    if (r0) *reinterpret_cast<float2*>(a.qf + ((size_t)(h0 + g) * 2 + which) * kDim + col) = make_float2(d[0], d[1]);
-    if (r1) *reinterpret_cast<float2*>(a.qf + ((size_t)(h0 + g + 8) * 2 + which) * kDim + col) = make_float2(d[2], d[3]);
-}
-
 // ------------------------------------------------------------------ split: tables
 // Entry e (a byte) of the 64 KiB table at kTabAddr is 256 bytes:
 //   bytes   0..127  region A, values:
@@ -313,17 +256,19 @@ __device__ void build_tables(const DecodeArgs& a, int e) {
 // The CTA's range [pos, end) of the pages of all units in order (unit u = b Hkv + h
 // holds the pages of sequence b), cut into pieces by unit.
 struct Pieces {
+    const int* pre;  // the CTA's page prefix sums
     long pos, end;
     int b;
-    __device__ void init(const DecodeArgs& a, long p, long e) {
+    __device__ void init(const DecodeArgs& a, const int* prefix, long p, long e) {
+        pre = prefix;
         pos = p;
         end = e;
         b = 0;
-        if (pos < end) {  // the last sequence b with Hkv * prefix[b] <= pos
+        if (pos < end) {  // the last sequence b with Hkv * pre[b] <= pos
             int lo = 0, hi = a.B - 1;
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
-                if ((long)a.Hkv * a.prefix[mid] <= pos) lo = mid;
+                if ((long)a.Hkv * pre[mid] <= pos) lo = mid;
                 else hi = mid - 1;
             }
             b = lo;
@@ -332,8 +277,8 @@ struct Pieces {
     // next piece: sequence bb, kv head hk, pages [p0, p1) of the sequence
     __device__ bool next(const DecodeArgs& a, int& bb, int& hk, int& p0, int& p1) {
         while (pos < end && b < a.B) {
-            const int np = a.prefix[b + 1] - a.prefix[b];
-            const long off = pos - (long)a.Hkv * a.prefix[b];
+            const int np = pre[b + 1] - pre[b];
+            const long off = pos - (long)a.Hkv * pre[b];
             if (np == 0 || off >= (long)a.Hkv * np) {
                 ++b;
                 continue;
@@ -357,6 +302,8 @@ struct PageCursor {
     int b, hk, p0, p1, ji, nj;
     bool live;
     int win, win_next, wbase;
+    uint32_t kb, vb;                    // chunk bytes
+    const uint8_t *kbase, *vbase;       // this lane's 16 bytes of kv head hk's chunks in physical block 0
     __device__ int load_win(const DecodeArgs& a, int warp, int lane, int base) const {
         const int jj = base + lane;
         return jj < nj ? a.block_table[(size_t)b * a.max_blocks + p0 + warp + jj * kNW] : -1;
@@ -370,12 +317,17 @@ struct PageCursor {
             wbase = 0;
             win = load_win(a, warp, lane, 0);
             win_next = -1;
+            kbase = a.kc + (size_t)hk * kb + 16 * lane;
+            vbase = a.vc + (size_t)hk * vb + 16 * lane;
             live = true;
             return;
         }
     }
-    __device__ void init(const DecodeArgs& a, long pos, long end, int warp, int lane) {
-        it.init(a, pos, end);
+    __device__ void init(const DecodeArgs& a, const int* pre, long pos, long end, int warp, int lane, uint32_t kbytes,
+                         uint32_t vbytes) {
+        kb = kbytes;
+        vb = vbytes;
+        it.init(a, pre, pos, end);
         enter(a, warp, lane);
     }
     // block id of the current page (warp-uniform; every lane calls it)
@@ -401,7 +353,7 @@ struct PageRegs {
     uint32_t s[2];       // sign word c of rows g, g+8
     float kn[2], kg[2];  // key norm * qscale, gamma * sscale of rows g, g+8
     uint32_t v[4][2];    // value code bytes of rows 2c, 2c+1, 2c+8, 2c+9 (coords 16g .. 16g+15)
-    float vn[2];         // value norm / sqrt(d) of rows g, g+8
+    float vn[2];         // value norm of rows g, g+8
 };
 
 // Byte geometry of a page's key and value chunks (the same as the library's chunk
@@ -461,7 +413,7 @@ __device__ __forceinline__ void load_page(PageRegs<KM, VM, PROD>& r, const uint8
             r.kg[i] = *reinterpret_cast<const float*>(nb + P::kGamma) * sscale;
         }
         r.kn[i] = *reinterpret_cast<const float*>(nb + P::kNorm) * qscale;
-        r.vn[i] = *reinterpret_cast<const float*>(nb + P::kBytes + P::vNorm) * 0.08838834764831845f;
+        r.vn[i] = *reinterpret_cast<const float*>(nb + P::kBytes + P::vNorm);  // (1/sqrt(d) in the epilogue)
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -489,13 +441,7 @@ __device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, 
                                              const uint32_t (&bs)[NT][8][2], float (&m)[NT][2], float (&l)[NT][2],
                                              float (&acc)[NT][8][4]) {
     // ---- scores: the key term (even and odd K-steps in separate accumulators) and the sign term
-    float d1[NT][2][4], d2[NT][2][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) d1[nt][h][e] = d2[nt][h][e] = 0.f;
+    float d1[NT][2][4], d2[NT][2][4];  // the first MMA of each accumulator starts it
     if (KM == kKPrmt || KM == kKByte4) {
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
@@ -519,7 +465,8 @@ __device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, 
             }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
-                mma16816(d1[nt][ks & 1], ak[0][0], ak[1][0], ak[0][1], ak[1][1], bq[nt][ks][0], bq[nt][ks][1]);
+                if (ks < 2) mma16816_z(d1[nt][ks & 1], ak[0][0], ak[1][0], ak[0][1], ak[1][1], bq[nt][ks][0], bq[nt][ks][1]);
+                else mma16816(d1[nt][ks & 1], ak[0][0], ak[1][0], ak[0][1], ak[1][1], bq[nt][ks][0], bq[nt][ks][1]);
         }
     } else {
         // +-1 bit planes: byte b of the thread's key bytes -> K-steps 2b, 2b+1
@@ -539,8 +486,13 @@ __device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, 
             }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                mma16816(d1[nt][0], t[0].x, t[1].x, t[0].y, t[1].y, bq[nt][2 * b][0], bq[nt][2 * b][1]);
-                mma16816(d1[nt][1], t[0].z, t[1].z, t[0].w, t[1].w, bq[nt][2 * b + 1][0], bq[nt][2 * b + 1][1]);
+                if (b == 0) {
+                    mma16816_z(d1[nt][0], t[0].x, t[1].x, t[0].y, t[1].y, bq[nt][0][0], bq[nt][0][1]);
+                    mma16816_z(d1[nt][1], t[0].z, t[1].z, t[0].w, t[1].w, bq[nt][1][0], bq[nt][1][1]);
+                } else {
+                    mma16816(d1[nt][0], t[0].x, t[1].x, t[0].y, t[1].y, bq[nt][2 * b][0], bq[nt][2 * b][1]);
+                    mma16816(d1[nt][1], t[0].z, t[1].z, t[0].w, t[1].w, bq[nt][2 * b + 1][0], bq[nt][2 * b + 1][1]);
+                }
             }
         }
     }
@@ -560,8 +512,13 @@ __device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, 
             }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                mma16816(d2[nt][0], t[0].x, t[1].x, t[0].y, t[1].y, bs[nt][2 * b][0], bs[nt][2 * b][1]);
-                mma16816(d2[nt][1], t[0].z, t[1].z, t[0].w, t[1].w, bs[nt][2 * b + 1][0], bs[nt][2 * b + 1][1]);
+                if (b == 0) {
+                    mma16816_z(d2[nt][0], t[0].x, t[1].x, t[0].y, t[1].y, bs[nt][0][0], bs[nt][0][1]);
+                    mma16816_z(d2[nt][1], t[0].z, t[1].z, t[0].w, t[1].w, bs[nt][1][0], bs[nt][1][1]);
+                } else {
+                    mma16816(d2[nt][0], t[0].x, t[1].x, t[0].y, t[1].y, bs[nt][2 * b][0], bs[nt][2 * b][1]);
+                    mma16816(d2[nt][1], t[0].z, t[1].z, t[0].w, t[1].w, bs[nt][2 * b + 1][0], bs[nt][2 * b + 1][1]);
+                }
             }
         }
     }
@@ -685,9 +642,230 @@ __device__ __forceinline__ int coord_of(int mt) {
     return VM == kVByte4 ? 2 * mt : 4 * (mt >> 1) + 2 * (mt & 1);
 }
 
-// ------------------------------------------------------------------ split kernel
+// ------------------------------------------------------------------ prologue helpers
+// Unit (b Hkv + hk) of page position p of the CTA's page order (0 <= p < total).
+__device__ __forceinline__ int unit_at(const DecodeArgs& a, const int* pre, long p) {
+    int lo = 0, hi = a.B - 1;  // the last sequence with Hkv pre[b] <= p (it has pages)
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((long)a.Hkv * pre[mid] <= p) lo = mid;
+        else hi = mid - 1;
+    }
+    const int np = pre[lo + 1] - pre[lo];
+    return lo * a.Hkv + (int)((p - (long)a.Hkv * pre[lo]) / np);
+}
+
+// [q' | s] = q [R | S^T] of the query heads of units u_lo .. u_hi (rows u G + h of q,
+// contiguous) into the CTA's slots (row u G + h + CTA G of qf), on mma.sync: fp16
+// inputs, fp32 accumulation; R^T enters as fp16 hi + lo, S (+-1) is exact.  rt: the
+// shared-memory copies [R^T hi | R^T lo | S], row-major fp16 with the 16-byte pieces of
+// row n in the order k ^ (n % 8) (the eight rows of a fragment load meet no bank
+// twice).  Per 16-row tile of q (A fragments loaded once) warp w takes the 8-column
+// output tiles w, w + kNW, ... of the 32 (q' then s), two at a time.
+__device__ void rotate_queries(const DecodeArgs& a, const uint8_t* rt, int u_lo, int u_hi, int warp, int lane) {
+    const int g = lane >> 2, c = lane & 3;
+    const int r_lo = u_lo * a.G, r_end = (u_hi + 1) * a.G;
+    const size_t slot_rows = (size_t)blockIdx.x * a.G;
+    auto word = [&](const uint8_t* row, int w) {  // word w of a row: piece (w / 4) ^ g, word w % 4
+        return *reinterpret_cast<const uint32_t*>(row + ((((w >> 2) ^ g) << 4) | ((w & 3) << 2)));
+    };
+    for (int r0 = r_lo; r0 < r_end; r0 += 16) {
+        const bool v0 = r0 + g < r_end, v1 = r0 + g + 8 < r_end;
+        const uint32_t* q0 = reinterpret_cast<const uint32_t*>(a.q + (size_t)(v0 ? r0 + g : r_lo) * kDim);
+        const uint32_t* q1 = reinterpret_cast<const uint32_t*>(a.q + (size_t)(v1 ? r0 + g + 8 : r_lo) * kDim);
+        uint32_t A[8][4];
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            A[ks][0] = v0 ? q0[8 * ks + c] : 0u;
+            A[ks][1] = v1 ? q1[8 * ks + c] : 0u;
+            A[ks][2] = v0 ? q0[8 * ks + c + 4] : 0u;
+            A[ks][3] = v1 ? q1[8 * ks + c + 4] : 0u;
+        }
+        for (int nt0 = warp; nt0 < 32; nt0 += 2 * kNW) {
+            float d[2][4];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {  // two independent accumulation chains
+                const int nt = nt0 + t * kNW;
+                const bool isq = nt < 16;
+                const int n = (nt & 15) * 8 + g;
+                const uint8_t* ph = rt + (isq ? 0 : 2 * kDim * kDim * 2) + n * kDim * 2;
+                const uint8_t* pl = rt + kDim * kDim * 2 + n * kDim * 2;
+                if (nt < 32) {
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        if (ks == 0) mma16816_z(d[t], A[0][0], A[0][1], A[0][2], A[0][3], word(ph, c), word(ph, c + 4));
+                        else mma16816(d[t], A[ks][0], A[ks][1], A[ks][2], A[ks][3], word(ph, 8 * ks + c), word(ph, 8 * ks + c + 4));
+                        if (isq)
+                            mma16816(d[t], A[ks][0], A[ks][1], A[ks][2], A[ks][3], word(pl, 8 * ks + c), word(pl, 8 * ks + c + 4));
+                    }
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int nt = nt0 + t * kNW;
+                if (nt >= 32) continue;
+                const int col = (nt & 15) * 8 + 2 * c, which = nt < 16 ? 0 : 1;
+                if (v0)
+                    *reinterpret_cast<float2*>(a.qf + ((slot_rows + r0 + g) * 2 + which) * kDim + col) =
+                        make_float2(d[t][0], d[t][1]);
+                if (v1)
+                    *reinterpret_cast<float2*>(a.qf + ((slot_rows + r0 + g + 8) * 2 + which) * kDim + col) =
+                        make_float2(d[t][2], d[t][3]);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ epilogue helpers
+// Slot flags: a piece that does not start its unit publishes its partial with the
+// launch's epoch; the CTA holding the unit's first page waits for them (bounded).
+__device__ __forceinline__ void flag_publish(unsigned long long* f, unsigned long long epoch) {
+    __threadfence();
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(f), "l"(epoch) : "memory");
+}
+__device__ __forceinline__ unsigned long long flag_load(const unsigned long long* f) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
+    return v;
+}
+// Warp-collective bounded wait: each active lane waits for its own flag to reach
+// `epoch`; false for a lane whose flag did not within the limit (or once another warp
+// of the CTA gave up).
+__device__ bool flag_wait_lanes(const unsigned long long* f, bool active, unsigned long long epoch,
+                                volatile int* gave_up) {
+    bool ok = !active || flag_load(f) == epoch;
+    if (__all_sync(0xffffffffu, ok)) return true;
+    const uint64_t t0 = sm100::globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (!ok) ok = flag_load(f) == epoch;
+        if (__all_sync(0xffffffffu, ok) || *gave_up) break;
+        if ((it & 63u) == 0 && sm100::globaltimer_ns() - t0 > kWaitNs) {
+            *gave_up = 1;
+            break;
+        }
+        __nanosleep(64);
+    }
+    return ok;
+}
+
+// Epilogue scratch in the merge area and the low stages (free once the pages are done).
+struct EpiSmem {
+    float arow[16][kDim + 4];  // a = acc / l of the compressed part (rotated), then o = R a (rows padded)
+    float ml[16][2];       // its M, L
+    float trow[16][kDim + 4];  // window: acc (original domain)
+    float tml[16][2];      // window: M, L
+    float sq[16][kDim];    // window: q of the unit's heads
+    float ts[kDecodeTailMax][16];  // window: scores, then probabilities
+    float red[2][kNW][16];
+    int gave_up;
+};
+static_assert(sizeof(EpiSmem) <= kOffPre - kOffMerge, "epilogue scratch fits below the prefix sums");
+static_assert(2 * kDim * kDim * 2 <= (kNW * kStages - kLowStages) * kStageBytes, "R hi, lo fit the ring");
+
+// The residual window of unit u (sequence b, kv head hk) for its G heads: rows r0 + h.
+__device__ void window_unit(const DecodeArgs& a, EpiSmem& e, int b, int hk, int r0) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = a.G;
+    int tl = a.tail_lens[b];
+    if (tl < 0 || tl > a.tail_cap) {
+        if (tid == 0 && hk == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
+        tl = 0;
+    }
+    for (int k = tid; k < G * kDim; k += kSplitThreads) {
+        const int h = k / kDim, i = k - h * kDim;
+        e.sq[h][i] = __half2float(__ushort_as_half(a.q[((size_t)b * a.Hq + hk * G + h) * kDim + i]));
+    }
+    __syncthreads();
+    float mx[16];
+#pragma unroll
+    for (int h = 0; h < 16; ++h) mx[h] = -INFINITY;
+    for (int t = tid; t < tl; t += kSplitThreads) {  // scores: a thread per token
+        const uint4* kr = reinterpret_cast<const uint4*>(a.tail_k + (((size_t)b * a.tail_cap + t) * a.Hkv + hk) * kDim);
+        float sc[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) sc[h] = 0.f;
+#pragma unroll 1
+        for (int c8 = 0; c8 < kDim / 8; ++c8) {
+            const uint4 w = kr[c8];
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const float2 kk = __half22float2(*reinterpret_cast<const __half2*>(&ww[jj]));
+#pragma unroll
+                for (int h = 0; h < 16; ++h)
+                    if (h < G) sc[h] = fmaf(e.sq[h][8 * c8 + 2 * jj + 1], kk.y, fmaf(e.sq[h][8 * c8 + 2 * jj], kk.x, sc[h]));
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+            sc[h] *= a.scale_log2;
+            e.ts[t][h] = sc[h];
+            mx[h] = fmaxf(mx[h], sc[h]);
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < 16; ++h) {
+        for (int off = 16; off > 0; off >>= 1) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], off));
+        if (lane == 0) e.red[0][warp][h] = mx[h];
+    }
+    __syncthreads();
+    float gm[16], sm[16];
+#pragma unroll
+    for (int h = 0; h < 16; ++h) {
+        gm[h] = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) gm[h] = fmaxf(gm[h], e.red[0][w][h]);
+        sm[h] = 0.f;
+    }
+    for (int t = tid; t < tl; t += kSplitThreads)
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+            const float pr = h < G ? exp2f(e.ts[t][h] - gm[h]) : 0.f;
+            e.ts[t][h] = pr;
+            sm[h] += pr;
+        }
+#pragma unroll
+    for (int h = 0; h < 16; ++h) {
+        for (int off = 16; off > 0; off >>= 1) sm[h] += __shfl_xor_sync(0xffffffffu, sm[h], off);
+        if (lane == 0) e.red[1][warp][h] = sm[h];
+    }
+    __syncthreads();
+    for (int h = warp; h < G; h += kNW) {  // values: (head h, coordinates 4 lane ..)
+        float tL = 0.f;
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) tL += e.red[1][w][h];
+        float4 tA = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int t = 0; t < tl; ++t) {
+            const uint2 w = reinterpret_cast<const uint2*>(a.tail_v + (((size_t)b * a.tail_cap + t) * a.Hkv + hk) * kDim)[lane];
+            const float2 v0 = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
+            const float2 v1 = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
+            const float pr = e.ts[t][h];
+            tA.x = fmaf(pr, v0.x, tA.x);
+            tA.y = fmaf(pr, v0.y, tA.y);
+            tA.z = fmaf(pr, v1.x, tA.z);
+            tA.w = fmaf(pr, v1.y, tA.w);
+        }
+        reinterpret_cast<float4*>(e.trow[r0 + h])[lane] = tA;
+        if (lane == 0) e.tml[r0 + h][0] = tl > 0 ? gm[h] : -INFINITY, e.tml[r0 + h][1] = tL;
+    }
+    __syncthreads();
+}
+
+// ------------------------------------------------------------------ the decode kernel
+// One persistent CTA per SM (cooperative launch: all CTAs resident) over an equal
+// range of the pages of all (sequence, kv head) units:
+//   prologue  the CTA's own page prefix sums (last warp) while the other warps build
+//             the lookup tables; the page stream starts; q' and s of the units of the
+//             range into the CTA's slots;
+//   pages     per piece (the range's part of one unit) the warps' online softmax
+//             states, merged per piece into the slot (unit + CTA); a piece that does
+//             not hold its unit's first page publishes the slot (epoch flag);
+//   epilogue  the CTA that holds a unit's first page (or, for units without pages, the
+//             CTA of that position) combines the unit's slots by log-sum-exp, adds the
+//             residual window, un-rotates (o = R a on mma.sync, R as fp16 hi + lo) and
+//             stores, 16 query heads at a time.
 template <int KM, int VM, bool PROD, int NT>
-__global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kSplitThreads, 1) decode_attn_kernel(DecodeArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t base = sm100::smem_u32(smem);
@@ -695,59 +873,103 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeAr
         if (tid == 0) atomicOr(a.err, TQ_DEVERR_INTERNAL);
         return;
     }
-    const uint32_t full_bar = base + kOffFull;
     // shared-window address of stage st
     auto stage_addr = [&](uint32_t st) -> uint32_t {
         return st < (uint32_t)kLowStages ? base + kOffLowStages + st * kStageBytes
                                          : kRingAddr + (st - kLowStages) * kStageBytes;
     };
-    int* valid = reinterpret_cast<int*>(smem + kOffValid);
-    volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffAbort);
-    if (tid < 256) build_tables<KM, VM, PROD>(a, tid);
-    if (tid == 0) {
-        for (int i = 0; i < kNW * kStages; ++i) sm100::mbar_init(full_bar + 8 * i, 1);
-        *abort = 0;
-        sm100::fence_mbar_init();
+    // ---- prologue: R^T hi, R^T lo and S into the ring by 16-byte copies (parameters,
+    // nothing to wait for; row n's pieces swizzled, see rotate_queries), meanwhile the
+    // page prefix sums of the sequences (exclusive; invalid lengths count as empty and
+    // raise the error word), this CTA's own copy, and the lookup tables
+    {
+        constexpr int kPieces = kDim * kDim * 2 / 16;  // per matrix
+        for (int i = tid; i < 3 * kPieces; i += kSplitThreads) {
+            const int mtx = i / kPieces, o = (i - mtx * kPieces) * 16;
+            const int n = o >> 8, k16 = (o >> 4) & 15;
+            const uint16_t* src = mtx == 0 ? a.RTh : (mtx == 1 ? a.RTl : a.Sh);
+            sm100::cp_async16(kRingAddr + mtx * (kPieces * 16) + n * 256 + ((k16 ^ (n & 7)) << 4),
+                              reinterpret_cast<const uint8_t*>(src) + o);
+        }
+        sm100::cp_async_commit();
     }
+    int* pre = a.B + 1 <= kPreCap && base + kOffPre + (a.B + 1) * 4 <= kTabAddr
+                   ? reinterpret_cast<int*>(smem + kOffPre)
+                   : a.prefix + (size_t)blockIdx.x * (a.B + 1);
+    if (warp == kNW - 1) {
+        int carry = 0;
+        for (int b0 = 0; b0 < a.B; b0 += 32) {
+            const int b = b0 + lane;
+            int n = 0;
+            if (b < a.B) {
+                const int L = a.seq_lens[b];
+                if (seq_len_ok(a, L)) n = (L + kPage - 1) / kPage;
+                else if (blockIdx.x == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
+            }
+            int x = n;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (b < a.B) pre[b] = carry + x - n;
+            carry += __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (lane == 0) pre[a.B] = carry;
+    }
+    if (tid < 256) build_tables<KM, VM, PROD>(a, tid);
+    sm100::cp_async_wait<0>();
     __syncthreads();
-    griddep_wait();  // q', s and the page prefix sums from the prep kernel; the caller's inputs
-    griddep_launch_dependents();  // the merge kernel may stage its rotation meanwhile
-    const long total = (long)a.Hkv * a.prefix[a.B];
+    const long total = (long)a.Hkv * pre[a.B];
     const long pos0 = total * (long)blockIdx.x / gridDim.x;
     const long end = total * (long)(blockIdx.x + 1) / gridDim.x;
-    constexpr uint32_t kb = PageGeom<KM, VM, PROD>::kBytes, vb = PageGeom<KM, VM, PROD>::vBytes;
+    // q' and s of the units the range touches
+    if (pos0 < end)
+        rotate_queries(a, smem + (kRingAddr - base), unit_at(a, pre, pos0), unit_at(a, pre, end - 1), warp, lane);
+    __syncthreads();  // the slots are written, the ring is free
+    using P = PageGeom<KM, VM, PROD>;
+    constexpr uint32_t kb = P::kBytes, vb = P::vBytes;
+    static_assert(kb % 16 == 0 && vb % 16 == 0 && kb + vb <= kStageBytes, "page chunks in 16-byte pieces");
+    static_assert(3 * kDim * kDim * 2 <= (kNW * kStages - kLowStages) * kStageBytes, "R^T, S fit the ring");
     const size_t kstride = (size_t)a.Hkv * kb, vstride = (size_t)a.Hkv * vb;  // bytes per physical block
 
-    // ---- this warp's page stream: issue cursor (runs kStages pages ahead) and the
-    // copies of page number `k` of the warp into stage k % kStages
+    // ---- this warp's page stream: the issue cursor runs kStages pages ahead; page k of
+    // the warp goes to stage k % kStages as 16-byte copies by every lane, one commit
+    // group per page (empty past the end), so waiting for all but the newest
+    // kStages - 1 groups means page k has landed.  vmask bit s: stage s holds a page
+    // with a valid block id.
     PageCursor icur;
-    icur.init(a, pos0, end, warp, lane);
-    uint32_t issued = 0, landed = 0;  // pages issued; pages whose copies were started (for the drain)
-    // A page is two bulk copies (key chunk, value chunk) into the stage, completing on
-    // its barrier.  (Per-lane 16-byte cp.async copies measured slower.)
+    icur.init(a, pre, pos0, end, warp, lane, kb, vb);
+    uint32_t issued = 0, vmask = 0;
+    // the warp's stages are consecutive (kLowStages is a multiple of kStages)
+    static_assert(kLowStages % kStages == 0, "a warp's stages in one region");
+    const uint32_t wstage_addr = stage_addr(warp * kStages) + 16 * lane;
+    const uint8_t* wstage = smem + (stage_addr(warp * kStages) - base);
     auto issue_next = [&]() {
-        if (!icur.live) return;
-        const int blk = icur.block();
-        const uint32_t st = warp * kStages + issued % kStages;
-        if (lane == 0) {
+        if (icur.live) {
+            const int blk = icur.block();
+            const uint32_t s = issued % kStages;
             const bool v = blk >= 0 && blk < a.num_blocks;
-            valid[st] = v ? 1 : 0;
-            if (a.stall) {
-                // test hook: nothing arrives on the stage
-            } else if (v) {
-                const uint32_t dst = stage_addr(st);
-                sm100::mbar_arrive_expect_tx(full_bar + 8 * st, kb + vb);
-                sm100::bulk_g2s(dst, a.kc + (size_t)blk * kstride + icur.hk * kb, kb, full_bar + 8 * st);
-                sm100::bulk_g2s(dst + kb, a.vc + (size_t)blk * vstride + icur.hk * vb, vb, full_bar + 8 * st);
-            } else {
+            vmask = (vmask & ~(1u << s)) | ((uint32_t)v << s);
+            if (v) {
+                const uint32_t dst = wstage_addr + s * kStageBytes;
+                const uint8_t* ks = icur.kbase + (size_t)blk * kstride;
+                const uint8_t* vs = icur.vbase + (size_t)blk * vstride;
+#pragma unroll
+                for (int i = 0; i < (int)(kb / 512 + 1); ++i)
+                    if (i * 32 + lane < (int)(kb / 16)) sm100::cp_async16(dst + 512 * i, ks + 512 * i);
+#pragma unroll
+                for (int i = 0; i < (int)(vb / 512 + 1); ++i)
+                    if (i * 32 + lane < (int)(vb / 16)) sm100::cp_async16(dst + kb + 512 * i, vs + 512 * i);
+            } else if (lane == 0) {
                 atomicOr(a.err, TQ_DEVERR_BLOCK);
-                sm100::mbar_arrive(full_bar + 8 * st);  // nothing to copy: the stage completes at once
             }
+            icur.advance(a, warp, lane);
         }
-        if (!a.stall) ++landed;
+        sm100::cp_async_commit();
         ++issued;
-        icur.advance(a, warp, lane);
     };
+#pragma unroll 1
     for (int i = 0; i < kStages; ++i) issue_next();
 
     // ---------------------------------------------------------------- pages
@@ -776,10 +998,9 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeAr
     }
     float* wml = reinterpret_cast<float*>(smem + kOffML);      // [warp][2][4]: m then l
     float* wacc = reinterpret_cast<float*>(smem + kOffMerge);  // [warp][4 heads][128]
-    uint32_t cnt = 0;   // pages this warp has consumed (all pieces)
-    bool dead = false;  // a page never arrived: this warp stops working
+    uint32_t cnt = 0;  // pages this warp has consumed (all pieces)
     Pieces it;
-    it.init(a, pos0, end);
+    it.init(a, pre, pos0, end);
     int b, hk, p0, p1;
     constexpr int KS = KeyTerm<KM>::kSteps;
     while (it.next(a, b, hk, p0, p1)) {
@@ -791,7 +1012,8 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeAr
         for (int nt = 0; nt < NT; ++nt) {
             const int h = nt * 8 + g;
             if (h < a.G) {
-                const float4* src = reinterpret_cast<const float4*>(a.qf + (((size_t)unit * a.G + h) * 2) * kDim + 32 * c);
+                const float4* src =
+                    reinterpret_cast<const float4*>(a.qf + (((size_t)(unit + blockIdx.x) * a.G + h) * 2) * kDim + 32 * c);
                 float4 x[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) x[i] = src[i];
@@ -838,26 +1060,16 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeAr
         // ---- the warp's pages of the piece: p0 + warp, + kNW, ...
         const int nj = p0 + warp < p1 ? (p1 - p0 - warp + kNW - 1) / kNW : 0;
         for (int j = 0; j < nj; ++j) {
-            const uint32_t st = warp * kStages + cnt % kStages;
-            if (!dead) {
-                const bool ok = sm100::mbar_wait(full_bar + 8 * st, (cnt / kStages) & 1u, abort, kWaitNs);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    if (lane == 0 && !*abort) {
-                        *abort = 1;
-                        atomicOr(a.err, TQ_DEVERR_TIMEOUT);
-                    }
-                    dead = true;
-                }
-            }
-            if (dead) continue;  // this warp stops: no more pages are consumed or issued
+            const uint32_t s = cnt % kStages;
+            sm100::cp_async_wait<kStages - 1>();  // this lane's copies of the page
+            __syncwarp();                           // ... and every other lane's
             const int page = p0 + warp + j * kNW;
             // the page's bytes into registers, then the stage goes back to the stream
             // before the page is worked, so every stage is in flight meanwhile
-            const bool vp = valid[st] != 0;
+            const bool vp = (vmask >> s) & 1u;
             PageRegs<KM, VM, PROD> r;
-            if (vp) load_page<KM, VM, PROD>(r, smem + (stage_addr(st) - base), po, a.qscale, a.sscale);
-            sm100::fence_proxy_async_shared();  // this lane's reads before the refill's bulk copy
-            __syncwarp();                       // every lane is done with the stage before it is refilled
+            if (vp) load_page<KM, VM, PROD>(r, wstage + s * kStageBytes, po, a.qscale, a.sscale);
+            __syncwarp();  // every lane is done with the stage before it is refilled
             ++cnt;
             issue_next();
             if (vp)
@@ -922,232 +1134,219 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_split_kernel(DecodeAr
                     reinterpret_cast<float2*>(part + 2)[2 * lane + 1] = make_float2(A.z, A.w);
                 }
             }
+        // a piece that does not start its unit publishes the slot for the unit's merge
+        if (p0 > 0) {
+            __syncthreads();  // every head of the slot is written
+            if (tid == 0 && !a.stall) flag_publish(a.flags + unit + blockIdx.x, a.epoch);
+        }
     }
-    if (dead && landed > cnt) {  // the copies this warp started land before the CTA exits
-        const volatile int never = 0;
-        for (uint32_t k = cnt; k < landed; ++k)
-            sm100::mbar_wait(full_bar + 8 * (warp * kStages + k % kStages), (k / kStages) & 1u, &never, kWaitNs);
-    }
-}
+    sm100::cp_async_wait<0>();  // only empty groups remain; nothing is in flight
+    __syncthreads();            // the stage ring is free for the epilogue
 
-// ------------------------------------------------------------------ merge
-// One CTA of 8 warps per (unit, group of up to 8 query heads).  Unit u's pieces sit
-// in slots u + c for the split CTAs c whose page range meets it: c(p) = ((p + 1)
-// grid - 1) / total is the CTA of page p.
-//   1. log-sum-exp over the slots, thread = (head = warp, coordinates 4 lane ..
-//      4 lane + 3), into a = acc / l (rotated domain) in shared memory;
-//   2. with a residual window, the window's (m, l, acc) in the original domain:
-//      scores with a thread per token, values with the (head, 4 coordinates) layout;
-//   3. o = R a on mma.sync: A = a as fp16 hi + lo (heads on M), B = R as fp16 hi +
-//      lo (outputs on N; warp w takes the 8-output tiles w and w + 8), three passes
-//      (hi hi, hi lo, lo hi) into fp32; R's fragments are loaded before waiting for
-//      the page kernel (R is a parameter, not its output);
-//   4. o = (w_c R a + w_t acc_t) / (w_c + w_t l_t) with the two parts' log-sum-exp
-//      weights, stored fp16 or fp32.
-constexpr int kMergeWarps = 8;
-constexpr int kMergeThreads = kMergeWarps * 32;
-constexpr int kTailMax = 256;  // most window tokens per sequence
-struct MergeSmem {
-    float a[8][kDim];          // combined a = acc / l of each head (rotated), then o = R a
-    float ml[8][2];            // M, L of the compressed part per head
-    float q[8][kDim];          // window: q of the heads
-    float ts[kTailMax][8];     // window: scores, then probabilities
-    float red[2][kMergeWarps][8];
-};
-__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs a) {
-    __shared__ MergeSmem sm;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-    const int groups = (a.G + 7) / 8;
-    const int unit = blockIdx.x / groups, h0 = (blockIdx.x - unit * groups) * 8;
-    const int nh = min(8, a.G - h0);
-    const int b = unit / a.Hkv, hk = unit - b * a.Hkv;
-    // R fragments (B operand: column n = output i, K-pair = consecutive j of row i)
-    uint32_t rb[2][8][2][2];  // [tile][k-step][b0 / b1][hi / lo]
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-        const int i = (warp + 8 * t) * 8 + g;
-        const uint32_t* rh = reinterpret_cast<const uint32_t*>(a.Rh + (size_t)i * kDim);
-        const uint32_t* rl = reinterpret_cast<const uint32_t*>(a.Rl + (size_t)i * kDim);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            rb[t][ks][0][0] = rh[8 * ks + c];
-            rb[t][ks][1][0] = rh[8 * ks + c + 4];
-            rb[t][ks][0][1] = rl[8 * ks + c];
-            rb[t][ks][1][1] = rl[8 * ks + c + 4];
-        }
-    }
-    griddep_wait();  // the split partials
-    // ---- 1. log-sum-exp over the unit's slots: head hh = warp, coordinates 4 lane ..
-    const long total = (long)a.Hkv * a.prefix[a.B];
-    const long grid = a.split_grid;
-    const int np = a.prefix[b + 1] - a.prefix[b];
-    int c_lo = 0, c_hi = -1;
-    if (np > 0) {
-        const long first = (long)a.Hkv * a.prefix[b] + (long)hk * np, last = first + np - 1;
-        c_lo = (int)(((first + 1) * grid - 1) / total);
-        c_hi = (int)(((last + 1) * grid - 1) / total);
-    }
-    const int hh = warp;
-    float M = -INFINITY, L = 0.f;
-    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (hh < nh) {
-#pragma unroll 4
-        for (int cc = c_lo; cc <= c_hi; ++cc) {
-            const float* pp = a.partial + (((size_t)unit + cc) * a.G + h0 + hh) * kPartStride;
-            const float2 ml = *reinterpret_cast<const float2*>(pp);
-            const float2 x = reinterpret_cast<const float2*>(pp + 2)[2 * lane];
-            const float2 y = reinterpret_cast<const float2*>(pp + 2)[2 * lane + 1];
-            const float mn = fmaxf(M, ml.x);
-            const float sa = (M == -INFINITY) ? 0.f : exp2f(M - mn);
-            const float sb = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - mn);
-            L = fmaf(L, sa, ml.y * sb);
-            A.x = fmaf(A.x, sa, x.x * sb);
-            A.y = fmaf(A.y, sa, x.y * sb);
-            A.z = fmaf(A.z, sa, y.x * sb);
-            A.w = fmaf(A.w, sa, y.y * sb);
-            M = mn;
-        }
-    }
+    // ---------------------------------------------------------------- epilogue
+    EpiSmem& ep = *reinterpret_cast<EpiSmem*>(smem + kOffMerge);
+    if (tid == 0) ep.gave_up = 0;
+    // R hi and lo into the ring, row i's 16-byte pieces in the order k ^ (i % 8) (the
+    // fragment loads below meet no bank twice); they land while the slots are read
     {
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        reinterpret_cast<float4*>(sm.a[hh])[lane] = make_float4(A.x * inv, A.y * inv, A.z * inv, A.w * inv);
-        if (lane == 0) sm.ml[hh][0] = M, sm.ml[hh][1] = L;
+        constexpr int kPieces = kDim * kDim * 2 / 16;  // per matrix
+        for (int i = tid; i < 2 * kPieces; i += kSplitThreads) {
+            const int mtx = i / kPieces, o = (i - mtx * kPieces) * 16;
+            const int n = o >> 8, k16 = (o >> 4) & 15;
+            sm100::cp_async16(kRingAddr + mtx * (kPieces * 16) + n * 256 + ((k16 ^ (n & 7)) << 4),
+                              reinterpret_cast<const uint8_t*>(mtx == 0 ? a.Rh : a.Rl) + o);
+        }
+        sm100::cp_async_commit();
     }
-    // ---- 2. the residual window of the unit's sequence (base 2, original domain)
-    float tM = -INFINITY, tL = 0.f;
-    float4 tA = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (a.tail_k) {
-        int tl = a.tail_lens[b];
-        if (tl < 0 || tl > a.tail_cap) {
-            if (threadIdx.x == 0 && h0 == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
-            tl = 0;
+    const uint8_t* rsm = smem + (kRingAddr - base);
+    __syncthreads();
+    const int grid = gridDim.x, cta = blockIdx.x;
+    // The units this CTA finishes: first page position in [pos0, end), or (last CTA) at
+    // total -- units without pages sit at their sequence's position.  Sequences from the
+    // first one that reaches pos0, in batches of 16 / G units (16 rows).
+    int b_lo;
+    {
+        int lo = 0, hi = a.B;  // first b with Hkv pre[b] >= pos0 or Hkv pre[b + 1] > pos0
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if ((long)a.Hkv * pre[mid] >= pos0 || (long)a.Hkv * pre[mid + 1] > pos0) hi = mid;
+            else lo = mid + 1;
         }
-        for (int k = threadIdx.x; k < 8 * kDim; k += kMergeThreads) {
-            const int e = k / kDim, i = k - e * kDim;
-            sm.q[e][i] = e < nh ? __half2float(__ushort_as_half(a.q[((size_t)b * a.Hq + hk * a.G + h0 + e) * kDim + i]))
-                                : 0.f;
-        }
-        __syncthreads();
-        float mx[8];
+        b_lo = lo;
+    }
+    const bool last_cta = cta == grid - 1;
+    const int per_batch = 16 / a.G;
+    int ulist[16];
+    int nu = 0;
+    auto finish_batch = [&]() {
+        const int rows = nu * a.G;
+        // 1. log-sum-exp of each row's slots, thread = (row r, coordinates 4 lane ..);
+        // the slots' flags and (m, l) a lane per slot, 32 slots at a time
+        for (int r = warp; r < 16; r += kNW) {
+            float M = -INFINITY, L = 0.f;
+            float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r < rows) {
+                const int j = r / a.G, h = r - j * a.G;
+                const int u = ulist[j], b = u / a.Hkv, hk = u - b * a.Hkv;
+                const int np = pre[b + 1] - pre[b];
+                if (np > 0) {
+                    const long first = (long)a.Hkv * pre[b] + (long)hk * np, last = first + np - 1;
+                    const int ncon = (int)(((last + 1) * grid - 1) / total) - cta + 1;  // slots u + cta ..
+                    for (int i0 = 0; i0 < ncon; i0 += 32) {
+                        const int i = i0 + lane;
+                        const bool later = i > 0 && i < ncon;
+                        const bool ok = flag_wait_lanes(a.flags + u + cta + (later ? i : 0), later, a.epoch, &ep.gave_up);
+                        if (!__all_sync(0xffffffffu, ok) && lane == 0)
+                            atomicOr(a.err, TQ_DEVERR_TIMEOUT);  // (the slot is read all the same)
+                        const size_t row0 = ((size_t)u + cta + i0) * a.G + h;  // slot u + cta + i0, head h
+                        const int n = min(32, ncon - i0);
+                        // the first (up to) 8 slots' coordinates are loaded with the (m, l)
+                        float4 pa[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
-        for (int u = threadIdx.x; u < tl; u += kMergeThreads) {  // scores: a thread per token
-            const uint4* kr = reinterpret_cast<const uint4*>(a.tail_k + (((size_t)b * a.tail_cap + u) * a.Hkv + hk) * kDim);
-            float sc[8];
+                        for (int k = 0; k < 8; ++k) {
+                            pa[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (k < n) {
+                                const float* pp = a.partial + (row0 + (size_t)k * a.G) * kPartStride + 2;
+                                const float2 x = __ldcg(reinterpret_cast<const float2*>(pp) + 2 * lane);
+                                const float2 y = __ldcg(reinterpret_cast<const float2*>(pp) + 2 * lane + 1);
+                                pa[k] = make_float4(x.x, x.y, y.x, y.y);
+                            }
+                        }
+                        float2 mli = make_float2(-INFINITY, 0.f);
+                        if (i < ncon) mli = __ldcg(reinterpret_cast<const float2*>(a.partial + (row0 + (size_t)lane * a.G) * kPartStride));
+                        float mx = mli.x;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) sc[e] = 0.f;
-#pragma unroll 2
-            for (int c8 = 0; c8 < kDim / 8; ++c8) {
-                const uint4 w = kr[c8];
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                        const float mn = fmaxf(M, mx);
+                        if (mn == -INFINITY) continue;  // nothing in these slots yet
+                        const float sa = M == -INFINITY ? 0.f : exp2f(M - mn);
+                        const float wi = mli.x == -INFINITY ? 0.f : exp2f(mli.x - mn);
+                        float li = wi * mli.y;
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const float2 kk = __half22float2(*reinterpret_cast<const __half2*>(&ww[jj]));
+                        for (int o = 16; o > 0; o >>= 1) li += __shfl_xor_sync(0xffffffffu, li, o);
+                        L = fmaf(L, sa, li);
+                        A.x *= sa, A.y *= sa, A.z *= sa, A.w *= sa;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        sc[e] = fmaf(sm.q[e][8 * c8 + 2 * jj + 1], kk.y, fmaf(sm.q[e][8 * c8 + 2 * jj], kk.x, sc[e]));
+                        for (int k = 0; k < 8; ++k) {
+                            const float w = __shfl_sync(0xffffffffu, wi, k);  // 0 past n
+                            A.x = fmaf(w, pa[k].x, A.x);
+                            A.y = fmaf(w, pa[k].y, A.y);
+                            A.z = fmaf(w, pa[k].z, A.z);
+                            A.w = fmaf(w, pa[k].w, A.w);
+                        }
+#pragma unroll 4
+                        for (int k = 8; k < n; ++k) {
+                            const float w = __shfl_sync(0xffffffffu, wi, k);
+                            const float* pp = a.partial + (row0 + (size_t)k * a.G) * kPartStride + 2;
+                            const float2 x = __ldcg(reinterpret_cast<const float2*>(pp) + 2 * lane);
+                            const float2 y = __ldcg(reinterpret_cast<const float2*>(pp) + 2 * lane + 1);
+                            A.x = fmaf(w, x.x, A.x);
+                            A.y = fmaf(w, x.y, A.y);
+                            A.z = fmaf(w, y.x, A.z);
+                            A.w = fmaf(w, y.y, A.w);
+                        }
+                        M = mn;
+                    }
                 }
             }
+            // a = acc / (l sqrt(d)): the value norms entered without their 1/sqrt(d)
+            const float inv = L > 0.f ? 0.08838834764831845f / L : 0.f;
+            reinterpret_cast<float4*>(ep.arow[r])[lane] = make_float4(A.x * inv, A.y * inv, A.z * inv, A.w * inv);
+            if (lane == 0) ep.ml[r][0] = M, ep.ml[r][1] = L;
+        }
+        // 2. the residual windows of the batch's units
+        if (a.tail_k)
+            for (int j = 0; j < nu; ++j) window_unit(a, ep, ulist[j] / a.Hkv, ulist[j] % a.Hkv, j * a.G);
+        __syncthreads();  // a, ml complete
+        // 3. o = R a: rows = the batch's heads, columns = outputs; warp w < 8 takes the
+        // output tiles w and w + 8 (B fragments: column n = output i, K-pair =
+        // consecutive j of row i of R)
+        sm100::cp_async_wait<0>();
+        __syncthreads();  // R landed (every thread's copies)
+        float d[2][4];
+        if (warp < 8) {
+            uint32_t ah[8][4], al[8][4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                sc[e] *= a.scale_log2;
-                sm.ts[u][e] = sc[e];
-                mx[e] = fmaxf(mx[e], sc[e]);
+            for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {  // rows g / g + 8, k-columns 2c.. / 2c + 8..
+                    const float2 x = *reinterpret_cast<const float2*>(&ep.arow[g + 8 * (q4 & 1)][16 * ks + 8 * (q4 >> 1) + 2 * c]);
+                    const __half2 hi = __floats2half2_rn(x.x, x.y);
+                    const float2 hif = __half22float2(hi);
+                    const __half2 lo = __floats2half2_rn(x.x - hif.x, x.y - hif.y);
+                    ah[ks][q4] = *reinterpret_cast<const uint32_t*>(&hi);
+                    al[ks][q4] = *reinterpret_cast<const uint32_t*>(&lo);
+                }
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) d[t][e4] = 0.f;
+#pragma unroll
+                const int i = (warp + 8 * t) * 8 + g;
+                const uint8_t* rh = rsm + i * 256;
+                const uint8_t* rl = rsm + kDim * kDim * 2 + i * 256;
+                auto word = [&](const uint8_t* row, int w) {  // word w: piece (w / 4) ^ g
+                    return *reinterpret_cast<const uint32_t*>(row + ((((w >> 2) ^ g) << 4) | ((w & 3) << 2)));
+                };
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t h0 = word(rh, 8 * ks + c), h1 = word(rh, 8 * ks + c + 4);
+                    const uint32_t l0 = word(rl, 8 * ks + c), l1 = word(rl, 8 * ks + c + 4);
+                    mma16816(d[t], al[ks][0], al[ks][1], al[ks][2], al[ks][3], h0, h1);
+                    mma16816(d[t], ah[ks][0], ah[ks][1], ah[ks][2], ah[ks][3], l0, l1);
+                    mma16816(d[t], ah[ks][0], ah[ks][1], ah[ks][2], ah[ks][3], h0, h1);
+                }
             }
         }
+        __syncthreads();  // every warp has read a
+        if (warp < 8) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            for (int off = 16; off > 0; off >>= 1) mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], off));
-            if (lane == 0) sm.red[0][warp][e] = mx[e];
-        }
-        __syncthreads();
-        float gm[8], sm8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            gm[e] = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < kMergeWarps; ++w) gm[e] = fmaxf(gm[e], sm.red[0][w][e]);
-            sm8[e] = 0.f;
-        }
-        for (int u = threadIdx.x; u < tl; u += kMergeThreads)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float p = exp2f(sm.ts[u][e] - gm[e]);
-                sm.ts[u][e] = p;
-                sm8[e] += p;
+            for (int t = 0; t < 2; ++t) {
+                const int col = (warp + 8 * t) * 8 + 2 * c;
+                *reinterpret_cast<float2*>(&ep.arow[g][col]) = make_float2(d[t][0], d[t][1]);
+                *reinterpret_cast<float2*>(&ep.arow[g + 8][col]) = make_float2(d[t][2], d[t][3]);
             }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            for (int off = 16; off > 0; off >>= 1) sm8[e] += __shfl_xor_sync(0xffffffffu, sm8[e], off);
-            if (lane == 0) sm.red[1][warp][e] = sm8[e];
         }
         __syncthreads();
-        tM = gm[hh];
-#pragma unroll
-        for (int w = 0; w < kMergeWarps; ++w) tL += sm.red[1][w][hh];
-        for (int u = 0; u < tl; ++u) {  // values: (head hh, coordinates 4 lane ..)
-            const uint2 w = reinterpret_cast<const uint2*>(a.tail_v + (((size_t)b * a.tail_cap + u) * a.Hkv + hk) * kDim)[lane];
-            const float2 v0 = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
-            const float2 v1 = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
-            const float p = sm.ts[u][hh];
-            tA.x = fmaf(p, v0.x, tA.x);
-            tA.y = fmaf(p, v0.y, tA.y);
-            tA.z = fmaf(p, v1.x, tA.z);
-            tA.w = fmaf(p, v1.y, tA.w);
+        // 4. combine with the window and store: thread = (row r, coordinates 4 lane ..)
+        for (int r = warp; r < rows; r += kNW) {
+            const int j = r / a.G, h = r - j * a.G;
+            float4 o = reinterpret_cast<const float4*>(ep.arow[r])[lane];
+            if (a.tail_k) {
+                const float Mc = ep.ml[r][0], Lc = ep.ml[r][1], tM = ep.tml[r][0], tL = ep.tml[r][1];
+                const float4 tA = reinterpret_cast<const float4*>(ep.trow[r])[lane];
+                const float Mx = fmaxf(Mc, tM);
+                const float wc = Lc > 0.f ? exp2f(Mc - Mx) * Lc : 0.f;
+                const float et = tL > 0.f ? exp2f(tM - Mx) : 0.f;
+                const float den = wc + et * tL;
+                const float inv = den > 0.f ? 1.f / den : 0.f;
+                o = make_float4((wc * o.x + et * tA.x) * inv, (wc * o.y + et * tA.y) * inv,
+                                (wc * o.z + et * tA.z) * inv, (wc * o.w + et * tA.w) * inv);
+            }
+            const size_t oi = ((size_t)ulist[j] * a.G + h) * kDim + 4 * lane;
+            if (a.out_fp32) {
+                *reinterpret_cast<float4*>(static_cast<float*>(a.out) + oi) = o;
+            } else {
+                const __half2 lo = __floats2half2_rn(o.x, o.y), hi = __floats2half2_rn(o.z, o.w);
+                *reinterpret_cast<uint2*>(static_cast<__half*>(a.out) + oi) =
+                    make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+            }
+        }
+        __syncthreads();  // the scratch is free for the next batch
+        nu = 0;
+    };
+    for (int b = b_lo; b < a.B; ++b) {
+        const long s0 = (long)a.Hkv * pre[b];
+        if (s0 >= end && !(last_cta && s0 == total)) break;
+        const int np = pre[b + 1] - pre[b];
+        for (int hk = 0; hk < a.Hkv; ++hk) {
+            const long first = s0 + (long)hk * np;
+            if (!((first >= pos0 && first < end) || (last_cta && first == total))) continue;
+            ulist[nu++] = b * a.Hkv + hk;
+            if (nu == per_batch) finish_batch();
         }
     }
-    __syncthreads();  // a and ml complete
-    // ---- 3. o = R a for the (up to 8) heads: rows g (heads), columns = outputs
-    uint32_t ah[8][2], al[8][2];  // [k-step][k-cols 2c.. / 2c+8..] of head row g
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            const float2 x = *reinterpret_cast<const float2*>(&sm.a[g][16 * ks + 8 * hf + 2 * c]);
-            const __half2 hi = __floats2half2_rn(x.x, x.y);
-            const float2 hif = __half22float2(hi);
-            const __half2 lo = __floats2half2_rn(x.x - hif.x, x.y - hif.y);
-            ah[ks][hf] = *reinterpret_cast<const uint32_t*>(&hi);
-            al[ks][hf] = *reinterpret_cast<const uint32_t*>(&lo);
-        }
-    float d[2][4];
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) d[t][e] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            mma16816(d[t], al[ks][0], 0u, al[ks][1], 0u, rb[t][ks][0][0], rb[t][ks][1][0]);
-            mma16816(d[t], ah[ks][0], 0u, ah[ks][1], 0u, rb[t][ks][0][1], rb[t][ks][1][1]);
-            mma16816(d[t], ah[ks][0], 0u, ah[ks][1], 0u, rb[t][ks][0][0], rb[t][ks][1][0]);
-        }
-    }
-    __syncthreads();  // every warp has read a
-#pragma unroll
-    for (int t = 0; t < 2; ++t)
-        *reinterpret_cast<float2*>(&sm.a[g][(warp + 8 * t) * 8 + 2 * c]) = make_float2(d[t][0], d[t][1]);
-    __syncthreads();
-    // ---- 4. combine with the window and store: thread = (head hh, coordinates 4 lane ..)
-    if (hh >= nh) return;
-    float4 o = reinterpret_cast<const float4*>(sm.a[hh])[lane];
-    if (a.tail_k) {
-        const float Mc = sm.ml[hh][0], Lc = sm.ml[hh][1];
-        const float Mx = fmaxf(Mc, tM);
-        const float wc = Lc > 0.f ? exp2f(Mc - Mx) * Lc : 0.f;
-        const float et = tL > 0.f ? exp2f(tM - Mx) : 0.f;
-        const float den = wc + et * tL;
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        o = make_float4((wc * o.x + et * tA.x) * inv, (wc * o.y + et * tA.y) * inv, (wc * o.z + et * tA.z) * inv,
-                        (wc * o.w + et * tA.w) * inv);
-    }
-    const size_t oi = ((size_t)unit * a.G + h0 + hh) * kDim + 4 * lane;
-    if (a.out_fp32) {
-        *reinterpret_cast<float4*>(static_cast<float*>(a.out) + oi) = o;
-    } else {
-        const __half2 lo = __floats2half2_rn(o.x, o.y), hi = __floats2half2_rn(o.z, o.w);
-        *reinterpret_cast<uint2*>(static_cast<__half*>(a.out) + oi) =
-            make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
-    }
+    if (nu > 0) finish_batch();
 }
 
 int kmode_of(const tq_ctx* ctx) {
@@ -1157,33 +1356,44 @@ int kmode_of(const tq_ctx* ctx) {
     return kKBit1;
 }
 
-// Launch with programmatic stream serialization (see griddep_wait).
-template <typename K>
-cudaError_t launch_dependent(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, const DecodeArgs& a) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, a);
-}
-
 template <int KM, int VM, bool PROD, int NT>
-cudaError_t launch_split(const DecodeArgs& a, int grid, cudaStream_t stream) {
+cudaError_t launch_attn(const DecodeArgs& a, int grid, cudaStream_t stream) {
     using P = PageGeom<KM, VM, PROD>;
     if (a.lk.bytes != P::kBytes || a.lv.bytes != P::vBytes || a.lk.code_row != P::kRow ||
         a.lv.code_row != P::vRow || a.lk.norm_off != P::kNorm || a.lv.norm_off != P::vNorm ||
         (PROD && (a.lk.signs_off != P::kSigns || a.lk.gamma_off != P::kGamma)))
         return cudaErrorInvalidValue;  // the kernel's fixed geometry must be the context's
-    auto k = decode_split_kernel<KM, VM, PROD, NT>;
+    auto k = decode_attn_kernel<KM, VM, PROD, NT>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSplitSmem);
     if (e != cudaSuccess) return e;
-    return launch_dependent(k, dim3(grid), dim3(kSplitThreads), kSplitSmem, stream, a);
+    // cooperative: every CTA resident at once (a unit's merge waits for later CTAs' slots)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kSplitThreads);
+    cfg.dynamicSmemBytes = kSplitSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, a);
+}
+
+// Launch tags: a process-wide counter from a time-derived start, so that no two
+// launches share one and stale or foreign workspace contents never match.
+std::atomic<unsigned long long> g_epoch{0};
+unsigned long long next_epoch() {
+    unsigned long long e = g_epoch.fetch_add(1, std::memory_order_relaxed);
+    if (e == 0) {  // first use: start from the clock, away from 0 and all-ones patterns
+        const unsigned long long t =
+            (unsigned long long)std::chrono::high_resolution_clock::now().time_since_epoch().count();
+        unsigned long long expect = 1;
+        const unsigned long long start = (t * 0x9E3779B97F4A7C15ull) | (1ull << 40);
+        g_epoch.compare_exchange_strong(expect, start + 1, std::memory_order_relaxed);
+        return start;
+    }
+    return e;
 }
 
 }  // namespace
@@ -1191,25 +1401,25 @@ cudaError_t launch_split(const DecodeArgs& a, int grid, cudaStream_t stream) {
 DecodePlan plan_decode(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_seq_len) {
     DecodePlan p{};
     p.max_pages = (max_seq_len + kPage - 1) / kPage;
-    const long resident = (long)ctx->sm_count;  // one split CTA per SM
+    const long resident = (long)ctx->sm_count;  // one CTA per SM
     const long units = (long)B * Hkv;
-    // every SM, but at least 4 pages per consumer warp for small batches
+    // every SM, but at least 4 pages per warp for small batches
     long grid = (units * p.max_pages + 4 * kNW - 1) / (4 * kNW);
     if (grid > resident) grid = resident;
     if (grid < 1) grid = 1;
     p.grid = (int)grid;
     p.slots = (int)(units + grid);
     const int G = Hkv > 0 ? Hq / Hkv : 0;
+    auto take = [](size_t& off, size_t n) {
+        const size_t at = off;
+        off = (off + n + 255) & ~size_t(255);
+        return at;
+    };
     size_t off = 0;
-    p.qprep_off = off;
-    off += (size_t)B * Hq * 2 * kDim * sizeof(float);
-    off = (off + 255) & ~size_t(255);
-    p.partial_off = off;
-    off += (size_t)p.slots * G * kPartStride * sizeof(float);
-    off = (off + 255) & ~size_t(255);
-    p.prefix_off = off;
-    off += (size_t)(B + 1) * sizeof(int);
-    off = (off + 255) & ~size_t(255);
+    p.qprep_off = take(off, (size_t)p.slots * G * 2 * kDim * sizeof(float));
+    p.partial_off = take(off, (size_t)p.slots * G * kPartStride * sizeof(float));
+    p.flags_off = take(off, (size_t)p.slots * sizeof(unsigned long long));
+    p.prefix_off = take(off, (size_t)grid * (B + 1) * sizeof(int));
     p.bytes = off;
     return p;
 }
@@ -1242,8 +1452,9 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
     a.qscale = scale_log2 / sqrtf((float)kDim);
     a.sscale = scale_log2 * 1.2533141373155003f / (float)kDim;
     a.partial = reinterpret_cast<float*>(ws + plan.partial_off);
+    a.flags = reinterpret_cast<unsigned long long*>(ws + plan.flags_off);
+    a.epoch = next_epoch();
     a.prefix = reinterpret_cast<int*>(ws + plan.prefix_off);
-    a.split_grid = plan.grid;
     a.RTh = ctx->dev.RTh;
     a.RTl = ctx->dev.RTl;
     a.Sh = ctx->dev.Sh;
@@ -1265,15 +1476,13 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
     a.kbeta = KM == kKByte2 ? 0.25f * (ck[3] - ck[2] + ck[1] - ck[0]) : 0.f;
     a.stall = take_stall(ctx) ? 1 : 0;
 
-    cudaError_t e = launch_dependent(decode_prep_kernel, dim3((B * Hq + 15) / 16, 4), dim3(kPrepThreads), 0, stream, a);
-    if (e != cudaSuccess) return e;
     const int VM = ctx->cb_value.width == 4 ? kVByte4 : kVByte2;
     const bool prod = ctx->lay_key.prod;
     const int NT = a.G <= 8 ? 1 : 2;
     const int grid = plan.grid;
-    e = cudaErrorInvalidValue;
+    cudaError_t e = cudaErrorInvalidValue;
 #define TQ_DEC_CASE(K_, V_, P_, N_) \
-    if (KM == K_ && VM == V_ && prod == P_ && NT == N_) e = launch_split<K_, V_, P_, N_>(a, grid, stream);
+    if (KM == K_ && VM == V_ && prod == P_ && NT == N_) e = launch_attn<K_, V_, P_, N_>(a, grid, stream);
 #define TQ_DEC_NT(K_, V_, P_) TQ_DEC_CASE(K_, V_, P_, 1) TQ_DEC_CASE(K_, V_, P_, 2)
     TQ_DEC_NT(kKPrmt, kVByte4, true)    // bits 4, prod keys (3-bit codes)
     TQ_DEC_NT(kKByte2, kVByte4, true)   // bits 3, prod keys (2-bit codes)
@@ -1284,10 +1493,7 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint1
 #undef TQ_DEC_NT
 #undef TQ_DEC_CASE
     if (e != cudaSuccess) return e;
-    const int mctas = B * Hkv * ((a.G + 7) / 8);
-    e = launch_dependent(decode_merge_kernel, dim3(mctas), dim3(kMergeThreads), 0, stream, a);
-    if (e != cudaSuccess) return e;
-    count_launches(3);
+    count_launches(1);
     return cudaGetLastError();
 }
 

@@ -111,16 +111,17 @@ cudaError_t launch_decompress(const tq_ctx* ctx, int kind, const uint8_t* cache,
                               const int32_t* slots, int T, int H, void* out, int out_fp32, cudaStream_t stream);
 
 // Split-K decode: the pages of all (sequence, kv head) units, in order, are cut
-// into `grid` equal ranges, one per CTA of the split kernel; the piece of unit u
+// into `grid` equal ranges, one per CTA of the decode kernel; the piece of unit u
 // in CTA c leaves its partial softmax state in slot u + c (unique: each slot index
 // counts the unit and CTA boundaries before the piece).
 struct DecodePlan {
-    int grid;            // CTAs of the split kernel
-    int slots;           // units + grid
+    int grid;            // CTAs of the decode kernel
+    int slots;           // units + grid: unit u's slot in CTA c is u + c
     int max_pages;       // ceil(max_seq_len / 16)
-    size_t qprep_off;    // workspace offsets (bytes)
-    size_t partial_off;
-    size_t prefix_off;   // int32 [B + 1]: pages of sequences 0 .. b-1
+    size_t qprep_off;    // workspace offsets (bytes): fp32 [slots][G][2][128] q' and s
+    size_t partial_off;  // fp32 [slots][G][130] m, l, acc
+    size_t flags_off;    // u64 [slots] launch tags of the published slots
+    size_t prefix_off;   // int32 [grid][B + 1]: each CTA's page prefix sums
     size_t bytes;        // total workspace
 };
 DecodePlan plan_decode(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_seq_len);

@@ -306,8 +306,9 @@ def tq_get_device_error(ctx: Context, stream=None) -> int:
 
 
 def tq_debug_stall(ctx: Context, launches: int):
-    """Test hook: the next `launches` streaming kernels of ctx skip their input
-    copies, so their bounded waits run out and TQ_DEVERR_TIMEOUT is set (see tq.h)."""
+    """Test hook: the next `launches` kernels of ctx withhold what their bounded
+    waits expect (compress: its input copies; decode: the partial results another
+    CTA merges), so the waits run out and TQ_DEVERR_TIMEOUT is set (see tq.h)."""
     _check(_lib.tq_debug_stall(ctx.handle, int(launches)), "tq_debug_stall")
 
 

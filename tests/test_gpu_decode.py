@@ -187,7 +187,7 @@ def test_decompress_matches_oracle(orc, rot, bits, km):
         assert np.abs(got - want).max() <= 1e-5 * scale.max()
 
 
-# Every instantiation of the split kernel: (key code mode, value code mode, QJL or not)
+# Every instantiation of the decode kernel: (key code mode, value code mode, QJL or not)
 # x (one or two tiles of 8 query heads).  bits 4 / 3 / 2 with prod keys (3-, 2-, 1-bit
 # key codes + signs) and with MSE keys (4-, 3-, 2-bit key codes).
 DECODE_MODES = [(0, 4, 0), (1, 3, 0), (1, 2, 0), (0, 4, 1), (1, 3, 1), (0, 2, 1)]

@@ -1,8 +1,9 @@
 """Failure detection on the GPU: a bounded wait that runs out.
 
-tq_debug_stall makes the next launches skip their input copies, so the waits
-that expect those copies (a flag nothing will set) give up after their bounded
-limit.  The kernel must then report TQ_DEVERR_TIMEOUT through the device error
+tq_debug_stall makes the next launches withhold what their waits expect (the
+compress kernels skip their input copies; the decode kernel's CTAs do not publish
+the partial results another CTA merges), so those waits (on a flag nothing will
+set) give up after their bounded limit.  The kernel must then report TQ_DEVERR_TIMEOUT through the device error
 word, release what it holds and return; the context must stay usable and the
 next ordinary call must again match the oracle exactly.  Nothing here faults,
 traps or hangs a GPU.
@@ -77,7 +78,7 @@ def test_decode_wait_runs_out_then_context_recovers(orc):
             torch.as_tensor(bt, device=dev), torch.as_tensor(seq, device=dev), T)
     ws = torch.full((tq.tq_decode_workspace_bytes(ctx, B, G * Hkv, Hkv, T),), 0xFF, dtype=torch.uint8, device=dev)
     out = torch.empty((B, G * Hkv, 128), dtype=torch.float32, device=dev)
-    tq.tq_debug_stall(ctx, 1)          # the page kernel of the next decode copies no page
+    tq.tq_debug_stall(ctx, 1)          # the next decode publishes no partial result (unit 1 spans 2 CTAs)
     t0 = time.time()
     tq.tq_decode_attention(ctx, *args, out, ws, Hkv=Hkv)
     torch.cuda.synchronize()
