@@ -408,7 +408,7 @@ def main():
     def roofline(kind):
         rec = traffic_record(kind)
         r = {"kernel": "tq_compress (K and V launches)" if kind == "compress" else
-             "tq_decode_attention (prep, page kernel, merge)",
+             "tq_decode_attention (one kernel launch)",
              "bound": "hbm", "achieved": comp_gbs if kind == "compress" else dec_gbs,
              "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
              "traffic": (rec["bytes_per_call"] if rec else None)}

@@ -287,3 +287,51 @@ def test_peaked_batched_decode_power(orc):
                  "decode batched peaked x4 (3 seqs, spread %.1f)" % spread)
     del k, v, kc, vc
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("B,Hkv,G,window", [(4000, 2, 3, False), (600, 1, 5, True)])
+def test_many_short_sequences(orc, B, Hkv, G, window):
+    """Thousands of short sequences (0 to 48 tokens): more sequences than the
+    shared-memory prefix sums hold (B = 4000), dozens of units and pieces per CTA,
+    units split across CTAs, several 16-row batches per CTA in the merge (G = 3, 5),
+    empty sequences; the second case adds an fp16 residual window to every unit."""
+    import torch
+    from kv_cache_vector_02_b200 import tq, workloads as W
+    maxlen = 48
+    w = W.WORKLOADS["llama8b"].with_(Hkv=Hkv, Hq=G * Hkv)
+    o = orc.Oracle(128, 4, w.param_seed)
+    pool = _pool_cache(orc, o, w, 64, seed=51)
+    rng = np.random.default_rng(B + G)
+    nbps = maxlen // 16
+    nb = B * nbps
+    pick = rng.integers(0, 64, size=nb)
+    kc, vc = pool[0][pick], pool[1][pick]
+    bt = rng.permutation(nb).reshape(B, nbps).astype(np.int32)
+    seq = rng.integers(0, maxlen + 1, size=B).astype(np.int32)
+    seq[:3] = 0
+    seq[-2:] = 0
+    seq[B // 2] = maxlen
+    q = (rng.standard_normal((B, G * Hkv, 128)) * 2 / math.sqrt(128)).astype(np.float16)
+    ctx = gpu_ctx(4, w.param_seed, 0, 0)
+    if not window:
+        got, err = _decode_gpu(ctx, q, kc, vc, bt, seq, maxlen, Hkv)
+        assert err == 0
+        want = o.decode(q.astype(np.float64), kc, vc, bt, seq, Hkv)
+    else:
+        cap = 20
+        tk = (rng.standard_normal((B, cap, Hkv, 128)) * 2).astype(np.float16)
+        tv = rng.standard_normal((B, cap, Hkv, 128)).astype(np.float16)
+        tl = rng.integers(0, cap + 1, size=B).astype(np.int32)
+        dev = torch.device("cuda")
+        out = torch.empty((B, G * Hkv, 128), dtype=torch.float32, device=dev)
+        ws = torch.full((tq.tq_decode_workspace_bytes(ctx, B, G * Hkv, Hkv, maxlen),), 0xFF, dtype=torch.uint8, device=dev)
+        args = [torch.as_tensor(x).to(dev) for x in (q, kc, vc, bt, seq)]
+        tq.tq_decode_attention_window(ctx, *args, maxlen, torch.as_tensor(tk).to(dev), torch.as_tensor(tv).to(dev),
+                                      torch.as_tensor(tl).to(dev), out, ws, Hkv=Hkv)
+        torch.cuda.synchronize()
+        err = tq.tq_get_device_error(ctx)
+        assert err == 0
+        got = out.cpu().numpy()
+        want = o.decode(q.astype(np.float64), kc, vc, bt, seq, Hkv, tail_k=tk, tail_v=tv, tail_lens=tl)
+    assert np.all(got[seq == 0] == 0) or window
+    check_decode(got, want, "decode %d short seqs Hkv%d G%d%s" % (B, Hkv, G, " + window" if window else ""))
