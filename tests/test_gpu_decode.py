@@ -333,5 +333,26 @@ def test_many_short_sequences(orc, B, Hkv, G, window):
         assert err == 0
         got = out.cpu().numpy()
         want = o.decode(q.astype(np.float64), kc, vc, bt, seq, Hkv, tail_k=tk, tail_v=tv, tail_lens=tl)
-    assert np.all(got[seq == 0] == 0) or window
-    check_decode(got, want, "decode %d short seqs Hkv%d G%d%s" % (B, Hkv, G, " + window" if window else ""))
+    if not window:
+        assert np.all(got[seq == 0] == 0)
+    # The bar scales with the attended values: the value centroids and P enter the
+    # MMA in fp16, so an output made of one or a few tokens carries about 2^-11 of
+    # their magnitude per rounding (these sequences have 1 to 48 tokens, and the
+    # llama8b law's outlier channels reach |v| ~ 30).
+    t = [np.arange(L) for L in seq]
+    slots = np.concatenate([bt[b][tt // 16] * 16 + tt % 16 for b, tt in enumerate(t)]).astype(np.int32)
+    vals = np.abs(o.decompress_paged(1, vc, slots, Hkv)).max(axis=2)            # [tokens, Hkv]
+    vmax = np.zeros((B, Hkv))
+    starts = np.concatenate([[0], np.cumsum(seq)])[:-1]
+    has = seq > 0
+    vmax[has] = np.maximum.reduceat(vals, starts[has], axis=0)
+    if window:
+        for b in range(B):
+            if tl[b] > 0:
+                vmax[b] = np.maximum(vmax[b], np.abs(tv[b, :tl[b]].astype(np.float64)).max(axis=(0, 2)))
+    bound = DECODE_ATOL + 2.0 ** -10 * np.repeat(vmax, G, axis=1)                # [B, Hq]
+    err = np.abs(got - want).max(axis=2)
+    label = "decode %d short seqs Hkv%d G%d%s" % (B, Hkv, G, " + window" if window else "")
+    record(label, {"decode_max_abs": float(err.max()), "outputs": int(want.size),
+                   "max_err_over_bound": float((err / bound).max())})
+    assert np.all(err <= bound), (label, float(err.max()), float((err / bound).max()))
