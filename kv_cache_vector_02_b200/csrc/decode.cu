@@ -55,16 +55,16 @@
 namespace tq {
 namespace {
 
-constexpr int kNW = 12;                       // warps per split CTA (one CTA per SM, three per scheduler)
+constexpr int kNW = 8;                        // warps per CTA (one CTA per SM, two per scheduler)
 constexpr int kSplitThreads = kNW * 32;
 constexpr int kPartStride = kDim + 2;         // m, l, acc[128]
-constexpr int kStages = 4;                    // page stages per warp
+constexpr int kStages = 6;                    // page stages per warp: 3 pairs
 constexpr uint32_t kStageBytes = 2496;        // >= key chunk + value chunk at every bit width (16-byte multiple)
 constexpr uint32_t kTabAddr = 65536;          // shared-window address of the lookup tables
 constexpr uint32_t kTabBytes = 65536;         // 256 entries x 256 bytes
 // Stages: the first kLowStages below the tables (after the fields below), the rest
 // from kRingAddr on (see stage_addr).
-constexpr int kLowStages = 8;
+constexpr int kLowStages = 12;
 constexpr uint32_t kRingAddr = kTabAddr + kTabBytes;
 constexpr uint32_t kSplitSmem = kRingAddr + (kNW * kStages - kLowStages) * kStageBytes;  // any window base >= 0
 // Below the tables, from the window base: the warps' (m, l), the CTA merge area (4
@@ -75,7 +75,8 @@ constexpr uint32_t kOffLowStages = (kOffMerge + kNW * 4 * kDim * 4 + 127) & ~127
 constexpr uint32_t kLowBytes = kOffLowStages + kLowStages * kStageBytes;
 // The page prefix sums of up to kPreCap - 1 sequences sit in the rest of the window
 // below the tables (more sequences: the CTA's copy in the workspace).
-constexpr uint32_t kOffPre = kLowBytes;
+constexpr uint32_t kEpiBytes = 45056;  // the epilogue's scratch (EpiSmem) from kOffMerge on
+constexpr uint32_t kOffPre = (kLowBytes > kOffMerge + kEpiBytes ? kLowBytes : kOffMerge + kEpiBytes);
 constexpr int kPreCap = 3840;
 static_assert(kOffPre + kPreCap * 4 + 1024 <= kTabAddr, "prefix sums below the tables");
 static_assert(kSplitSmem <= 232448, "shared memory budget");
@@ -294,9 +295,11 @@ struct Pieces {
     }
 };
 
-// The pages of one warp (p0 + warp, + kNW, ...) of every piece of the CTA, in
-// order, with their block ids: lane l holds the block id of the warp's page
-// wbase + l of the piece, and the next 32 are loaded 16 pages ahead of their use.
+// The page pairs of one warp (p0 + 2 warp + {0, 1}, + 2 kNW, ...) of every piece of the
+// CTA, in order, with their block ids: lane l holds the block id of page l % 2 of
+// the warp's pair wbase + l / 2 of the piece (-2: past the piece's end), and the next
+// 16 pairs are loaded 8 pairs ahead of their use.
+constexpr int kNoPage = -2;
 struct PageCursor {
     Pieces it;
     int b, hk, p0, p1, ji, nj;
@@ -305,18 +308,18 @@ struct PageCursor {
     uint32_t kb, vb;                    // chunk bytes
     const uint8_t *kbase, *vbase;       // this lane's 16 bytes of kv head hk's chunks in physical block 0
     __device__ int load_win(const DecodeArgs& a, int warp, int lane, int base) const {
-        const int jj = base + lane;
-        return jj < nj ? a.block_table[(size_t)b * a.max_blocks + p0 + warp + jj * kNW] : -1;
+        const int jj = base + (lane >> 1), p = p0 + 2 * warp + (lane & 1) + jj * (2 * kNW);
+        return jj < nj && p < p1 ? a.block_table[(size_t)b * a.max_blocks + p] : kNoPage;
     }
     __device__ void enter(const DecodeArgs& a, int warp, int lane) {  // the next piece with pages for this warp
         live = false;
         while (it.next(a, b, hk, p0, p1)) {
-            nj = p0 + warp < p1 ? (p1 - p0 - warp + kNW - 1) / kNW : 0;
+            nj = p0 + 2 * warp < p1 ? (p1 - p0 - 2 * warp + 2 * kNW - 1) / (2 * kNW) : 0;
             if (nj == 0) continue;
             ji = 0;
             wbase = 0;
             win = load_win(a, warp, lane, 0);
-            win_next = -1;
+            win_next = kNoPage;
             kbase = a.kc + (size_t)hk * kb + 16 * lane;
             vbase = a.vc + (size_t)hk * vb + 16 * lane;
             live = true;
@@ -330,16 +333,16 @@ struct PageCursor {
         it.init(a, pre, pos, end);
         enter(a, warp, lane);
     }
-    // block id of the current page (warp-uniform; every lane calls it)
-    __device__ int block() const { return __shfl_sync(0xffffffffu, win, ji - wbase); }
+    // block id of page h (0, 1) of the current pair (warp-uniform; every lane calls it)
+    __device__ int block(int h) const { return __shfl_sync(0xffffffffu, win, 2 * (ji - wbase) + h); }
     __device__ void advance(const DecodeArgs& a, int warp, int lane) {
         ++ji;
         if (ji >= nj) {
             enter(a, warp, lane);
             return;
         }
-        if (ji - wbase == 16 && wbase + 32 < nj) win_next = load_win(a, warp, lane, wbase + 32);
-        if (ji - wbase == 32) {
+        if (ji - wbase == 8 && wbase + 16 < nj) win_next = load_win(a, warp, lane, wbase + 16);
+        if (ji - wbase == 16) {
             wbase = ji;
             win = win_next;
         }
@@ -432,15 +435,15 @@ struct KeyTerm {
     static constexpr int kSteps = KM == kKByte2 ? 16 : 8;  // 2-bit codes: 128 coordinates x 2 bit planes
 };
 
-// Scores, online softmax and the value accumulation of one page (ntok valid rows).
+// Base-2 logits of one page (ntok valid rows; 0: none): sc[nt][i][e] for rows g, g + 8
+// (i) and heads nt*8 + 2c + e.  The key term (even and odd K-steps in separate
+// accumulators) and the sign term on mma.sync.
 template <int KM, int VM, bool PROD, int NT>
-__device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, int ntok, const int (&tk)[2],
-                                             uint32_t klo0, uint32_t klo1, uint32_t khi0, uint32_t khi1,
-                                             uint32_t LA, uint32_t LB,
-                                             const uint32_t (&bq)[NT][KeyTerm<KM>::kSteps][2],
-                                             const uint32_t (&bs)[NT][8][2], float (&m)[NT][2], float (&l)[NT][2],
-                                             float (&acc)[NT][8][4]) {
-    // ---- scores: the key term (even and odd K-steps in separate accumulators) and the sign term
+__device__ __forceinline__ void page_logits(const PageRegs<KM, VM, PROD>& cur, int ntok, const int (&tk)[2],
+                                            uint32_t klo0, uint32_t klo1, uint32_t khi0, uint32_t khi1,
+                                            uint32_t LA, uint32_t LB,
+                                            const uint32_t (&bq)[NT][KeyTerm<KM>::kSteps][2],
+                                            const uint32_t (&bs)[NT][8][2], float (&sc)[NT][2][2]) {
     float d1[NT][2][4], d2[NT][2][4];  // the first MMA of each accumulator starts it
     if (KM == kKPrmt || KM == kKByte4) {
 #pragma unroll
@@ -524,71 +527,35 @@ __device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, 
     }
     const bool full = ntok >= kPage;
     const bool valid0 = full || tk[0] < ntok, valid1 = full || tk[1] < ntok;
-    uint32_t pb[NT][2];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        // ---- base-2 logits of rows g, g+8 for heads nt*8 + 2c + e
-        float sc[2][2];
-#pragma unroll
-        for (int i = 0; i < 2; ++i)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float s = cur.kn[i] * (d1[nt][0][2 * i + e] + d1[nt][1][2 * i + e]);
-                if (PROD) s = fmaf(cur.kg[i], d2[nt][0][2 * i + e] + d2[nt][1][2 * i + e], s);
-                sc[i][e] = s;
-            }
-        if (!full) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                sc[0][e] = valid0 ? sc[0][e] : -INFINITY;
-                sc[1][e] = valid1 ? sc[1][e] : -INFINITY;
-            }
-        }
-        // Lazy maximum: each lane checks its own two logits per column against
-        // m + kSlack; only when one exceeds it is the page maximum reduced over the
-        // column's lanes and the state rescaled.  l holds this lane's partial sum
-        // (its rows), reduced over the column's lanes once per piece.
-        bool over = false;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) over |= fmaxf(sc[0][e], sc[1][e]) > m[nt][e] + kSlack;
-        if (__any_sync(0xffffffffu, over)) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float mx = fmaxf(sc[0][e], sc[1][e]);
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                const float mnew = mx > m[nt][e] + kSlack ? mx : m[nt][e];
-                const float corr = ex2(m[nt][e] - mnew);  // 1 when unchanged, 0 from -inf
-                l[nt][e] *= corr;
-#pragma unroll
-                for (int mt = 0; mt < 8; ++mt) {
-                    acc[nt][mt][e] *= corr;
-                    acc[nt][mt][2 + e] *= corr;
-                }
-                m[nt][e] = mnew;
-            }
-        }
-        float pw[2][2];
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            const float p0v = ex2(sc[0][e] - m[nt][e]), p1v = ex2(sc[1][e] - m[nt][e]);
-            l[nt][e] += p0v + p1v;
-            pw[0][e] = p0v * cur.vn[0];
-            pw[1][e] = p1v * cur.vn[1];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                float x = cur.kn[i] * (d1[nt][0][2 * i + e] + d1[nt][1][2 * i + e]);
+                if (PROD) x = fmaf(cur.kg[i], d2[nt][0][2 * i + e] + d2[nt][1][2 * i + e], x);
+                sc[nt][i][e] = x;
+            }
+            if (!full) {
+                sc[nt][0][e] = valid0 ? sc[nt][0][e] : -INFINITY;
+                sc[nt][1][e] = valid1 ? sc[nt][1][e] : -INFINITY;
+            }
         }
-        // ---- P' to the B-operand layout: each 8-row half of the C fragment (row g,
-        // heads 2c, 2c + 1) transposed in registers to (rows 2c, 2c + 1, head g)
-        pb[nt][0] = movmatrix_trans(f2h2(pw[0][0], pw[0][1]));
-        pb[nt][1] = movmatrix_trans(f2h2(pw[1][0], pw[1][1]));
-    }
+}
+
+// Value accumulation of one page: acc += Vhat^T P' (v: the page's value code bytes,
+// pb: its P').
+template <int VM, int NT>
+__device__ __forceinline__ void page_values(const uint32_t (&v)[4][2], const uint32_t (&pb)[NT][2], uint32_t LA,
+                                            uint32_t LB, float (&acc)[NT][8][4]) {
     // ---- values: m-tile mt, row g -> coordinate c0(mt) of the thread's 16, row g+8 -> c0 + 1
     if (VM == kVByte4) {
         // pair bytes of rows (2c, 2c+1) and (2c+8, 2c+9): lo -> even coordinates, hi -> odd
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             constexpr uint32_t M4 = 0x0F0F0F0Fu;
-            const uint32_t A = cur.v[0][hf], B = cur.v[1][hf], C = cur.v[2][hf], D = cur.v[3][hf];
+            const uint32_t A = v[0][hf], B = v[1][hf], C = v[2][hf], D = v[3][hf];
             const uint32_t pl0 = (A & M4) | ((B << 4) & ~M4), ph0 = ((A >> 4) & M4) | (B & ~M4);
             const uint32_t pl1 = (C & M4) | ((D << 4) & ~M4), ph1 = ((C >> 4) & M4) | (D & ~M4);
 #pragma unroll
@@ -611,7 +578,7 @@ __device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, 
     } else {
         // crumb pair bytes: X -> coordinates 4m, 4m+2 of the 16, Y -> 4m+1, 4m+3
         constexpr uint32_t M2 = 0x33333333u;
-        const uint32_t A = cur.v[0][0], B = cur.v[1][0], C = cur.v[2][0], D = cur.v[3][0];
+        const uint32_t A = v[0][0], B = v[1][0], C = v[2][0], D = v[3][0];
         const uint32_t x0 = (A & M2) | ((B << 2) & ~M2), y0 = ((A >> 2) & M2) | (B & ~M2);
         const uint32_t x1 = (C & M2) | ((D << 2) & ~M2), y1 = ((C >> 2) & M2) | (D & ~M2);
 #pragma unroll
@@ -636,6 +603,68 @@ __device__ __forceinline__ void process_page(const PageRegs<KM, VM, PROD>& cur, 
     }
 }
 
+// Two pages (A, B) of one piece: logits of both, one online-softmax update over
+// their 32 rows, then both value contractions.  Lazy maximum: each lane checks its
+// own four logits per column against m + kSlack; only when one exceeds it is the
+// maximum reduced over the column's lanes and the state rescaled.  l holds this
+// lane's partial sum (its rows), reduced over the column's lanes once per piece.
+template <int KM, int VM, bool PROD, int NT>
+__device__ __forceinline__ void process_pair(const PageRegs<KM, VM, PROD>& ra, const PageRegs<KM, VM, PROD>& rb,
+                                             int ntok_a, int ntok_b, const int (&tk)[2], uint32_t klo0,
+                                             uint32_t klo1, uint32_t khi0, uint32_t khi1, uint32_t LA, uint32_t LB,
+                                             const uint32_t (&bq)[NT][KeyTerm<KM>::kSteps][2],
+                                             const uint32_t (&bs)[NT][8][2], float (&m)[NT][2], float (&l)[NT][2],
+                                             float (&acc)[NT][8][4]) {
+    float sa[NT][2][2], sb[NT][2][2];
+    page_logits<KM, VM, PROD, NT>(ra, ntok_a, tk, klo0, klo1, khi0, khi1, LA, LB, bq, bs, sa);
+    page_logits<KM, VM, PROD, NT>(rb, ntok_b, tk, klo0, klo1, khi0, khi1, LA, LB, bq, bs, sb);
+    uint32_t pa[NT][2], pbb[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        bool over = false;
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+            over |= fmaxf(fmaxf(sa[nt][0][e], sa[nt][1][e]), fmaxf(sb[nt][0][e], sb[nt][1][e])) > m[nt][e] + kSlack;
+        if (__any_sync(0xffffffffu, over)) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float mx = fmaxf(fmaxf(sa[nt][0][e], sa[nt][1][e]), fmaxf(sb[nt][0][e], sb[nt][1][e]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                const float mnew = mx > m[nt][e] + kSlack ? mx : m[nt][e];
+                const float corr = ex2(m[nt][e] - mnew);  // 1 when unchanged, 0 from -inf
+                l[nt][e] *= corr;
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    acc[nt][mt][e] *= corr;
+                    acc[nt][mt][2 + e] *= corr;
+                }
+                m[nt][e] = mnew;
+            }
+        }
+        float wa[2][2], wb[2][2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float a0 = ex2(sa[nt][0][e] - m[nt][e]), a1 = ex2(sa[nt][1][e] - m[nt][e]);
+            const float b0 = ex2(sb[nt][0][e] - m[nt][e]), b1 = ex2(sb[nt][1][e] - m[nt][e]);
+            l[nt][e] += (a0 + a1) + (b0 + b1);
+            wa[0][e] = a0 * ra.vn[0];
+            wa[1][e] = a1 * ra.vn[1];
+            wb[0][e] = b0 * rb.vn[0];
+            wb[1][e] = b1 * rb.vn[1];
+        }
+        // P' to the B-operand layout: each 8-row half of the C fragment (row g, heads
+        // 2c, 2c + 1) transposed in registers to (rows 2c, 2c + 1, head g)
+        pa[nt][0] = movmatrix_trans(f2h2(wa[0][0], wa[0][1]));
+        pa[nt][1] = movmatrix_trans(f2h2(wa[1][0], wa[1][1]));
+        pbb[nt][0] = movmatrix_trans(f2h2(wb[0][0], wb[0][1]));
+        pbb[nt][1] = movmatrix_trans(f2h2(wb[1][0], wb[1][1]));
+    }
+    page_values<VM, NT>(ra.v, pa, LA, LB, acc);
+    page_values<VM, NT>(rb.v, pbb, LA, LB, acc);
+}
+
 // Coordinate of row g of m-tile mt among the thread's 16 (16 g + c0; row g+8 -> c0 + 1).
 template <int VM>
 __device__ __forceinline__ int coord_of(int mt) {
@@ -657,8 +686,8 @@ __device__ __forceinline__ int unit_at(const DecodeArgs& a, const int* pre, long
 
 // [q' | s] = q [R | S^T] of the query heads of units u_lo .. u_hi (rows u G + h of q,
 // contiguous) into the CTA's slots (row u G + h + CTA G of qf), on mma.sync: fp16
-// inputs, fp32 accumulation; R^T enters as fp16 hi + lo, S (+-1) is exact.  rt: the
-// shared-memory copies [R^T hi | R^T lo | S], row-major fp16 with the 16-byte pieces of
+// inputs, fp32 accumulation; R^T enters as fp16 hi + lo, S (+-1) is exact and read from
+// global memory.  rt: the shared-memory copies [R^T hi | R^T lo], row-major fp16 with the 16-byte pieces of
 // row n in the order k ^ (n % 8) (the eight rows of a fragment load meet no bank
 // twice).  Per 16-row tile of q (A fragments loaded once) warp w takes the 8-column
 // output tiles w, w + kNW, ... of the 32 (q' then s), two at a time.
@@ -688,15 +717,24 @@ __device__ void rotate_queries(const DecodeArgs& a, const uint8_t* rt, int u_lo,
                 const int nt = nt0 + t * kNW;
                 const bool isq = nt < 16;
                 const int n = (nt & 15) * 8 + g;
-                const uint8_t* ph = rt + (isq ? 0 : 2 * kDim * kDim * 2) + n * kDim * 2;
+                const uint8_t* ph = rt + n * kDim * 2;
                 const uint8_t* pl = rt + kDim * kDim * 2 + n * kDim * 2;
-                if (nt < 32) {
+                const uint32_t* ps = reinterpret_cast<const uint32_t*>(a.Sh + (size_t)n * kDim);  // S: global, row-major
+                if (nt < 32 && isq) {
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
                         if (ks == 0) mma16816_z(d[t], A[0][0], A[0][1], A[0][2], A[0][3], word(ph, c), word(ph, c + 4));
                         else mma16816(d[t], A[ks][0], A[ks][1], A[ks][2], A[ks][3], word(ph, 8 * ks + c), word(ph, 8 * ks + c + 4));
-                        if (isq)
-                            mma16816(d[t], A[ks][0], A[ks][1], A[ks][2], A[ks][3], word(pl, 8 * ks + c), word(pl, 8 * ks + c + 4));
+                        mma16816(d[t], A[ks][0], A[ks][1], A[ks][2], A[ks][3], word(pl, 8 * ks + c), word(pl, 8 * ks + c + 4));
+                    }
+                } else if (nt < 32) {
+                    uint32_t sb[8][2];
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) sb[ks][0] = ps[8 * ks + c], sb[ks][1] = ps[8 * ks + c + 4];
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        if (ks == 0) mma16816_z(d[t], A[0][0], A[0][1], A[0][2], A[0][3], sb[0][0], sb[0][1]);
+                        else mma16816(d[t], A[ks][0], A[ks][1], A[ks][2], A[ks][3], sb[ks][0], sb[ks][1]);
                     }
                 }
             }
@@ -759,7 +797,7 @@ struct EpiSmem {
     float red[2][kNW][16];
     int gave_up;
 };
-static_assert(sizeof(EpiSmem) <= kOffPre - kOffMerge, "epilogue scratch fits below the prefix sums");
+static_assert(sizeof(EpiSmem) <= kEpiBytes, "epilogue scratch fits below the prefix sums");
 static_assert(2 * kDim * kDim * 2 <= (kNW * kStages - kLowStages) * kStageBytes, "R hi, lo fit the ring");
 
 // The residual window of unit u (sequence b, kv head hk) for its G heads: rows r0 + h.
@@ -869,7 +907,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_attn_kernel(DecodeArg
     extern __shared__ __align__(16) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t base = sm100::smem_u32(smem);
-    if (base + kLowBytes > kTabAddr) {  // the window leaves no room below the tables
+    if (base + kOffPre > kTabAddr) {  // the window leaves no room below the tables
         if (tid == 0) atomicOr(a.err, TQ_DEVERR_INTERNAL);
         return;
     }
@@ -878,16 +916,16 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_attn_kernel(DecodeArg
         return st < (uint32_t)kLowStages ? base + kOffLowStages + st * kStageBytes
                                          : kRingAddr + (st - kLowStages) * kStageBytes;
     };
-    // ---- prologue: R^T hi, R^T lo and S into the ring by 16-byte copies (parameters,
+    // ---- prologue: R^T hi and R^T lo into the ring by 16-byte copies (parameters,
     // nothing to wait for; row n's pieces swizzled, see rotate_queries), meanwhile the
     // page prefix sums of the sequences (exclusive; invalid lengths count as empty and
     // raise the error word), this CTA's own copy, and the lookup tables
     {
         constexpr int kPieces = kDim * kDim * 2 / 16;  // per matrix
-        for (int i = tid; i < 3 * kPieces; i += kSplitThreads) {
+        for (int i = tid; i < 2 * kPieces; i += kSplitThreads) {
             const int mtx = i / kPieces, o = (i - mtx * kPieces) * 16;
             const int n = o >> 8, k16 = (o >> 4) & 15;
-            const uint16_t* src = mtx == 0 ? a.RTh : (mtx == 1 ? a.RTl : a.Sh);
+            const uint16_t* src = mtx == 0 ? a.RTh : a.RTl;
             sm100::cp_async16(kRingAddr + mtx * (kPieces * 16) + n * 256 + ((k16 ^ (n & 7)) << 4),
                               reinterpret_cast<const uint8_t*>(src) + o);
         }
@@ -930,39 +968,43 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_attn_kernel(DecodeArg
     using P = PageGeom<KM, VM, PROD>;
     constexpr uint32_t kb = P::kBytes, vb = P::vBytes;
     static_assert(kb % 16 == 0 && vb % 16 == 0 && kb + vb <= kStageBytes, "page chunks in 16-byte pieces");
-    static_assert(3 * kDim * kDim * 2 <= (kNW * kStages - kLowStages) * kStageBytes, "R^T, S fit the ring");
+    static_assert(2 * kDim * kDim * 2 <= (kNW * kStages - kLowStages) * kStageBytes, "R^T hi, lo fit the ring");
     const size_t kstride = (size_t)a.Hkv * kb, vstride = (size_t)a.Hkv * vb;  // bytes per physical block
 
-    // ---- this warp's page stream: the issue cursor runs kStages pages ahead; page k of
-    // the warp goes to stage k % kStages as 16-byte copies by every lane, one commit
-    // group per page (empty past the end), so waiting for all but the newest
-    // kStages - 1 groups means page k has landed.  vmask bit s: stage s holds a page
-    // with a valid block id.
+    // ---- this warp's page stream, by pairs of pages: the issue cursor runs kPairs pairs
+    // ahead; pair k of the warp goes to stages 2 (k % kPairs) and + 1 as 16-byte copies
+    // by every lane, one commit group per pair (empty past the end), so waiting for all
+    // but the newest kPairs - 1 groups means pair k has landed.  vmask bit s: stage s
+    // holds a page with a valid block id.
+    constexpr int kPairs = kStages / 2;
     PageCursor icur;
     icur.init(a, pre, pos0, end, warp, lane, kb, vb);
     uint32_t issued = 0, vmask = 0;
     // the warp's stages are consecutive (kLowStages is a multiple of kStages)
-    static_assert(kLowStages % kStages == 0, "a warp's stages in one region");
+    static_assert(kLowStages % kStages == 0 && kStages % 2 == 0, "a warp's stages in one region, in pairs");
     const uint32_t wstage_addr = stage_addr(warp * kStages) + 16 * lane;
     const uint8_t* wstage = smem + (stage_addr(warp * kStages) - base);
     auto issue_next = [&]() {
         if (icur.live) {
-            const int blk = icur.block();
-            const uint32_t s = issued % kStages;
-            const bool v = blk >= 0 && blk < a.num_blocks;
-            vmask = (vmask & ~(1u << s)) | ((uint32_t)v << s);
-            if (v) {
-                const uint32_t dst = wstage_addr + s * kStageBytes;
-                const uint8_t* ks = icur.kbase + (size_t)blk * kstride;
-                const uint8_t* vs = icur.vbase + (size_t)blk * vstride;
 #pragma unroll
-                for (int i = 0; i < (int)(kb / 512 + 1); ++i)
-                    if (i * 32 + lane < (int)(kb / 16)) sm100::cp_async16(dst + 512 * i, ks + 512 * i);
+            for (int h = 0; h < 2; ++h) {
+                const int blk = icur.block(h);
+                const uint32_t s = 2 * (issued % kPairs) + h;
+                const bool v = blk >= 0 && blk < a.num_blocks;
+                vmask = (vmask & ~(1u << s)) | ((uint32_t)v << s);
+                if (v) {
+                    const uint32_t dst = wstage_addr + s * kStageBytes;
+                    const uint8_t* ks = icur.kbase + (size_t)blk * kstride;
+                    const uint8_t* vs = icur.vbase + (size_t)blk * vstride;
 #pragma unroll
-                for (int i = 0; i < (int)(vb / 512 + 1); ++i)
-                    if (i * 32 + lane < (int)(vb / 16)) sm100::cp_async16(dst + kb + 512 * i, vs + 512 * i);
-            } else if (lane == 0) {
-                atomicOr(a.err, TQ_DEVERR_BLOCK);
+                    for (int i = 0; i < (int)(kb / 512 + 1); ++i)
+                        if (i * 32 + lane < (int)(kb / 16)) sm100::cp_async16(dst + 512 * i, ks + 512 * i);
+#pragma unroll
+                    for (int i = 0; i < (int)(vb / 512 + 1); ++i)
+                        if (i * 32 + lane < (int)(vb / 16)) sm100::cp_async16(dst + kb + 512 * i, vs + 512 * i);
+                } else if (blk != kNoPage && lane == 0) {
+                    atomicOr(a.err, TQ_DEVERR_BLOCK);
+                }
             }
             icur.advance(a, warp, lane);
         }
@@ -970,7 +1012,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_attn_kernel(DecodeArg
         ++issued;
     };
 #pragma unroll 1
-    for (int i = 0; i < kStages; ++i) issue_next();
+    for (int i = 0; i < kPairs; ++i) issue_next();
 
     // ---------------------------------------------------------------- pages
     const int g = lane >> 2, c = lane & 3;
@@ -1057,24 +1099,28 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_attn_kernel(DecodeArg
             for (int mt = 0; mt < 8; ++mt) acc[nt][mt][0] = acc[nt][mt][1] = acc[nt][mt][2] = acc[nt][mt][3] = 0.f;
         }
 
-        // ---- the warp's pages of the piece: p0 + warp, + kNW, ...
-        const int nj = p0 + warp < p1 ? (p1 - p0 - warp + kNW - 1) / kNW : 0;
+        // ---- the warp's page pairs of the piece: p0 + 2 warp + {0, 1}, + 2 kNW, ...
+        const int nj = p0 + 2 * warp < p1 ? (p1 - p0 - 2 * warp + 2 * kNW - 1) / (2 * kNW) : 0;
         for (int j = 0; j < nj; ++j) {
-            const uint32_t s = cnt % kStages;
-            sm100::cp_async_wait<kStages - 1>();  // this lane's copies of the page
-            __syncwarp();                           // ... and every other lane's
-            const int page = p0 + warp + j * kNW;
-            // the page's bytes into registers, then the stage goes back to the stream
-            // before the page is worked, so every stage is in flight meanwhile
-            const bool vp = (vmask >> s) & 1u;
-            PageRegs<KM, VM, PROD> r;
-            if (vp) load_page<KM, VM, PROD>(r, wstage + s * kStageBytes, po, a.qscale, a.sscale);
-            __syncwarp();  // every lane is done with the stage before it is refilled
+            const uint32_t s = 2 * (cnt % kPairs);
+            sm100::cp_async_wait<kPairs - 1>();  // this lane's copies of the pair
+            __syncwarp();                          // ... and every other lane's
+            const int page = p0 + 2 * warp + j * (2 * kNW);
+            // the pages' bytes into registers, then the stages go back to the stream
+            // before the pages are worked, so every stage is in flight meanwhile
+            const bool va = (vmask >> s) & 1u, vbb = (vmask >> (s + 1)) & 1u;
+            PageRegs<KM, VM, PROD> ra, rb;
+            if (va) load_page<KM, VM, PROD>(ra, wstage + s * kStageBytes, po, a.qscale, a.sscale);
+            else ra = PageRegs<KM, VM, PROD>{};
+            if (vbb) load_page<KM, VM, PROD>(rb, wstage + (s + 1) * kStageBytes, po, a.qscale, a.sscale);
+            else rb = PageRegs<KM, VM, PROD>{};
+            __syncwarp();  // every lane is done with the stages before they are refilled
             ++cnt;
             issue_next();
-            if (vp)
-                process_page<KM, VM, PROD, NT>(r, min(kPage, Ls - page * kPage), tk, klo0, klo1, khi0, khi1, LA, LB,
-                                               bq, bs, m, l, acc);
+            const int ntok_a = va ? min(kPage, Ls - page * kPage) : 0;
+            const int ntok_b = vbb && page + 1 < p1 ? min(kPage, Ls - (page + 1) * kPage) : 0;
+            process_pair<KM, VM, PROD, NT>(ra, rb, ntok_a, ntok_b, tk, klo0, klo1, khi0, khi1, LA, LB, bq, bs, m, l,
+                                           acc);
         }
 
         // ---- merge the CTA's warps (one tile of 8 heads at a time; coordinates back in order)
@@ -1281,7 +1327,6 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_attn_kernel(DecodeArg
             for (int t = 0; t < 2; ++t) {
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) d[t][e4] = 0.f;
-#pragma unroll
                 const int i = (warp + 8 * t) * 8 + g;
                 const uint8_t* rh = rsm + i * 256;
                 const uint8_t* rl = rsm + kDim * kDim * 2 + i * 256;
