@@ -11,18 +11,18 @@
 //
 // One kernel (decode_attn_kernel), cooperative: one persistent CTA per SM over an
 // equal range of the pages of all (sequence, kv head) units, all CTAs resident.
-//   prologue  R^T (fp16 hi, lo) and S staged in shared memory; the CTA's own page
-//             prefix sums of the sequences; the lookup tables; q' = R^T q and s = S q
-//             of the units of the range (mma.sync) into the CTA's workspace slots.
-//   pages     page p of a unit's piece (the range's part of one unit) goes to warp
-//             p % kNW.  Each warp streams its own pages (16-byte async copies by
-//             every lane of the key and the value chunk, one commit group per page)
-//             into its ring of shared-memory stages, its issue cursor running ahead
-//             across pieces, and per 16-token page:
+//   prologue  R^T (fp16 hi, lo) staged in shared memory; the CTA's own page prefix
+//             sums of the sequences; the lookup tables; q' = R^T q and s = S q of the
+//             units of the range (mma.sync) into the CTA's workspace slots.
+//   pages     pages p, p + 1 (p = 2 (w + kNW j)) of a unit's piece (the range's part
+//             of one unit) go to warp w.  Each warp streams its own pairs of pages
+//             (16-byte async copies by every lane of the key and the value chunks,
+//             one commit group per pair) into its ring of shared-memory stages, its
+//             issue cursor running ahead across pieces, and per pair of 16-token pages:
 //               scores  D[16 tok x 8 heads] = sum_k Khat[tok][k] q'[k][h]  (mma m16n8k16)
-//                       plus the sign term with +-1 fragments against s
-//               softmax online, base 2, per head column
-//               values  D[16 coords x 8 heads] += Vhat^T[coord][tok] P'[tok][h]
+//                       plus the sign term with +-1 fragments against s, per page
+//               softmax online, base 2, per head column, one update for both pages
+//               values  D[16 coords x 8 heads] += Vhat^T[coord][tok] P'[tok][h], per page
 //             The warps of the CTA merge their states per piece into the slot (unit
 //             + CTA); a piece that does not start its unit publishes the slot with
 //             the launch's tag.
