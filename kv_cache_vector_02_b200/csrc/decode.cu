@@ -691,6 +691,7 @@ __device__ __forceinline__ int unit_at(const DecodeArgs& a, const int* pre, long
 // row n in the order k ^ (n % 8) (the eight rows of a fragment load meet no bank
 // twice).  Per 16-row tile of q (A fragments loaded once) warp w takes the 8-column
 // output tiles w, w + kNW, ... of the 32 (q' then s), two at a time.
+static_assert(kNW == 8, "rotate_queries: warp w takes the output tiles w, w + 8 (q') and w + 16, w + 24 (s)");
 __device__ void rotate_queries(const DecodeArgs& a, const uint8_t* rt, int u_lo, int u_hi, int warp, int lane) {
     const int g = lane >> 2, c = lane & 3;
     const int r_lo = u_lo * a.G, r_end = (u_hi + 1) * a.G;
@@ -698,6 +699,15 @@ __device__ void rotate_queries(const DecodeArgs& a, const uint8_t* rt, int u_lo,
     auto word = [&](const uint8_t* row, int w) {  // word w of a row: piece (w / 4) ^ g, word w % 4
         return *reinterpret_cast<const uint32_t*>(row + ((((w >> 2) ^ g) << 4) | ((w & 3) << 2)));
     };
+    // S fragments of the tiles w + 16, w + 24 (rows 8 (w + 8 t) + g of S), loaded with
+    // the first tile's q rows
+    uint32_t sb[2][8][2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const uint32_t* ps = reinterpret_cast<const uint32_t*>(a.Sh + (size_t)((warp + 8 * t) * 8 + g) * kDim);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) sb[t][ks][0] = ps[8 * ks + c], sb[t][ks][1] = ps[8 * ks + c + 4];
+    }
     for (int r0 = r_lo; r0 < r_end; r0 += 16) {
         const bool v0 = r0 + g < r_end, v1 = r0 + g + 8 < r_end;
         const uint32_t* q0 = reinterpret_cast<const uint32_t*>(a.q + (size_t)(v0 ? r0 + g : r_lo) * kDim);
@@ -710,46 +720,30 @@ __device__ void rotate_queries(const DecodeArgs& a, const uint8_t* rt, int u_lo,
             A[ks][2] = v0 ? q0[8 * ks + c + 4] : 0u;
             A[ks][3] = v1 ? q1[8 * ks + c + 4] : 0u;
         }
-        for (int nt0 = warp; nt0 < 32; nt0 += 2 * kNW) {
-            float d[2][4];
+        float d[4][4];  // tiles w, w + 8 (q'), w + 16, w + 24 (s): four independent chains
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {  // two independent accumulation chains
-                const int nt = nt0 + t * kNW;
-                const bool isq = nt < 16;
-                const int n = (nt & 15) * 8 + g;
-                const uint8_t* ph = rt + n * kDim * 2;
-                const uint8_t* pl = rt + kDim * kDim * 2 + n * kDim * 2;
-                const uint32_t* ps = reinterpret_cast<const uint32_t*>(a.Sh + (size_t)n * kDim);  // S: global, row-major
-                if (nt < 32 && isq) {
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        if (ks == 0) mma16816_z(d[t], A[0][0], A[0][1], A[0][2], A[0][3], word(ph, c), word(ph, c + 4));
-                        else mma16816(d[t], A[ks][0], A[ks][1], A[ks][2], A[ks][3], word(ph, 8 * ks + c), word(ph, 8 * ks + c + 4));
-                        mma16816(d[t], A[ks][0], A[ks][1], A[ks][2], A[ks][3], word(pl, 8 * ks + c), word(pl, 8 * ks + c + 4));
-                    }
-                } else if (nt < 32) {
-                    uint32_t sb[8][2];
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) sb[ks][0] = ps[8 * ks + c], sb[ks][1] = ps[8 * ks + c + 4];
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        if (ks == 0) mma16816_z(d[t], A[0][0], A[0][1], A[0][2], A[0][3], sb[0][0], sb[0][1]);
-                        else mma16816(d[t], A[ks][0], A[ks][1], A[ks][2], A[ks][3], sb[ks][0], sb[ks][1]);
-                    }
-                }
-            }
+        for (int ks = 0; ks < 8; ++ks) {
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
-                const int nt = nt0 + t * kNW;
-                if (nt >= 32) continue;
-                const int col = (nt & 15) * 8 + 2 * c, which = nt < 16 ? 0 : 1;
-                if (v0)
-                    *reinterpret_cast<float2*>(a.qf + ((slot_rows + r0 + g) * 2 + which) * kDim + col) =
-                        make_float2(d[t][0], d[t][1]);
-                if (v1)
-                    *reinterpret_cast<float2*>(a.qf + ((slot_rows + r0 + g + 8) * 2 + which) * kDim + col) =
-                        make_float2(d[t][2], d[t][3]);
+                const int n = (warp + 8 * t) * 8 + g;
+                const uint8_t* ph = rt + n * kDim * 2;
+                const uint8_t* pl = rt + kDim * kDim * 2 + n * kDim * 2;
+                if (ks == 0) mma16816_z(d[t], A[0][0], A[0][1], A[0][2], A[0][3], word(ph, c), word(ph, c + 4));
+                else mma16816(d[t], A[ks][0], A[ks][1], A[ks][2], A[ks][3], word(ph, 8 * ks + c), word(ph, 8 * ks + c + 4));
+                mma16816(d[t], A[ks][0], A[ks][1], A[ks][2], A[ks][3], word(pl, 8 * ks + c), word(pl, 8 * ks + c + 4));
+                if (ks == 0) mma16816_z(d[2 + t], A[0][0], A[0][1], A[0][2], A[0][3], sb[t][0][0], sb[t][0][1]);
+                else mma16816(d[2 + t], A[ks][0], A[ks][1], A[ks][2], A[ks][3], sb[t][ks][0], sb[t][ks][1]);
             }
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int col = (warp + 8 * (t & 1)) * 8 + 2 * c, which = t >> 1;
+            if (v0)
+                *reinterpret_cast<float2*>(a.qf + ((slot_rows + r0 + g) * 2 + which) * kDim + col) =
+                    make_float2(d[t][0], d[t][1]);
+            if (v1)
+                *reinterpret_cast<float2*>(a.qf + ((slot_rows + r0 + g + 8) * 2 + which) * kDim + col) =
+                    make_float2(d[t][2], d[t][3]);
         }
     }
 }
