@@ -326,6 +326,18 @@ class Oracle:
             raise ValueError("block id or sequence length out of range")
         return out
 
+    def prefill(self, q, kcache, vcache, block_table, q_start: int, Hkv: int, scale=None):
+        """Causal prefill attention of one sequence over its paged cache: q [Tq, Hq, d]
+        are the queries at positions q_start .. q_start + Tq - 1, whose keys and values
+        are already in the cache; query i attends to the tokens 0 .. q_start + i with the
+        decode estimator.  It is the decode of Tq sequences that share the block table,
+        query i's of length q_start + i + 1."""
+        q = _f64(q)
+        Tq = q.shape[0]
+        bt = np.tile(np.ascontiguousarray(block_table, np.int32).reshape(1, -1), (Tq, 1))
+        lens = (q_start + 1 + np.arange(Tq)).astype(np.int32)
+        return self.decode(q, kcache, vcache, bt, lens, Hkv, scale)
+
     def _decode_window(self, q, kcache, vcache, block_table, seq_lens, Hkv, scale, form, tail_k, tail_v, tail_lens):
         q = _f64(q)
         B, Hq, d = q.shape
