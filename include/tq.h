@@ -250,6 +250,30 @@ TQ_API tq_status tq_decode_attention_window(const tq_ctx* ctx, const uint16_t* q
                                             int out_fp32, void* workspace_dev, size_t workspace_bytes, void* stream);
 
 /*
+ * tq_prefill_attention -- causal attention of a chunk of queries of one sequence over
+ * the sequence's compressed, paged cache [FQ-TQ "架构设计": the fused prefill attention
+ * kernel, the compressed keys dequantized inline; estimator of "注意力计算的特殊挑战与
+ * QJL校正"].  Query i (position q_start + i) attends to the tokens 0 .. q_start + i,
+ * whose keys and values must already be in the cache (compress the chunk first):
+ *   s_t = scale * ( <q_i, k_hat_t> + gamma_t*sqrt(pi/2)/d * <S q_i, 2 sigma_t - 1> ),
+ *   o_i = sum_{t <= q_start + i} softmax(s)_t * v_hat_t.
+ * (Reading: the pages name the kernel and its inline decompression; the causal
+ * prefix and the decode's estimator are the plainest reading.)
+ *   q_dev          : [Tq][Hq][128] fp16, device, 16-byte aligned.
+ *   block_table_dev: [max_blocks] int32, device; page p of the sequence lives in
+ *                    physical block block_table[p].  A block id outside
+ *                    [0, num_blocks) skips the page and sets TQ_DEVERR_BLOCK.
+ *   q_start + Tq   : <= max_blocks * 16 (TQ_ERR_INVALID_ARG otherwise).
+ *   scale          : softmax scale; 0 for the default 1/sqrt(d).
+ *   out_dev        : [Tq][Hq][128], fp16 (out_fp32 = 0) or fp32 (out_fp32 = 1).
+ * No workspace.  One kernel launch; Tq = 0 launches nothing.
+ */
+TQ_API tq_status tq_prefill_attention(const tq_ctx* ctx, const uint16_t* q_dev, const uint8_t* k_cache_dev,
+                                      const uint8_t* v_cache_dev, int num_blocks, const int32_t* block_table_dev,
+                                      int max_blocks, int q_start, int Tq, int Hq, int Hkv, float scale, void* out_dev,
+                                      int out_fp32, void* stream);
+
+/*
  * Size of the device array behind tq_decode_attention_noalloc.  Every GPU that
  * loads libtq reserves this much device memory for it until the process exits.
  */

@@ -50,6 +50,7 @@
 #include <mutex>
 
 #include "device_util.cuh"
+#include "mma_sync.cuh"
 #include "sm100.cuh"
 
 namespace tq {
@@ -128,25 +129,6 @@ __device__ __forceinline__ bool seq_len_ok(const DecodeArgs& a, int L) {
 
 // ------------------------------------------------------------------ helpers
 
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// D = A B (no accumulator input).
-__device__ __forceinline__ void mma16816_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                           uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%10,%10,%10,%10};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
-}
-
 // Transpose of an 8x8 fp16 matrix held as m8n8 fragments (thread 4 g + c holds row g,
 // columns 2c, 2c + 1): afterwards it holds row g of the transpose.
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
@@ -154,11 +136,6 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
     asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
     return d;
 }
-
-__device__ __forceinline__ uint32_t h2bits(__half lo, __half hi) {
-    return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
-}
-__device__ __forceinline__ uint32_t f2h2(float lo, float hi) { return h2bits(__float2half_rn(lo), __float2half_rn(hi)); }
 
 __device__ __forceinline__ __half cb_half(const Codebook& cb, int code) {
     float v = 0.f;
@@ -618,6 +595,14 @@ __device__ __forceinline__ void process_pair(const PageRegs<KM, VM, PROD>& ra, c
     float sa[NT][2][2], sb[NT][2][2];
     page_logits<KM, VM, PROD, NT>(ra, ntok_a, tk, klo0, klo1, khi0, khi1, LA, LB, bq, bs, sa);
     page_logits<KM, VM, PROD, NT>(rb, ntok_b, tk, klo0, klo1, khi0, khi1, LA, LB, bq, bs, sb);
+    // value norms of the rows past a page's valid tokens are not used (a partial page's
+    // unused rows may hold anything)
+    float van[2], vbn[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        van[i] = (ntok_a >= kPage || tk[i] < ntok_a) ? ra.vn[i] : 0.f;
+        vbn[i] = (ntok_b >= kPage || tk[i] < ntok_b) ? rb.vn[i] : 0.f;
+    }
     uint32_t pa[NT][2], pbb[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -649,10 +634,10 @@ __device__ __forceinline__ void process_pair(const PageRegs<KM, VM, PROD>& ra, c
             const float a0 = ex2(sa[nt][0][e] - m[nt][e]), a1 = ex2(sa[nt][1][e] - m[nt][e]);
             const float b0 = ex2(sb[nt][0][e] - m[nt][e]), b1 = ex2(sb[nt][1][e] - m[nt][e]);
             l[nt][e] += (a0 + a1) + (b0 + b1);
-            wa[0][e] = a0 * ra.vn[0];
-            wa[1][e] = a1 * ra.vn[1];
-            wb[0][e] = b0 * rb.vn[0];
-            wb[1][e] = b1 * rb.vn[1];
+            wa[0][e] = a0 * van[0];
+            wa[1][e] = a1 * van[1];
+            wb[0][e] = b0 * vbn[0];
+            wb[1][e] = b1 * vbn[1];
         }
         // P' to the B-operand layout: each 8-row half of the C fragment (row g, heads
         // 2c, 2c + 1) transposed in registers to (rows 2c, 2c + 1, head g)

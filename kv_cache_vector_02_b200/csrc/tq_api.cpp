@@ -364,6 +364,25 @@ tq_status tq_decode_attention(const tq_ctx* ctx, const uint16_t* q, const uint8_
                          max_seq_len, tq::DecodeTail{}, scale, out, out_fp32, workspace, workspace_bytes, stream);
 }
 
+tq_status tq_prefill_attention(const tq_ctx* ctx, const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                               int num_blocks, const int32_t* block_table, int max_blocks, int q_start, int Tq, int Hq,
+                               int Hkv, float scale, void* out, int out_fp32, void* stream) {
+    if (!ctx || ctx->host_only || Tq < 0 || q_start < 0 || Hq < 1 || Hkv < 1 || max_blocks < 0 || num_blocks < 0)
+        return TQ_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return TQ_ERR_INVALID_ARG;
+    if (Tq == 0) return TQ_OK;
+    if ((long long)q_start + Tq > (long long)max_blocks * tq::kPage) return TQ_ERR_INVALID_ARG;
+    if (!q || !k_cache || !v_cache || !block_table || !out) return TQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return TQ_ERR_INVALID_ARG;
+    if (!(scale >= 0.f) || !std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
+    if (scale == 0.f) scale = 1.0f / std::sqrt(float(kDim));
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (tq::launch_prefill(ctx, q, k_cache, v_cache, num_blocks, block_table, max_blocks, q_start, Tq, Hq, Hkv, scale,
+                           out, out_fp32, s) != cudaSuccess)
+        return TQ_ERR_CUDA;
+    return note_use(ctx, s) ? TQ_OK : TQ_ERR_CUDA;
+}
+
 tq_status tq_decode_attention_window(const tq_ctx* ctx, const uint16_t* q, const uint8_t* k_cache,
                                      const uint8_t* v_cache, int num_blocks, const int32_t* block_table,
                                      int max_blocks, const int32_t* seq_lens, int B, int Hq, int Hkv,

@@ -134,6 +134,10 @@ struct DecodeTail {
     int cap = 0;
 };
 constexpr int kDecodeTailMax = 256;
+// Causal prefill attention of one sequence (queries at q_start .. q_start + Tq - 1).
+cudaError_t launch_prefill(const tq_ctx* ctx, const uint16_t* q, const uint8_t* kc, const uint8_t* vc, int num_blocks,
+                           const int32_t* block_table, int max_blocks, int q_start, int Tq, int Hq, int Hkv, float scale,
+                           void* out, int out_fp32, cudaStream_t stream);
 cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const uint16_t* q, const uint8_t* kc,
                           const uint8_t* vc, int num_blocks, const int32_t* block_table, int max_blocks,
                           const int32_t* seq_lens, int B, int Hq, int Hkv, int max_seq_len, const DecodeTail& tail,

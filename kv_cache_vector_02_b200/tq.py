@@ -27,6 +27,7 @@ FLAG_SPHERE_CODEBOOK, FLAG_HOST_ONLY = 0x1, 0x4
 
 EXPORTED = ("tq_init", "tq_init_ex", "tq_init_host", "tq_destroy", "tq_chunk_bytes", "tq_code_bits", "tq_export_params", "tq_compress",
             "tq_decompress", "tq_decode_workspace_bytes", "tq_decode_attention", "tq_decode_attention_window",
+            "tq_prefill_attention",
             "tq_decode_attention_noalloc",
             "tq_get_device_error", "tq_debug_stall", "tq_launch_count", "tq_status_string")
 
@@ -55,6 +56,7 @@ def _load():
         "tq_decode_workspace_bytes": (Z, [P, I, I, I, I]),
         "tq_decode_attention": (I, [P, P, P, P, I, P, I, P, I, I, I, I, F, P, I, P, Z, P]),
         "tq_decode_attention_window": (I, [P, P, P, P, I, P, I, P, I, I, I, I, P, P, P, I, F, P, I, P, Z, P]),
+        "tq_prefill_attention": (I, [P, P, P, P, I, P, I, I, I, I, I, F, P, I, P]),
         "tq_decode_attention_noalloc": (I, [P, P, P, P, I, P, I, P, I, I, I, I, F, P, I, P]),
         "tq_get_device_error": (I, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
         "tq_debug_stall": (I, [P, I]),
@@ -264,6 +266,27 @@ def tq_decode_attention_window(ctx: Context, q, k_cache, v_cache, block_table, s
                                            float(scale), _ptr(out), 1 if out.dtype == torch.float32 else 0,
                                            _ptr(workspace), int(workspace.numel() * workspace.element_size()),
                                            _stream(stream)), what)
+
+
+def tq_prefill_attention(ctx: Context, q, k_cache, v_cache, block_table, q_start: int, out, scale: float = 0.0,
+                         Hkv: int | None = None, stream=None):
+    """Causal prefill attention of one sequence: q [Tq, Hq, 128] fp16 at positions
+    q_start .. q_start + Tq - 1, block_table [max_blocks] int32, out [Tq, Hq, 128]
+    fp16 or fp32 (see tq.h)."""
+    import torch
+    Tq, Hq = int(q.shape[0]), int(q.shape[1])
+    if Hkv is None:
+        Hkv = int(k_cache.shape[1])
+    what = "tq_prefill_attention"
+    _expect(q, (Tq, Hq, ctx.head_dim), (torch.float16,), what, "q")
+    _expect(k_cache, (None, Hkv, tq_chunk_bytes(ctx, KIND_KEY)), (torch.uint8,), what, "k_cache")
+    _expect(v_cache, (int(k_cache.shape[0]), Hkv, tq_chunk_bytes(ctx, KIND_VALUE)), (torch.uint8,), what, "v_cache")
+    _expect(block_table, (None,), (torch.int32,), what, "block_table")
+    _expect(out, (Tq, Hq, ctx.head_dim), (torch.float16, torch.float32), what, "out")
+    _check(_lib.tq_prefill_attention(ctx.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache), int(k_cache.shape[0]),
+                                     _ptr(block_table), int(block_table.shape[0]), int(q_start), Tq, Hq, Hkv,
+                                     float(scale), _ptr(out), 1 if out.dtype == torch.float32 else 0,
+                                     _stream(stream)), what)
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20

@@ -356,3 +356,29 @@ def test_many_short_sequences(orc, B, Hkv, G, window):
     record(label, {"decode_max_abs": float(err.max()), "outputs": int(want.size),
                    "max_err_over_bound": float((err / bound).max())})
     assert np.all(err <= bound), (label, float(err.max()), float((err / bound).max()))
+
+
+def test_partial_pages_ignore_unused_rows(orc):
+    """The unused rows of each sequence's last page hold 0xFF bytes (NaN norms, maximal
+    codes): the decode reads only the sequence's tokens."""
+    o = orc.Oracle(128, 4, 31)
+    rng = np.random.default_rng(31)
+    B, Hkv, G, maxlen = 5, 2, 4, 100
+    nbps = (maxlen + 15) // 16
+    nb = B * nbps
+    bt = rng.permutation(nb).reshape(B, nbps).astype(np.int32)
+    seq = np.array([100, 1, 37, 64, 85], np.int32)
+    kc = np.full_like(o.new_cache(0, nb, Hkv), 0xFF)
+    vc = np.full_like(o.new_cache(1, nb, Hkv), 0xFF)
+    for b in range(B):
+        t = np.arange(seq[b])
+        sl = (bt[b][t // 16] * 16 + t % 16).astype(np.int32)
+        o.compress_paged(0, (rng.standard_normal((seq[b], Hkv, 128)) * 2).astype(np.float16), sl, kc)
+        o.compress_paged(1, rng.standard_normal((seq[b], Hkv, 128)).astype(np.float16), sl, vc)
+    q = (rng.standard_normal((B, G * Hkv, 128)) / math.sqrt(128)).astype(np.float16)
+    ctx = gpu_ctx(4, 31, 0, 0)
+    got, err = _decode_gpu(ctx, q, kc, vc, bt, seq, maxlen, Hkv)
+    assert err == 0
+    assert np.all(np.isfinite(got))
+    want = o.decode(q.astype(np.float64), kc, vc, bt, seq, Hkv)
+    check_decode(got, want, "decode with 0xFF in unused page rows")
