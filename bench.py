@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--rotation", default="haar", choices=["haar", "hadamard"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill", action="store_true",
+                    help="time the causal prefill attention of one sequence of the workload instead (1 GPU)")
     return ap.parse_args()
 
 
@@ -321,10 +323,71 @@ def bench_slots(w):
 
 
 # ---------------------------------------------------------------- GPU arm
+def run_prefill(args):
+    """Causal prefill attention of the workload's first sequence (all T tokens as one
+    chunk) over its compressed cache: one JSON line, attended (query head, token) pairs
+    per second, and the tensor-pipe roofline of its contractions."""
+    import numpy as np
+    import torch
+    from kv_cache_vector_02_b200 import tq, workloads as W
+    dev = torch.device("cuda")
+    rot = 1 if args.rotation == "hadamard" else 0
+    w = W.WORKLOADS[args.workload].with_(bits=args.bits, rotation=rot, decode_steps=0, B=1)
+    ctx = tq.tq_init(D, w.bits, w.param_seed, w.rotation, w.key_mode)
+    slots_np, bt_np = bench_slots(w)
+    slots = torch.as_tensor(slots_np, device=dev)
+    ck, cv = tq.tq_chunk_bytes(ctx, tq.KIND_KEY), tq.tq_chunk_bytes(ctx, tq.KIND_VALUE)
+    kc = torch.zeros((w.num_blocks, w.Hkv, ck), dtype=torch.uint8, device=dev)
+    vc = torch.zeros((w.num_blocks, w.Hkv, cv), dtype=torch.uint8, device=dev)
+    tq.tq_compress(ctx, W.gen_kv(w, 0, device=dev), W.gen_kv(w, 1, device=dev), slots, kc, vc)
+    Tq = w.T
+    q = (torch.randn((Tq, w.Hq, D), device=dev, generator=torch.Generator(device=dev).manual_seed(5)) /
+         math.sqrt(D)).to(torch.float16)
+    bt = torch.as_tensor(np.asarray(bt_np)[0], device=dev)
+    out = torch.empty((Tq, w.Hq, D), dtype=torch.float16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        tq.tq_prefill_attention(ctx, q, kc, vc, bt, 0, out)
+    torch.cuda.synchronize()
+    steps = min(args.steps, 50)
+    ts = []
+    for i in range(steps):
+        flush.fill_(i & 0xff)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        tq.tq_prefill_attention(ctx, q, kc, vc, bt, 0, out)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    if tq.tq_get_device_error(ctx) != 0:
+        raise RuntimeError("device error word set during the prefill")
+    ms = statistics.median(ts)
+    pairs = w.Hq * Tq * (Tq + 1) / 2  # attended (query head, token) pairs, causal
+    per_pair = (6 if w.key_mode == 0 else 4) * D  # QK^T (+ the QJL sign term) and PV, 2 flops per MAC
+    tflops = pairs * per_pair / (ms * 1e-3) / 1e12
+    peak = None
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak = float(json.load(f)["bf16_tflops"])
+    except Exception:
+        peak = None
+    line = {"metric": "prefill attention (query head, token) pairs/s over the compressed cache", "impl": "tq",
+            "value": pairs / (ms * 1e-3), "unit": "pairs/s", "ms": ms, "higher_is_better": True, "n_gpus": 1,
+            "steps": steps, "dtype": "f16 operands, f32 accumulate", "data": "synthetic",
+            "config": {"workload": "%s: one sequence of %d tokens as one causal chunk, %d kv / %d q heads, TQ%d, %s"
+                       % (w.name, Tq, w.Hkv, w.Hq, w.bits, args.rotation), "l2": "flushed (256 MB write) before each call"},
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": (tflops / peak) if peak else None,
+                         "flops": "%d per attended pair (QK^T, QJL sign term, PV)" % per_pair}}
+    print(json.dumps(line))
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.prefill:
+        return run_prefill(args)
     ws, rank, local = dist_setup("nccl")
     import numpy as np
     import torch

@@ -12,7 +12,7 @@
 // (+ the sign term against S q), values accumulated as sum_t p_t n_t c[idx_t]/sqrt(d)
 // and un-rotated once per query row (o = R acc / l).
 //
-// One CTA of 4 warps per (block of 64 queries, query head); warp w takes 16 queries.
+// One CTA of 8 warps per (block of 128 queries, query head); warp w takes 16 queries.
 //   prologue  R^T (fp16 hi, lo) and S staged in shared memory (16-byte async copies,
 //             rows swizzled); each warp computes q' and s of its 16 queries on
 //             mma.sync and keeps them as fp16 A fragments in registers.
@@ -32,7 +32,7 @@
 namespace tq {
 namespace {
 
-constexpr int kPW = 4;                 // warps per CTA
+constexpr int kPW = 8;                 // warps per CTA
 constexpr int kPThreads = kPW * 32;
 constexpr int kPQ = 16 * kPW;          // queries per CTA
 constexpr int kKS = kDim + 8;          // K / sign tile row stride (halves): rows 16 bytes apart in banks
@@ -95,38 +95,60 @@ __device__ __forceinline__ uint64_t load_codes16(const uint8_t* row, int t8, int
     return *reinterpret_cast<const uint16_t*>(row + 2 * t8);
 }
 
-// The page's key codes, sign bits and value codes as fp16 tiles (thread t: token t / 8,
-// coordinates 16 (t % 8) .. + 15; levels from the shared-memory codebooks ck, cv), and
-// the tokens' scalars.
-__device__ void decode_page_tiles(const PrefillArgs& a, const uint8_t* kch, const uint8_t* vch, uint8_t* smem,
-                                  const __half* ck, const __half* cv) {
+// One page's bytes for thread i < 128 (token i % 16, coordinates 16 (i / 16) .. + 15):
+// its packed key codes, sign bits and value codes, and (threads < 16) the token's
+// scalars.  Loaded a page ahead of their use.
+struct PageBytes {
+    uint64_t kw, vw;
+    uint32_t sw;
+    float kn, kg, vn;
+};
+__device__ __forceinline__ PageBytes fetch_page(const PrefillArgs& a, int blk, int hk) {
+    PageBytes r{};
+    if (threadIdx.x >= 128 || blk < 0 || blk >= a.num_blocks) return r;
+    const uint8_t* kch = a.kc + ((size_t)blk * a.Hkv + hk) * a.lk.bytes;
+    const uint8_t* vch = a.vc + ((size_t)blk * a.Hkv + hk) * a.lv.bytes;
+    const int t = threadIdx.x & 15, t8 = threadIdx.x >> 4;
+    r.kw = load_codes16(kch + t * a.lk.code_row, t8, a.cbk.width);
+    r.vw = load_codes16(vch + t * a.lv.code_row, t8, a.cbv.width);
+    if (a.lk.prod) r.sw = *reinterpret_cast<const uint16_t*>(kch + a.lk.signs_off + t * (kDim / 8) + 2 * t8);
+    if (threadIdx.x < kPage) {
+        r.kn = reinterpret_cast<const float*>(kch + a.lk.norm_off)[t] * a.qscale;
+        r.kg = a.lk.prod ? reinterpret_cast<const float*>(kch + a.lk.gamma_off)[t] * a.sscale : 0.f;
+        r.vn = reinterpret_cast<const float*>(vch + a.lv.norm_off)[t];
+    }
+    return r;
+}
+
+// A page's fp16 tiles from its bytes (levels from the shared-memory codebooks ck, cv):
+// a half-warp writes one coordinate's 16 tokens side by side in the transposed value
+// tile.
+__device__ __forceinline__ void store_page_tiles(const PrefillArgs& a, const PageBytes& r, uint8_t* smem,
+                                                 const __half* ck, const __half* cv) {
+    if (threadIdx.x >= 128) return;
     __half* kt = reinterpret_cast<__half*>(smem + kPOffK);
     __half* st = reinterpret_cast<__half*>(smem + kPOffS);
     __half* vt = reinterpret_cast<__half*>(smem + kPOffV);
     float* ts = reinterpret_cast<float*>(smem + kPOffT);
-    const int t = threadIdx.x >> 3, t8 = threadIdx.x & 7, j0 = 16 * t8;
+    const int t = threadIdx.x & 15, j0 = 16 * (threadIdx.x >> 4);
     const int wk = a.cbk.width, wv = a.cbv.width;
-    const uint64_t kw = load_codes16(kch + t * a.lk.code_row, t8, wk);
-    const uint64_t vw = load_codes16(vch + t * a.lv.code_row, t8, wv);
-    const uint32_t sw = a.lk.prod ? *reinterpret_cast<const uint16_t*>(kch + a.lk.signs_off + t * (kDim / 8) + 2 * t8) : 0u;
     const uint32_t mk = (1u << wk) - 1u, mv = (1u << wv) - 1u;
 #pragma unroll
     for (int j = 0; j < 16; j += 2) {
-        const __half k0 = ck[(uint32_t)(kw >> (j * wk)) & mk], k1 = ck[(uint32_t)(kw >> ((j + 1) * wk)) & mk];
+        const __half k0 = ck[(uint32_t)(r.kw >> (j * wk)) & mk], k1 = ck[(uint32_t)(r.kw >> ((j + 1) * wk)) & mk];
         *reinterpret_cast<__half2*>(kt + t * kKS + j0 + j) = __halves2half2(k0, k1);
         if (a.lk.prod) {
-            const __half s0 = ((sw >> j) & 1u) ? __float2half_rn(1.f) : __float2half_rn(-1.f);
-            const __half s1 = ((sw >> (j + 1)) & 1u) ? __float2half_rn(1.f) : __float2half_rn(-1.f);
+            const __half s0 = ((r.sw >> j) & 1u) ? __float2half_rn(1.f) : __float2half_rn(-1.f);
+            const __half s1 = ((r.sw >> (j + 1)) & 1u) ? __float2half_rn(1.f) : __float2half_rn(-1.f);
             *reinterpret_cast<__half2*>(st + t * kKS + j0 + j) = __halves2half2(s0, s1);
         }
-        vt[(j0 + j) * kVS + t] = cv[(uint32_t)(vw >> (j * wv)) & mv];
-        vt[(j0 + j + 1) * kVS + t] = cv[(uint32_t)(vw >> ((j + 1) * wv)) & mv];
+        vt[(j0 + j) * kVS + t] = cv[(uint32_t)(r.vw >> (j * wv)) & mv];
+        vt[(j0 + j + 1) * kVS + t] = cv[(uint32_t)(r.vw >> ((j + 1) * wv)) & mv];
     }
     if (threadIdx.x < kPage) {
-        const int r = threadIdx.x;
-        ts[r] = reinterpret_cast<const float*>(kch + a.lk.norm_off)[r] * a.qscale;
-        ts[kPage + r] = a.lk.prod ? reinterpret_cast<const float*>(kch + a.lk.gamma_off)[r] * a.sscale : 0.f;
-        ts[2 * kPage + r] = reinterpret_cast<const float*>(vch + a.lv.norm_off)[r];
+        ts[t] = r.kn;
+        ts[kPage + t] = r.kg;
+        ts[2 * kPage + t] = r.vn;
     }
 }
 
@@ -207,16 +229,21 @@ __global__ void __launch_bounds__(kPThreads) prefill_attn_kernel(PrefillArgs a) 
     const __half* st = reinterpret_cast<const __half*>(smem + kPOffS);
     const __half* vt = reinterpret_cast<const __half*>(smem + kPOffV);
     const float* ts = reinterpret_cast<const float*>(smem + kPOffT);
+    // block ids two pages ahead, page bytes one page ahead of their use
+    int blk_next = n_pages > 0 ? a.block_table[0] : 0;
+    PageBytes nxt = fetch_page(a, blk_next, hk);
+    int blk_after = n_pages > 1 ? a.block_table[1] : 0;
     for (int p = 0; p < n_pages; ++p) {
-        const int blk = a.block_table[p];
-        const bool ok = blk >= 0 && blk < a.num_blocks;
-        __syncthreads();  // the previous page's tiles are read
-        if (ok) {
-            decode_page_tiles(a, a.kc + ((size_t)blk * a.Hkv + hk) * a.lk.bytes,
-                              a.vc + ((size_t)blk * a.Hkv + hk) * a.lv.bytes, smem, ck, cv);
-        } else if (threadIdx.x == 0 && h == 0 && blockIdx.x == 0) {
-            atomicOr(a.err, TQ_DEVERR_BLOCK);
+        const PageBytes cur = nxt;
+        const bool ok = blk_next >= 0 && blk_next < a.num_blocks;
+        if (p + 1 < n_pages) {
+            blk_next = blk_after;
+            nxt = fetch_page(a, blk_next, hk);
+            blk_after = p + 2 < n_pages ? a.block_table[p + 2] : 0;
         }
+        __syncthreads();  // the previous page's tiles are read
+        if (ok) store_page_tiles(a, cur, smem, ck, cv);
+        else if (threadIdx.x == 0) atomicOr(a.err, TQ_DEVERR_BLOCK);
         __syncthreads();
         if (!ok) continue;
         // scores of tokens nt*8 + 2c + e for rows g (i = 0), g + 8 (i = 1)
