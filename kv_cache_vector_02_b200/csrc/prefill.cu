@@ -16,11 +16,12 @@
 //   prologue  R^T (fp16 hi, lo) and S staged in shared memory (16-byte async copies,
 //             rows swizzled); each warp computes q' and s of its 16 queries on
 //             mma.sync and keeps them as fp16 A fragments in registers.
-//   pages     per 16-token page up to the block's last query: the CTA's threads
-//             decode the key codes, sign bits and value codes into fp16 tiles in
-//             shared memory (K: [token][coord], V: [coord][token]); each warp takes
-//             scores S[16 queries x 16 tokens] (two n-tiles, key term and sign term),
-//             the causal mask, an online-softmax step (base 2), and O += P' V.
+//   pages     per step of two 16-token pages up to the block's last query: the CTA's
+//             threads decode the key codes, sign bits and value codes (fetched a step
+//             ahead) into fp16 tiles in shared memory (K: [token][coord], V:
+//             [coord][token]); each warp takes scores S[16 queries x 32 tokens] (four
+//             n-tiles, key term and sign term), the causal mask, an online-softmax
+//             step (base 2), and O += P' V.
 //   epilogue  R (fp16 hi, lo) staged over R^T; o = R (O / l) / sqrt(d) on mma.sync
 //             (three passes), stored fp16 or fp32.
 #include <cmath>
@@ -35,17 +36,18 @@ namespace {
 constexpr int kPW = 8;                 // warps per CTA
 constexpr int kPThreads = kPW * 32;
 constexpr int kPQ = 16 * kPW;          // queries per CTA
+constexpr int kPT = 2 * kPage;         // tokens per step: two pages
 constexpr int kKS = kDim + 8;          // K / sign tile row stride (halves): rows 16 bytes apart in banks
-constexpr int kVS = kPage + 8;         // V tile row stride (halves)
+constexpr int kVS = kPT + 8;           // V tile row stride (halves)
 // Shared memory: [0, 96 KiB) staged matrices (R^T hi | R^T lo | S, then R hi | R lo),
 // then the page tiles and the per-token scalars.
 constexpr uint32_t kPOffMat = 0;
 constexpr uint32_t kPMatBytes = 3 * kDim * kDim * 2;
-constexpr uint32_t kPOffK = kPOffMat + kPMatBytes;                  // half [16][kKS]: c[key code]
-constexpr uint32_t kPOffS = kPOffK + kPage * kKS * 2;               // half [16][kKS]: +-1 signs
-constexpr uint32_t kPOffV = kPOffS + kPage * kKS * 2;               // half [128][kVS]: c[value code], transposed
-constexpr uint32_t kPOffT = kPOffV + kDim * kVS * 2;                // float [3][16]: key norm, gamma, value norm
-constexpr uint32_t kPOffCB = kPOffT + 3 * kPage * 4;               // half [2][16]: key, value levels
+constexpr uint32_t kPOffK = kPOffMat + kPMatBytes;                  // half [32][kKS]: c[key code]
+constexpr uint32_t kPOffS = kPOffK + kPT * kKS * 2;                 // half [32][kKS]: +-1 signs
+constexpr uint32_t kPOffV = kPOffS + kPT * kKS * 2;                 // half [128][kVS]: c[value code], transposed
+constexpr uint32_t kPOffT = kPOffV + kDim * kVS * 2;                // float [3][32]: key norm, gamma, value norm
+constexpr uint32_t kPOffCB = kPOffT + 3 * kPT * 4;                  // half [2][16]: key, value levels
 constexpr uint32_t kPSmem = kPOffCB + 2 * 16 * 2;
 
 struct PrefillArgs {
@@ -95,9 +97,10 @@ __device__ __forceinline__ uint64_t load_codes16(const uint8_t* row, int t8, int
     return *reinterpret_cast<const uint16_t*>(row + 2 * t8);
 }
 
-// One page's bytes for thread i < 128 (token i % 16, coordinates 16 (i / 16) .. + 15):
-// its packed key codes, sign bits and value codes, and (threads < 16) the token's
-// scalars.  Loaded a page ahead of their use.
+// One step's bytes for thread i (page i / 128 of the step's two, token i % 16,
+// coordinates 16 (i / 16 % 8) .. + 15): its packed key codes, sign bits and value
+// codes, and (threads i % 128 < 16) the token's scalars.  Loaded a step ahead of use.
+static_assert(kPThreads == 256, "one thread per (page, token, 16 coordinates) of a step");
 struct PageBytes {
     uint64_t kw, vw;
     uint32_t sw;
@@ -105,14 +108,14 @@ struct PageBytes {
 };
 __device__ __forceinline__ PageBytes fetch_page(const PrefillArgs& a, int blk, int hk) {
     PageBytes r{};
-    if (threadIdx.x >= 128 || blk < 0 || blk >= a.num_blocks) return r;
+    if (blk < 0 || blk >= a.num_blocks) return r;
     const uint8_t* kch = a.kc + ((size_t)blk * a.Hkv + hk) * a.lk.bytes;
     const uint8_t* vch = a.vc + ((size_t)blk * a.Hkv + hk) * a.lv.bytes;
-    const int t = threadIdx.x & 15, t8 = threadIdx.x >> 4;
+    const int t = threadIdx.x & 15, t8 = (threadIdx.x >> 4) & 7;
     r.kw = load_codes16(kch + t * a.lk.code_row, t8, a.cbk.width);
     r.vw = load_codes16(vch + t * a.lv.code_row, t8, a.cbv.width);
     if (a.lk.prod) r.sw = *reinterpret_cast<const uint16_t*>(kch + a.lk.signs_off + t * (kDim / 8) + 2 * t8);
-    if (threadIdx.x < kPage) {
+    if ((threadIdx.x & 127) < kPage) {
         r.kn = reinterpret_cast<const float*>(kch + a.lk.norm_off)[t] * a.qscale;
         r.kg = a.lk.prod ? reinterpret_cast<const float*>(kch + a.lk.gamma_off)[t] * a.sscale : 0.f;
         r.vn = reinterpret_cast<const float*>(vch + a.lv.norm_off)[t];
@@ -120,17 +123,16 @@ __device__ __forceinline__ PageBytes fetch_page(const PrefillArgs& a, int blk, i
     return r;
 }
 
-// A page's fp16 tiles from its bytes (levels from the shared-memory codebooks ck, cv):
+// A step's fp16 tiles from its bytes (levels from the shared-memory codebooks ck, cv):
 // a half-warp writes one coordinate's 16 tokens side by side in the transposed value
 // tile.
 __device__ __forceinline__ void store_page_tiles(const PrefillArgs& a, const PageBytes& r, uint8_t* smem,
                                                  const __half* ck, const __half* cv) {
-    if (threadIdx.x >= 128) return;
     __half* kt = reinterpret_cast<__half*>(smem + kPOffK);
     __half* st = reinterpret_cast<__half*>(smem + kPOffS);
     __half* vt = reinterpret_cast<__half*>(smem + kPOffV);
     float* ts = reinterpret_cast<float*>(smem + kPOffT);
-    const int t = threadIdx.x & 15, j0 = 16 * (threadIdx.x >> 4);
+    const int t = (threadIdx.x >> 7) * kPage + (threadIdx.x & 15), j0 = 16 * ((threadIdx.x >> 4) & 7);
     const int wk = a.cbk.width, wv = a.cbv.width;
     const uint32_t mk = (1u << wk) - 1u, mv = (1u << wv) - 1u;
 #pragma unroll
@@ -145,10 +147,10 @@ __device__ __forceinline__ void store_page_tiles(const PrefillArgs& a, const Pag
         vt[(j0 + j) * kVS + t] = cv[(uint32_t)(r.vw >> (j * wv)) & mv];
         vt[(j0 + j + 1) * kVS + t] = cv[(uint32_t)(r.vw >> ((j + 1) * wv)) & mv];
     }
-    if (threadIdx.x < kPage) {
+    if ((threadIdx.x & 127) < kPage) {
         ts[t] = r.kn;
-        ts[kPage + t] = r.kg;
-        ts[2 * kPage + t] = r.vn;
+        ts[kPT + t] = r.kg;
+        ts[2 * kPT + t] = r.vn;
     }
 }
 
@@ -229,75 +231,85 @@ __global__ void __launch_bounds__(kPThreads) prefill_attn_kernel(PrefillArgs a) 
     const __half* st = reinterpret_cast<const __half*>(smem + kPOffS);
     const __half* vt = reinterpret_cast<const __half*>(smem + kPOffV);
     const float* ts = reinterpret_cast<const float*>(smem + kPOffT);
-    // block ids two pages ahead, page bytes one page ahead of their use
-    int blk_next = n_pages > 0 ? a.block_table[0] : 0;
+    // steps of two pages: this thread's page id two steps ahead, its bytes one step ahead
+    const int sub = threadIdx.x >> 7;  // the page of the step this thread fetches
+    const int n_steps = (n_pages + 1) / 2;
+    auto block_of = [&](int pg) { return pg < n_pages ? a.block_table[pg] : -1; };
+    int blk_next = block_of(sub);
     PageBytes nxt = fetch_page(a, blk_next, hk);
-    int blk_after = n_pages > 1 ? a.block_table[1] : 0;
-    for (int p = 0; p < n_pages; ++p) {
+    int blk_after = block_of(2 + sub);
+    for (int step = 0; step < n_steps; ++step) {
         const PageBytes cur = nxt;
-        const bool ok = blk_next >= 0 && blk_next < a.num_blocks;
-        if (p + 1 < n_pages) {
+        const int blk_cur = blk_next;
+        if (step + 1 < n_steps) {
             blk_next = blk_after;
             nxt = fetch_page(a, blk_next, hk);
-            blk_after = p + 2 < n_pages ? a.block_table[p + 2] : 0;
+            blk_after = block_of(2 * (step + 2) + sub);
         }
-        __syncthreads();  // the previous page's tiles are read
-        if (ok) store_page_tiles(a, cur, smem, ck, cv);
-        else if (threadIdx.x == 0) atomicOr(a.err, TQ_DEVERR_BLOCK);
+        // pages of the step with a valid block (a page past the last is masked by the
+        // causal limit: its positions exceed every query's)
+        const int b0 = block_of(2 * step), b1 = block_of(2 * step + 1);
+        const bool ok0 = b0 >= 0 && b0 < a.num_blocks;
+        const bool ok1 = (2 * step + 1 >= n_pages) || (b1 >= 0 && b1 < a.num_blocks);
+        __syncthreads();  // the previous step's tiles are read
+        if (blk_cur >= 0 && blk_cur < a.num_blocks) store_page_tiles(a, cur, smem, ck, cv);
+        if (threadIdx.x == 0 && !(ok0 && ok1)) atomicOr(a.err, TQ_DEVERR_BLOCK);
         __syncthreads();
-        if (!ok) continue;
-        // scores of tokens nt*8 + 2c + e for rows g (i = 0), g + 8 (i = 1)
-        float sc[2][2][2];  // [nt][i][e]
+        // scores of tokens nt*8 + 2c + e (nt = 0..3) for rows g (i = 0), g + 8 (i = 1)
+        float sc[4][2][2];  // [nt][i][e]
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
+        for (int nt = 0; nt < 4; ++nt) {
             const int tok = nt * 8 + g;  // B column of this lane
             float d1[4], d2[4];
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kt + tok * kKS + 16 * ks + 2 * c);
-                const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kt + tok * kKS + 16 * ks + 2 * c + 8);
-                if (ks == 0) mma16816_z(d1, ra[0][0], ra[0][1], ra[0][2], ra[0][3], b0, b1);
-                else mma16816(d1, ra[ks][0], ra[ks][1], ra[ks][2], ra[ks][3], b0, b1);
+                const uint32_t b0w = *reinterpret_cast<const uint32_t*>(kt + tok * kKS + 16 * ks + 2 * c);
+                const uint32_t b1w = *reinterpret_cast<const uint32_t*>(kt + tok * kKS + 16 * ks + 2 * c + 8);
+                if (ks == 0) mma16816_z(d1, ra[0][0], ra[0][1], ra[0][2], ra[0][3], b0w, b1w);
+                else mma16816(d1, ra[ks][0], ra[ks][1], ra[ks][2], ra[ks][3], b0w, b1w);
             }
             if (a.lk.prod) {
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t b0 = *reinterpret_cast<const uint32_t*>(st + tok * kKS + 16 * ks + 2 * c);
-                    const uint32_t b1 = *reinterpret_cast<const uint32_t*>(st + tok * kKS + 16 * ks + 2 * c + 8);
-                    if (ks == 0) mma16816_z(d2, sa[0][0], sa[0][1], sa[0][2], sa[0][3], b0, b1);
-                    else mma16816(d2, sa[ks][0], sa[ks][1], sa[ks][2], sa[ks][3], b0, b1);
+                    const uint32_t b0w = *reinterpret_cast<const uint32_t*>(st + tok * kKS + 16 * ks + 2 * c);
+                    const uint32_t b1w = *reinterpret_cast<const uint32_t*>(st + tok * kKS + 16 * ks + 2 * c + 8);
+                    if (ks == 0) mma16816_z(d2, sa[0][0], sa[0][1], sa[0][2], sa[0][3], b0w, b1w);
+                    else mma16816(d2, sa[ks][0], sa[ks][1], sa[ks][2], sa[ks][3], b0w, b1w);
                 }
             } else {
                 d2[0] = d2[1] = d2[2] = d2[3] = 0.f;
             }
+            const bool okp = nt < 2 ? ok0 : ok1;
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const int tt = nt * 8 + 2 * c + e, pos = p * kPage + tt;
-                const float kn = ts[tt], kg = ts[kPage + tt];
+                const int tt = nt * 8 + 2 * c + e, pos = step * kPT + tt;
+                const float kn = ts[tt], kg = ts[kPT + tt];
                 const float s0 = fmaf(kg, d2[e], kn * d1[e]), s1 = fmaf(kg, d2[2 + e], kn * d1[2 + e]);
-                sc[nt][0][e] = pos <= qp0 ? s0 : -INFINITY;
-                sc[nt][1][e] = pos <= qp1 ? s1 : -INFINITY;
+                sc[nt][0][e] = okp && pos <= qp0 ? s0 : -INFINITY;
+                sc[nt][1][e] = okp && pos <= qp1 ? s1 : -INFINITY;
             }
         }
-        // online softmax per row (the row's 16 scores sit in the quad's 4 lanes)
-        uint32_t pa[4];
+        // online softmax per row (the row's 32 scores sit in the quad's 4 lanes)
+        uint32_t pa[2][4];  // [K-step: tokens 0-15 / 16-31][A register]
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-            float mx = fmaxf(fmaxf(sc[0][i][0], sc[0][i][1]), fmaxf(sc[1][i][0], sc[1][i][1]));
+            float mx = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) mx = fmaxf(mx, fmaxf(sc[nt][i][0], sc[nt][i][1]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
             const float mnew = fmaxf(m[i], mx);
             const float corr = (m[i] == -INFINITY) ? 0.f : exp2f(m[i] - mnew);
-            float pw[2][2];
+            float pw[4][2];
             float sum = 0.f;
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const float pr = (sc[nt][i][e] == -INFINITY) ? 0.f : exp2f(sc[nt][i][e] - mnew);
                     sum += pr;
-                    // (a masked token's value norm is not read: past the chunk it may be anything)
-                    pw[nt][e] = pr > 0.f ? pr * ts[2 * kPage + nt * 8 + 2 * c + e] : 0.f;
+                    // (a masked token's value norm is not read: it may be anything)
+                    pw[nt][e] = pr > 0.f ? pr * ts[2 * kPT + nt * 8 + 2 * c + e] : 0.f;
                 }
             l[i] = l[i] * corr + sum;
             m[i] = mnew;
@@ -306,17 +318,23 @@ __global__ void __launch_bounds__(kPThreads) prefill_attn_kernel(PrefillArgs a) 
                 acc[nt][2 * i] *= corr;
                 acc[nt][2 * i + 1] *= corr;
             }
-            // P' as the A fragment of the value contraction (K = the page's 16 tokens)
-            pa[i] = f2h2(pw[0][0], pw[0][1]);      // tokens 2c, 2c + 1
-            pa[2 + i] = f2h2(pw[1][0], pw[1][1]);  // tokens 2c + 8, 2c + 9
+            // P' as A fragments of the value contraction (K-steps: tokens 0-15, 16-31)
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                pa[k][i] = f2h2(pw[2 * k][0], pw[2 * k][1]);          // tokens 16k + 2c, + 1
+                pa[k][2 + i] = f2h2(pw[2 * k + 1][0], pw[2 * k + 1][1]);  // tokens 16k + 2c + 8, + 9
+            }
         }
         // O[16 x 128] += P' V: n-tile nt = coordinates 8 nt .. 8 nt + 7
 #pragma unroll
         for (int nt = 0; nt < 16; ++nt) {
             const int coord = nt * 8 + g;
-            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(vt + coord * kVS + 2 * c);
-            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(vt + coord * kVS + 2 * c + 8);
-            mma16816(acc[nt], pa[0], pa[1], pa[2], pa[3], b0, b1);
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const uint32_t b0w = *reinterpret_cast<const uint32_t*>(vt + coord * kVS + 16 * k + 2 * c);
+                const uint32_t b1w = *reinterpret_cast<const uint32_t*>(vt + coord * kVS + 16 * k + 2 * c + 8);
+                mma16816(acc[nt], pa[k][0], pa[k][1], pa[k][2], pa[k][3], b0w, b1w);
+            }
         }
     }
 
