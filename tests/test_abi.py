@@ -97,3 +97,17 @@ def test_noalloc_raw_call_refuses_bad_arguments(tq):
     ctx = tq.tq_init_host(128, 4, 0)
     assert f(ctx.handle, *args) == tq.TQ_ERR_INVALID_ARG
     tq.tq_destroy(ctx)
+
+
+def test_prefill_raw_call_refuses_bad_arguments(tq):
+    """tq_prefill_attention through the raw symbol: a null or host-only context, and a
+    chunk that reaches past the block table, are refused on the host before any device
+    is touched; an empty chunk is a no-op."""
+    L = tq._lib
+    f = L.tq_prefill_attention
+    # (q, k_cache, v_cache, num_blocks, block_table, max_blocks, q_start, Tq, Hq, Hkv, scale, out, out_fp32, stream)
+    good = (16, 16, 16, 4, 16, 4, 0, 16, 2, 1, 0.0, 16, 1, None)
+    assert f(None, *good) == tq.TQ_ERR_INVALID_ARG
+    ctx = tq.tq_init_host(128, 4, 0)
+    assert f(ctx.handle, *good) == tq.TQ_ERR_INVALID_ARG
+    tq.tq_destroy(ctx)
