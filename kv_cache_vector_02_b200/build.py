@@ -1,6 +1,7 @@
 """Build libtq.so (CUDA sm_100a + host C++) in-tree with nvcc.
 
     python -m kv_cache_vector_02_b200.build [--force] [--verbose]
+    TQ_DEBUG=1 python -m kv_cache_vector_02_b200.build --force   # with device invariant checks
 
 Every .cu / .cpp under csrc/ is compiled to an object under _build/ (in
 parallel) and linked into kv_cache_vector_02_b200/libtq.so with a static CUDA
@@ -23,6 +24,11 @@ INCLUDE = PKG.parent / "include"
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden", "-I", str(INCLUDE)]
+# TQ_DEBUG=1 in the environment: device-side invariant checks (index bounds of slots,
+# rows and pages), each setting TQ_DEVERR_INTERNAL instead of touching memory out of
+# range.  Build with --force when switching.
+if os.environ.get("TQ_DEBUG", "") not in ("", "0"):
+    COMMON += ["-DTQ_DEBUG"]
 
 
 def _nvcc() -> str:

@@ -1024,8 +1024,10 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_attn_kernel(DecodeArg
     it.init(a, pre, pos0, end);
     int b, hk, p0, p1;
     constexpr int KS = KeyTerm<KM>::kSteps;
+    const long n_slots = (long)a.B * a.Hkv + gridDim.x;
     while (it.next(a, b, hk, p0, p1)) {
         const int unit = b * a.Hkv + hk;
+        if (!TQ_DCHECK(unit >= 0 && unit + (long)blockIdx.x < n_slots && p0 >= 0 && p1 <= a.max_blocks, a.err)) break;
         const int Ls = a.seq_lens[b];  // valid: the sequence has pages
         // query fragments (B operand) of heads nt*8 + g: key term and sign term
         uint32_t bq[NT][KS][2], bs[NT][8][2];
@@ -1366,6 +1368,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_attn_kernel(DecodeArg
         for (int hk = 0; hk < a.Hkv; ++hk) {
             const long first = s0 + (long)hk * np;
             if (!((first >= pos0 && first < end) || (last_cta && first == total))) continue;
+            if (!TQ_DCHECK(nu < per_batch && b * a.Hkv + hk + (long)cta < n_slots, a.err)) continue;
             ulist[nu++] = b * a.Hkv + hk;
             if (nu == per_batch) finish_batch();
         }

@@ -234,7 +234,9 @@ __global__ void __launch_bounds__(kPThreads) prefill_attn_kernel(PrefillArgs a) 
     // steps of two pages: this thread's page id two steps ahead, its bytes one step ahead
     const int sub = threadIdx.x >> 7;  // the page of the step this thread fetches
     const int n_steps = (n_pages + 1) / 2;
-    auto block_of = [&](int pg) { return pg < n_pages ? a.block_table[pg] : -1; };
+    auto block_of = [&](int pg) {
+        return pg < n_pages && TQ_DCHECK(pg < a.max_blocks, a.err) ? a.block_table[pg] : -1;
+    };
     int blk_next = block_of(sub);
     PageBytes nxt = fetch_page(a, blk_next, hk);
     int blk_after = block_of(2 + sub);

@@ -1,6 +1,7 @@
 // C ABI of libtq: validation, parameter upload, dispatch.  The arithmetic of
 // the hot path runs in the CUDA translation units; this file only checks
 // arguments, owns the context and launches.
+#include <nvtx3/nvToolsExt.h>
 #include <algorithm>
 #include <atomic>
 #include <cmath>
@@ -65,6 +66,15 @@ tq::Codebook make_codebook(const std::vector<double>& c, const std::vector<doubl
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// An NVTX range around each device entry point, named after it, for Nsight timelines;
+// with no tool attached a push / pop costs a pointer test.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Records that ctx's parameters are in use by work queued on `stream` up to now.
 // Returns false if the event could not be created or recorded.
@@ -295,6 +305,7 @@ tq_status tq_export_params(const tq_ctx* ctx, double* R, int8_t* S, int8_t* hsig
 tq_status tq_compress(const tq_ctx* ctx, const uint16_t* k, const uint16_t* v, int T, int Hkv,
                       const int32_t* slot_mapping, uint8_t* k_cache, uint8_t* v_cache, int num_blocks,
                       void* stream) {
+    NvtxRange nvtx("tq_compress");
     if (!ctx || ctx->host_only || T < 0 || Hkv < 1 || num_blocks < 0) return TQ_ERR_INVALID_ARG;
     if (T == 0) return TQ_OK;
     if (!slot_mapping || (!k && !v)) return TQ_ERR_INVALID_ARG;
@@ -312,6 +323,7 @@ tq_status tq_compress(const tq_ctx* ctx, const uint16_t* k, const uint16_t* v, i
 
 tq_status tq_decompress(const tq_ctx* ctx, int kind, const uint8_t* cache, int num_blocks,
                         const int32_t* slot_mapping, int T, int Hkv, void* out, int out_fp32, void* stream) {
+    NvtxRange nvtx("tq_decompress");
     if (!ctx || ctx->host_only || T < 0 || Hkv < 1 || num_blocks < 0) return TQ_ERR_INVALID_ARG;
     if (kind != TQ_KIND_KEY && kind != TQ_KIND_VALUE) return TQ_ERR_INVALID_ARG;
     if (T == 0) return TQ_OK;
@@ -333,6 +345,7 @@ tq_status decode_common(const tq_ctx* ctx, const uint16_t* q, const uint8_t* k_c
                         int num_blocks, const int32_t* block_table, int max_blocks, const int32_t* seq_lens, int B,
                         int Hq, int Hkv, int max_seq_len, const tq::DecodeTail& tail, float scale, void* out,
                         int out_fp32, void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx("tq_decode_attention");
     if (!ctx || ctx->host_only || B < 0 || Hq < 1 || Hkv < 1 || max_blocks < 0 || num_blocks < 0 || max_seq_len < 0)
         return TQ_ERR_INVALID_ARG;
     if (Hq % Hkv != 0 || Hq / Hkv > 16) return TQ_ERR_INVALID_ARG;
@@ -367,6 +380,7 @@ tq_status tq_decode_attention(const tq_ctx* ctx, const uint16_t* q, const uint8_
 tq_status tq_prefill_attention(const tq_ctx* ctx, const uint16_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
                                int num_blocks, const int32_t* block_table, int max_blocks, int q_start, int Tq, int Hq,
                                int Hkv, float scale, void* out, int out_fp32, void* stream) {
+    NvtxRange nvtx("tq_prefill_attention");
     if (!ctx || ctx->host_only || Tq < 0 || q_start < 0 || Hq < 1 || Hkv < 1 || max_blocks < 0 || num_blocks < 0)
         return TQ_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return TQ_ERR_INVALID_ARG;
