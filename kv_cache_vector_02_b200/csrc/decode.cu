@@ -57,7 +57,7 @@ namespace tq {
 namespace {
 
 constexpr int kNW = 8;                        // warps per CTA (one CTA per SM, two per scheduler)
-constexpr int kSplitThreads = kNW * 32;
+constexpr int kThreads = kNW * 32;
 constexpr int kPartStride = kDim + 2;         // m, l, acc[128]
 constexpr int kStages = 6;                    // page stages per warp: 3 pairs
 constexpr uint32_t kStageBytes = 2496;        // >= key chunk + value chunk at every bit width (16-byte multiple)
@@ -67,7 +67,7 @@ constexpr uint32_t kTabBytes = 65536;         // 256 entries x 256 bytes
 // from kRingAddr on (see stage_addr).
 constexpr int kLowStages = 12;
 constexpr uint32_t kRingAddr = kTabAddr + kTabBytes;
-constexpr uint32_t kSplitSmem = kRingAddr + (kNW * kStages - kLowStages) * kStageBytes;  // any window base >= 0
+constexpr uint32_t kSmemBytes = kRingAddr + (kNW * kStages - kLowStages) * kStageBytes;  // any window base >= 0
 // Below the tables, from the window base: the warps' (m, l), the CTA merge area (4
 // heads at a time), the low stages.
 constexpr uint32_t kOffML = 0;                                  // [kNW][2][4] float: m, l
@@ -80,7 +80,7 @@ constexpr uint32_t kEpiBytes = 45056;  // the epilogue's scratch (EpiSmem) from 
 constexpr uint32_t kOffPre = (kLowBytes > kOffMerge + kEpiBytes ? kLowBytes : kOffMerge + kEpiBytes);
 constexpr int kPreCap = 3840;
 static_assert(kOffPre + kPreCap * 4 + 1024 <= kTabAddr, "prefix sums below the tables");
-static_assert(kSplitSmem <= 232448, "shared memory budget");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint64_t kWaitNs = 2000000000ull;  // bounded waits for another CTA's slot
 
 enum KMode { kKPrmt = 0, kKByte4 = 1, kKByte2 = 2, kKBit1 = 3 };
@@ -188,7 +188,7 @@ constexpr float kSlack = 8.f;
 // Token of page row r (see the file comment).
 __host__ __device__ constexpr int row_token(int r) { return r ^ ((r >> 1) & 1); }
 
-// ------------------------------------------------------------------ split: tables
+// ------------------------------------------------------------------ page loop: tables
 // Entry e (a byte) of the 64 KiB table at kTabAddr is 256 bytes:
 //   bytes   0..127  region A, values:
 //                     nibble pair bytes (low nibble: token t, high: token t + 1):
@@ -230,7 +230,7 @@ __device__ void build_tables(const DecodeArgs& a, int e) {
     }
 }
 
-// ------------------------------------------------------------------ split: pieces
+// ------------------------------------------------------------------ page loop: pieces
 // The CTA's range [pos, end) of the pages of all units in order (unit u = b Hkv + h
 // holds the pages of sequence b), cut into pieces by unit.
 struct Pieces {
@@ -326,7 +326,7 @@ struct PageCursor {
     }
 };
 
-// ------------------------------------------------------------------ split: one page
+// ------------------------------------------------------------------ page loop: one page
 template <int KM, int VM, bool PROD>
 struct PageRegs {
     uint32_t k[2][4];    // key code bytes of token rows g, g+8 (coords 32c .. 32c+31)
@@ -788,7 +788,7 @@ __device__ void window_unit(const DecodeArgs& a, EpiSmem& e, int b, int hk, int 
         if (tid == 0 && hk == 0) atomicOr(a.err, TQ_DEVERR_SEQLEN);
         tl = 0;
     }
-    for (int k = tid; k < G * kDim; k += kSplitThreads) {
+    for (int k = tid; k < G * kDim; k += kThreads) {
         const int h = k / kDim, i = k - h * kDim;
         e.sq[h][i] = __half2float(__ushort_as_half(a.q[((size_t)b * a.Hq + hk * G + h) * kDim + i]));
     }
@@ -796,7 +796,7 @@ __device__ void window_unit(const DecodeArgs& a, EpiSmem& e, int b, int hk, int 
     float mx[16];
 #pragma unroll
     for (int h = 0; h < 16; ++h) mx[h] = -INFINITY;
-    for (int t = tid; t < tl; t += kSplitThreads) {  // scores: a thread per token
+    for (int t = tid; t < tl; t += kThreads) {  // scores: a thread per token
         const uint4* kr = reinterpret_cast<const uint4*>(a.tail_k + (((size_t)b * a.tail_cap + t) * a.Hkv + hk) * kDim);
         float sc[16];
 #pragma unroll
@@ -834,7 +834,7 @@ __device__ void window_unit(const DecodeArgs& a, EpiSmem& e, int b, int hk, int 
         for (int w = 0; w < kNW; ++w) gm[h] = fmaxf(gm[h], e.red[0][w][h]);
         sm[h] = 0.f;
     }
-    for (int t = tid; t < tl; t += kSplitThreads)
+    for (int t = tid; t < tl; t += kThreads)
 #pragma unroll
         for (int h = 0; h < 16; ++h) {
             const float pr = h < G ? exp2f(e.ts[t][h] - gm[h]) : 0.f;
@@ -882,7 +882,7 @@ __device__ void window_unit(const DecodeArgs& a, EpiSmem& e, int b, int hk, int 
 //             residual window, un-rotates (o = R a on mma.sync, R as fp16 hi + lo) and
 //             stores, 16 query heads at a time.
 template <int KM, int VM, bool PROD, int NT>
-__global__ void __launch_bounds__(kSplitThreads, 1) decode_attn_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) decode_attn_kernel(DecodeArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t base = sm100::smem_u32(smem);
@@ -901,7 +901,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_attn_kernel(DecodeArg
     // raise the error word), this CTA's own copy, and the lookup tables
     {
         constexpr int kPieces = kDim * kDim * 2 / 16;  // per matrix
-        for (int i = tid; i < 2 * kPieces; i += kSplitThreads) {
+        for (int i = tid; i < 2 * kPieces; i += kThreads) {
             const int mtx = i / kPieces, o = (i - mtx * kPieces) * 16;
             const int n = o >> 8, k16 = (o >> 4) & 15;
             const uint16_t* src = mtx == 0 ? a.RTh : a.RTl;
@@ -1177,7 +1177,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1) decode_attn_kernel(DecodeArg
     // fragment loads below meet no bank twice); they land while the slots are read
     {
         constexpr int kPieces = kDim * kDim * 2 / 16;  // per matrix
-        for (int i = tid; i < 2 * kPieces; i += kSplitThreads) {
+        for (int i = tid; i < 2 * kPieces; i += kThreads) {
             const int mtx = i / kPieces, o = (i - mtx * kPieces) * 16;
             const int n = o >> 8, k16 = (o >> 4) & 15;
             sm100::cp_async16(kRingAddr + mtx * (kPieces * 16) + n * 256 + ((k16 ^ (n & 7)) << 4),
@@ -1391,13 +1391,13 @@ cudaError_t launch_attn(const DecodeArgs& a, int grid, cudaStream_t stream) {
         (PROD && (a.lk.signs_off != P::kSigns || a.lk.gamma_off != P::kGamma)))
         return cudaErrorInvalidValue;  // the kernel's fixed geometry must be the context's
     auto k = decode_attn_kernel<KM, VM, PROD, NT>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSplitSmem);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     // cooperative: every CTA resident at once (a unit's merge waits for later CTAs' slots)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kSplitThreads);
-    cfg.dynamicSmemBytes = kSplitSmem;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
