@@ -18,10 +18,10 @@
 //             mma.sync and keeps them as fp16 A fragments in registers.
 //   pages     per step of two 16-token pages up to the block's last query: the CTA's
 //             threads decode the key codes, sign bits and value codes (fetched a step
-//             ahead) into fp16 tiles in shared memory (K: [token][coord], V:
-//             [coord][token]); each warp takes scores S[16 queries x 32 tokens] (four
-//             n-tiles, key term and sign term), the causal mask, an online-softmax
-//             step (base 2), and O += P' V.
+//             ahead) into fp16 [token][coordinate] tiles in shared memory; each warp
+//             takes scores S[16 queries x 32 tokens] (four n-tiles, key term and sign
+//             term; B fragments by ldmatrix), the causal mask, an online-softmax step
+//             (base 2), and O += P' V (B fragments by transposing ldmatrix).
 //   epilogue  R (fp16 hi, lo) staged over R^T; o = R (O / l) / sqrt(d) on mma.sync
 //             (three passes), stored fp16 or fp32.
 #include <cmath>
@@ -37,16 +37,15 @@ constexpr int kPW = 8;                 // warps per CTA
 constexpr int kPThreads = kPW * 32;
 constexpr int kPQ = 16 * kPW;          // queries per CTA
 constexpr int kPT = 2 * kPage;         // tokens per step: two pages
-constexpr int kKS = kDim + 8;          // K / sign tile row stride (halves): rows 16 bytes apart in banks
-constexpr int kVS = kPT + 8;           // V tile row stride (halves)
+constexpr int kKS = kDim + 8;          // tile row stride (halves): rows 16 bytes apart in banks
 // Shared memory: [0, 96 KiB) staged matrices (R^T hi | R^T lo | S, then R hi | R lo),
 // then the page tiles and the per-token scalars.
 constexpr uint32_t kPOffMat = 0;
 constexpr uint32_t kPMatBytes = 3 * kDim * kDim * 2;
 constexpr uint32_t kPOffK = kPOffMat + kPMatBytes;                  // half [32][kKS]: c[key code]
 constexpr uint32_t kPOffS = kPOffK + kPT * kKS * 2;                 // half [32][kKS]: +-1 signs
-constexpr uint32_t kPOffV = kPOffS + kPT * kKS * 2;                 // half [128][kVS]: c[value code], transposed
-constexpr uint32_t kPOffT = kPOffV + kDim * kVS * 2;                // float [3][32]: key norm, gamma, value norm
+constexpr uint32_t kPOffV = kPOffS + kPT * kKS * 2;                 // half [32][kKS]: c[value code]
+constexpr uint32_t kPOffT = kPOffV + kPT * kKS * 2;                 // float [3][32]: key norm, gamma, value norm
 constexpr uint32_t kPOffCB = kPOffT + 3 * kPT * 4;                  // half [2][16]: key, value levels
 constexpr uint32_t kPSmem = kPOffCB + 2 * 16 * 2;
 
@@ -82,6 +81,22 @@ __device__ __forceinline__ void stage_matrices(uint32_t dst, const uint16_t* con
                           reinterpret_cast<const uint8_t*>(src[mtx]) + o);
     }
     sm100::cp_async_commit();
+}
+
+// Four 8x8 fp16 matrices from shared memory (lane l gives the address of row l % 8 of
+// matrix l / 8); register j holds matrix j in the mma fragment layout.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// The same, each matrix transposed: register j holds column (not row) pairs of matrix j.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                                  uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
 }
 
 // Word w (two halves: columns 2w, 2w + 1) of row r of a staged matrix.
@@ -124,28 +139,33 @@ __device__ __forceinline__ PageBytes fetch_page(const PrefillArgs& a, int blk, i
 }
 
 // A step's fp16 tiles from its bytes (levels from the shared-memory codebooks ck, cv):
-// a half-warp writes one coordinate's 16 tokens side by side in the transposed value
-// tile.
+// each thread writes its token's 16 coordinates of the three [token][coordinate] tiles
+// as two 16-byte stores each (eight consecutive tokens of a quarter-warp cover the 32
+// banks once: rows are 16 bytes apart modulo 128).
 __device__ __forceinline__ void store_page_tiles(const PrefillArgs& a, const PageBytes& r, uint8_t* smem,
                                                  const __half* ck, const __half* cv) {
-    __half* kt = reinterpret_cast<__half*>(smem + kPOffK);
-    __half* st = reinterpret_cast<__half*>(smem + kPOffS);
-    __half* vt = reinterpret_cast<__half*>(smem + kPOffV);
     float* ts = reinterpret_cast<float*>(smem + kPOffT);
     const int t = (threadIdx.x >> 7) * kPage + (threadIdx.x & 15), j0 = 16 * ((threadIdx.x >> 4) & 7);
     const int wk = a.cbk.width, wv = a.cbv.width;
     const uint32_t mk = (1u << wk) - 1u, mv = (1u << wv) - 1u;
+    const uint32_t row = (uint32_t)(t * kKS + j0) * 2;
 #pragma unroll
-    for (int j = 0; j < 16; j += 2) {
-        const __half k0 = ck[(uint32_t)(r.kw >> (j * wk)) & mk], k1 = ck[(uint32_t)(r.kw >> ((j + 1) * wk)) & mk];
-        *reinterpret_cast<__half2*>(kt + t * kKS + j0 + j) = __halves2half2(k0, k1);
-        if (a.lk.prod) {
-            const __half s0 = ((r.sw >> j) & 1u) ? __float2half_rn(1.f) : __float2half_rn(-1.f);
-            const __half s1 = ((r.sw >> (j + 1)) & 1u) ? __float2half_rn(1.f) : __float2half_rn(-1.f);
-            *reinterpret_cast<__half2*>(st + t * kKS + j0 + j) = __halves2half2(s0, s1);
+    for (int hb = 0; hb < 2; ++hb) {  // coordinates j0 + 8 hb .. + 7: one 16-byte store per tile
+        uint32_t kw[4], sw[4], vw[4];
+#pragma unroll
+        for (int jj = 0; jj < 8; jj += 2) {
+            const int j = 8 * hb + jj;
+            const __half k0 = ck[(uint32_t)(r.kw >> (j * wk)) & mk], k1 = ck[(uint32_t)(r.kw >> ((j + 1) * wk)) & mk];
+            const __half v0 = cv[(uint32_t)(r.vw >> (j * wv)) & mv], v1 = cv[(uint32_t)(r.vw >> ((j + 1) * wv)) & mv];
+            kw[jj / 2] = h2bits(k0, k1);
+            vw[jj / 2] = h2bits(v0, v1);
+            // +-1 in fp16: 0xBC00 (-1) with bit 15 cleared where the sign bit is set
+            sw[jj / 2] = 0xBC00BC00u ^ (((r.sw >> j) & 1u) << 15) ^ (((r.sw >> (j + 1)) & 1u) << 31);
         }
-        vt[(j0 + j) * kVS + t] = cv[(uint32_t)(r.vw >> (j * wv)) & mv];
-        vt[(j0 + j + 1) * kVS + t] = cv[(uint32_t)(r.vw >> ((j + 1) * wv)) & mv];
+        *reinterpret_cast<uint4*>(smem + kPOffK + row + 16 * hb) = make_uint4(kw[0], kw[1], kw[2], kw[3]);
+        *reinterpret_cast<uint4*>(smem + kPOffV + row + 16 * hb) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
+        if (a.lk.prod)
+            *reinterpret_cast<uint4*>(smem + kPOffS + row + 16 * hb) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
     }
     if ((threadIdx.x & 127) < kPage) {
         ts[t] = r.kn;
@@ -227,10 +247,11 @@ __global__ void __launch_bounds__(kPThreads) prefill_attn_kernel(PrefillArgs a) 
     float acc[16][4];
 #pragma unroll
     for (int nt = 0; nt < 16; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-    const __half* kt = reinterpret_cast<const __half*>(smem + kPOffK);
-    const __half* st = reinterpret_cast<const __half*>(smem + kPOffS);
-    const __half* vt = reinterpret_cast<const __half*>(smem + kPOffV);
+    const uint32_t kt_addr = sm100::smem_u32(smem) + kPOffK, st_addr = sm100::smem_u32(smem) + kPOffS;
+    const uint32_t vt_addr = sm100::smem_u32(smem) + kPOffV;
     const float* ts = reinterpret_cast<const float*>(smem + kPOffT);
+    static_assert(kPOffK % 16 == 0 && kPOffS % 16 == 0 && kPOffV % 16 == 0 && (kKS * 2) % 16 == 0,
+                  "ldmatrix rows and tile stores 16-byte aligned");
     // steps of two pages: this thread's page id two steps ahead, its bytes one step ahead
     const int sub = threadIdx.x >> 7;  // the page of the step this thread fetches
     const int n_steps = (n_pages + 1) / 2;
@@ -261,22 +282,26 @@ __global__ void __launch_bounds__(kPThreads) prefill_attn_kernel(PrefillArgs a) 
         float sc[4][2][2];  // [nt][i][e]
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
-            const int tok = nt * 8 + g;  // B column of this lane
+            // B fragments of two K-steps per ldmatrix.x4: lane l addresses token nt*8 + l % 8,
+            // coordinates 16 (ks + l / 16) + 8 (l / 8 % 2)
+            const uint32_t krow = (uint32_t)((nt * 8 + (lane & 7)) * kKS + 8 * ((lane >> 3) & 1) + 16 * (lane >> 4)) * 2;
             float d1[4], d2[4];
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t b0w = *reinterpret_cast<const uint32_t*>(kt + tok * kKS + 16 * ks + 2 * c);
-                const uint32_t b1w = *reinterpret_cast<const uint32_t*>(kt + tok * kKS + 16 * ks + 2 * c + 8);
-                if (ks == 0) mma16816_z(d1, ra[0][0], ra[0][1], ra[0][2], ra[0][3], b0w, b1w);
-                else mma16816(d1, ra[ks][0], ra[ks][1], ra[ks][2], ra[ks][3], b0w, b1w);
+            for (int ks = 0; ks < 8; ks += 2) {
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4(kt_addr + krow + 32 * ks, b0, b1, b2, b3);
+                if (ks == 0) mma16816_z(d1, ra[0][0], ra[0][1], ra[0][2], ra[0][3], b0, b1);
+                else mma16816(d1, ra[ks][0], ra[ks][1], ra[ks][2], ra[ks][3], b0, b1);
+                mma16816(d1, ra[ks + 1][0], ra[ks + 1][1], ra[ks + 1][2], ra[ks + 1][3], b2, b3);
             }
             if (a.lk.prod) {
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t b0w = *reinterpret_cast<const uint32_t*>(st + tok * kKS + 16 * ks + 2 * c);
-                    const uint32_t b1w = *reinterpret_cast<const uint32_t*>(st + tok * kKS + 16 * ks + 2 * c + 8);
-                    if (ks == 0) mma16816_z(d2, sa[0][0], sa[0][1], sa[0][2], sa[0][3], b0w, b1w);
-                    else mma16816(d2, sa[ks][0], sa[ks][1], sa[ks][2], sa[ks][3], b0w, b1w);
+                for (int ks = 0; ks < 8; ks += 2) {
+                    uint32_t b0, b1, b2, b3;
+                    ldmatrix_x4(st_addr + krow + 32 * ks, b0, b1, b2, b3);
+                    if (ks == 0) mma16816_z(d2, sa[0][0], sa[0][1], sa[0][2], sa[0][3], b0, b1);
+                    else mma16816(d2, sa[ks][0], sa[ks][1], sa[ks][2], sa[ks][3], b0, b1);
+                    mma16816(d2, sa[ks + 1][0], sa[ks + 1][1], sa[ks + 1][2], sa[ks + 1][3], b2, b3);
                 }
             } else {
                 d2[0] = d2[1] = d2[2] = d2[3] = 0.f;
@@ -293,6 +318,7 @@ __global__ void __launch_bounds__(kPThreads) prefill_attn_kernel(PrefillArgs a) 
         }
         // online softmax per row (the row's 32 scores sit in the quad's 4 lanes)
         uint32_t pa[2][4];  // [K-step: tokens 0-15 / 16-31][A register]
+        float mnew[2], corr[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             float mx = -INFINITY;
@@ -300,26 +326,35 @@ __global__ void __launch_bounds__(kPThreads) prefill_attn_kernel(PrefillArgs a) 
             for (int nt = 0; nt < 4; ++nt) mx = fmaxf(mx, fmaxf(sc[nt][i][0], sc[nt][i][1]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float mnew = fmaxf(m[i], mx);
-            const float corr = (m[i] == -INFINITY) ? 0.f : exp2f(m[i] - mnew);
+            mnew[i] = fmaxf(m[i], mx);
+            corr[i] = (m[i] == -INFINITY) ? 0.f : exp2f(m[i] - mnew[i]);
+        }
+        // rescale O only when a row of the warp has a new maximum (after the first steps
+        // of a long sequence, seldom)
+        if (__any_sync(0xffffffffu, corr[0] != 1.f || corr[1] != 1.f)) {
+#pragma unroll
+            for (int nt = 0; nt < 16; ++nt) {
+                acc[nt][0] *= corr[0];
+                acc[nt][1] *= corr[0];
+                acc[nt][2] *= corr[1];
+                acc[nt][3] *= corr[1];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
             float pw[4][2];
             float sum = 0.f;
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const float pr = (sc[nt][i][e] == -INFINITY) ? 0.f : exp2f(sc[nt][i][e] - mnew);
+                    const float pr = (sc[nt][i][e] == -INFINITY) ? 0.f : exp2f(sc[nt][i][e] - mnew[i]);
                     sum += pr;
                     // (a masked token's value norm is not read: it may be anything)
                     pw[nt][e] = pr > 0.f ? pr * ts[2 * kPT + nt * 8 + 2 * c + e] : 0.f;
                 }
-            l[i] = l[i] * corr + sum;
-            m[i] = mnew;
-#pragma unroll
-            for (int nt = 0; nt < 16; ++nt) {
-                acc[nt][2 * i] *= corr;
-                acc[nt][2 * i + 1] *= corr;
-            }
+            l[i] = l[i] * corr[i] + sum;
+            m[i] = mnew[i];
             // P' as A fragments of the value contraction (K-steps: tokens 0-15, 16-31)
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
@@ -327,16 +362,15 @@ __global__ void __launch_bounds__(kPThreads) prefill_attn_kernel(PrefillArgs a) 
                 pa[k][2 + i] = f2h2(pw[2 * k + 1][0], pw[2 * k + 1][1]);  // tokens 16k + 2c + 8, + 9
             }
         }
-        // O[16 x 128] += P' V: n-tile nt = coordinates 8 nt .. 8 nt + 7
+        // O[16 x 128] += P' V: n-tile nt = coordinates 8 nt .. 8 nt + 7; one transposing
+        // ldmatrix.x4 gives both K-steps' B fragments (lane l addresses token l,
+        // coordinates 8 nt .. 8 nt + 7)
 #pragma unroll
         for (int nt = 0; nt < 16; ++nt) {
-            const int coord = nt * 8 + g;
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const uint32_t b0w = *reinterpret_cast<const uint32_t*>(vt + coord * kVS + 16 * k + 2 * c);
-                const uint32_t b1w = *reinterpret_cast<const uint32_t*>(vt + coord * kVS + 16 * k + 2 * c + 8);
-                mma16816(acc[nt], pa[k][0], pa[k][1], pa[k][2], pa[k][3], b0w, b1w);
-            }
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4_trans(vt_addr + (uint32_t)(lane * kKS + 8 * nt) * 2, b0, b1, b2, b3);
+            mma16816(acc[nt], pa[0][0], pa[0][1], pa[0][2], pa[0][3], b0, b1);
+            mma16816(acc[nt], pa[1][0], pa[1][1], pa[1][2], pa[1][3], b2, b3);
         }
     }
 
