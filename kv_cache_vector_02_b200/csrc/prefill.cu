@@ -104,11 +104,12 @@ __device__ __forceinline__ uint32_t staged_word(const uint8_t* m, int r, int w) 
     return *reinterpret_cast<const uint32_t*>(m + r * 256 + ((((w >> 2) ^ (r & 7)) << 4) | ((w & 3) << 2)));
 }
 
-// The 16 packed codes of width w from bit 16 w t8 of a row (t8 = 0..7): 2 w bytes at a
-// 2 w-aligned offset.
-__device__ __forceinline__ uint64_t load_codes16(const uint8_t* row, int t8, int w) {
-    if (w == 4) return *reinterpret_cast<const uint64_t*>(row + 8 * t8);
-    if (w == 2) return *reinterpret_cast<const uint32_t*>(row + 4 * t8);
+// The 16 packed codes of width W from bit 16 W t8 of a row (t8 = 0..7): 2 W bytes at a
+// 2 W-aligned offset.
+template <int W>
+__device__ __forceinline__ uint64_t load_codes16(const uint8_t* row, int t8) {
+    if (W == 4) return *reinterpret_cast<const uint64_t*>(row + 8 * t8);
+    if (W == 2) return *reinterpret_cast<const uint32_t*>(row + 4 * t8);
     return *reinterpret_cast<const uint16_t*>(row + 2 * t8);
 }
 
@@ -121,14 +122,15 @@ struct PageBytes {
     uint32_t sw;
     float kn, kg, vn;
 };
+template <int WK, int WV>
 __device__ __forceinline__ PageBytes fetch_page(const PrefillArgs& a, int blk, int hk) {
     PageBytes r{};
     if (blk < 0 || blk >= a.num_blocks) return r;
     const uint8_t* kch = a.kc + ((size_t)blk * a.Hkv + hk) * a.lk.bytes;
     const uint8_t* vch = a.vc + ((size_t)blk * a.Hkv + hk) * a.lv.bytes;
     const int t = threadIdx.x & 15, t8 = (threadIdx.x >> 4) & 7;
-    r.kw = load_codes16(kch + t * a.lk.code_row, t8, a.cbk.width);
-    r.vw = load_codes16(vch + t * a.lv.code_row, t8, a.cbv.width);
+    r.kw = load_codes16<WK>(kch + t * a.lk.code_row, t8);
+    r.vw = load_codes16<WV>(vch + t * a.lv.code_row, t8);
     if (a.lk.prod) r.sw = *reinterpret_cast<const uint16_t*>(kch + a.lk.signs_off + t * (kDim / 8) + 2 * t8);
     if ((threadIdx.x & 127) < kPage) {
         r.kn = reinterpret_cast<const float*>(kch + a.lk.norm_off)[t] * a.qscale;
@@ -138,16 +140,17 @@ __device__ __forceinline__ PageBytes fetch_page(const PrefillArgs& a, int blk, i
     return r;
 }
 
-// A step's fp16 tiles from its bytes (levels from the shared-memory codebooks ck, cv):
+// A step's fp16 tiles from its bytes (levels from the shared-memory codebooks ck, cv;
+// code widths WK, WV):
 // each thread writes its token's 16 coordinates of the three [token][coordinate] tiles
 // as two 16-byte stores each (eight consecutive tokens of a quarter-warp cover the 32
 // banks once: rows are 16 bytes apart modulo 128).
+template <int WK, int WV>
 __device__ __forceinline__ void store_page_tiles(const PrefillArgs& a, const PageBytes& r, uint8_t* smem,
                                                  const __half* ck, const __half* cv) {
     float* ts = reinterpret_cast<float*>(smem + kPOffT);
     const int t = (threadIdx.x >> 7) * kPage + (threadIdx.x & 15), j0 = 16 * ((threadIdx.x >> 4) & 7);
-    const int wk = a.cbk.width, wv = a.cbv.width;
-    const uint32_t mk = (1u << wk) - 1u, mv = (1u << wv) - 1u;
+    constexpr uint32_t mk = (1u << WK) - 1u, mv = (1u << WV) - 1u;
     const uint32_t row = (uint32_t)(t * kKS + j0) * 2;
 #pragma unroll
     for (int hb = 0; hb < 2; ++hb) {  // coordinates j0 + 8 hb .. + 7: one 16-byte store per tile
@@ -155,8 +158,8 @@ __device__ __forceinline__ void store_page_tiles(const PrefillArgs& a, const Pag
 #pragma unroll
         for (int jj = 0; jj < 8; jj += 2) {
             const int j = 8 * hb + jj;
-            const __half k0 = ck[(uint32_t)(r.kw >> (j * wk)) & mk], k1 = ck[(uint32_t)(r.kw >> ((j + 1) * wk)) & mk];
-            const __half v0 = cv[(uint32_t)(r.vw >> (j * wv)) & mv], v1 = cv[(uint32_t)(r.vw >> ((j + 1) * wv)) & mv];
+            const __half k0 = ck[(uint32_t)(r.kw >> (j * WK)) & mk], k1 = ck[(uint32_t)(r.kw >> ((j + 1) * WK)) & mk];
+            const __half v0 = cv[(uint32_t)(r.vw >> (j * WV)) & mv], v1 = cv[(uint32_t)(r.vw >> ((j + 1) * WV)) & mv];
             kw[jj / 2] = h2bits(k0, k1);
             vw[jj / 2] = h2bits(v0, v1);
             // +-1 in fp16: 0xBC00 (-1) with bit 15 cleared where the sign bit is set
@@ -174,6 +177,7 @@ __device__ __forceinline__ void store_page_tiles(const PrefillArgs& a, const Pag
     }
 }
 
+template <int WK, int WV>
 __global__ void __launch_bounds__(kPThreads) prefill_attn_kernel(PrefillArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
@@ -259,23 +263,22 @@ __global__ void __launch_bounds__(kPThreads) prefill_attn_kernel(PrefillArgs a) 
         return pg < n_pages && TQ_DCHECK(pg < a.max_blocks, a.err) ? a.block_table[pg] : -1;
     };
     int blk_next = block_of(sub);
-    PageBytes nxt = fetch_page(a, blk_next, hk);
+    PageBytes nxt = fetch_page<WK, WV>(a, blk_next, hk);
     int blk_after = block_of(2 + sub);
     for (int step = 0; step < n_steps; ++step) {
-        const PageBytes cur = nxt;
-        const int blk_cur = blk_next;
-        if (step + 1 < n_steps) {
-            blk_next = blk_after;
-            nxt = fetch_page(a, blk_next, hk);
-            blk_after = block_of(2 * (step + 2) + sub);
-        }
         // pages of the step with a valid block (a page past the last is masked by the
         // causal limit: its positions exceed every query's)
         const int b0 = block_of(2 * step), b1 = block_of(2 * step + 1);
         const bool ok0 = b0 >= 0 && b0 < a.num_blocks;
         const bool ok1 = (2 * step + 1 >= n_pages) || (b1 >= 0 && b1 < a.num_blocks);
         __syncthreads();  // the previous step's tiles are read
-        if (blk_cur >= 0 && blk_cur < a.num_blocks) store_page_tiles(a, cur, smem, ck, cv);
+        if (blk_next >= 0 && blk_next < a.num_blocks) store_page_tiles<WK, WV>(a, nxt, smem, ck, cv);
+        // the next step's bytes, in flight during this step's contractions
+        if (step + 1 < n_steps) {
+            blk_next = blk_after;
+            nxt = fetch_page<WK, WV>(a, blk_next, hk);
+            blk_after = block_of(2 * (step + 2) + sub);
+        }
         if (threadIdx.x == 0 && !(ok0 && ok1)) atomicOr(a.err, TQ_DEVERR_BLOCK);
         __syncthreads();
         // scores of tokens nt*8 + 2c + e (nt = 0..3) for rows g (i = 0), g + 8 (i = 1)
@@ -465,10 +468,19 @@ cudaError_t launch_prefill(const tq_ctx* ctx, const uint16_t* q, const uint8_t* 
     a.out = out;
     a.out_fp32 = out_fp32;
     a.err = ctx->dev_error;
-    cudaError_t e = cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPSmem);
+    // code container widths (key, value): TQ4 and 3/4-bit MSE keys (4, 4), bits 3 prod
+    // keys (2, 4), TQ2 (1, 2), 2-bit MSE keys (2, 2)
+    void (*kern)(PrefillArgs) = nullptr;
+    const int wk = a.cbk.width, wv = a.cbv.width;
+    if (wk == 4 && wv == 4) kern = prefill_attn_kernel<4, 4>;
+    else if (wk == 2 && wv == 4) kern = prefill_attn_kernel<2, 4>;
+    else if (wk == 1 && wv == 2) kern = prefill_attn_kernel<1, 2>;
+    else if (wk == 2 && wv == 2) kern = prefill_attn_kernel<2, 2>;
+    else return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPSmem);
     if (e != cudaSuccess) return e;
     const dim3 grid((Tq + kPQ - 1) / kPQ, Hq);
-    prefill_attn_kernel<<<grid, kPThreads, kPSmem, stream>>>(a);
+    kern<<<grid, kPThreads, kPSmem, stream>>>(a);
     count_launches(1);
     return cudaGetLastError();
 }

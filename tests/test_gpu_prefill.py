@@ -61,6 +61,8 @@ def _oracle_cache(orc, o, T, Hkv, rng, law_scale=2.0):
     (16, 20, 2, 2, 2, 0, 0),     # TQ2: 1-bit key codes + signs, 2-bit values
     (3, 64, 1, 8, 3, 0, 1),      # MSE keys (3-bit), 3-bit values
     (100, 130, 2, 1, 4, 1, 1),   # MSE keys (4-bit), one query head per kv head
+    (40, 45, 2, 4, 3, 0, 0),     # bits 3 prod: 2-bit key codes + signs, 3-bit values
+    (0, 33, 1, 2, 2, 1, 1),      # MSE keys (2-bit), 2-bit values
 ])
 def test_prefill_on_oracle_cache(orc, q_start, Tq, Hkv, G, bits, rot, km):
     rng = np.random.default_rng(q_start * 7 + Tq)
