@@ -259,7 +259,8 @@ TQ_API tq_status tq_decode_attention_window(const tq_ctx* ctx, const uint16_t* q
  *   o_i = sum_{t <= q_start + i} softmax(s)_t * v_hat_t.
  * (Reading: the pages name the kernel and its inline decompression; the causal
  * prefix and the decode's estimator are the plainest reading.)
- *   q_dev          : [Tq][Hq][128] fp16, device, 16-byte aligned.
+ *   q_dev          : [Tq][Hq][128] fp16, device, 16-byte aligned; Hq 1 .. 65535, a
+ *                    multiple of Hkv (TQ_ERR_INVALID_ARG otherwise).
  *   block_table_dev: [max_blocks] int32, device; page p of the sequence lives in
  *                    physical block block_table[p].  A block id outside
  *                    [0, num_blocks) skips the page and sets TQ_DEVERR_BLOCK.

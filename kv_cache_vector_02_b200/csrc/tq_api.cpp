@@ -383,7 +383,7 @@ tq_status tq_prefill_attention(const tq_ctx* ctx, const uint16_t* q, const uint8
     NvtxRange nvtx("tq_prefill_attention");
     if (!ctx || ctx->host_only || Tq < 0 || q_start < 0 || Hq < 1 || Hkv < 1 || max_blocks < 0 || num_blocks < 0)
         return TQ_ERR_INVALID_ARG;
-    if (Hq % Hkv != 0) return TQ_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0 || Hq > 65535) return TQ_ERR_INVALID_ARG;  // one grid row per query head
     if (Tq == 0) return TQ_OK;
     if ((long long)q_start + Tq > (long long)max_blocks * tq::kPage) return TQ_ERR_INVALID_ARG;
     if (!q || !k_cache || !v_cache || !block_table || !out) return TQ_ERR_INVALID_ARG;

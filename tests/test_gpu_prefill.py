@@ -152,6 +152,12 @@ def test_prefill_bad_block_and_empty_chunk(orc):
                             torch.as_tensor(bt).to(dev), 0, out, Hkv=1)
     torch.cuda.synchronize()
     assert tq.tq_get_device_error(ctx) == 0
+    # more query heads than grid rows: refused on the host
+    qh = torch.zeros((1, 65536, 128), dtype=torch.float16, device=dev)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_prefill_attention(ctx, qh, torch.as_tensor(kc).to(dev), torch.as_tensor(vc).to(dev),
+                                torch.as_tensor(bt).to(dev), 0, torch.zeros_like(qh), Hkv=1)
+    assert e.value.status == tq.TQ_ERR_INVALID_ARG
 
 
 def test_prefill_ignores_rows_past_the_chunk(orc):
