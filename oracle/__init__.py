@@ -28,7 +28,14 @@ KIND_KEY, KIND_VALUE = 0, 1
 
 
 def build(force: bool = False) -> Path:
-    """Compile the oracle into ``oracle/liboracle.so`` (gcc, -O2, OpenMP)."""
+    """Compile the oracle into ``oracle/liboracle.so`` (gcc, -O2, OpenMP).
+
+    With ``TQ_ORACLE_LIB`` set in the environment, that library (a copy of the
+    oracle compiled elsewhere: the planted-mistake tests' mutants) is loaded
+    instead and nothing is compiled."""
+    override = os.environ.get("TQ_ORACLE_LIB")
+    if override:
+        return Path(override)
     if force or not _LIB.exists() or _LIB.stat().st_mtime < _SRC.stat().st_mtime:
         tmp = _LIB.with_suffix(".so.tmp%d" % os.getpid())
         cmd = ["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
