@@ -45,7 +45,11 @@ def test_whole_job_throughput_sums_the_ranks():
 
 
 def test_peak_is_the_measured_copy_bandwidth():
-    with open(os.path.join(bench.ROOT, "MEASURED_PEAKS.json")) as f:
+    p = os.path.join(bench.ROOT, "MEASURED_PEAKS.json")
+    if not os.path.exists(p):   # a checkout without the measured file: the stated fallback
+        assert bench.measured_peak() == (bench.FALLBACK_HBM_GBS, "fallback")
+        return
+    with open(p) as f:
         want = float(json.load(f)["hbm_gbs"])
     assert bench.measured_peak() == (want, "measured")
 
